@@ -1,0 +1,176 @@
+/*
+ * redlite_moe.h -- C ABI of the B200 (sm_100a) routed top-k MoE layer over
+ * codebook-quantised experts.
+ *
+ * The layer ("Red Metal dev8 -- resident routed top-k layer", steps 1-6):
+ * for every (token, slot) the selected expert runs gate, up, SiLU(gate)*up
+ * and down from its resident slot, and the layer accumulates
+ * out += router_weight * expert_output; an optional shared expert is added
+ * with weight 1 ("Red Lite dev16 -- complete full-attention parity", block
+ * composition: routed top-10 MoE plus shared expert).  Expert weights are
+ * packed in one of two codebook formats whose grids are expanded once before
+ * use ("Red Lite dev10 -- standalone native Metal path", section "Quant
+ * grids").
+ *
+ * Conventions for every entry point:
+ *   - Pointers documented "device" must be CUDA device (or managed) memory
+ *     of the current device; "host" pointers are ordinary CPU memory.
+ *   - The caller owns every buffer.  Entry points do not allocate device
+ *     memory and do not keep pointers after they return (the kernels they
+ *     enqueue read them until they complete).
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ *     stream).  Work is enqueued asynchronously; nothing synchronises except
+ *     where stated.
+ *   - Return values: REDLITE_OK (0) or a negative REDLITE_E* code for errors
+ *     found on the host (bad argument, unsupported shape, launch failure).
+ *     Errors only visible on the device (an expert id out of range, an
+ *     expert slot without matrices, a bounded wait that gave up) are ORed
+ *     into the caller's device status word as REDLITE_STATUS_* bits; the
+ *     offending (token, slot) pair contributes nothing.  No kernel traps.
+ *
+ * Packed matrix layout.  A matrix with `rows` outputs and `k` inputs is its
+ * rows*k weights in row-major order cut into consecutive 256-weight blocks
+ * (k a multiple of 256, or a divisor of 256 that is a multiple of 32).
+ *   IQ2_XS-style block, 74 bytes / 256 weights:
+ *     u16 d (fp16) | u8 scales[4] | u8 qs[32] | u8 qh[4] | u8 signs[32]
+ *     group g (weights 8g..8g+7): idx = qs[g] | bit (g&7) of qh[g>>3] << 8,
+ *     sc = nibble (g>>2)&1 of scales[g>>3],
+ *     w = d * (2sc+1)/8 * grid2[idx][j] * (bit j of signs[g] ? -1 : +1)
+ *   IQ1_M-style block, 56 bytes / 256 weights:
+ *     u16 d (fp16) | u8 qs[32] | u8 qh[16] | u8 scales[6]
+ *     nib = nibble (g&1) of qh[g>>1], idx = qs[g] | (nib&7) << 8,
+ *     delta = (nib & 8) ? -1/8 : +1/8, sc = bits 3(g>>1).. of the 48-bit
+ *     little-endian scales field,
+ *     w = d * (2sc+1) * (grid1[idx][j] + delta)
+ *   An expert is three matrices: gate [ffn x hidden], up [ffn x hidden],
+ *   down [hidden x ffn], each 16-byte aligned.
+ */
+#ifndef REDLITE_MOE_H
+#define REDLITE_MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum { REDLITE_Q_IQ2XS_STYLE = 1, REDLITE_Q_IQ1M_STYLE = 2 } redlite_qtype;
+
+enum {
+  REDLITE_OK = 0,
+  REDLITE_EINVAL = -1,       /* null pointer, bad size, bad enum, bad grid symbol */
+  REDLITE_EUNSUPPORTED = -2, /* shape outside what the kernels support */
+  REDLITE_ENOMEM = -3,       /* caller-provided workspace or pool too small */
+  REDLITE_ECUDA = -4         /* a CUDA call or kernel launch failed */
+};
+
+/* Bits ORed into the device status word. */
+enum {
+  REDLITE_STATUS_BAD_ID = 1,     /* an expert id outside [0, n_experts) */
+  REDLITE_STATUS_BAD_EXPERT = 2, /* selected slot has null matrices, bad qtype or shape */
+  REDLITE_STATUS_TIMEOUT = 4     /* a bounded in-kernel wait gave up */
+};
+
+/* One expert slot.  gate/up/down are device pointers to packed matrices. */
+typedef struct {
+  int32_t qtype; /* redlite_qtype */
+  int32_t ffn;   /* F, rows of gate and up, inputs of down */
+  const void *gate;
+  const void *up;
+  const void *down;
+} redlite_moe_expert;
+
+/* Everything a layer call needs besides its per-call tensors. */
+typedef struct {
+  int32_t hidden;    /* H */
+  int32_t n_experts; /* entries of `experts` */
+  int32_t max_ffn;   /* largest F of any expert (and of the shared expert) */
+  int32_t max_tokens;/* largest n_tokens the workspace was sized for */
+  const redlite_moe_expert *experts; /* device array [n_experts]: the slot table */
+  const void *grids;                 /* device, redlite_moe_grids_bytes(), from expand_grids */
+  void *workspace;                   /* device, caller-owned scratch */
+  size_t workspace_bytes;            /* >= redlite_moe_workspace_bytes(...) */
+  int32_t *status;                   /* device word; REDLITE_STATUS_* bits are ORed in */
+  void *stream;                      /* cudaStream_t */
+} redlite_moe_table;
+
+/* Bytes of the expanded-grid buffer expand_grids writes. */
+size_t redlite_moe_grids_bytes(void);
+
+/* Grid expansion ("Red Lite dev10", section "Quant grids"; done once before
+ * the pool is used).  iq2_compact: host [512] uint16, iq1_compact: host
+ * [2048] uint16; entry value j is symbol (c >> 2j) & 3, symbols 0,1,2 map to
+ * 8/25/43 (IQ2_XS-style) and -1/0/+1 (IQ1_M-style).  A symbol 3 anywhere
+ * returns REDLITE_EINVAL before anything is enqueued.  grids_dev: device,
+ * redlite_moe_grids_bytes() bytes, 256-byte aligned.  The host arrays may
+ * be reused as soon as the call returns (they are staged synchronously). */
+int redlite_moe_expand_grids(const uint16_t *iq2_compact, const uint16_t *iq1_compact, void *grids_dev,
+                             void *stream);
+
+/* Packed bytes of a rows x k matrix, or 0 if the shape is not supported. */
+size_t redlite_moe_matrix_bytes(int32_t qtype, int64_t rows, int64_t k);
+
+/* Device scratch a layer call needs for these limits. */
+size_t redlite_moe_workspace_bytes(int32_t hidden, int32_t n_experts, int32_t max_tokens, int32_t top_k,
+                                   int32_t max_ffn);
+
+/* Zero the workspace's control words (call once after allocating it, and
+ * after a call reported REDLITE_STATUS_TIMEOUT).  Enqueued on table->stream. */
+int redlite_moe_workspace_reset(const redlite_moe_table *table);
+
+/* The routed layer ("Red Metal dev8", steps 4-6).
+ *   x              device [n_tokens, hidden] fp32, row-major
+ *   n_tokens       0 .. table->max_tokens (0 returns REDLITE_OK, enqueues nothing)
+ *   expert_ids     device [n_tokens, top_k] int32
+ *   router_weights device [n_tokens, top_k] fp32, used as given (no renormalisation)
+ *   top_k          1 .. 16
+ *   expert_table   host struct (its device pointers are read by the kernels)
+ *   shared_expert  host struct with device matrix pointers, or NULL
+ *   out            device [n_tokens, hidden] fp32, overwritten (not accumulated into)
+ * Enqueued on expert_table->stream; x, ids, weights and out must not be
+ * written by other work until it completes.  Two calls that share a
+ * workspace must be ordered on one stream.  Decode-sized calls run one
+ * fused kernel; calls with many tokens per expert run the bucketed
+ * tensor-core path (bf16 operands, fp32 accumulation). */
+int redlite_moe_layer(const float *x, int32_t n_tokens, const int32_t *expert_ids, const float *router_weights,
+                      int32_t top_k, const redlite_moe_table *expert_table, const redlite_moe_expert *shared_expert,
+                      float *out);
+
+/* Dequantise one packed matrix (the bit-exactness check of the decoders).
+ * packed: device; out_f32: device [rows*k] fp32 or NULL; out_bf16: device
+ * [rows*k] bf16 bits (round to nearest even) or NULL.  grids: expanded. */
+int redlite_moe_dequant(int32_t qtype, const void *packed, int64_t rows, int64_t k, const void *grids, float *out_f32,
+                        uint16_t *out_bf16, void *stream);
+
+/* Slot-table builder: copies experts from host memory into a device pool
+ * and writes their slot descriptors ("Red Metal dev8", steps 1-3: every
+ * selected expert made resident, three positional reads per expert).
+ *   hidden       H of the layer (sizes the matrices with each expert's ffn)
+ *   ids          host [n] expert ids (slot index in table_dev)
+ *   host_experts host [n]; gate/up/down are HOST pointers to packed bytes
+ *   pool         device, pool_bytes, 16-byte aligned; matrices are placed
+ *                back to back at 16-byte aligned offsets from `pool_offset`
+ *   table_dev    device [n_experts] slot table; entries ids[i] are written
+ *   counters     host, optional: {loads, copies, bytes} are added to it
+ *   pool_end     host, optional: receives the first free pool offset
+ * Shapes are checked and placement is planned before anything is copied:
+ * REDLITE_EUNSUPPORTED for a shape the kernels do not take, REDLITE_ENOMEM
+ * if the pool is too small.  Three host->device copies per expert plus one
+ * descriptor copy are enqueued on `stream`, then the call synchronises the
+ * stream, so host buffers may be released when it returns. */
+typedef struct {
+  int64_t loads;  /* experts made resident */
+  int64_t copies; /* host->device matrix copies (3 per expert) */
+  int64_t bytes;  /* packed bytes copied */
+} redlite_moe_upload_counters;
+
+int redlite_moe_upload_experts(int32_t hidden, const int32_t *ids, const redlite_moe_expert *host_experts, int32_t n,
+                               void *pool, size_t pool_bytes, size_t pool_offset, redlite_moe_expert *table_dev,
+                               int32_t n_experts, void *stream, redlite_moe_upload_counters *counters,
+                               size_t *pool_end);
+
+#ifdef __cplusplus
+}
+#endif
+#endif

@@ -1,0 +1,102 @@
+"""The C-ABI library loads without a GPU and exports every entry point that
+include/redlite_moe.h declares; host-only argument checks answer without
+touching the device."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _declared():
+    names = set()
+    for fn in os.listdir(os.path.join(ROOT, "include")):
+        if fn.endswith(".h"):
+            txt = open(os.path.join(ROOT, "include", fn)).read()
+            txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
+            names |= set(re.findall(r"^\s*(?:[\w\s\*]+?)\b(redlite_\w+)\s*\(", txt, flags=re.M))
+    return names
+
+
+@pytest.fixture(scope="module")
+def native():
+    from routed_expert_ffn_iq2_b200 import build
+
+    build.build()
+    import routed_expert_ffn_iq2_b200 as P
+
+    return P
+
+
+def test_every_declared_symbol_exported(native):
+    declared = _declared()
+    assert len(declared) >= 8
+    lib = native.lib()
+    for name in declared:
+        assert hasattr(lib, name), name
+    assert declared == set(native.EXPORTS), (declared ^ set(native.EXPORTS))
+
+
+def test_host_only_sizes(native):
+    assert native.redlite_moe_matrix_bytes(1, 512, 2048) == 303104
+    assert native.redlite_moe_matrix_bytes(2, 512, 2048) == 229376
+    assert native.redlite_moe_matrix_bytes(1, 2048, 512) == 303104
+    assert native.redlite_moe_matrix_bytes(1, 256, 64) == 64 * 74
+    assert native.redlite_moe_matrix_bytes(1, 256, 48) == 0
+    assert native.redlite_moe_matrix_bytes(3, 512, 2048) == 0
+    assert native.redlite_moe_grids_bytes() >= 512 * 8 + 2048 * 8
+    assert native.redlite_moe_workspace_bytes(2048, 512, 64, 10, 512) > 64 * 11 * 512 * 4
+    assert native.redlite_moe_workspace_bytes(0, 512, 64, 10, 512) == 0
+
+
+def test_expand_grids_rejects_symbol3_before_device_work(native):
+    g2 = np.zeros(512, np.uint16)
+    g1 = np.zeros(2048, np.uint16)
+    g2[7] = 0x0300
+    rc = native.lib().redlite_moe_expand_grids(g2.ctypes.data_as(ctypes.c_void_p), g1.ctypes.data_as(ctypes.c_void_p),
+                                               ctypes.c_void_p(256), None)
+    assert rc == native.REDLITE_EINVAL
+    rc = native.lib().redlite_moe_expand_grids(None, g1.ctypes.data_as(ctypes.c_void_p), ctypes.c_void_p(256), None)
+    assert rc == native.REDLITE_EINVAL
+
+
+def test_layer_rejects_bad_arguments_on_host(native):
+    L = native.lib()
+    t = native.redlite_moe_table(2048, 512, 512, 64, 0x1000, 0x2000, 0x3000, 1 << 30, 0x4000, None)
+    p = ctypes.c_void_p(0x10000)
+    # null table
+    assert L.redlite_moe_layer(p, 1, p, p, 10, None, None, p) == native.REDLITE_EINVAL
+    # top_k out of range
+    assert L.redlite_moe_layer(p, 1, p, p, 0, ctypes.byref(t), None, p) == native.REDLITE_EINVAL
+    assert L.redlite_moe_layer(p, 1, p, p, 17, ctypes.byref(t), None, p) == native.REDLITE_EINVAL
+    # n_tokens above the table's limit, negative
+    assert L.redlite_moe_layer(p, 65, p, p, 10, ctypes.byref(t), None, p) == native.REDLITE_EINVAL
+    assert L.redlite_moe_layer(p, -1, p, p, 10, ctypes.byref(t), None, p) == native.REDLITE_EINVAL
+    # zero tokens: nothing to do
+    assert L.redlite_moe_layer(None, 0, None, None, 10, ctypes.byref(t), None, None) == native.REDLITE_OK
+    # null tensors
+    assert L.redlite_moe_layer(None, 1, p, p, 10, ctypes.byref(t), None, p) == native.REDLITE_EINVAL
+    # misaligned x
+    assert L.redlite_moe_layer(ctypes.c_void_p(0x10004), 1, p, p, 10, ctypes.byref(t), None, p) == native.REDLITE_EINVAL
+    # workspace too small
+    t2 = native.redlite_moe_table(2048, 512, 512, 64, 0x1000, 0x2000, 0x3000, 1024, 0x4000, None)
+    assert L.redlite_moe_layer(p, 1, p, p, 10, ctypes.byref(t2), None, p) == native.REDLITE_ENOMEM
+    # bad shared expert (bad qtype / unsupported shape)
+    sh = native.redlite_moe_expert(3, 512, 0x1000, 0x2000, 0x3000)
+    assert L.redlite_moe_layer(p, 1, p, p, 10, ctypes.byref(t), ctypes.byref(sh), p) == native.REDLITE_EINVAL
+    sh = native.redlite_moe_expert(1, 48, 0x1000, 0x2000, 0x3000)
+    assert L.redlite_moe_layer(p, 1, p, p, 10, ctypes.byref(t), ctypes.byref(sh), p) == native.REDLITE_EINVAL
+    # hidden not a multiple of 32
+    t3 = native.redlite_moe_table(2047, 512, 512, 64, 0x1000, 0x2000, 0x3000, 1 << 30, 0x4000, None)
+    assert L.redlite_moe_layer(p, 1, p, p, 10, ctypes.byref(t3), None, p) == native.REDLITE_EINVAL
+
+
+def test_dequant_rejects_on_host(native):
+    L = native.lib()
+    p = ctypes.c_void_p(0x10000)
+    assert L.redlite_moe_dequant(3, p, 1, 256, p, p, None, None) == native.REDLITE_EINVAL
+    assert L.redlite_moe_dequant(1, p, 1, 300, p, p, None, None) == native.REDLITE_EUNSUPPORTED
+    assert L.redlite_moe_dequant(1, p, 1, 256, p, None, None, None) == native.REDLITE_EINVAL

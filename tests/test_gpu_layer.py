@@ -1,0 +1,178 @@
+"""Layer parity of the CUDA path against the fp64 oracle on the seeded
+workloads, plus invariants and device-side error reporting.
+
+Tolerance: max|gpu - oracle| <= tol * max|oracle| with tol = 1e-4 for the
+fp32-accumulate decode path and 2e-2 for the bf16 tensor-core path."""
+import numpy as np
+import pytest
+import torch
+
+import fixtures
+
+pytestmark = pytest.mark.gpu
+
+TOL_FP32 = 1e-4
+TOL_BF16 = 2e-2
+
+
+@pytest.fixture(scope="module")
+def P():
+    from routed_expert_ffn_iq2_b200 import build
+
+    build.build()
+    import routed_expert_ffn_iq2_b200 as P
+
+    return P
+
+
+def _dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def _run(L, x, ids, wt):
+    out = L(_dev(x), _dev(ids), _dev(wt))
+    torch.cuda.synchronize()
+    return out.cpu().numpy().astype(np.float64)
+
+
+def _rel_err(got, ref):
+    return np.abs(got - ref).max() / np.abs(ref).max()
+
+
+@pytest.mark.parametrize("cfg", [1, 2, 3])
+def test_decode_workloads(P, oracle_lib, cfg):
+    w = fixtures.workload(cfg)
+    L = P.layer_for_workload(w)
+    got = _run(L, w.x, w.ids, w.weights)
+    ref = oracle_lib.workload_layer(w)
+    assert L.read_status() == 0
+    assert _rel_err(got, ref) <= TOL_FP32
+
+
+def test_cold_upload_counters(P):
+    """A cold top-10 selection makes 10 experts resident with 30 matrix copies."""
+    w = fixtures.workload(3)
+    L = P.layer_for_workload(w)
+    assert (L.counters.loads, L.counters.copies) == (10, 30)
+    assert L.counters.bytes == 10 * fixtures.expert_bytes(2, 2048, 512)
+
+
+def test_batched_decode_workload(P, oracle_lib):
+    w = fixtures.workload(4)
+    L = P.layer_for_workload(w)
+    got = _run(L, w.x, w.ids, w.weights)
+    ref = oracle_lib.workload_layer(w)
+    assert L.read_status() == 0
+    assert _rel_err(got, ref) <= TOL_FP32
+
+
+def test_prefill_small(P, oracle_lib):
+    w = fixtures.workload(5, n_tokens=192)
+    L = P.layer_for_workload(w)
+    got = _run(L, w.x, w.ids, w.weights)
+    ref = oracle_lib.workload_layer(w)
+    assert L.read_status() == 0
+    assert _rel_err(got, ref) <= TOL_BF16
+
+
+def test_prefill_full_sampled(P, oracle_lib):
+    w = fixtures.workload(5)
+    L = P.layer_for_workload(w)
+    got = _run(L, w.x, w.ids, w.weights)
+    sample = np.arange(0, 4096, 173)
+    ref = oracle_lib.workload_layer(w, tokens=sample)
+    assert L.read_status() == 0
+    assert _rel_err(got[sample], ref) <= TOL_BF16
+    assert np.isfinite(got).all()
+
+
+def test_slot_order_and_zero_weight(P):
+    w = fixtures.workload(2)
+    L = P.layer_for_workload(w)
+    base = _run(L, w.x, w.ids, w.weights)
+    perm = np.array([3, 9, 0, 5, 1, 8, 2, 7, 4, 6])
+    permuted = _run(L, w.x, w.ids[:, perm], w.weights[:, perm])
+    assert _rel_err(permuted, base) <= TOL_FP32
+    w0 = w.weights.copy()
+    w0[0, 4] = 0.0
+    zeroed = _run(L, w.x, w.ids, w0)
+    dropped = _run(L, w.x, np.delete(w.ids, 4, axis=1), np.delete(w.weights, 4, axis=1))
+    assert _rel_err(zeroed, dropped) <= TOL_FP32
+
+
+def test_aliased_ids_equal_single_expert(P):
+    w = fixtures.workload(2)
+    L = P.layer_for_workload(w)
+    e = int(w.ids[0, 0])
+    ids = np.full((1, 4), e, np.int32)
+    wt = np.array([[0.125, 0.25, 0.375, 0.25]], np.float32)
+    many = _run(L, w.x, ids, wt)
+    one = _run(L, w.x, ids[:, :1], np.ones((1, 1), np.float32))
+    assert _rel_err(many, one) <= TOL_FP32
+
+
+def test_bad_ids_reported_and_skipped(P, oracle_lib):
+    w = fixtures.workload(2)
+    L = P.layer_for_workload(w)
+    ids = w.ids.copy()
+    ids[0, 2] = 512
+    ids[0, 6] = -3
+    got = _run(L, w.x, ids, w.weights)
+    assert L.read_status() & P.REDLITE_STATUS_BAD_ID
+    L.clear_status()
+    w0 = w.weights.copy()
+    w0[0, 2] = w0[0, 6] = 0
+    ref = _run(L, w.x, w.ids, w0)
+    assert _rel_err(got, ref) <= TOL_FP32
+    assert L.read_status() == 0
+
+
+def test_missing_expert_reported(P):
+    w = fixtures.workload(2)
+    L = P.layer_for_workload(w)
+    ids = w.ids.copy()
+    free = next(e for e in range(512) if e not in set(w.ids[0].tolist()))
+    ids[0, 0] = free  # slot never uploaded: null matrices
+    _run(L, w.x, ids, w.weights)
+    assert L.read_status() & P.REDLITE_STATUS_BAD_EXPERT
+
+
+def test_max_topk_and_ragged_shapes(P, oracle_lib):
+    """top_k = 16, hidden 768, ffn 128 (down rows of half a block), a shared expert of width 256,
+    7 tokens (ragged against the 4-token passes)."""
+    H, E, F, k, T = 768, 24, 128, 16, 7
+    seed = 4242
+    g2 = fixtures.make_grid(seed, 1)
+    g1 = fixtures.make_grid(seed, 2)
+    experts = [fixtures.make_expert(seed, 1 + (e % 2), H, F, e) for e in range(E)]
+    st = fixtures.Stream(seed, 3)
+    ids = st.randint(T * k, E).astype(np.int32).reshape(T, k)
+    wt = (0.1 + st.uniform(T * k)).astype(np.float32).reshape(T, k)
+    x = fixtures.make_x(seed, T, H)
+    shared = fixtures.make_expert(seed, 2, H, 2 * F, 777)
+    L = P.MoeLayer(H, E, 2 * F, T, k, g2, g1, pool_bytes=(E + 2) * fixtures.expert_bytes(1, H, 2 * F) + 4096)
+    assert L.upload(list(range(E)), experts) == 0
+    assert L.set_shared(shared) == 0
+    got = _run(L, x, ids, wt)
+    ref = oracle_lib.moe_layer(x, ids, wt, experts, shared, oracle_lib.expand_grid(1, g2),
+                               oracle_lib.expand_grid(2, g1))
+    assert _rel_err(got, ref) <= TOL_FP32
+
+
+def test_zero_tokens_noop(P):
+    w = fixtures.workload(1)
+    L = P.layer_for_workload(w)
+    out = torch.full((1, 256), 7.0, device="cuda")
+    e = torch.zeros((1, 4), dtype=torch.int32, device="cuda")
+    rc = P.redlite_moe_layer(out, 0, e, out, 4, L.table, None, out)
+    torch.cuda.synchronize()
+    assert rc == 0 and float(out[0, 0]) == 7.0
+
+
+def test_repeat_calls_reuse_workspace(P):
+    w = fixtures.workload(2)
+    L = P.layer_for_workload(w)
+    a = _run(L, w.x, w.ids, w.weights)
+    for _ in range(3):
+        b = _run(L, w.x, w.ids, w.weights)
+    assert _rel_err(b, a) <= TOL_FP32
