@@ -1,0 +1,405 @@
+"""Benchmark of the routed top-k MoE layer (one JSON line on rank 0).
+
+Default workload: the Qwen3-Next-shaped decode layer with IQ2_XS-style
+experts (hidden 2048, 512 experts of width 512, top-10, one token per call).
+A step is one layer call over one token.  All 512 experts are resident; the
+steps cycle through 48 pairwise-disjoint top-10 sets (480 experts, 436 MB of
+packed weights, far above the 126 MB L2), so every step streams its experts
+from HBM.  Steps are issued as CUDA-graph replays of the C-ABI call.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config 2..5]
+  python bench.py --impl reference ...   # the fp64 CPU oracle, timed on host cores
+
+Multi-GPU (torchrun): every rank runs an independent replica (the layer has no
+exchange step); value = all ranks' tokens / the slowest rank's device time.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import fixtures  # noqa: E402
+
+METRIC = "routed-MoE-layer tokens/sec on 1 B200; achieved HBM GB/s vs ~8 TB/s peak"
+N_SETS = 48
+GRAPH_CYCLES = 5  # graph = GRAPH_CYCLES * N_SETS calls for the decode workloads
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": d["hbm_gbs"], "bf16_tflops": d["bf16_tflops"],
+                "bf16_tflops_sustained": d.get("bf16_tflops_sustained", d["bf16_tflops"]), "src": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "src": "fallback"}
+
+
+class ClockSampler:
+    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+             "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+             "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.QUERY}",
+                                          "--format=csv,noheader,nounits", "-lms", "100"],
+                                         stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        out, _ = self.proc.communicate(timeout=10)
+        rows = [r.split(",") for r in out.strip().splitlines() if r.count(",") >= 8]
+        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if "Active" in r[5 + i] and "Not" not in r[5 + i]})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+def _source_sha():
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "routed_expert_ffn_iq2_b200", "csrc")
+    for fn in sorted(os.listdir(csrc)):
+        h.update(open(os.path.join(csrc, fn), "rb").read())
+    return h.hexdigest()[:16]
+
+
+def _traffic(kernel_key: str):
+    """DRAM bytes per launch from the committed ncu summary, if the kernel
+    sources have not changed since it was taken (else None)."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    d = json.load(open(p)).get(kernel_key)
+    if not d or d.get("source_sha") != _source_sha():
+        return None
+    return d.get("dram_bytes_per_launch")
+
+
+# ------------------------------------------------------------------ workloads
+
+
+class Problem:
+    """Per-config inputs: `sets` of (x [T,H], ids [T,k], weights [T,k]) cycled by the steps."""
+
+    def __init__(self, cfg: int):
+        self.cfg = cfg
+        seed = fixtures.SEED_BASE + cfg
+        if cfg in (2, 3):
+            self.w = fixtures.workload(cfg)
+            ids = fixtures.decode_id_sets(seed, N_SETS, self.w.top_k, self.w.n_experts)
+            st = fixtures.Stream(seed, 6)
+            wts = [fixtures.normalised_positive_weights(st, self.w.top_k)[None, :] for _ in range(N_SETS)]
+            xs = fixtures.make_x(seed, N_SETS, self.w.hidden, tag=7)
+            self.sets = [(xs[i:i + 1], ids[i:i + 1], wts[i]) for i in range(N_SETS)]
+            self.resident = sorted(set(ids.reshape(-1).tolist()))
+        elif cfg in (4, 5):
+            self.w = fixtures.workload(cfg)
+            self.sets = [(self.w.x, self.w.ids, self.w.weights)]
+            self.resident = self.w.selected()
+        else:
+            raise SystemExit("bench supports --config 2..5 (config 1 is a parity case)")
+        w = self.w
+        self.tokens_per_step = self.sets[0][0].shape[0]
+        self.step_bytes = []
+        self.step_flops = []
+        sh = w.shared()
+        for x, ids, _ in self.sets:
+            uniq = sorted(set(ids.reshape(-1).tolist()))
+            b = sum(fixtures.expert_bytes(int(w.qtypes[e]), w.hidden, w.ffn) for e in uniq)
+            if sh is not None:
+                b += sh.nbytes
+            b += x.nbytes * 2 + ids.nbytes * 2  # x in, out back, ids and weights in
+            self.step_bytes.append(b)
+            pairs = ids.size + (x.shape[0] if sh is not None else 0)
+            self.step_flops.append(2.0 * 3 * w.hidden * w.ffn * pairs)
+
+    def name(self):
+        return self.w.name
+
+
+def _oracle_step(oracle, P: Problem, i: int, cache):
+    w = P.w
+    x, ids, wt = P.sets[i % len(P.sets)]
+    experts = [None] * w.n_experts
+    for e in set(ids.reshape(-1).tolist()):
+        experts[e] = w.expert(e)
+    if "grids" not in cache:
+        cache["grids"] = (oracle.expand_grid(1, w.grid_iq2), oracle.expand_grid(2, w.grid_iq1))
+    g2, g1 = cache["grids"]
+    return oracle.moe_layer(x, ids, wt, experts, w.shared(), g2, g1)
+
+
+def cpu_oracle_rate(P: Problem, budget_s: float, max_steps: int):
+    """Time the fp64 oracle as it stands on the host cores: steps/s (tokens/s)."""
+    import oracle
+
+    cores = oracle.set_threads(0)
+    cache = {}
+    if P.cfg == 5:
+        # bounded sample: the first 32 tokens of the prefill batch
+        sub = Problem.__new__(Problem)
+        sub.__dict__.update(P.__dict__)
+        x, ids, wt = P.sets[0]
+        sub.sets = [(x[:32], ids[:32], wt[:32])]
+        P = sub
+    _oracle_step(oracle, P, 0, cache)  # warm (grid expansion, expert bytes)
+    t0 = time.perf_counter()
+    n = 0
+    while n < max_steps:
+        _oracle_step(oracle, P, n, cache)
+        n += 1
+        if time.perf_counter() - t0 > budget_s:
+            break
+    dt = time.perf_counter() - t0
+    toks = n * P.sets[0][0].shape[0]
+    sample = f"{n} layer calls x {P.sets[0][0].shape[0]} token(s) of {P.name()}, fp64 oracle, {dt:.1f} s"
+    return toks / dt, cores, sample
+
+
+# ------------------------------------------------------------------ main
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=0)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", type=int, default=2)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--cpu-budget", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        P = Problem(args.config)
+        rate, cores, sample = cpu_oracle_rate(P, args.cpu_budget, max_steps=max(args.steps, 1) * 48)
+        peaks = _peaks()
+        line = {
+            "impl": "reference", "metric": METRIC, "value": rate, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * P.tokens_per_step / rate,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": P.name(), "tokens_per_step": P.tokens_per_step},
+            "cpu_baseline": {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": rate, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "peaks_src": peaks["src"],
+        }
+        print(json.dumps(line), flush=True)
+        return
+
+    import torch
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    from routed_expert_ffn_iq2_b200 import build as B
+
+    B.build()
+    import routed_expert_ffn_iq2_b200 as R
+
+    P = Problem(args.config)
+    w = P.w
+    stream = torch.cuda.Stream(dev)
+    torch.cuda.set_stream(stream)
+    per = max(fixtures.expert_bytes(q, w.hidden, w.ffn) for q in (1, 2)) + 64
+    sh = w.shared()
+    pool = per * len(P.resident) + (sh.nbytes + 64 if sh is not None else 0)
+    max_tok = P.tokens_per_step
+    L = R.MoeLayer(w.hidden, w.n_experts, max(w.ffn, w.shared_ffn), max_tok, w.top_k, w.grid_iq2, w.grid_iq1,
+                   pool, device=str(dev), stream=stream)
+    for i in range(0, len(P.resident), 32):
+        chunk = P.resident[i:i + 32]
+        R._native._check(L.upload(chunk, [w.expert(e) for e in chunk]), "upload")
+        if rank != 0:
+            for e in chunk:
+                w._experts.pop(e, None)
+    if sh is not None:
+        R._native._check(L.set_shared(sh), "set_shared")
+
+    dx = [torch.from_numpy(np.ascontiguousarray(s[0])).to(dev) for s in P.sets]
+    di = [torch.from_numpy(np.ascontiguousarray(s[1])).to(dev) for s in P.sets]
+    dw = [torch.from_numpy(np.ascontiguousarray(s[2])).to(dev) for s in P.sets]
+    do = [torch.empty((s[0].shape[0], w.hidden), dtype=torch.float32, device=dev) for s in P.sets]
+    nsets = len(P.sets)
+
+    def call(i):
+        j = i % nsets
+        rc = R.redlite_moe_layer(dx[j], dx[j].shape[0], di[j], dw[j], w.top_k, L.table, L.shared, do[j])
+        if rc != 0:
+            raise RuntimeError(f"redlite_moe_layer rc={rc}")
+
+    # graph of G calls
+    G = GRAPH_CYCLES * nsets if nsets > 1 else 10
+    steps = args.steps if args.steps > 0 else (G * 800 if nsets > 1 else (200 if P.cfg == 4 else 30))
+    steps = ((steps + G - 1) // G) * G
+    for i in range(max(args.warmup, 3)):
+        call(i)
+    stream.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph, stream=stream):
+        for i in range(G):
+            call(i)
+    reps_w = max(1, (max(args.warmup, 3) + G - 1) // G)
+    for _ in range(reps_w):
+        graph.replay()
+    stream.synchronize()
+    if L.read_status() != 0:
+        raise RuntimeError(f"device status {L.read_status()}")
+
+    def barrier():
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.barrier()
+
+    clk = ClockSampler(local)
+    barrier()
+    torch.cuda.synchronize()
+    clk.start()
+    time.sleep(0.3)
+    ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    ev0.record(stream)
+    for _ in range(steps // G):
+        graph.replay()
+    ev1.record(stream)
+    ev1.synchronize()
+    torch.cuda.synchronize()
+    barrier()
+    clocks = clk.stop()
+    ms = ev0.elapsed_time(ev1)
+    if world > 1:
+        import torch.distributed as dist
+
+        t = torch.tensor([ms], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    launches_per_call = R.launches_per_call(dx[0].shape[0], w.top_k, sh is not None)
+    del graph
+
+    # end-to-end through the public call with host buffers (pinned), per step:
+    # H2D of x, ids, weights; the layer; D2H of out.
+    e2e = None
+    if not args.no_e2e:
+        hx = [torch.from_numpy(np.ascontiguousarray(s[0])).pin_memory() for s in P.sets]
+        hi = [torch.from_numpy(np.ascontiguousarray(s[1])).pin_memory() for s in P.sets]
+        hw = [torch.from_numpy(np.ascontiguousarray(s[2])).pin_memory() for s in P.sets]
+        ho = [torch.empty((s[0].shape[0], w.hidden), dtype=torch.float32).pin_memory() for s in P.sets]
+        e_steps = min(steps, 2000 if nsets > 1 else steps)
+
+        def e2e_step(i):
+            j = i % nsets
+            dx[j].copy_(hx[j], non_blocking=True)
+            di[j].copy_(hi[j], non_blocking=True)
+            dw[j].copy_(hw[j], non_blocking=True)
+            call(j)
+            ho[j].copy_(do[j], non_blocking=True)
+
+        for i in range(3):
+            e2e_step(i)
+        stream.synchronize()
+        barrier()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for i in range(e_steps):
+            e2e_step(i)
+        e1.record(stream)
+        e1.synchronize()
+        barrier()
+        ems = e0.elapsed_time(e1)
+        if world > 1:
+            import torch.distributed as dist
+
+            t = torch.tensor([ems], device=dev)
+            dist.all_reduce(t, op=dist.ReduceOp.MAX)
+            ems = float(t.item())
+        h2d = hx[0].nbytes + hi[0].nbytes + hw[0].nbytes
+        e2e = {"value": world * e_steps * P.tokens_per_step / (ems / 1e3), "unit": "tokens/s",
+               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(ho[0].nbytes), "steps": e_steps}
+
+    if L.read_status() != 0:
+        raise RuntimeError(f"device status {L.read_status()}")
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, cores, sample = cpu_oracle_rate(P, args.cpu_budget, max_steps=10 ** 6)
+        cpu = {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample}
+
+    if rank == 0:
+        peaks = _peaks()
+        sec = ms / 1e3
+        per_step_s = sec / steps
+        mean_bytes = float(np.mean([P.step_bytes[i % nsets] for i in range(G)]))
+        mean_flops = float(np.mean([P.step_flops[i % nsets] for i in range(G)]))
+        tok_s = world * steps * P.tokens_per_step / sec
+        if P.cfg == 5:
+            ach = mean_flops / per_step_s / 1e12
+            peak = peaks["bf16_tflops_sustained"]
+            roof = {"bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s", "frac": ach / peak,
+                    "traffic": _traffic("prefill"), "peak_kind": f"{peaks['src']} bf16 sustained"}
+        else:
+            ach = mean_bytes / per_step_s / 1e9
+            peak = peaks["hbm_gbs"]
+            roof = {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak,
+                    "traffic": _traffic("decode" if P.cfg in (2, 3) else "batched"),
+                    "peak_kind": f"{peaks['src']} HBM copy"}
+        line = {
+            "metric": METRIC, "value": tok_s, "unit": "tokens/s", "n_gpus": world, "steps": steps,
+            "warmup": args.warmup, "ms_per_step": ms / steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32" if P.cfg != 5 else "bf16", "data": "synthetic",
+            "config": {"workload": P.name(), "tokens_per_step": P.tokens_per_step,
+                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                       "l2": ("inputs larger than L2: steps cycle 48 disjoint top-10 sets over 480 resident "
+                              "experts (436 MB)" if nsets > 1 else "inputs larger than L2 (expert bytes per step "
+                              f"{mean_bytes / 1e6:.0f} MB)"),
+                       "issue": f"CUDA graph of {G} layer calls, replayed"},
+            "weight_gbs": mean_bytes / per_step_s / 1e9,
+            "roofline": roof,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": launches_per_call * steps,
+            "clocks": clocks,
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -44,6 +44,14 @@
  *     w = d * (2sc+1) * (grid1[idx][j] + delta)
  *   An expert is three matrices: gate [ffn x hidden], up [ffn x hidden],
  *   down [hidden x ffn], each 16-byte aligned.
+ *
+ * Resident layout.  Matrices held in a slot (and read by every kernel) are
+ * in the library's resident layout: for rows a multiple of 16 and k a
+ * multiple of 256 it is the same bytes regrouped per tile of 16 rows x 256
+ * inputs so that each tensor-core lane reads its fields with wide loads
+ * (redlite_moe_pack_matrix converts; redlite_moe_upload_experts does it
+ * for you); for other shapes it is the interchange layout unchanged.  Both
+ * layouts have the same size (redlite_moe_matrix_bytes).
  */
 #ifndef REDLITE_MOE_H
 #define REDLITE_MOE_H
@@ -87,6 +95,12 @@ typedef struct {
   int32_t n_experts; /* entries of `experts` */
   int32_t max_ffn;   /* largest F of any expert (and of the shared expert) */
   int32_t max_tokens;/* largest n_tokens the workspace was sized for */
+  int32_t min_ffn;   /* smallest F of any expert (incl. shared), 0 if unknown.
+                      * Valid widths are 32, 64, 128 or multiples of 256, so
+                      * min_ffn >= 256 tells the call that every expert has
+                      * the tiled layout the fast paths need; otherwise the
+                      * general path runs. */
+  int32_t reserved;  /* 0 */
   const redlite_moe_expert *experts; /* device array [n_experts]: the slot table */
   const void *grids;                 /* device, redlite_moe_grids_bytes(), from expand_grids */
   void *workspace;                   /* device, caller-owned scratch */
@@ -137,18 +151,27 @@ int redlite_moe_layer(const float *x, int32_t n_tokens, const int32_t *expert_id
                       int32_t top_k, const redlite_moe_table *expert_table, const redlite_moe_expert *shared_expert,
                       float *out);
 
-/* Dequantise one packed matrix (the bit-exactness check of the decoders).
- * packed: device; out_f32: device [rows*k] fp32 or NULL; out_bf16: device
- * [rows*k] bf16 bits (round to nearest even) or NULL.  grids: expanded. */
+/* Host-side conversion of one matrix from the interchange layout to the
+ * resident layout.  src, dst: host buffers of redlite_moe_matrix_bytes()
+ * bytes, not overlapping.  REDLITE_EUNSUPPORTED for shapes the kernels do
+ * not take.  Pure host code: no device work. */
+int redlite_moe_pack_matrix(int32_t qtype, int64_t rows, int64_t k, const void *src, void *dst);
+
+/* Dequantise one matrix held in the resident layout (the bit-exactness
+ * check of the decoders).  packed: device; out_f32: device [rows*k] fp32 or
+ * NULL; out_bf16: device [rows*k] bf16 bits (round to nearest even) or
+ * NULL; outputs 16-byte aligned.  grids: expanded.  Enqueued on stream. */
 int redlite_moe_dequant(int32_t qtype, const void *packed, int64_t rows, int64_t k, const void *grids, float *out_f32,
                         uint16_t *out_bf16, void *stream);
 
 /* Slot-table builder: copies experts from host memory into a device pool
  * and writes their slot descriptors ("Red Metal dev8", steps 1-3: every
  * selected expert made resident, three positional reads per expert).
+ * Matrices are converted to the resident layout on the way.
  *   hidden       H of the layer (sizes the matrices with each expert's ffn)
  *   ids          host [n] expert ids (slot index in table_dev)
  *   host_experts host [n]; gate/up/down are HOST pointers to packed bytes
+ *                in the interchange layout
  *   pool         device, pool_bytes, 16-byte aligned; matrices are placed
  *                back to back at 16-byte aligned offsets from `pool_offset`
  *   table_dev    device [n_experts] slot table; entries ids[i] are written

@@ -16,6 +16,7 @@ from ._native import (  # noqa: F401
     REDLITE_STATUS_BAD_EXPERT,
     REDLITE_STATUS_BAD_ID,
     REDLITE_STATUS_TIMEOUT,
+    launches_per_call,
     lib,
     redlite_moe_dequant,
     redlite_moe_expand_grids,
@@ -23,6 +24,7 @@ from ._native import (  # noqa: F401
     redlite_moe_grids_bytes,
     redlite_moe_layer,
     redlite_moe_matrix_bytes,
+    redlite_moe_pack_matrix,
     redlite_moe_table,
     redlite_moe_upload_counters,
     redlite_moe_upload_experts,

@@ -37,7 +37,8 @@ class redlite_moe_expert(ctypes.Structure):
 class redlite_moe_table(ctypes.Structure):
     _fields_ = [
         ("hidden", ctypes.c_int32), ("n_experts", ctypes.c_int32), ("max_ffn", ctypes.c_int32),
-        ("max_tokens", ctypes.c_int32), ("experts", _c_void_p), ("grids", _c_void_p), ("workspace", _c_void_p),
+        ("max_tokens", ctypes.c_int32), ("min_ffn", ctypes.c_int32), ("reserved", ctypes.c_int32),
+        ("experts", _c_void_p), ("grids", _c_void_p), ("workspace", _c_void_p),
         ("workspace_bytes", ctypes.c_size_t), ("status", _c_void_p), ("stream", _c_void_p),
     ]
 
@@ -55,6 +56,8 @@ EXPORTS = {
     "redlite_moe_layer": (ctypes.c_int, [_c_void_p, ctypes.c_int32, _c_void_p, _c_void_p, ctypes.c_int32,
                                          ctypes.POINTER(redlite_moe_table), ctypes.POINTER(redlite_moe_expert),
                                          _c_void_p]),
+    "redlite_moe_pack_matrix": (ctypes.c_int, [ctypes.c_int32, ctypes.c_int64, ctypes.c_int64, _c_void_p,
+                                               _c_void_p]),
     "redlite_moe_dequant": (ctypes.c_int, [ctypes.c_int32, _c_void_p, ctypes.c_int64, ctypes.c_int64, _c_void_p,
                                            _c_void_p, _c_void_p, _c_void_p]),
     "redlite_moe_upload_experts": (ctypes.c_int, [ctypes.c_int32, _c_void_p, _c_void_p, ctypes.c_int32, _c_void_p,
@@ -128,6 +131,17 @@ def redlite_moe_dequant(qtype: int, packed: torch.Tensor, rows: int, k: int, gri
                                      _stream_handle(stream))
 
 
+def redlite_moe_pack_matrix(qtype: int, rows: int, k: int, src):
+    """Interchange -> resident layout on the host (numpy uint8 in, numpy uint8 out)."""
+    import numpy as np
+
+    a = np.ascontiguousarray(src, dtype=np.uint8)
+    out = np.zeros_like(a)
+    rc = lib().redlite_moe_pack_matrix(qtype, rows, k, a.ctypes.data_as(_c_void_p), out.ctypes.data_as(_c_void_p))
+    _check(rc, "redlite_moe_pack_matrix")
+    return out
+
+
 def redlite_moe_workspace_reset(table: redlite_moe_table) -> int:
     return lib().redlite_moe_workspace_reset(ctypes.byref(table))
 
@@ -161,3 +175,13 @@ def redlite_moe_upload_experts(hidden: int, ids, host_experts, pool: torch.Tenso
                                           ctypes.byref(ctr), ctypes.byref(end))
     del keep
     return rc, int(end.value)
+
+
+def launches_per_call(n_tokens: int, top_k: int, has_shared: bool, fast: bool = True) -> int:
+    """Kernels one redlite_moe_layer call enqueues: the fused decode kernel for
+    decode-sized calls on tiled tables, else bucketing + gate/up + down."""
+    if n_tokens == 0:
+        return 0
+    if fast and n_tokens * top_k <= 640 and (not has_shared or n_tokens <= 64):
+        return 1
+    return 3

@@ -82,6 +82,26 @@ int redlite_moe_layer(const float *x, int32_t n_tokens, const int32_t *expert_id
   cudaStream_t s = (cudaStream_t)t->stream;
   uint8_t *ws = (uint8_t *)t->workspace;
 
+  if (t->min_ffn >= 256 && fused_supported(t->hidden, t->max_ffn, n_tokens, top_k, t->n_experts, shared != nullptr)) {
+    FusedArgs fa{};
+    fa.x = x;
+    fa.ids = expert_ids;
+    fa.weights = router_weights;
+    fa.out = out;
+    fa.n_tokens = n_tokens;
+    fa.top_k = top_k;
+    fa.n_experts = t->n_experts;
+    fa.hidden = t->hidden;
+    fa.max_ffn = t->max_ffn;
+    fa.experts = t->experts;
+    if (shared) fa.shared = *shared;
+    fa.has_shared = shared != nullptr;
+    fa.grids = (const uint8_t *)t->grids;
+    fa.ws = ws;
+    fa.L = L;
+    fa.status = t->status;
+    return launch_fused(fa, s) == cudaSuccess ? REDLITE_OK : REDLITE_ECUDA;
+  }
   if (cudaMemsetAsync(out, 0, sizeof(float) * (size_t)n_tokens * t->hidden, s) != cudaSuccess) return REDLITE_ECUDA;
   RouteArgs ra{expert_ids, router_weights, n_tokens, top_k, t->n_experts, t->hidden, t->max_ffn,
                t->experts, shared != nullptr, ws, L, t->status};
@@ -144,12 +164,21 @@ int redlite_moe_upload_experts(int32_t hidden, const int32_t *ids, const redlite
   }
   if (off > pool_bytes) return REDLITE_ENOMEM;
   cudaStream_t s = (cudaStream_t)stream;
+  // resident-layout copies stay alive until the stream is synchronised below
+  std::vector<std::vector<uint8_t>> staged((size_t)n * 3);
   for (int i = 0; i < n; ++i) {
     const void *src[3] = {host_experts[i].gate, host_experts[i].up, host_experts[i].down};
     const void *dst[3] = {desc[i].gate, desc[i].up, desc[i].down};
-    for (int m = 0; m < 3; ++m)
-      if (cudaMemcpyAsync((void *)dst[m], src[m], sizes[3 * i + m], cudaMemcpyHostToDevice, s) != cudaSuccess)
+    const int64_t shp[3][2] = {{host_experts[i].ffn, hidden}, {host_experts[i].ffn, hidden}, {hidden, host_experts[i].ffn}};
+    for (int m = 0; m < 3; ++m) {
+      std::vector<uint8_t> &buf = staged[3 * i + m];
+      buf.resize(sizes[3 * i + m]);
+      if (pack_matrix_host(host_experts[i].qtype, shp[m][0], shp[m][1], (const uint8_t *)src[m], buf.data()) !=
+          REDLITE_OK)
+        return REDLITE_EUNSUPPORTED;
+      if (cudaMemcpyAsync((void *)dst[m], buf.data(), buf.size(), cudaMemcpyHostToDevice, s) != cudaSuccess)
         return REDLITE_ECUDA;
+    }
     if (cudaMemcpyAsync(table_dev + ids[i], &desc[i], sizeof(redlite_moe_expert), cudaMemcpyHostToDevice, s) !=
         cudaSuccess)
       return REDLITE_ECUDA;

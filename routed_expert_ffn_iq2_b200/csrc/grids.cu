@@ -26,6 +26,14 @@ __global__ void expand_grids_kernel(const uint16_t *__restrict__ comp2, const ui
       vb[j] = __int2bfloat16_rn(val);
     }
     reinterpret_cast<uint16_t *>(grids + kGridQ2Comp)[t] = c;
+    uint32_t sel = 0;
+    for (int j = 0; j < 8; ++j) sel |= (uint32_t)((c >> (2 * j)) & 3) << (4 * j);
+    reinterpret_cast<uint32_t *>(grids + kGridQ2Sel)[t] = sel;
+    if (t < 256) {
+      uint32_t sg = 0;
+      for (int j = 0; j < 8; ++j) sg |= (uint32_t)((t >> j) & 1) << (4 * j + 2);
+      reinterpret_cast<uint32_t *>(grids + kGridSign)[t] = sg;
+    }
   } else if (t < kQ2GridEntries + kQ1GridEntries) {
     const int e = t - kQ2GridEntries;
     const uint16_t c = comp1[e];
@@ -41,17 +49,22 @@ __global__ void expand_grids_kernel(const uint16_t *__restrict__ comp2, const ui
       p1[j] = __int2bfloat16_rn(8 * val - 1);  // 8 * (val - 1/8)
     }
     reinterpret_cast<uint16_t *>(grids + kGridQ1Comp)[e] = c;
+    uint32_t sel = 0;
+    for (int j = 0; j < 8; ++j) sel |= (uint32_t)((c >> (2 * j)) & 3) << (4 * j);
+    reinterpret_cast<uint32_t *>(grids + kGridQ1Sel)[e] = sel;
+    reinterpret_cast<uint32_t *>(grids + kGridQ1Sel)[e + 2048] = sel | 0x44444444u;
   }
 }
 
 // Dequantise a packed matrix: one thread per 8-weight group.
 template <int QT>
-__global__ void dequant_kernel(const uint8_t *__restrict__ mat, int64_t n_groups, const int8_t *__restrict__ grid,
-                               float *__restrict__ out_f32, uint16_t *__restrict__ out_bf16) {
+__global__ void dequant_kernel(const uint8_t *__restrict__ mat, int64_t n_groups, int64_t k, bool tiled,
+                               const int8_t *__restrict__ grid, float *__restrict__ out_f32,
+                               uint16_t *__restrict__ out_bf16) {
   for (int64_t G = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; G < n_groups;
        G += (int64_t)gridDim.x * blockDim.x) {
     float w[8];
-    decode_group_f32<QT>(mat, G, grid, w);
+    decode_group_f32<QT>(mat, k, tiled, G, grid, w);
     if (out_f32) {
       float4 *o = reinterpret_cast<float4 *>(out_f32 + 8 * G);
       o[0] = make_float4(w[0], w[1], w[2], w[3]);
@@ -83,12 +96,13 @@ cudaError_t launch_dequant(int qtype, const void *packed, int64_t rows, int64_t 
   int64_t blocks = (groups + threads - 1) / threads;
   if (blocks > 148 * 64) blocks = 148 * 64;
   const uint8_t *g = (const uint8_t *)grids;
+  const bool tiled = tiled_shape(rows, k);
   if (qtype == kQ2)
     dequant_kernel<kQ2><<<(unsigned)blocks, threads, 0, stream>>>(
-        (const uint8_t *)packed, groups, (const int8_t *)(g + kGridQ2Vals), out_f32, out_bf16);
+        (const uint8_t *)packed, groups, k, tiled, (const int8_t *)(g + kGridQ2Vals), out_f32, out_bf16);
   else
     dequant_kernel<kQ1><<<(unsigned)blocks, threads, 0, stream>>>(
-        (const uint8_t *)packed, groups, (const int8_t *)(g + kGridQ1Vals), out_f32, out_bf16);
+        (const uint8_t *)packed, groups, k, tiled, (const int8_t *)(g + kGridQ1Vals), out_f32, out_bf16);
   return cudaGetLastError();
 }
 

@@ -10,7 +10,10 @@
 #include <cuda_runtime.h>
 #include <stdint.h>
 
+#include <algorithm>
+
 #include "../../include/redlite_moe.h"
+#include "layout.cuh"
 
 namespace redlite {
 
@@ -30,13 +33,23 @@ constexpr int kQ1GridEntries = 2048;
 //   kGridQ1Bf16p: bf16  [2][2048][8] IQ1 (grid + delta) * 8 as bf16, delta
 //                 +1/8 (plane 0) and -1/8 (plane 1): values -9,-7,-1,1,7,9
 //   kGridQ2Comp : u16 [512], kGridQ1Comp : u16 [2048] (compact, as given)
+//   kGridQ2Sel  : u32 [512]   byte-permute selectors: nibble j = symbol j
+//   kGridSign   : u32 [256]   nibble j bit 2 = sign bit j of a sign byte
+//   kGridQ1Sel  : u32 [4096]  index e = idx | delta_bit << 11: nibble j =
+//                 symbol j of grid entry idx | delta_bit << 2
+// A selector nibble picks one byte of a constant 8-byte table (see the
+// decode kernels), so two byte-permutes turn a selector into eight signed
+// int8 weights.
 constexpr size_t kGridQ2Vals = 0;
 constexpr size_t kGridQ1Vals = kGridQ2Vals + 512 * 8;
 constexpr size_t kGridQ2Bf16 = kGridQ1Vals + 2048 * 8;
 constexpr size_t kGridQ1Bf16p = kGridQ2Bf16 + 512 * 8 * 2;
 constexpr size_t kGridQ2Comp = kGridQ1Bf16p + 2 * 2048 * 8 * 2;
 constexpr size_t kGridQ1Comp = kGridQ2Comp + 512 * 2;
-constexpr size_t kGridBytes = kGridQ1Comp + 2048 * 2;
+constexpr size_t kGridQ2Sel = kGridQ1Comp + 2048 * 2;
+constexpr size_t kGridSign = kGridQ2Sel + 512 * 4;
+constexpr size_t kGridQ1Sel = kGridSign + 256 * 4;
+constexpr size_t kGridBytes = kGridQ1Sel + 4096 * 4;
 
 inline __host__ __device__ int block_bytes(int qtype) {
   return qtype == kQ2 ? kQ2BlockBytes : (qtype == kQ1 ? kQ1BlockBytes : 0);
@@ -77,22 +90,24 @@ struct Ctrl {
   int n_pairs;         // pairs in the sorted list
   int ticket;          // next work ticket
   int exit_count;      // CTAs that finished (the last one resets)
-  int phase1_done;     // gate/up tickets completed
-  int zero_done;       // output-zeroing tickets completed
+  int phase1_done;     // CTAs past the gate/up phase (fused decode kernel)
+  int phase0_done;     // CTAs past the activation-conversion phase
   int pad[58];
 };
 static_assert(sizeof(Ctrl) == 256, "ctrl block is 256 bytes");
 
 struct WorkspaceLayout {
-  size_t ctrl, active, pairs, counts, done, h, total;
+  size_t ctrl, active, pairs, counts, done, h, gu, limbs, exps, total;
   int max_active, max_pairs;
 };
+
+// Largest (token, slot) pair count the fused decode kernel takes.
+constexpr int kFusedMaxPairs = 640;
 
 inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
 inline WorkspaceLayout workspace_layout(int hidden, int n_experts, int max_tokens, int top_k, int max_ffn) {
   WorkspaceLayout L;
-  (void)hidden;
   int64_t routed = (int64_t)max_tokens * top_k;
   L.max_pairs = (int)(routed + max_tokens);  // + shared expert pairs
   L.max_active = (int)((routed < n_experts ? routed : n_experts) + 1);
@@ -109,6 +124,15 @@ inline WorkspaceLayout workspace_layout(int hidden, int n_experts, int max_token
   off = align256(off + sizeof(int) * (size_t)L.max_active);
   L.h = off;
   off = align256(off + sizeof(float) * (size_t)L.max_pairs * (size_t)max_ffn);
+  // fused decode kernel: gate/up results per pair, activation limbs per token
+  const int64_t ft = std::min<int64_t>(max_tokens, kFusedMaxPairs / (top_k > 0 ? top_k : 1));
+  const int64_t fpairs = ft * top_k + ft;
+  L.gu = off;
+  off = align256(off + sizeof(float) * (size_t)fpairs * 2 * (size_t)max_ffn);
+  L.limbs = off;
+  off = align256(off + (size_t)ft * 3 * (size_t)(hidden + 32));
+  L.exps = off;
+  off = align256(off + sizeof(int) * (size_t)(ft + 1));
   L.total = off;
   return L;
 }
@@ -120,38 +144,66 @@ __device__ __forceinline__ float fp16_bits_to_float(uint16_t h) { return __half2
 __device__ __forceinline__ uint16_t ld_u16(const uint8_t *p) { return (uint16_t)(p[0] | (p[1] << 8)); }
 
 // Eight weights of group G (weights 8G..8G+7 of the matrix's row-major
-// sequence), exact in fp32.  grid: expanded int8 values of the format.
+// sequence), exact in fp32, read from the resident layout of a rows x k
+// matrix (tiled when tiled_shape(rows, k), else the interchange layout).
+// grid: expanded int8 values of the format.
 template <int QT>
-__device__ __forceinline__ void decode_group_f32(const uint8_t *__restrict__ mat, int64_t G,
+__device__ __forceinline__ void decode_group_f32(const uint8_t *__restrict__ mat, int64_t k, bool tiled, int64_t G,
                                                  const int8_t *__restrict__ grid, float w[8]) {
-  const int64_t blk_i = G >> 5;
-  const int g = (int)(G & 31);
+  int idx, sc, nib = 0;
+  unsigned s = 0;
+  float d;
+  if (tiled) {
+    const int64_t n = 8 * G, r = n / k, kk = n % k;
+    const int64_t kb = kk >> 8;
+    const int g = (int)((kk & 255) >> 3), rr = (int)(r & 15);
+    const uint8_t *tb = mat + tile_block_offset(QT, k, r, kb);
+    if constexpr (QT == kQ2) {
+      const Q2Loc o = q2_loc(rr, g);
+      idx = tb[o.qs] | (((ld_u16(tb + o.qh_word) >> o.qh_bit) & 1) << 8);
+      sc = (tb[o.scales + (g >> 3)] >> (4 * ((g >> 2) & 1))) & 15;
+      s = tb[o.sign];
+      d = fp16_bits_to_float(ld_u16(tb + o.d));
+    } else {
+      const Q1Loc o = q1_loc(rr, g);
+      nib = (tb[o.nib_byte] >> o.nib_shift) & 15;
+      idx = tb[o.qs] | ((nib & 7) << 8);
+      const int bit = 3 * (g >> 1);
+      const unsigned two = tb[o.scales + (bit >> 3)] | ((bit >> 3) < 5 ? (unsigned)tb[o.scales + (bit >> 3) + 1] << 8 : 0u);
+      sc = (two >> (bit & 7)) & 7;
+      d = fp16_bits_to_float(ld_u16(tb + o.d));
+    }
+  } else {
+    const int64_t blk_i = G >> 5;
+    const int g = (int)(G & 31);
+    if constexpr (QT == kQ2) {
+      const uint8_t *b = mat + blk_i * kQ2BlockBytes;
+      d = fp16_bits_to_float(ld_u16(b));
+      idx = b[6 + g] | (((b[38 + (g >> 3)] >> (g & 7)) & 1) << 8);
+      sc = (b[2 + (g >> 3)] >> (4 * ((g >> 2) & 1))) & 15;
+      s = b[42 + g];
+    } else {
+      const uint8_t *b = mat + blk_i * kQ1BlockBytes;
+      d = fp16_bits_to_float(ld_u16(b));
+      nib = (b[34 + (g >> 1)] >> (4 * (g & 1))) & 15;
+      idx = b[2 + g] | ((nib & 7) << 8);
+      const int bit = 3 * (g >> 1);
+      // the 3-bit field may straddle two bytes of the 48-bit scales field
+      const unsigned two = b[50 + (bit >> 3)] | ((bit >> 3) < 5 ? (unsigned)b[51 + (bit >> 3)] << 8 : 0u);
+      sc = (two >> (bit & 7)) & 7;
+    }
+  }
+  const int8_t *gv = grid + idx * 8;
   if constexpr (QT == kQ2) {
-    const uint8_t *b = mat + blk_i * kQ2BlockBytes;
-    const float d = fp16_bits_to_float(ld_u16(b));
-    const int idx = b[6 + g] | (((b[38 + (g >> 3)] >> (g & 7)) & 1) << 8);
-    const int sc = (b[2 + (g >> 3)] >> (4 * ((g >> 2) & 1))) & 15;
-    const unsigned s = b[42 + g];
     const float scale = d * (float)(2 * sc + 1) * 0.125f;
-    const int8_t *gv = grid + idx * 8;
 #pragma unroll
     for (int j = 0; j < 8; ++j) {
-      float v = scale * (float)gv[j];
+      const float v = scale * (float)gv[j];
       w[j] = ((s >> j) & 1) ? -v : v;
     }
   } else {
-    const uint8_t *b = mat + blk_i * kQ1BlockBytes;
-    const float d = fp16_bits_to_float(ld_u16(b));
-    const int nib = (b[34 + (g >> 1)] >> (4 * (g & 1))) & 15;
-    const int idx = b[2 + g] | ((nib & 7) << 8);
-    const float delta = (nib & 8) ? -0.125f : 0.125f;
-    const int sub = g >> 1;
-    const int bit = 3 * sub;
-    // the 3-bit field may straddle two bytes of the 48-bit scales field
-    const unsigned two = b[50 + (bit >> 3)] | ((bit >> 3) < 5 ? (unsigned)b[51 + (bit >> 3)] << 8 : 0u);
-    const int sc = (two >> (bit & 7)) & 7;
     const float scale = d * (float)(2 * sc + 1);
-    const int8_t *gv = grid + idx * 8;
+    const float delta = (nib & 8) ? -0.125f : 0.125f;
 #pragma unroll
     for (int j = 0; j < 8; ++j) w[j] = scale * ((float)gv[j] + delta);
   }
@@ -198,5 +250,23 @@ cudaError_t launch_dequant(int qtype, const void *packed, int64_t rows, int64_t 
                            uint16_t *out_bf16, cudaStream_t stream);
 cudaError_t launch_route(const RouteArgs &a, cudaStream_t stream);
 cudaError_t launch_simt_tiles(const TileArgs &a, int max_active, cudaStream_t stream);
+int pack_matrix_host(int qtype, int64_t rows, int64_t k, const uint8_t *src, uint8_t *dst);
+
+struct FusedArgs {
+  const float *x;
+  const int32_t *ids;
+  const float *weights;
+  float *out;
+  int n_tokens, top_k, n_experts, hidden, max_ffn;
+  const redlite_moe_expert *experts;
+  redlite_moe_expert shared;
+  int has_shared;
+  const uint8_t *grids;
+  uint8_t *ws;
+  WorkspaceLayout L;
+  int32_t *status;
+};
+bool fused_supported(int hidden, int max_ffn, int n_tokens, int top_k, int n_experts, bool has_shared);
+cudaError_t launch_fused(const FusedArgs &a, cudaStream_t stream);
 
 }  // namespace redlite

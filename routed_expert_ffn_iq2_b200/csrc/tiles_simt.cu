@@ -27,14 +27,14 @@ __device__ __forceinline__ void load_grids_smem(const uint8_t *grids, int8_t *g2
 
 // dot of one packed row (k inputs, groups G0..G0+k/8) with NT vectors in smem
 template <int QT>
-__device__ __forceinline__ void row_dot(const uint8_t *mat, int64_t G0, int k, const int8_t *grid, const float *vs,
-                                        int vstride, int nt, float acc[kSimtNT]) {
+__device__ __forceinline__ void row_dot(const uint8_t *mat, int64_t G0, int k, bool tiled, const int8_t *grid,
+                                        const float *vs, int vstride, int nt, float acc[kSimtNT]) {
   const int lane = threadIdx.x & 31;
 #pragma unroll
   for (int j = 0; j < kSimtNT; ++j) acc[j] = 0.f;
   for (int gq = lane; gq < k / 8; gq += 32) {
     float w[8];
-    decode_group_f32<QT>(mat, G0 + gq, grid, w);
+    decode_group_f32<QT>(mat, k, tiled, G0 + gq, grid, w);
 #pragma unroll
     for (int j = 0; j < kSimtNT; ++j) {
       if (j < nt) {
@@ -88,12 +88,13 @@ __global__ void __launch_bounds__(kSimtThreads) gateup_simt_kernel(TileArgs a) {
       if (i >= F) break;
       const int64_t G0 = (int64_t)i * H / 8;
       float gacc[kSimtNT], uacc[kSimtNT];
+      const bool tiled = tiled_shape(F, H);
       if (ex.qtype == kQ2) {
-        row_dot<kQ2>((const uint8_t *)ex.gate, G0, H, g2, xs, H, nt, gacc);
-        row_dot<kQ2>((const uint8_t *)ex.up, G0, H, g2, xs, H, nt, uacc);
+        row_dot<kQ2>((const uint8_t *)ex.gate, G0, H, tiled, g2, xs, H, nt, gacc);
+        row_dot<kQ2>((const uint8_t *)ex.up, G0, H, tiled, g2, xs, H, nt, uacc);
       } else {
-        row_dot<kQ1>((const uint8_t *)ex.gate, G0, H, g1, xs, H, nt, gacc);
-        row_dot<kQ1>((const uint8_t *)ex.up, G0, H, g1, xs, H, nt, uacc);
+        row_dot<kQ1>((const uint8_t *)ex.gate, G0, H, tiled, g1, xs, H, nt, gacc);
+        row_dot<kQ1>((const uint8_t *)ex.up, G0, H, tiled, g1, xs, H, nt, uacc);
       }
 #pragma unroll
       for (int j = 0; j < kSimtNT; ++j)
@@ -136,10 +137,11 @@ __global__ void __launch_bounds__(kSimtThreads) down_simt_kernel(TileArgs a) {
       if (r >= H) break;
       const int64_t G0 = (int64_t)r * F / 8;
       float y[kSimtNT];
+      const bool tiled = tiled_shape(H, F);
       if (ex.qtype == kQ2)
-        row_dot<kQ2>((const uint8_t *)ex.down, G0, F, g2, hs, F, nt, y);
+        row_dot<kQ2>((const uint8_t *)ex.down, G0, F, tiled, g2, hs, F, nt, y);
       else
-        row_dot<kQ1>((const uint8_t *)ex.down, G0, F, g1, hs, F, nt, y);
+        row_dot<kQ1>((const uint8_t *)ex.down, G0, F, tiled, g1, hs, F, nt, y);
 #pragma unroll
       for (int j = 0; j < kSimtNT; ++j)
         if (lane == j && j < nt) atomicAdd(a.out + (size_t)s_pair[j].token * H + r, s_pair[j].weight * y[j]);

@@ -34,7 +34,7 @@ class MoeLayer:
         self.counters = N.redlite_moe_upload_counters()
         self.shared: Optional[N.redlite_moe_expert] = None
         self.table = N.redlite_moe_table(
-            hidden, n_experts, max_ffn, max_tokens, self.table_dev.data_ptr(), self.grids.data_ptr(),
+            hidden, n_experts, max_ffn, max_tokens, 0, 0, self.table_dev.data_ptr(), self.grids.data_ptr(),
             self.workspace.data_ptr(), self.workspace.numel(), self.status.data_ptr(), self.stream.cuda_stream)
         N._check(N.redlite_moe_workspace_reset(self.table), "redlite_moe_workspace_reset")
 
@@ -43,6 +43,8 @@ class MoeLayer:
                                                self.table_dev, self.n_experts + 1, self.counters, self.stream)
         if rc == N.REDLITE_OK:
             self.pool_used = end
+            f = min(int(e.ffn) for e in experts) if len(experts) else 0
+            self.table.min_ffn = f if self.table.min_ffn == 0 else min(self.table.min_ffn, f)
         return rc
 
     def set_shared(self, expert) -> int:

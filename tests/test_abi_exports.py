@@ -65,7 +65,7 @@ def test_expand_grids_rejects_symbol3_before_device_work(native):
 
 def test_layer_rejects_bad_arguments_on_host(native):
     L = native.lib()
-    t = native.redlite_moe_table(2048, 512, 512, 64, 0x1000, 0x2000, 0x3000, 1 << 30, 0x4000, None)
+    t = native.redlite_moe_table(2048, 512, 512, 64, 0, 0, 0x1000, 0x2000, 0x3000, 1 << 30, 0x4000, None)
     p = ctypes.c_void_p(0x10000)
     # null table
     assert L.redlite_moe_layer(p, 1, p, p, 10, None, None, p) == native.REDLITE_EINVAL
@@ -82,7 +82,7 @@ def test_layer_rejects_bad_arguments_on_host(native):
     # misaligned x
     assert L.redlite_moe_layer(ctypes.c_void_p(0x10004), 1, p, p, 10, ctypes.byref(t), None, p) == native.REDLITE_EINVAL
     # workspace too small
-    t2 = native.redlite_moe_table(2048, 512, 512, 64, 0x1000, 0x2000, 0x3000, 1024, 0x4000, None)
+    t2 = native.redlite_moe_table(2048, 512, 512, 64, 0, 0, 0x1000, 0x2000, 0x3000, 1024, 0x4000, None)
     assert L.redlite_moe_layer(p, 1, p, p, 10, ctypes.byref(t2), None, p) == native.REDLITE_ENOMEM
     # bad shared expert (bad qtype / unsupported shape)
     sh = native.redlite_moe_expert(3, 512, 0x1000, 0x2000, 0x3000)
@@ -90,7 +90,7 @@ def test_layer_rejects_bad_arguments_on_host(native):
     sh = native.redlite_moe_expert(1, 48, 0x1000, 0x2000, 0x3000)
     assert L.redlite_moe_layer(p, 1, p, p, 10, ctypes.byref(t), ctypes.byref(sh), p) == native.REDLITE_EINVAL
     # hidden not a multiple of 32
-    t3 = native.redlite_moe_table(2047, 512, 512, 64, 0x1000, 0x2000, 0x3000, 1 << 30, 0x4000, None)
+    t3 = native.redlite_moe_table(2047, 512, 512, 64, 0, 0, 0x1000, 0x2000, 0x3000, 1 << 30, 0x4000, None)
     assert L.redlite_moe_layer(p, 1, p, p, 10, ctypes.byref(t3), None, p) == native.REDLITE_EINVAL
 
 

@@ -29,7 +29,7 @@ def grids(P):
 
 
 def _gpu_dequant(P, g, qtype, packed, rows, k):
-    dev = torch.from_numpy(packed).cuda()
+    dev = torch.from_numpy(P.redlite_moe_pack_matrix(qtype, rows, k, packed)).cuda()
     f = torch.empty(rows * k, dtype=torch.float32, device="cuda")
     b = torch.empty(rows * k, dtype=torch.int16, device="cuda")
     assert P.redlite_moe_dequant(qtype, dev, rows, k, g, f, b) == 0
@@ -55,7 +55,7 @@ def _edge_blocks(qtype, n):
 
 
 @pytest.mark.parametrize("qtype,rows,k", [(1, 64, 2048), (2, 64, 2048), (1, 256, 64), (2, 2048, 512), (1, 3, 256),
-                                          (2, 128, 128)])
+                                          (2, 128, 128), (1, 48, 768), (2, 32, 256)])
 def test_dequant_bit_exact(P, grids, oracle_lib, qtype, rows, k):
     w, g = grids
     packed = fixtures.make_matrix(17, qtype, rows, k, 5)

@@ -176,3 +176,25 @@ def test_repeat_calls_reuse_workspace(P):
     for _ in range(3):
         b = _run(L, w.x, w.ids, w.weights)
     assert _rel_err(b, a) <= TOL_FP32
+
+
+@pytest.mark.parametrize("T", [1, 3, 5, 17])
+def test_batched_token_counts(P, oracle_lib, T):
+    """Mixed-format batched decode with the shared expert at several token
+    counts: local activation limbs (T <= 4) and the cooperative conversion."""
+    w = fixtures.workload(4, n_tokens=T)
+    L = P.layer_for_workload(w)
+    got = _run(L, w.x, w.ids, w.weights)
+    ref = oracle_lib.workload_layer(w)
+    assert L.read_status() == 0
+    assert _rel_err(got, ref) <= TOL_FP32
+
+
+def test_general_path_agrees_with_fast_path(P):
+    w = fixtures.workload(4, n_tokens=9)
+    L = P.layer_for_workload(w)
+    fast = _run(L, w.x, w.ids, w.weights)
+    L.table.min_ffn = 0  # unknown widths: the general CUDA-core path runs
+    general = _run(L, w.x, w.ids, w.weights)
+    assert L.read_status() == 0
+    assert _rel_err(fast, general) <= TOL_FP32
