@@ -5,20 +5,23 @@
 // the layer accumulates out += router_weight * expert_output (plus the
 // shared expert with weight 1, "Red Lite dev16", block composition).
 //
-// Structure (one CTA per SM, cooperative launch so all CTAs are resident):
+// Structure (one CTA per SM, cooperative launch so all CTAs are resident;
+// 8 consumer warps + 1 producer warp per CTA):
 //   prologue  every CTA copies the byte-permute selector tables into shared
 //             memory, buckets the (token, slot) pairs by expert (stable,
 //             identical in every CTA), reads the selected slots'
-//             descriptors and enumerates the work items;
-//   phase 1   gate and up tiles (16 rows x hidden) of every selected expert,
-//             split evenly over the CTAs; each tile's packed bytes arrive
-//             by TMA bulk copy into a ring of shared-memory stages;
-//             results g, u go to the workspace; each CTA also zeroes a
-//             slice of `out`;
+//             descriptors, enumerates the work items and converts the
+//             activations to fixed-point limbs;
+//   phase 1   16-row tiles of gate and of up of every selected expert, split
+//             evenly over the CTAs; the producer warp streams each tile's
+//             packed bytes by TMA bulk copy into a ring of shared-memory
+//             stages; each consumer warp decodes one 16x256 tile-block and
+//             the last warp to finish a tile reduces it and writes g or u to
+//             the workspace; each CTA also zeroes a slice of `out`;
 //   barrier   one grid-wide counter (bounded wait);
-//   phase 2   down tiles: h = SiLU(g) * u per token, then y = W_down h and
-//             out[token] += weight * y with fp32 atomics.
-// Down tiles are prefetched into the ring while phase 1 finishes.
+//   phase 2   groups of down tiles: h = SiLU(g) * u per token, y = W_down h,
+//             out[token] += weight * y with fp32 atomics.  Down tiles are
+//             prefetched into the ring while phase 1 finishes.
 //
 // Arithmetic: weights are decoded to exact signed int8 values (IQ2: +-8,
 // +-25, +-43; IQ1: 8*(grid + delta) in {+-1, +-7, +-9}) by two byte
@@ -32,12 +35,16 @@
 
 namespace redlite {
 
-constexpr int kFThreads = 256;
-constexpr int kFWarps = kFThreads / 32;
+constexpr int kCWarps = 8;                 // consumer warps
+constexpr int kCThreads = 32 * kCWarps;    // 256
+constexpr int kFThreads = kCThreads + 32;  // + producer warp
 constexpr int kRing = 6;
 constexpr int kStageBytes = 8 * kQ2TileBlock;  // 9472 >= 8 * kQ1TileBlock
 constexpr int kTokChunk = 4;
-constexpr int kRep2 = 16;  // replicas of the IQ2 selector/sign tables (bank spread)
+#ifndef REDLITE_REP2
+#define REDLITE_REP2 16
+#endif
+constexpr int kRep2 = REDLITE_REP2;  // replicas of the IQ2 selector/sign tables (bank spread)
 constexpr int kRep1 = 2;   // replicas of the IQ1 selector table
 constexpr int kFusedMaxInst = kFusedMaxPairs + 2;
 constexpr int kLimbPad = 32;  // padding per limb plane (spreads shared-memory banks)
@@ -48,7 +55,7 @@ constexpr uint32_t kSpinLimit = 1u << 24;
 constexpr uint32_t kQ2Pos = 0x002B1908u, kQ2Neg = 0x00D5E7F8u;
 constexpr uint32_t kQ1Pos = 0x000901F9u, kQ1Neg = 0x0007FFF7u;
 
-struct Inst {          // one selected expert (or the shared expert)
+struct Inst {  // one selected expert (or the shared expert)
   const uint8_t *gate, *up, *down;
   int qtype, ffn;
   int pair_start, count;
@@ -63,14 +70,16 @@ struct ItemInfo {
 struct Smem {
   uint32_t *sel2, *sgn2, *sel1;
   uint8_t *ring;
+  float *red;  // [kRing][kCWarps][16 rows][4 tokens]
   uint8_t *limbs;
   Inst *inst;
   int *pair_tok;
   float *pair_w;
-  float *red;
-  uint64_t *full;
+  uint64_t *full, *empty;
+  int *done;  // per stage: consumer warps finished
   ItemInfo *info;
-  int *tok_exp;
+  float *tok_scale;  // per token slot: 2^(e - 20)
+  float *wmax;       // [kCWarps][4] partial maxima
 };
 
 // ------------------------------------------------------------------ PTX wrappers
@@ -87,6 +96,10 @@ __device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
   asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
 }
 
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
 __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
@@ -95,6 +108,13 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
       : "r"(smem_u32(bar)), "r"(parity)
       : "memory");
   return ok != 0;
+}
+
+// Bounded wait on an mbarrier phase; returns false if it gave up.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity) {
+  for (uint32_t it = 0; it < kSpinLimit; ++it)
+    if (mbar_try_wait(bar, parity)) return true;
+  return false;
 }
 
 // 1-D bulk copy global -> shared, completion counted on an mbarrier.
@@ -111,21 +131,67 @@ __device__ __forceinline__ int ld_acquire(const int *p) {
   return v;
 }
 
+// named barrier over the consumer warps only
+__device__ __forceinline__ void consumers_sync() { asm volatile("bar.sync 1, %0;" ::"n"(kCThreads) : "memory"); }
+
 __device__ __forceinline__ void mma_k32(int32_t d[4], const uint32_t a[4], uint32_t b0, uint32_t b1) {
-  asm volatile(
+  asm(
       "mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, {%10,%10,%10,%10};"
       : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
       : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1), "r"(0));
 }
 
 __device__ __forceinline__ void mma_k16(int32_t d[4], uint32_t a0, uint32_t a1, uint32_t b0) {
-  asm volatile(
+  asm(
       "mma.sync.aligned.m16n8k16.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5}, {%6}, {%7,%7,%7,%7};"
       : "=r"(d[0]), "=r"(d[1]), "=r"(d[2]), "=r"(d[3])
       : "r"(a0), "r"(a1), "r"(b0), "r"(0));
 }
 
+// Optional timeline (build with -DREDLITE_TRACE): CTA c writes %globaltimer
+// stamps to the 32 words after the workspace layout's end, slot c * 32 + i.
+#ifdef REDLITE_TRACE
+#define TRACE(i)                                                                  \
+  do {                                                                            \
+    if (threadIdx.x == 0) {                                                       \
+      uint64_t t_;                                                                \
+      asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_));                      \
+      reinterpret_cast<uint64_t *>(a.ws + a.L.total)[blockIdx.x * 32 + (i)] = t_; \
+    }                                                                             \
+  } while (0)
+#define TRACEC(i, v)                                                                                 \
+  do {                                                                                               \
+    if ((threadIdx.x & 31) == 0)                                                                     \
+      reinterpret_cast<uint64_t *>(a.ws + a.L.total)[148 * 32 + (blockIdx.x * 16 + (i))] = (v);       \
+  } while (0)
+#else
+#define TRACE(i) \
+  do {           \
+  } while (0)
+#define TRACEC(i, v) \
+  do {               \
+  } while (0)
+#endif
+
 __device__ __forceinline__ float half_bits(uint32_t h) { return __half2float(__ushort_as_half((unsigned short)h)); }
+
+// Power-of-two exponent e with m < 2^e (m >= 0), clamped to [-106, 128] so
+// that 2^(20-e) and 2^(e-20) are both normal floats.
+__device__ __forceinline__ int pow2_above(float m) {
+  const uint32_t E = __float_as_uint(m) >> 23;  // m >= 0: biased exponent
+  int e = E ? (int)E - 126 : -126;
+  return e < -106 ? -106 : e;
+}
+__device__ __forceinline__ float pow2f(int e) { return __uint_as_float((uint32_t)(e + 127) << 23); }
+
+// limbs of one value scaled by 2^(20-e) (a power of two: exact)
+__device__ __forceinline__ void to_limbs(float v, float scale, int &l0, int &l1, int &l2) {
+  const int X = __float2int_rn(v * scale);
+  l2 = ((X + 64) & 127) - 64;
+  const int X1 = (X - l2) >> 7;
+  l1 = ((X1 + 64) & 127) - 64;
+  l0 = (X1 - l1) >> 7;
+}
 
 // ------------------------------------------------------------------ tile-block math
 //
@@ -145,7 +211,10 @@ __device__ __forceinline__ void b_planes(const uint8_t *limbs, int lstride, cons
 }
 
 // IQ2_XS-style tile-block (16 rows x 256 inputs): acc[p][.] += partial dot
-// products of the block's rows with token pair p (mma C layout, limb columns).
+// products of the block's rows with token pair p (mma C layout, limb
+// columns).  Lane (q, t) decodes groups 4c + t of rows q and q+8.  All
+// selector and activation loads are issued before the first mma so their
+// latencies overlap.
 template <int NP>
 __device__ __forceinline__ void tb_q2(const uint8_t *__restrict__ tb, const uint32_t *__restrict__ sel2,
                                       const uint32_t *__restrict__ sgn2, const uint8_t *const bp[NP], int kbase,
@@ -158,29 +227,35 @@ __device__ __forceinline__ void tb_q2(const uint8_t *__restrict__ tb, const uint
   const uint32_t dw = *reinterpret_cast<const uint32_t *>(tb + 1152 + 4 * q);
   const uint32_t qsw[4] = {qs.x, qs.y, qs.z, qs.w};
   const uint32_t sgw[4] = {sg.x, sg.y, sg.z, sg.w};
+  uint32_t sel[16];  // field i = 2c + h
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const uint32_t idx = ((qsw[i >> 2] >> (8 * (i & 3))) & 0xFFu) | (((qh >> i) & 1u) << 8);
+    const uint32_t sgb = (sgw[i >> 2] >> (8 * (i & 3))) & 0xFFu;
+    sel[i] = sel2[idx * kRep2 + r] | sgn2[sgb * kRep2 + r];
+  }
+  uint2 b[NP][8];
+#pragma unroll
+  for (int p = 0; p < NP; ++p)
+#pragma unroll
+    for (int c = 0; c < 8; ++c)
+      b[p][c] = bp[p] ? *reinterpret_cast<const uint2 *>(bp[p] + kbase + 32 * c + 8 * t) : make_uint2(0u, 0u);
   int32_t cb[NP][4];
 #pragma unroll
   for (int p = 0; p < NP; ++p) cb[p][0] = cb[p][1] = cb[p][2] = cb[p][3] = 0;
 #pragma unroll
   for (int c = 0; c < 8; ++c) {
     uint32_t a[4];
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int i = 2 * c + h;
-      const uint32_t qsb = (qsw[i >> 2] >> (8 * (i & 3))) & 0xFFu;
-      const uint32_t idx = qsb | (((qh >> i) & 1u) << 8);
-      const uint32_t sgb = (sgw[i >> 2] >> (8 * (i & 3))) & 0xFFu;
-      const uint32_t sel = sel2[idx * kRep2 + r] | sgn2[sgb * kRep2 + r];
-      a[h] = __byte_perm(kQ2Pos, kQ2Neg, sel);
-      a[2 + h] = __byte_perm(kQ2Pos, kQ2Neg, sel >> 16);
-    }
+    a[0] = __byte_perm(kQ2Pos, kQ2Neg, sel[2 * c]);
+    a[2] = __byte_perm(kQ2Pos, kQ2Neg, sel[2 * c] >> 16);
+    a[1] = __byte_perm(kQ2Pos, kQ2Neg, sel[2 * c + 1]);
+    a[3] = __byte_perm(kQ2Pos, kQ2Neg, sel[2 * c + 1] >> 16);
     const int m0 = 2 * (int)((scw.x >> (4 * c)) & 15u) + 1;
     const int m1 = 2 * (int)((scw.y >> (4 * c)) & 15u) + 1;
 #pragma unroll
     for (int p = 0; p < NP; ++p) {
-      const uint2 b = bp[p] ? *reinterpret_cast<const uint2 *>(bp[p] + kbase + 32 * c + 8 * t) : make_uint2(0u, 0u);
       int32_t d[4];
-      mma_k32(d, a, b.x, b.y);
+      mma_k32(d, a, b[p][c].x, b[p][c].y);
       cb[p][0] += m0 * d[0];
       cb[p][1] += m0 * d[1];
       cb[p][2] += m1 * d[2];
@@ -212,30 +287,34 @@ __device__ __forceinline__ void tb_q1(const uint8_t *__restrict__ tb, const uint
   const uint64_t row0 = (uint64_t)s0 | ((uint64_t)(s1 & 0xFFFFu) << 32);
   const uint64_t row1 = (uint64_t)(s1 >> 16) | ((uint64_t)s2 << 16);
   const uint32_t dw = *reinterpret_cast<const uint32_t *>(tb + 864 + 4 * q);
+  const int hshift = 16 * (t & 1);
   const uint32_t qsw[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
   const uint32_t nbw[4] = {nb.x, nb.y, nb.z, nb.w};
-  const int hshift = 16 * (t & 1);
+  uint32_t sel[32];  // entry i = 2s + h
+#pragma unroll
+  for (int i = 0; i < 32; ++i) {
+    const uint32_t qsb = (qsw[i >> 2] >> (8 * (i & 3))) & 0xFFu;
+    const uint32_t nib = (nbw[i >> 3] >> (4 * (i & 7))) & 0xFu;
+    sel[i] = sel1[(qsb | (nib << 8)) * kRep1 + r] >> hshift;
+  }
+  uint32_t b[NP][16];
+#pragma unroll
+  for (int p = 0; p < NP; ++p)
+#pragma unroll
+    for (int s = 0; s < 16; ++s) b[p][s] = bp[p] ? *reinterpret_cast<const uint32_t *>(bp[p] + kbase + 16 * s + 4 * t) : 0u;
   int32_t cb[NP][4];
 #pragma unroll
   for (int p = 0; p < NP; ++p) cb[p][0] = cb[p][1] = cb[p][2] = cb[p][3] = 0;
 #pragma unroll
   for (int s = 0; s < 16; ++s) {
-    uint32_t a[2];
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int i = 2 * s + h;
-      const uint32_t qsb = (qsw[i >> 2] >> (8 * (i & 3))) & 0xFFu;
-      const uint32_t nib = (nbw[i >> 3] >> (4 * (i & 7))) & 0xFu;
-      const uint32_t sel = sel1[(qsb | (nib << 8)) * kRep1 + r];
-      a[h] = __byte_perm(kQ1Pos, kQ1Neg, sel >> hshift);
-    }
+    const uint32_t a0 = __byte_perm(kQ1Pos, kQ1Neg, sel[2 * s]);
+    const uint32_t a1 = __byte_perm(kQ1Pos, kQ1Neg, sel[2 * s + 1]);
     const int m0 = 2 * (int)((row0 >> (3 * s)) & 7u) + 1;
     const int m1 = 2 * (int)((row1 >> (3 * s)) & 7u) + 1;
 #pragma unroll
     for (int p = 0; p < NP; ++p) {
-      const uint32_t b = bp[p] ? *reinterpret_cast<const uint32_t *>(bp[p] + kbase + 16 * s + 4 * t) : 0u;
       int32_t d[4];
-      mma_k16(d, a[0], a[1], b);
+      mma_k16(d, a0, a1, b[p][s]);
       cb[p][0] += m0 * d[0];
       cb[p][1] += m0 * d[1];
       cb[p][2] += m1 * d[2];
@@ -252,11 +331,11 @@ __device__ __forceinline__ void tb_q1(const uint8_t *__restrict__ tb, const uint
   }
 }
 
-// Combine the limb columns of each token and store the warp's partial sums:
-// red[warp][row 0..15][token slot 0..3].
+// Combine the limb columns of each token and store this warp's partial sums
+// to red[row 0..15][token position 0..3].
 template <int NP>
 __device__ __forceinline__ void store_partials(const float acc[NP][4], float *red) {
-  const int lane = threadIdx.x & 31, q = lane >> 2, t = lane & 3, w = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31, q = lane >> 2, t = lane & 3;
   const int n0 = 2 * t, n1 = 2 * t + 1;
   const float f0 = n0 < 6 ? (n0 % 3 == 0 ? 16384.f : (n0 % 3 == 1 ? 128.f : 1.f)) : 0.f;
   const float f1 = n1 < 6 ? (n1 % 3 == 0 ? 16384.f : (n1 % 3 == 1 ? 128.f : 1.f)) : 0.f;
@@ -274,65 +353,126 @@ __device__ __forceinline__ void store_partials(const float acc[NP][4], float *re
       v[j] += __shfl_xor_sync(0xffffffffu, v[j], 2);
     }
     if (t == 0) {
-      float *rw = red + w * 64;
-      rw[q * 4 + 2 * p] = v[0];
-      rw[q * 4 + 2 * p + 1] = v[1];
-      rw[(q + 8) * 4 + 2 * p] = v[2];
-      rw[(q + 8) * 4 + 2 * p + 1] = v[3];
+      red[q * 4 + 2 * p] = v[0];
+      red[q * 4 + 2 * p + 1] = v[1];
+      red[(q + 8) * 4 + 2 * p] = v[2];
+      red[(q + 8) * 4 + 2 * p + 1] = v[3];
     }
   }
 }
 
-// Run one tile-block of either format for up to 4 token positions and
-// store this warp's partials.
-__device__ __forceinline__ void warp_tile_block(int qtype, const uint8_t *tb, const Smem &S, const uint8_t *limbs,
-                                                int lstride, int kbase, const int slots[4], int ntok) {
-  if (ntok <= 2) {
-    const uint8_t *bp[1];
-    b_planes<1>(limbs, lstride, slots, ntok, bp);
-    float acc[1][4] = {{0.f, 0.f, 0.f, 0.f}};
-    if (qtype == kQ2)
-      tb_q2<1>(tb, S.sel2, S.sgn2, bp, kbase, acc);
-    else
-      tb_q1<1>(tb, S.sel1, bp, kbase, acc);
-    store_partials<1>(acc, S.red);
-  } else {
-    const uint8_t *bp[2];
-    b_planes<2>(limbs, lstride, slots, ntok, bp);
-    float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-    if (qtype == kQ2)
-      tb_q2<2>(tb, S.sel2, S.sgn2, bp, kbase, acc);
-    else
-      tb_q1<2>(tb, S.sel1, bp, kbase, acc);
-    store_partials<2>(acc, S.red);
-  }
-}
-
-// Fixed-point limbs of one vector v[0..n) (n a multiple of 32) by one warp:
-// X = round(v * 2^(20-e)) with 2^e > max|v|, X = l0*2^14 + l1*2^7 + l2,
-// each limb in [-64, 64].  Returns e.
-__device__ int warp_limbs(const float *v, int n, uint8_t *dst, int lstride) {
-  const int lane = threadIdx.x & 31;
-  float m = 0.f;
-  for (int i = lane; i < n; i += 32) m = fmaxf(m, fabsf(v[i]));
+// One tile-block of one format for 1-2 (NP = 1) or 3-4 (NP = 2) token
+// positions; the warp's partials go to red (16 x 4 floats).  Kept out of
+// line: one copy of each variant keeps the hot loop inside the
+// instruction cache.
+template <int QT, int NP>
+__device__ __noinline__ void warp_tb(const uint8_t *tb, const uint32_t *sel_a, const uint32_t *sel_b,
+                                     const uint8_t *limbs, int lstride, int kbase, int s0, int s1, int s2, int s3,
+                                     int ntok, float *red) {
+  const int slots[4] = {s0, s1, s2, s3};
+  const uint8_t *bp[NP];
+  b_planes<NP>(limbs, lstride, slots, ntok, bp);
+  float acc[NP][4];
 #pragma unroll
-  for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-  int e = 0;
-  if (m > 0.f) frexpf(m, &e);  // m < 2^e
-  for (int i = lane; i < n; i += 32) {
-    const int X = __float2int_rn(ldexpf(v[i], 20 - e));
-    const int l2 = ((X + 64) & 127) - 64;
-    const int X1 = (X - l2) >> 7;
-    const int l1 = ((X1 + 64) & 127) - 64;
-    const int l0 = (X1 - l1) >> 7;
-    dst[i] = (uint8_t)(int8_t)l0;
-    dst[lstride + i] = (uint8_t)(int8_t)l1;
-    dst[2 * lstride + i] = (uint8_t)(int8_t)l2;
-  }
-  return e;
+  for (int p = 0; p < NP; ++p) acc[p][0] = acc[p][1] = acc[p][2] = acc[p][3] = 0.f;
+  if constexpr (QT == kQ2)
+    tb_q2<NP>(tb, sel_a, sel_b, bp, kbase, acc);
+  else
+    tb_q1<NP>(tb, sel_a, bp, kbase, acc);
+  store_partials<NP>(acc, red);
 }
 
-__device__ __forceinline__ float exp2i(int e) { return ldexpf(1.0f, e); }
+__device__ __forceinline__ void warp_tile_block(int qtype, const uint8_t *tb, const Smem &S, const uint8_t *limbs,
+                                                int lstride, int kbase, const int slots[4], int ntok, float *red) {
+  if (qtype == kQ2) {
+    if (ntok <= 2)
+      warp_tb<kQ2, 1>(tb, S.sel2, S.sgn2, limbs, lstride, kbase, slots[0], slots[1], slots[2], slots[3], ntok, red);
+    else
+      warp_tb<kQ2, 2>(tb, S.sel2, S.sgn2, limbs, lstride, kbase, slots[0], slots[1], slots[2], slots[3], ntok, red);
+  } else {
+    if (ntok <= 2)
+      warp_tb<kQ1, 1>(tb, S.sel1, nullptr, limbs, lstride, kbase, slots[0], slots[1], slots[2], slots[3], ntok, red);
+    else
+      warp_tb<kQ1, 2>(tb, S.sel1, nullptr, limbs, lstride, kbase, slots[0], slots[1], slots[2], slots[3], ntok, red);
+  }
+}
+
+// Vectors are handled as float4 slots: consumer thread tid owns slot
+// g = tid + kCThreads * i (i < 8) of the concatenation of nvec vectors of
+// n floats (n a multiple of 4, nvec * n / 4 <= 8 * kCThreads).
+template <class Load>
+__device__ __forceinline__ void load_slots(int nvec, int n, Load load, float4 v[8]) {
+  const int per = n / 4, total = nvec * per;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int g = threadIdx.x + kCThreads * i;
+    if (g < total) v[i] = load(g / per, g % per);
+  }
+}
+
+// Limbs of up to 4 vectors held in slots (see load_slots): vector j's limb
+// planes go to dst[j] + limb * lstride, scale_out[j] = 2^(e_j - 20) with
+// 2^e_j > max |vector j|.  Two consumer-only syncs (partial maxima).
+__device__ __noinline__ void block_limbs(int nvec, int n, const float4 v[8], uint8_t *const dst[4], int lstride,
+                                         float *wmax, float *scale_out) {
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int per = n / 4, total = nvec * per;
+  float m[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int g = tid + kCThreads * i;
+    if (g < total) {
+      const float mm = fmaxf(fmaxf(fabsf(v[i].x), fabsf(v[i].y)), fmaxf(fabsf(v[i].z), fabsf(v[i].w)));
+      const int j = g / per;
+#pragma unroll
+      for (int jj = 0; jj < 4; ++jj)
+        if (jj == j) m[jj] = fmaxf(m[jj], mm);
+    }
+  }
+#pragma unroll
+  for (int jj = 0; jj < 4; ++jj) {
+#pragma unroll
+    for (int o = 16; o; o >>= 1) m[jj] = fmaxf(m[jj], __shfl_xor_sync(0xffffffffu, m[jj], o));
+    if (lane == 0) wmax[warp * 4 + jj] = m[jj];
+  }
+  consumers_sync();
+  float scale[4];
+#pragma unroll
+  for (int jj = 0; jj < 4; ++jj) {
+    float mm = 0.f;
+#pragma unroll
+    for (int w = 0; w < kCWarps; ++w) mm = fmaxf(mm, wmax[w * 4 + jj]);
+    const int e = pow2_above(mm);
+    scale[jj] = pow2f(20 - e);
+    if (tid == 0 && jj < nvec) scale_out[jj] = pow2f(e - 20);
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int g = tid + kCThreads * i;
+    if (g < total) {
+      const int j = g / per, e4 = g % per;
+      float sc = scale[0];
+#pragma unroll
+      for (int jj = 1; jj < 4; ++jj)
+        if (jj == j) sc = scale[jj];
+      const float f[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
+      uint32_t p0 = 0, p1 = 0, p2 = 0;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        int l0, l1, l2;
+        to_limbs(f[c], sc, l0, l1, l2);
+        p0 |= (uint32_t)(l0 & 0xFF) << (8 * c);
+        p1 |= (uint32_t)(l1 & 0xFF) << (8 * c);
+        p2 |= (uint32_t)(l2 & 0xFF) << (8 * c);
+      }
+      uint8_t *d = dst[j] + 4 * e4;
+      *reinterpret_cast<uint32_t *>(d) = p0;
+      *reinterpret_cast<uint32_t *>(d + lstride) = p1;
+      *reinterpret_cast<uint32_t *>(d + 2 * lstride) = p2;
+    }
+  }
+  consumers_sync();
+}
 
 // ------------------------------------------------------------------ the kernel
 
@@ -356,10 +496,11 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(FusedArgs a)
   const int H = a.hidden, T = a.n_tokens, K = a.top_k, E = a.n_experts;
   const int npairs = T * K;
   const int lstrideX = H + kLimbPad;
+  const bool local_x = T <= kTokChunk;
   Ctrl *ctrl = reinterpret_cast<Ctrl *>(a.ws + a.L.ctrl);
   float *gu = reinterpret_cast<float *>(a.ws + a.L.gu);
   uint8_t *glimbs = a.ws + a.L.limbs;
-  int *gexps = reinterpret_cast<int *>(a.ws + a.L.exps);
+  float *gscale = reinterpret_cast<float *>(a.ws + a.L.exps);
 
   // ---- shared memory carve
   Smem S;
@@ -372,6 +513,8 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(FusedArgs a)
   off += 4096 * kRep1 * 4;
   S.ring = smem + off;
   off += (size_t)kRing * kStageBytes;
+  S.red = reinterpret_cast<float *>(smem + off);
+  off += sizeof(float) * kRing * kCWarps * 64;
   S.limbs = smem + off;
   const int lmax = (H > a.max_ffn ? H : a.max_ffn) + kLimbPad;
   off += (size_t)kTokChunk * 3 * lmax;
@@ -382,68 +525,114 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(FusedArgs a)
   off += sizeof(int) * (kFusedMaxPairs + 64);
   S.pair_w = reinterpret_cast<float *>(smem + off);
   off += sizeof(float) * (kFusedMaxPairs + 64);
-  S.red = reinterpret_cast<float *>(smem + off);
-  off += sizeof(float) * kFWarps * 64;
   S.full = reinterpret_cast<uint64_t *>(smem + off);
   off += sizeof(uint64_t) * kRing;
+  S.empty = reinterpret_cast<uint64_t *>(smem + off);
+  off += sizeof(uint64_t) * kRing;
+  S.done = reinterpret_cast<int *>(smem + off);
+  off += sizeof(int) * kRing;
   S.info = reinterpret_cast<ItemInfo *>(smem + off);
   off += sizeof(ItemInfo) * kRing;
-  S.tok_exp = reinterpret_cast<int *>(smem + off);
-  off += sizeof(int) * kTokChunk;
+  S.tok_scale = reinterpret_cast<float *>(smem + off);
+  off += sizeof(float) * kTokChunk;
+  S.wmax = reinterpret_cast<float *>(smem + off);
+  off += sizeof(float) * kCWarps * 4;
   __shared__ int s_n_inst, s_n1, s_n2, s_bad, s_scan[33];
+  TRACE(0);
 
-  // ---- prologue: selector tables with replication, barriers
-  {
+  // ---- prologue part 1: every independent global load first
+  int my_ids[3];
+  float my_w[3];
+  float4 xv[8];  // activation slots of the (<= 4) tokens when they are converted locally
+  if (tid < kCThreads && local_x)
+    load_slots(T, H, [&](int j, int i4) { return __ldcg(reinterpret_cast<const float4 *>(a.x + (size_t)j * H) + i4); },
+               xv);
+  if (tid < kCThreads) {
+    // selector tables with replication: thread tid fills words tid + 256 j of
+    // each replicated table (consecutive lanes -> consecutive banks); the
+    // source words are fetched in batches so their latencies overlap
     const uint32_t *g2 = reinterpret_cast<const uint32_t *>(a.grids + kGridQ2Sel);
     const uint32_t *gs = reinterpret_cast<const uint32_t *>(a.grids + kGridSign);
     const uint32_t *g1 = reinterpret_cast<const uint32_t *>(a.grids + kGridQ1Sel);
-    for (int i = tid; i < 512 * kRep2; i += kFThreads) S.sel2[i] = g2[i / kRep2];
-    for (int i = tid; i < 256 * kRep2; i += kFThreads) S.sgn2[i] = gs[i / kRep2];
-    for (int i = tid; i < 4096 * kRep1; i += kFThreads) S.sel1[i] = g1[i / kRep1];
-  }
-  if (tid == 0) {
-    for (int s = 0; s < kRing; ++s) mbar_init(&S.full[s], 1);
+#pragma unroll
+    for (int j = 0; j < 3; ++j) {
+      const int p = tid + kCThreads * j;
+      my_ids[j] = p < npairs ? __ldg(a.ids + p) : -1;
+      my_w[j] = p < npairs ? __ldg(a.weights + p) : 0.f;
+    }
+    auto fill = [&](uint32_t *dst, const uint32_t *src, int words, int rep) {
+      for (int j0 = 0; j0 < words; j0 += 16 * kCThreads) {
+        uint32_t v[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const int w = j0 + tid + kCThreads * j;
+          v[j] = w < words ? __ldg(src + w / rep) : 0u;
+        }
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const int w = j0 + tid + kCThreads * j;
+          if (w < words) dst[w] = v[j];
+        }
+      }
+    };
+    fill(S.sel2, g2, 512 * kRep2, kRep2);
+    fill(S.sgn2, gs, 256 * kRep2, kRep2);
+    fill(S.sel1, g1, 4096 * kRep1, kRep1);
+  } else if (lane == 0) {
+    for (int s = 0; s < kRing; ++s) {
+      mbar_init(&S.full[s], 1);
+      mbar_init(&S.empty[s], 1);
+      S.done[s] = 0;
+    }
     mbar_fence_init();
     s_bad = 0;
   }
+  TRACE(1);
 
   // ---- bucketing: counts per expert in the ring (scratch before any copy)
   int *cnt = reinterpret_cast<int *>(S.ring);  // [E]
   int *ids_s = cnt + E;                        // [npairs]
+  float *w_s = reinterpret_cast<float *>(ids_s + npairs);
   for (int e = tid; e < E; e += kFThreads) cnt[e] = 0;
   __syncthreads();
   int bad = 0;
-  for (int p = tid; p < npairs; p += kFThreads) {
-    const int e = a.ids[p];
-    ids_s[p] = e;
-    if (e < 0 || e >= E) {
-      bad |= REDLITE_STATUS_BAD_ID;
-      continue;
+  if (tid < kCThreads) {
+#pragma unroll
+    for (int j = 0; j < 3; ++j) {
+      const int p = tid + kCThreads * j;
+      if (p >= npairs) continue;
+      const int e = my_ids[j];
+      ids_s[p] = e;
+      w_s[p] = my_w[j];
+      if (e < 0 || e >= E) {
+        bad |= REDLITE_STATUS_BAD_ID;
+        continue;
+      }
+      atomicAdd(&cnt[e], 1);
     }
-    atomicAdd(&cnt[e], 1);
   }
   __syncthreads();
   // active experts in ascending id: exclusive scans of (count > 0) and counts
+  int n_routed_pairs = 0;
   {
-    const int per = (E + kFThreads - 1) / kFThreads;
-    const int e0 = tid * per, e1 = min(E, e0 + per);
+    const int per = (E + kCThreads - 1) / kCThreads;
+    const int e0 = tid < kCThreads ? tid * per : E, e1 = min(E, e0 + per);
     int my_act = 0, my_pairs = 0;
     for (int e = e0; e < e1; ++e) {
       my_act += cnt[e] > 0;
       my_pairs += cnt[e];
     }
-    // two block scans (warp shuffles + one shared array)
     int incl_a = my_act, incl_p = my_pairs;
 #pragma unroll
     for (int o = 1; o < 32; o <<= 1) {
       const int ya = __shfl_up_sync(0xffffffffu, incl_a, o), yp = __shfl_up_sync(0xffffffffu, incl_p, o);
       if (lane >= o) incl_a += ya, incl_p += yp;
     }
-    if (lane == 31) s_scan[warp] = incl_a, s_scan[16 + warp] = incl_p;
+    if (lane == 31 && warp < kCWarps) s_scan[warp] = incl_a, s_scan[16 + warp] = incl_p;
     __syncthreads();
     if (tid == 0) {
       int sa = 0, sp = 0;
-      for (int w = 0; w < kFWarps; ++w) {
+      for (int w = 0; w < kCWarps; ++w) {
         const int ta = s_scan[w], tp = s_scan[16 + w];
         s_scan[w] = sa, s_scan[16 + w] = sp;
         sa += ta, sp += tp;
@@ -452,23 +641,26 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(FusedArgs a)
       s_scan[32] = sp;
     }
     __syncthreads();
-    int act = s_scan[warp] + incl_a - my_act, pst = s_scan[16 + warp] + incl_p - my_pairs;
-    for (int e = e0; e < e1; ++e) {
-      if (cnt[e] > 0) {
-        Inst &I = S.inst[act];
-        I.qtype = e;  // expert id for now; descriptor below
-        I.pair_start = pst;
-        I.count = cnt[e];
-        cnt[e] = pst;  // becomes the running cursor of the stable fill
-        ++act;
-        pst += I.count;
+    if (tid < kCThreads) {
+      int act = s_scan[warp] + incl_a - my_act, pst = s_scan[16 + warp] + incl_p - my_pairs;
+      for (int e = e0; e < e1; ++e) {
+        if (cnt[e] > 0) {
+          Inst &I = S.inst[act];
+          I.qtype = e;  // expert id for now; descriptor below
+          I.pair_start = pst;
+          I.count = cnt[e];
+          cnt[e] = pst;  // becomes the running cursor of the stable fill
+          ++act;
+          pst += I.count;
+        }
       }
     }
+    __syncthreads();
+    n_routed_pairs = s_scan[32];
   }
-  __syncthreads();
-  const int n_routed_pairs = s_scan[32];
-  // stable fill of the pair list (one warp, pairs in index order)
-  if (warp == 0) {
+  int n_inst = s_n_inst;
+  if (warp == kCWarps) {
+    // stable fill of the pair list (the producer warp, pairs in index order)
     for (int p0 = 0; p0 < npairs; p0 += 32) {
       const int p = p0 + lane;
       const int e = p < npairs ? ids_s[p] : -1;
@@ -478,277 +670,317 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(FusedArgs a)
         const int rank = __popc(m & ((1u << lane) - 1u));
         const int pos = cnt[e] + rank;
         S.pair_tok[pos] = p / K;
-        S.pair_w[pos] = a.weights[p];
+        S.pair_w[pos] = w_s[p];
       }
       __syncwarp();
       if (ok && (m & ((1u << lane) - 1u)) == 0) cnt[e] += __popc(m);
       __syncwarp();
     }
-  }
-  // descriptors; the shared expert is the last instance
-  int n_inst = s_n_inst;
-  for (int u = tid; u < n_inst; u += kFThreads) {
-    Inst &I = S.inst[u];
-    const redlite_moe_expert d = a.experts[I.qtype];
-    if (fused_expert_ok(d, H, a.max_ffn)) {
-      I.gate = (const uint8_t *)d.gate, I.up = (const uint8_t *)d.up, I.down = (const uint8_t *)d.down;
-      I.qtype = d.qtype, I.ffn = d.ffn;
-    } else {
-      bad |= REDLITE_STATUS_BAD_EXPERT;
-      I.gate = I.up = I.down = nullptr;
-      I.qtype = kQ2, I.ffn = 256, I.count = 0;
+  } else {
+    // descriptors (consumer threads, one instance each)
+    for (int u = tid; u < n_inst; u += kCThreads) {
+      Inst &I = S.inst[u];
+      const redlite_moe_expert d = a.experts[I.qtype];
+      if (fused_expert_ok(d, H, a.max_ffn)) {
+        I.gate = (const uint8_t *)d.gate, I.up = (const uint8_t *)d.up, I.down = (const uint8_t *)d.down;
+        I.qtype = d.qtype, I.ffn = d.ffn;
+      } else {
+        bad |= REDLITE_STATUS_BAD_EXPERT;
+        I.gate = I.up = I.down = nullptr;
+        I.qtype = kQ2, I.ffn = 256, I.count = 0;
+      }
+    }
+    if (a.has_shared) {
+      if (tid == 0) {
+        Inst &I = S.inst[n_inst];
+        I.gate = (const uint8_t *)a.shared.gate, I.up = (const uint8_t *)a.shared.up;
+        I.down = (const uint8_t *)a.shared.down, I.qtype = a.shared.qtype, I.ffn = a.shared.ffn;
+        I.pair_start = n_routed_pairs, I.count = T;
+      }
+      for (int t = tid; t < T; t += kCThreads) S.pair_tok[n_routed_pairs + t] = t, S.pair_w[n_routed_pairs + t] = 1.f;
     }
   }
-  if (a.has_shared && tid == 0) {
-    Inst &I = S.inst[n_inst];
-    I.gate = (const uint8_t *)a.shared.gate, I.up = (const uint8_t *)a.shared.up;
-    I.down = (const uint8_t *)a.shared.down, I.qtype = a.shared.qtype, I.ffn = a.shared.ffn;
-    I.pair_start = n_routed_pairs, I.count = T;
-  }
-  if (a.has_shared)
-    for (int t = tid; t < T; t += kFThreads) S.pair_tok[n_routed_pairs + t] = t, S.pair_w[n_routed_pairs + t] = 1.f;
   if (a.has_shared) n_inst += 1;
   if (bad) atomicOr(&s_bad, bad);
   __syncthreads();
-  // work items per instance and their prefix sums (thread 0; n_inst is small)
-  if (tid == 0) {
-    int n1 = 0, n2 = 0;
-    for (int u = 0; u < n_inst; ++u) {
-      Inst &I = S.inst[u];
-      const int nch = (I.count + kTokChunk - 1) / kTokChunk;
-      const int it = item_tiles_of(I.ffn);
-      const int ngrp = (H / 16 + it - 1) / it;
-      I.p1_base = n1, I.p2_base = n2;
-      n1 += nch * 2 * (I.ffn / 16);
-      n2 += nch * ngrp;
+  // work items per instance and their prefix sums (one warp; n_inst is small)
+  if (warp == 0) {
+    int base1 = 0, base2 = 0;
+    for (int u0 = 0; u0 < n_inst; u0 += 32) {
+      const int u = u0 + lane;
+      int c1 = 0, c2 = 0;
+      if (u < n_inst) {
+        const Inst &I = S.inst[u];
+        const int nch = (I.count + kTokChunk - 1) / kTokChunk;
+        const int it = item_tiles_of(I.ffn);
+        c1 = nch * 2 * (I.ffn / 16);
+        c2 = nch * ((H / 16 + it - 1) / it);
+      }
+      int i1 = c1, i2 = c2;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int y1 = __shfl_up_sync(0xffffffffu, i1, o), y2 = __shfl_up_sync(0xffffffffu, i2, o);
+        if (lane >= o) i1 += y1, i2 += y2;
+      }
+      if (u < n_inst) S.inst[u].p1_base = base1 + i1 - c1, S.inst[u].p2_base = base2 + i2 - c2;
+      base1 += __shfl_sync(0xffffffffu, i1, 31);
+      base2 += __shfl_sync(0xffffffffu, i2, 31);
     }
-    s_n1 = n1, s_n2 = n2;
-    if (s_bad) atomicOr(a.status, s_bad);
+    if (lane == 0) {
+      s_n1 = base1, s_n2 = base2;
+      if (s_bad) atomicOr(a.status, s_bad);
+    }
   }
   __syncthreads();
+  TRACE(2);
   const int N1 = s_n1, N2 = s_n2;
   const int b1 = (int)((int64_t)cta * N1 / G), e1i = (int)((int64_t)(cta + 1) * N1 / G);
   const int rc = G - 1 - cta;
   const int b2 = (int)((int64_t)rc * N2 / G), e2i = (int)((int64_t)(rc + 1) * N2 / G);
   const int my1 = e1i - b1, my2 = e2i - b2, my_items = my1 + my2;
 
-  // ---- item lookup: instance of global phase item j (binary search on bases)
-  auto find_inst = [&](int j, int phase) {
-    int lo = 0, hi = n_inst - 1;
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      const int base = phase == 1 ? S.inst[mid].p1_base : S.inst[mid].p2_base;
-      if (base <= j) lo = mid; else hi = mid - 1;
-    }
-    return lo;
-  };
-  // issue item k of this CTA into its ring stage (thread 0 only)
-  auto issue = [&](int k) {
-    const int s = k % kRing;
-    ItemInfo inf;
-    const uint8_t *src;
-    uint32_t bytes;
-    if (k < my1) {
-      const int j = b1 + k, u = find_inst(j, 1);
-      const Inst &I = S.inst[u];
-      const int per = 2 * (I.ffn / 16), loc = j - I.p1_base;
-      inf.phase = 1, inf.inst = u, inf.chunk = loc / per;
-      const int rem = loc % per;
-      inf.sub = rem / (I.ffn / 16), inf.tile = rem % (I.ffn / 16);
-      const int tbb = tile_block_bytes(I.qtype);
-      bytes = (uint32_t)((H / 256) * tbb);
-      src = (inf.sub ? I.up : I.gate) + (size_t)inf.tile * bytes;
-    } else {
-      const int j = b2 + (k - my1), u = find_inst(j, 2);
-      const Inst &I = S.inst[u];
-      const int it = item_tiles_of(I.ffn), ngrp = (H / 16 + it - 1) / it, loc = j - I.p2_base;
-      inf.phase = 2, inf.inst = u, inf.chunk = loc / ngrp, inf.tile = loc % ngrp, inf.sub = 0;
-      const int tiles = min(it, H / 16 - inf.tile * it);
-      const int tbb = tile_block_bytes(I.qtype);
-      const size_t tile_bytes = (size_t)(I.ffn / 256) * tbb;
-      bytes = (uint32_t)(tiles * tile_bytes);
-      src = I.down + (size_t)inf.tile * it * tile_bytes;
-    }
-    S.info[s] = inf;
-    mbar_expect_tx(&S.full[s], bytes);
-    bulk_g2s(S.ring + (size_t)s * kStageBytes, src, bytes, &S.full[s]);
-  };
-
-  // ---- activations: T <= chunk: every CTA builds all limbs locally;
-  // otherwise phase 0 converts tokens cooperatively into the workspace.
-  const bool local_x = T <= kTokChunk;
-  __syncthreads();  // the ring scratch (counts, ids) is dead from here on
-  if (tid == 0) {
-    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // generic writes before bulk copies
-    for (int k = 0; k < min(kRing, my_items); ++k) issue(k);
-  }
-  if (local_x) {
-    for (int t = warp; t < T; t += kFWarps) {
-      const int e = warp_limbs(a.x + (size_t)t * H, H, S.limbs + (size_t)t * 3 * lstrideX, lstrideX);
-      if (lane == 0) S.tok_exp[t] = e;
-    }
-  } else {
-    for (int t = cta * kFWarps + warp; t < T; t += G * kFWarps) {
-      const int e = warp_limbs(a.x + (size_t)t * H, H, glimbs + (size_t)t * 3 * lstrideX, lstrideX);
-      if (lane == 0) gexps[t] = e;
-    }
-    __syncthreads();
-    if (tid == 0) {
-      __threadfence();
-      atomicAdd(&ctrl->phase0_done, 1);
-      uint32_t it = 0;
-      while (ld_acquire(&ctrl->phase0_done) < G) {
-        if (++it > kSpinLimit) {
+  // ---- producer warp: streams this CTA's items through the ring
+  if (warp == kCWarps) {
+    if (lane == 0) {
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // generic writes before bulk copies
+      for (int k = 0; k < my_items; ++k) {
+        const int s = k % kRing;
+        if (k >= kRing && !mbar_wait(&S.empty[s], (uint32_t)(((k / kRing) - 1) & 1))) {
           atomicOr(a.status, REDLITE_STATUS_TIMEOUT);
           break;
         }
-        __nanosleep(64);
+        ItemInfo inf;
+        const uint8_t *src;
+        uint32_t bytes;
+        const bool p1 = k < my1;
+        const int j = p1 ? b1 + k : b2 + (k - my1);
+        int lo = 0, hi = n_inst - 1;  // last instance whose base <= j
+        while (lo < hi) {
+          const int mid = (lo + hi + 1) >> 1;
+          if ((p1 ? S.inst[mid].p1_base : S.inst[mid].p2_base) <= j) lo = mid; else hi = mid - 1;
+        }
+        const Inst &I = S.inst[lo];
+        const int tbb = tile_block_bytes(I.qtype);
+        inf.inst = lo;
+        if (p1) {
+          const int nt = I.ffn / 16, per = 2 * nt, loc = j - I.p1_base;
+          inf.phase = 1, inf.chunk = loc / per, inf.sub = (loc % per) / nt, inf.tile = loc % nt;
+          bytes = (uint32_t)((H / 256) * tbb);
+          src = (inf.sub ? I.up : I.gate) + (size_t)inf.tile * bytes;
+        } else {
+          const int it = item_tiles_of(I.ffn), ngrp = (H / 16 + it - 1) / it, loc = j - I.p2_base;
+          inf.phase = 2, inf.chunk = loc / ngrp, inf.tile = loc % ngrp, inf.sub = 0;
+          const int tiles = min(it, H / 16 - inf.tile * it);
+          const size_t tile_bytes = (size_t)(I.ffn / 256) * tbb;
+          bytes = (uint32_t)(tiles * tile_bytes);
+          src = I.down + (size_t)inf.tile * it * tile_bytes;
+        }
+        S.info[s] = inf;
+        mbar_expect_tx(&S.full[s], bytes);
+        bulk_g2s(S.ring + (size_t)s * kStageBytes, src, bytes, &S.full[s]);
       }
     }
-  }
-  __syncthreads();
-
-  // ---- main loop over this CTA's items
-  int cur_inst = -1, cur_chunk = -1, cur_phase = 0;
-  int ntok = 0;
-  int slots[kTokChunk] = {0, 0, 0, 0};  // limb slot of each token position of the chunk
-  for (int k = 0; k < my_items; ++k) {
-    const int s = k % kRing;
-    if (k == my1) {
-      // end of phase 1: zero a slice of out, then the grid barrier
-      const size_t total4 = (size_t)T * H / 4;
-      const size_t z0 = total4 * cta / G, z1 = total4 * (cta + 1) / G;
-      for (size_t i = z0 + tid; i < z1; i += kFThreads) reinterpret_cast<float4 *>(a.out)[i] = make_float4(0, 0, 0, 0);
-      __syncthreads();
+  } else {
+    // ---- consumers: activations to limbs (locally, or phase 0 cooperative)
+    if (local_x) {
+      uint8_t *dst[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) dst[j] = S.limbs + (size_t)j * 3 * lstrideX;
+      TRACE(12);
+      block_limbs(T, H, xv, dst, lstrideX, S.wmax, S.tok_scale);
+    } else {
+      for (int t = cta; t < T; t += G) {
+        uint8_t *dst[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) dst[j] = glimbs + (size_t)t * 3 * lstrideX;
+        float4 v[8];
+        load_slots(1, H, [&](int, int i4) { return __ldcg(reinterpret_cast<const float4 *>(a.x + (size_t)t * H) + i4); },
+                   v);
+        block_limbs(1, H, v, dst, lstrideX, S.wmax, gscale + t);
+      }
+      consumers_sync();
       if (tid == 0) {
         __threadfence();
-        atomicAdd(&ctrl->phase1_done, 1);
+        atomicAdd(&ctrl->phase0_done, 1);
         uint32_t it = 0;
-        while (ld_acquire(&ctrl->phase1_done) < G) {
+        while (ld_acquire(&ctrl->phase0_done) < G) {
           if (++it > kSpinLimit) {
             atomicOr(a.status, REDLITE_STATUS_TIMEOUT);
             break;
           }
-          __nanosleep(32);
+          __nanosleep(64);
         }
         __threadfence();
       }
-      __syncthreads();
+      consumers_sync();
     }
-    // wait for this stage's bytes (bounded)
-    {
-      uint32_t it = 0;
-      const uint32_t parity = (uint32_t)((k / kRing) & 1);
-      while (!mbar_try_wait(&S.full[s], parity)) {
-        if (++it > kSpinLimit) {
-          if (tid == 0) atomicOr(a.status, REDLITE_STATUS_TIMEOUT);
-          break;
-        }
-      }
-    }
-    const ItemInfo inf = S.info[s];
-    const Inst I = S.inst[inf.inst];
-    const uint8_t *stage = S.ring + (size_t)s * kStageBytes;
-    const int tbb = tile_block_bytes(I.qtype);
-    const int pbase = I.pair_start + kTokChunk * inf.chunk;
-    // (re)load the token chunk's limbs when the instance/chunk/phase changes
-    if (inf.inst != cur_inst || inf.chunk != cur_chunk || inf.phase != cur_phase) {
-      cur_inst = inf.inst, cur_chunk = inf.chunk, cur_phase = inf.phase;
-      ntok = min(kTokChunk, I.count - kTokChunk * inf.chunk);
-      for (int j = 0; j < kTokChunk; ++j) slots[j] = j;
-      if (inf.phase == 1) {
-        if (local_x) {
-          for (int j = 0; j < ntok; ++j) slots[j] = S.pair_tok[pbase + j];  // limbs are indexed by token
-        } else {
-          const int nvec = 3 * lstrideX / 16;
-          for (int j = 0; j < ntok; ++j) {
-            const int t = S.pair_tok[pbase + j];
-            const uint4 *src = reinterpret_cast<const uint4 *>(glimbs + (size_t)t * 3 * lstrideX);
-            uint4 *dst = reinterpret_cast<uint4 *>(S.limbs + (size_t)j * 3 * lstrideX);
-            for (int v = tid; v < nvec; v += kFThreads) dst[v] = __ldcg(src + v);
-            if (tid == 0) S.tok_exp[j] = __ldcg(gexps + t);
+    TRACE(3);
+
+    // ---- main loop over this CTA's items
+    int cur_inst = -1, cur_chunk = -1, cur_phase = 0;
+    int ntok = 0;
+    int slots[kTokChunk] = {0, 0, 0, 0};  // limb slot of each token position of the chunk
+    for (int k = 0; k < my_items; ++k) {
+      const int s = k % kRing;
+      if (k == my1) {
+        TRACE(4);
+        // end of phase 1: zero a slice of out, then the grid barrier
+        const size_t total4 = (size_t)T * H / 4;
+        const size_t z0 = total4 * cta / G, z1 = total4 * (cta + 1) / G;
+        for (size_t i = z0 + tid; i < z1; i += kCThreads)
+          reinterpret_cast<float4 *>(a.out)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+        consumers_sync();
+        if (tid == 0) {
+          __threadfence();
+          atomicAdd(&ctrl->phase1_done, 1);
+          uint32_t it = 0;
+          while (ld_acquire(&ctrl->phase1_done) < G) {
+            if (++it > kSpinLimit) {
+              atomicOr(a.status, REDLITE_STATUS_TIMEOUT);
+              break;
+            }
+            __nanosleep(32);
           }
+          __threadfence();
         }
-      } else {
-        // h = SiLU(g) * u for each token of the chunk, then its limbs
-        const int F = I.ffn, lstrideH = F + kLimbPad;
-        for (int j = warp; j < ntok; j += kFWarps) {
-          const float *g = gu + (size_t)(pbase + j) * 2 * a.max_ffn;
-          const float *u = g + a.max_ffn;
-          float m = 0.f;
-          for (int i = lane; i < F; i += 32) m = fmaxf(m, fabsf(silu_mul(__ldcg(g + i), __ldcg(u + i))));
+        consumers_sync();
+        TRACE(5);
+      }
+      if (!mbar_wait(&S.full[s], (uint32_t)((k / kRing) & 1))) {
+        if (lane == 0) atomicOr(a.status, REDLITE_STATUS_TIMEOUT);
+      }
+      const ItemInfo inf = S.info[s];
+      const Inst &I = S.inst[inf.inst];
+      const int qtype = I.qtype, F = I.ffn;
+      const uint8_t *stage = S.ring + (size_t)s * kStageBytes;
+      const int tbb = tile_block_bytes(qtype);
+      const int pbase = I.pair_start + kTokChunk * inf.chunk;
+      // (re)load the token chunk's limbs when the instance/chunk/phase changes
+      if (inf.inst != cur_inst || inf.chunk != cur_chunk || inf.phase != cur_phase) {
+        cur_inst = inf.inst, cur_chunk = inf.chunk, cur_phase = inf.phase;
+        ntok = min(kTokChunk, I.count - kTokChunk * inf.chunk);
 #pragma unroll
-          for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-          int e = 0;
-          if (m > 0.f) frexpf(m, &e);
-          uint8_t *dst = S.limbs + (size_t)j * 3 * lstrideH;
-          for (int i = lane; i < F; i += 32) {
-            const int X = __float2int_rn(ldexpf(silu_mul(__ldcg(g + i), __ldcg(u + i)), 20 - e));
-            const int l2 = ((X + 64) & 127) - 64;
-            const int X1 = (X - l2) >> 7;
-            const int l1 = ((X1 + 64) & 127) - 64;
-            const int l0 = (X1 - l1) >> 7;
-            dst[i] = (uint8_t)(int8_t)l0;
-            dst[lstrideH + i] = (uint8_t)(int8_t)l1;
-            dst[2 * lstrideH + i] = (uint8_t)(int8_t)l2;
+        for (int j = 0; j < kTokChunk; ++j) slots[j] = j;
+        if (inf.phase == 1) {
+          if (local_x) {
+            for (int j = 0; j < ntok; ++j) slots[j] = S.pair_tok[pbase + j];  // limbs are indexed by token
+          } else {
+            consumers_sync();  // every warp is done with the previous chunk's limbs
+            const int nvec = 3 * lstrideX / 16;  // <= 390 for H <= 2048
+            uint4 buf[kTokChunk][2];
+#pragma unroll
+            for (int j = 0; j < kTokChunk; ++j) {
+              const int t = j < ntok ? S.pair_tok[pbase + j] : 0;
+              const uint4 *src = reinterpret_cast<const uint4 *>(glimbs + (size_t)t * 3 * lstrideX);
+#pragma unroll
+              for (int h = 0; h < 2; ++h)
+                if (j < ntok && tid + kCThreads * h < nvec) buf[j][h] = __ldcg(src + tid + kCThreads * h);
+            }
+#pragma unroll
+            for (int j = 0; j < kTokChunk; ++j) {
+              uint4 *dst = reinterpret_cast<uint4 *>(S.limbs + (size_t)j * 3 * lstrideX);
+#pragma unroll
+              for (int h = 0; h < 2; ++h)
+                if (j < ntok && tid + kCThreads * h < nvec) dst[tid + kCThreads * h] = buf[j][h];
+            }
+            if (tid < ntok) S.tok_scale[tid] = __ldcg(gscale + S.pair_tok[pbase + tid]);
+            consumers_sync();
           }
-          if (lane == 0) S.tok_exp[j] = e;
+        } else {
+          // h = SiLU(g) * u of each token of the chunk, then its limbs
+          consumers_sync();
+          const int lstrideH = F + kLimbPad;
+          uint8_t *dst[4];
+#pragma unroll
+          for (int j = 0; j < 4; ++j) dst[j] = S.limbs + (size_t)j * 3 * lstrideH;
+          const float *gbase = gu + (size_t)pbase * 2 * a.max_ffn;
+          const int mf = a.max_ffn;
+          float4 v[8];
+          load_slots(
+              ntok, F,
+              [&](int j, int i4) {
+                const float4 g = __ldcg(reinterpret_cast<const float4 *>(gbase + (size_t)j * 2 * mf) + i4);
+                const float4 u = __ldcg(reinterpret_cast<const float4 *>(gbase + (size_t)j * 2 * mf + mf) + i4);
+                return make_float4(silu_mul(g.x, u.x), silu_mul(g.y, u.y), silu_mul(g.z, u.z), silu_mul(g.w, u.w));
+              },
+              v);
+          block_limbs(ntok, F, v, dst, lstrideH, S.wmax, S.tok_scale);
         }
       }
-      __syncthreads();
-    }
-    if (inf.phase == 1) {
-      // one 16-row tile of gate or up: warp w takes input blocks w, w+8, ...
-      const int nkb = H / 256;
-      if (warp < nkb) {
-        for (int kb = warp; kb < nkb; kb += kFWarps) {
-          // warps with several input blocks accumulate through the partials
-          // area: only H <= 2048 is routed here, so kb == warp
-          warp_tile_block(I.qtype, stage + kb * tbb, S, S.limbs, lstrideX, kb * 256, slots, ntok);
+      float *red = S.red + (size_t)s * kCWarps * 64;
+      int nw;  // warps holding partials of this item
+      if (inf.phase == 1) {
+        const int nkb = H / 256;  // <= 8: warp w takes input block w
+        nw = nkb;
+#ifdef REDLITE_TRACE
+        const long long c0 = clock64();
+#endif
+        if (warp < nkb)
+          warp_tile_block(qtype, stage + warp * tbb, S, S.limbs, lstrideX, warp * 256, slots, ntok, red + warp * 64);
+#ifdef REDLITE_TRACE
+        if (k < 4 && warp < 4) TRACEC(k * 4 + warp, (uint64_t)(clock64() - c0));
+#endif
+      } else {
+        const int nkb = F / 256, it = item_tiles_of(F);
+        const int tiles = min(it, H / 16 - inf.tile * it);
+        nw = tiles * nkb;  // <= 8: warp w takes tile w / nkb, input block w % nkb
+        if (warp < nw)
+          warp_tile_block(qtype, stage + warp * tbb, S, S.limbs, F + kLimbPad, (warp % nkb) * 256, slots, ntok,
+                          red + warp * 64);
+      }
+      // the last consumer warp to finish reduces the item and frees the stage
+      __syncwarp();
+      int prev = 0;
+      if (lane == 0) {
+        __threadfence_block();
+        prev = atomicAdd(&S.done[s], 1);
+      }
+      prev = __shfl_sync(0xffffffffu, prev, 0);
+      if (prev == kCWarps - 1) {
+        __threadfence_block();
+        if (inf.phase == 1) {
+          for (int j2 = lane; j2 < 16 * ntok; j2 += 32) {
+            const int row = j2 & 15, j = j2 >> 4;
+            float v = 0.f;
+            for (int w = 0; w < nw; ++w) v += red[w * 64 + row * 4 + j];
+            const float sc = local_x ? S.tok_scale[slots[j]] : S.tok_scale[j];
+            gu[(size_t)(pbase + j) * 2 * a.max_ffn + (size_t)inf.sub * a.max_ffn + inf.tile * 16 + row] = v * sc;
+          }
+        } else {
+          const int nkb = F / 256, it = item_tiles_of(F);
+          const int tiles = nw / nkb;
+          for (int j2 = lane; j2 < tiles * 16 * ntok; j2 += 32) {
+            const int j = j2 % ntok, rt = j2 / ntok;
+            const int tile = rt >> 4, row = rt & 15;
+            float v = 0.f;
+            for (int kb = 0; kb < nkb; ++kb) v += red[(tile * nkb + kb) * 64 + row * 4 + j];
+            const int r = (inf.tile * it + tile) * 16 + row;
+            atomicAdd(a.out + (size_t)S.pair_tok[pbase + j] * H + r, S.pair_w[pbase + j] * (v * S.tok_scale[j]));
+          }
+        }
+        __syncwarp();
+        if (lane == 0) {
+          S.done[s] = 0;
+          mbar_arrive(&S.empty[s]);
         }
       }
-      __syncthreads();
-      if (tid < 16 * ntok) {
-        const int row = tid & 15, j = tid >> 4;
-        float v = 0.f;
-        for (int w = 0; w < min(nkb, kFWarps); ++w) v += S.red[w * 64 + row * 4 + j];
-        gu[(size_t)(pbase + j) * 2 * a.max_ffn + (size_t)inf.sub * a.max_ffn + inf.tile * 16 + row] =
-            v * exp2i(S.tok_exp[slots[j]] - 20);
-      }
-    } else {
-      // a group of down tiles: warp w takes tile-block w (tile w / nkb, input block w % nkb)
-      const int F = I.ffn, nkb = F / 256, lstrideH = F + kLimbPad;
-      const int it = item_tiles_of(F);
-      const int tiles = min(it, H / 16 - inf.tile * it);
-      const int ntb = tiles * nkb;  // <= 8
-      if (warp < ntb) warp_tile_block(I.qtype, stage + warp * tbb, S, S.limbs, lstrideH, (warp % nkb) * 256, slots, ntok);
-      __syncthreads();
-      for (int j2 = tid; j2 < tiles * 16 * ntok; j2 += kFThreads) {
-        const int j = j2 % ntok, rt = j2 / ntok;
-        const int tile = rt / 16, row = rt % 16;
-        float v = 0.f;
-        for (int kb = 0; kb < nkb; ++kb) v += S.red[(tile * nkb + kb) * 64 + row * 4 + j];
-        const int r = (inf.tile * it + tile) * 16 + row;
-        const float y = v * exp2i(S.tok_exp[j] - 20);
-        atomicAdd(a.out + (size_t)S.pair_tok[pbase + j] * H + r, S.pair_w[pbase + j] * y);
-      }
     }
-    __syncthreads();  // stage and partials consumed
-    if (tid == 0 && k + kRing < my_items) issue(k + kRing);
-  }
-  if (my1 == my_items) {
-    // no phase-2 items: still zero the slice and pass the barrier
-    const size_t total4 = (size_t)T * H / 4;
-    const size_t z0 = total4 * cta / G, z1 = total4 * (cta + 1) / G;
-    for (size_t i = z0 + tid; i < z1; i += kFThreads) reinterpret_cast<float4 *>(a.out)[i] = make_float4(0, 0, 0, 0);
-    __syncthreads();
-    if (tid == 0) {
-      __threadfence();
-      atomicAdd(&ctrl->phase1_done, 1);
+    if (my1 == my_items) {
+      // no phase-2 items: still zero the slice and count at the barrier
+      const size_t total4 = (size_t)T * H / 4;
+      const size_t z0 = total4 * cta / G, z1 = total4 * (cta + 1) / G;
+      for (size_t i = z0 + tid; i < z1; i += kCThreads)
+        reinterpret_cast<float4 *>(a.out)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+      consumers_sync();
+      if (tid == 0) {
+        __threadfence();
+        atomicAdd(&ctrl->phase1_done, 1);
+      }
     }
   }
   // ---- exit: the last CTA resets the counters for the next call
   __syncthreads();
+  TRACE(6);
   if (tid == 0) {
     __threadfence();
     const int prev = atomicAdd(&ctrl->exit_count, 1);
@@ -764,13 +996,14 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(FusedArgs a)
 size_t fused_smem_bytes(int hidden, int max_ffn) {
   size_t off = 512 * kRep2 * 4 + 256 * kRep2 * 4 + 4096 * kRep1 * 4;
   off += (size_t)kRing * kStageBytes;
+  off += sizeof(float) * kRing * kCWarps * 64;
   const int lmax = (hidden > max_ffn ? hidden : max_ffn) + kLimbPad;
   off += (size_t)kTokChunk * 3 * lmax;
   off = (off + 15) & ~size_t(15);
   off += sizeof(Inst) * kFusedMaxInst;
   off += 2 * sizeof(int) * (kFusedMaxPairs + 64);
-  off += sizeof(float) * kFWarps * 64 * 2;
-  off += sizeof(uint64_t) * kRing + sizeof(ItemInfo) * kRing + sizeof(int) * kTokChunk;
+  off += 2 * sizeof(uint64_t) * kRing + sizeof(int) * kRing + sizeof(ItemInfo) * kRing;
+  off += sizeof(float) * kTokChunk + sizeof(float) * kCWarps * 4;
   return off + 64;
 }
 
@@ -778,7 +1011,8 @@ bool fused_supported(int hidden, int max_ffn, int n_tokens, int top_k, int n_exp
   if (hidden % 256 || hidden > 2048 || max_ffn % 256 || max_ffn > 2048) return false;
   if ((int64_t)n_tokens * top_k > kFusedMaxPairs) return false;
   if (has_shared && n_tokens > 64) return false;
-  if (n_experts > (kRing * kStageBytes) / 4 - kFusedMaxPairs) return false;
+  // bucketing scratch (counts, ids, weights) lives in the ring
+  if ((size_t)n_experts * 4 + 8 * (size_t)kFusedMaxPairs > (size_t)kRing * kStageBytes) return false;
   return fused_smem_bytes(hidden, max_ffn) <= 227 * 1024;
 }
 
