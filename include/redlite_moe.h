@@ -151,6 +151,34 @@ int redlite_moe_layer(const float *x, int32_t n_tokens, const int32_t *expert_id
                       int32_t top_k, const redlite_moe_table *expert_table, const redlite_moe_expert *shared_expert,
                       float *out);
 
+/* The layer for callers that cannot allocate device memory.  Some callers
+ * have no way to call cudaMalloc for the workspace: for example a plugin
+ * running inside a host application that owns the whole device-memory
+ * budget and hands out only the tensors it manages, or code with no
+ * allocator at hand.  This entry point runs the same fused decode kernel as
+ * redlite_moe_layer but keeps the kernel's scratch in a fixed 4 MiB array
+ * that the library itself holds in device memory (every GPU that loads the
+ * library keeps it until the process exits).  It allocates nothing.
+ * There is no counterpart on the pages: it is an interface convenience.
+ *   Arguments as redlite_moe_layer; table->workspace and
+ *   table->workspace_bytes are ignored.
+ *   Only decode-sized calls the fused kernel takes are accepted
+ *   (n_tokens * top_k <= 640, hidden and every expert width multiples of
+ *   256 up to 2048, table->min_ffn >= 256): otherwise REDLITE_EUNSUPPORTED.
+ *   A call whose scratch (control block + 2 * 4 * max_ffn bytes per
+ *   (token, slot) pair incl. the shared expert + about 3 * hidden bytes per
+ *   token) exceeds 4 MiB returns REDLITE_ENOMEM before enqueuing anything.
+ *   The first call on a device looks the array up (cudaGetSymbolAddress)
+ *   and clears its control words on table->stream; make that first call
+ *   before any stream capture.
+ *   Every call on a device shares the one array, which keeps the last
+ *   call's contents: calls that overlap on the GPU (different streams, or
+ *   different host threads without ordering) race and must not be issued;
+ *   order them on one stream. */
+int redlite_moe_layer_noalloc(const float *x, int32_t n_tokens, const int32_t *expert_ids,
+                              const float *router_weights, int32_t top_k, const redlite_moe_table *expert_table,
+                              const redlite_moe_expert *shared_expert, float *out);
+
 /* Host-side conversion of one matrix from the interchange layout to the
  * resident layout.  src, dst: host buffers of redlite_moe_matrix_bytes()
  * bytes, not overlapping.  REDLITE_EUNSUPPORTED for shapes the kernels do

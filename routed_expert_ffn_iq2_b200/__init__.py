@@ -23,6 +23,7 @@ from ._native import (  # noqa: F401
     redlite_moe_expert,
     redlite_moe_grids_bytes,
     redlite_moe_layer,
+    redlite_moe_layer_noalloc,
     redlite_moe_matrix_bytes,
     redlite_moe_pack_matrix,
     redlite_moe_table,

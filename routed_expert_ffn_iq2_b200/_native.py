@@ -56,6 +56,9 @@ EXPORTS = {
     "redlite_moe_layer": (ctypes.c_int, [_c_void_p, ctypes.c_int32, _c_void_p, _c_void_p, ctypes.c_int32,
                                          ctypes.POINTER(redlite_moe_table), ctypes.POINTER(redlite_moe_expert),
                                          _c_void_p]),
+    "redlite_moe_layer_noalloc": (ctypes.c_int, [_c_void_p, ctypes.c_int32, _c_void_p, _c_void_p, ctypes.c_int32,
+                                                 ctypes.POINTER(redlite_moe_table),
+                                                 ctypes.POINTER(redlite_moe_expert), _c_void_p]),
     "redlite_moe_pack_matrix": (ctypes.c_int, [ctypes.c_int32, ctypes.c_int64, ctypes.c_int64, _c_void_p,
                                                _c_void_p]),
     "redlite_moe_dequant": (ctypes.c_int, [ctypes.c_int32, _c_void_p, ctypes.c_int64, ctypes.c_int64, _c_void_p,
@@ -152,6 +155,16 @@ def redlite_moe_layer(x: torch.Tensor, n_tokens: int, expert_ids: torch.Tensor, 
     return lib().redlite_moe_layer(_ptr(x), n_tokens, _ptr(expert_ids), _ptr(router_weights), top_k,
                                    ctypes.byref(expert_table),
                                    ctypes.byref(shared_expert) if shared_expert is not None else None, _ptr(out))
+
+
+def redlite_moe_layer_noalloc(x: torch.Tensor, n_tokens: int, expert_ids: torch.Tensor, router_weights: torch.Tensor,
+                              top_k: int, expert_table: redlite_moe_table, shared_expert: Optional[redlite_moe_expert],
+                              out: torch.Tensor) -> int:
+    """The layer without a caller workspace (scratch held by the library)."""
+    return lib().redlite_moe_layer_noalloc(_ptr(x), n_tokens, _ptr(expert_ids), _ptr(router_weights), top_k,
+                                           ctypes.byref(expert_table),
+                                           ctypes.byref(shared_expert) if shared_expert is not None else None,
+                                           _ptr(out))
 
 
 def redlite_moe_upload_experts(hidden: int, ids, host_experts, pool: torch.Tensor, pool_offset: int,
