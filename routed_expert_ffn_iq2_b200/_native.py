@@ -192,7 +192,8 @@ def redlite_moe_upload_experts(hidden: int, ids, host_experts, pool: torch.Tenso
 
 def launches_per_call(n_tokens: int, top_k: int, has_shared: bool, fast: bool = True) -> int:
     """Kernels one redlite_moe_layer call enqueues: the fused decode kernel for
-    decode-sized calls on tiled tables, else bucketing + gate/up + down."""
+    decode-sized calls on tiled tables; otherwise bucketing, then gate/up and
+    down (tensor-core kernels on tiled tables, CUDA-core tiles otherwise)."""
     if n_tokens == 0:
         return 0
     if fast and n_tokens * top_k <= 640 and (not has_shared or n_tokens <= 64):

@@ -104,7 +104,7 @@ int redlite_moe_layer(const float *x, int32_t n_tokens, const int32_t *expert_id
   }
   if (cudaMemsetAsync(out, 0, sizeof(float) * (size_t)n_tokens * t->hidden, s) != cudaSuccess) return REDLITE_ECUDA;
   RouteArgs ra{expert_ids, router_weights, n_tokens, top_k, t->n_experts, t->hidden, t->max_ffn,
-               t->experts, shared != nullptr, ws, L, t->status};
+               t->experts, shared != nullptr, shared ? shared->ffn : 0, shared ? shared->qtype : 0, ws, L, t->status};
   if (launch_route(ra, s) != cudaSuccess) return REDLITE_ECUDA;
   TileArgs ta{};
   ta.x = x;
@@ -117,6 +117,9 @@ int redlite_moe_layer(const float *x, int32_t n_tokens, const int32_t *expert_id
   ta.grids = (const uint8_t *)t->grids;
   ta.ws = ws;
   ta.L = L;
+  ta.status = t->status;
+  if (t->min_ffn >= 256 && tc_supported(t->hidden, t->max_ffn))
+    return launch_tc(ta, s) == cudaSuccess ? REDLITE_OK : REDLITE_ECUDA;
   const int64_t routed = (int64_t)n_tokens * top_k;
   const int max_active = (int)((routed < t->n_experts ? routed : t->n_experts) + (shared ? 1 : 0));
   if (launch_simt_tiles(ta, max_active, s) != cudaSuccess) return REDLITE_ECUDA;

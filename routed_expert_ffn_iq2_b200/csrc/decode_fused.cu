@@ -214,15 +214,21 @@ __device__ __forceinline__ void b_planes(const uint8_t *limbs, int lstride, cons
 // products of the block's rows with token pair p (mma C layout, limb
 // columns).  Lane (q, t) decodes groups 4c + t of rows q and q+8.  All
 // selector and activation loads are issued before the first mma so their
-// latencies overlap.
+// latencies overlap.  Per 8-weight group: two byte extracts, the index bit,
+// two multiply-adds for the table offsets (entry stride 64 bytes = 16
+// replicas), two table loads, one OR, two byte permutes and one shift.
 template <int NP>
 __device__ __forceinline__ void tb_q2(const uint8_t *__restrict__ tb, const uint32_t *__restrict__ sel2,
                                       const uint32_t *__restrict__ sgn2, const uint8_t *const bp[NP], int kbase,
                                       float acc[NP][4]) {
-  const int lane = threadIdx.x & 31, q = lane >> 2, t = lane & 3, r = lane & (kRep2 - 1);
+  static_assert(kRep2 == 16, "table offsets below assume 16 replicas (64-byte entries)");
+  const int lane = threadIdx.x & 31, q = lane >> 2, t = lane & 3;
+  const uint32_t r4 = (uint32_t)(lane & 15) << 2;
+  const uint8_t *g2 = reinterpret_cast<const uint8_t *>(sel2);
+  const uint8_t *gs = reinterpret_cast<const uint8_t *>(sgn2);
   const uint4 qs = *reinterpret_cast<const uint4 *>(tb + 32 * lane);
   const uint4 sg = *reinterpret_cast<const uint4 *>(tb + 32 * lane + 16);
-  const uint32_t qh = *reinterpret_cast<const uint16_t *>(tb + 1024 + 2 * lane);
+  const uint32_t qh14 = (uint32_t)(*reinterpret_cast<const uint16_t *>(tb + 1024 + 2 * lane)) << 14;
   const uint2 scw = *reinterpret_cast<const uint2 *>(tb + 1088 + 8 * q);
   const uint32_t dw = *reinterpret_cast<const uint32_t *>(tb + 1152 + 4 * q);
   const uint32_t qsw[4] = {qs.x, qs.y, qs.z, qs.w};
@@ -230,9 +236,12 @@ __device__ __forceinline__ void tb_q2(const uint8_t *__restrict__ tb, const uint
   uint32_t sel[16];  // field i = 2c + h
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
-    const uint32_t idx = ((qsw[i >> 2] >> (8 * (i & 3))) & 0xFFu) | (((qh >> i) & 1u) << 8);
-    const uint32_t sgb = (sgw[i >> 2] >> (8 * (i & 3))) & 0xFFu;
-    sel[i] = sel2[idx * kRep2 + r] | sgn2[sgb * kRep2 + r];
+    const uint32_t qsb = __byte_perm(qsw[i >> 2], 0u, 0x4440u | (uint32_t)(i & 3));
+    const uint32_t sgb = __byte_perm(sgw[i >> 2], 0u, 0x4440u | (uint32_t)(i & 3));
+    const uint32_t hi = ((qh14 >> i) & 0x4000u) | r4;  // index bit 8, times 64, plus replica
+    const uint32_t go = qsb * 64u + hi;
+    const uint32_t so = sgb * 64u + r4;
+    sel[i] = *reinterpret_cast<const uint32_t *>(g2 + go) | *reinterpret_cast<const uint32_t *>(gs + so);
   }
   uint2 b[NP][8];
 #pragma unroll
@@ -240,6 +249,10 @@ __device__ __forceinline__ void tb_q2(const uint8_t *__restrict__ tb, const uint
 #pragma unroll
     for (int c = 0; c < 8; ++c)
       b[p][c] = bp[p] ? *reinterpret_cast<const uint2 *>(bp[p] + kbase + 32 * c + 8 * t) : make_uint2(0u, 0u);
+  // sub-block multipliers 2sc+1 as bytes: chunk c is byte c >> 1 of the even
+  // (c even) or odd (c odd) nibble word of its row
+  const uint32_t me0 = ((scw.x & 0x0F0F0F0Fu) << 1) | 0x01010101u, mo0 = ((scw.x >> 3) & 0x1E1E1E1Eu) | 0x01010101u;
+  const uint32_t me1 = ((scw.y & 0x0F0F0F0Fu) << 1) | 0x01010101u, mo1 = ((scw.y >> 3) & 0x1E1E1E1Eu) | 0x01010101u;
   int32_t cb[NP][4];
 #pragma unroll
   for (int p = 0; p < NP; ++p) cb[p][0] = cb[p][1] = cb[p][2] = cb[p][3] = 0;
@@ -250,8 +263,8 @@ __device__ __forceinline__ void tb_q2(const uint8_t *__restrict__ tb, const uint
     a[2] = __byte_perm(kQ2Pos, kQ2Neg, sel[2 * c] >> 16);
     a[1] = __byte_perm(kQ2Pos, kQ2Neg, sel[2 * c + 1]);
     a[3] = __byte_perm(kQ2Pos, kQ2Neg, sel[2 * c + 1] >> 16);
-    const int m0 = 2 * (int)((scw.x >> (4 * c)) & 15u) + 1;
-    const int m1 = 2 * (int)((scw.y >> (4 * c)) & 15u) + 1;
+    const int m0 = (int)__byte_perm((c & 1) ? mo0 : me0, 0u, 0x4440u | (uint32_t)(c >> 1));
+    const int m1 = (int)__byte_perm((c & 1) ? mo1 : me1, 0u, 0x4440u | (uint32_t)(c >> 1));
 #pragma unroll
     for (int p = 0; p < NP; ++p) {
       int32_t d[4];
@@ -361,39 +374,40 @@ __device__ __forceinline__ void store_partials(const float acc[NP][4], float *re
   }
 }
 
-// One tile-block of one format for 1-2 (NP = 1) or 3-4 (NP = 2) token
-// positions; the warp's partials go to red (16 x 4 floats).  Kept out of
-// line: one copy of each variant keeps the hot loop inside the
-// instruction cache.
-template <int QT, int NP>
-__device__ __noinline__ void warp_tb(const uint8_t *tb, const uint32_t *sel_a, const uint32_t *sel_b,
-                                     const uint8_t *limbs, int lstride, int kbase, int s0, int s1, int s2, int s3,
-                                     int ntok, float *red) {
-  const int slots[4] = {s0, s1, s2, s3};
-  const uint8_t *bp[NP];
-  b_planes<NP>(limbs, lstride, slots, ntok, bp);
-  float acc[NP][4];
-#pragma unroll
-  for (int p = 0; p < NP; ++p) acc[p][0] = acc[p][1] = acc[p][2] = acc[p][3] = 0.f;
-  if constexpr (QT == kQ2)
-    tb_q2<NP>(tb, sel_a, sel_b, bp, kbase, acc);
-  else
-    tb_q1<NP>(tb, sel_a, bp, kbase, acc);
-  store_partials<NP>(acc, red);
-}
-
+// One tile-block of either format for 1-2 (NP = 1) or 3-4 (NP = 2) token
+// positions; the warp's partials go to red (16 x 4 floats).  Inlined at one
+// call site so the table and stage pointers keep their shared-memory
+// provenance (shared loads, not generic loads).
 __device__ __forceinline__ void warp_tile_block(int qtype, const uint8_t *tb, const Smem &S, const uint8_t *limbs,
                                                 int lstride, int kbase, const int slots[4], int ntok, float *red) {
   if (qtype == kQ2) {
-    if (ntok <= 2)
-      warp_tb<kQ2, 1>(tb, S.sel2, S.sgn2, limbs, lstride, kbase, slots[0], slots[1], slots[2], slots[3], ntok, red);
-    else
-      warp_tb<kQ2, 2>(tb, S.sel2, S.sgn2, limbs, lstride, kbase, slots[0], slots[1], slots[2], slots[3], ntok, red);
+    if (ntok <= 2) {
+      const uint8_t *bp[1];
+      b_planes<1>(limbs, lstride, slots, ntok, bp);
+      float acc[1][4] = {{0.f, 0.f, 0.f, 0.f}};
+      tb_q2<1>(tb, S.sel2, S.sgn2, bp, kbase, acc);
+      store_partials<1>(acc, red);
+    } else {
+      const uint8_t *bp[2];
+      b_planes<2>(limbs, lstride, slots, ntok, bp);
+      float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+      tb_q2<2>(tb, S.sel2, S.sgn2, bp, kbase, acc);
+      store_partials<2>(acc, red);
+    }
   } else {
-    if (ntok <= 2)
-      warp_tb<kQ1, 1>(tb, S.sel1, nullptr, limbs, lstride, kbase, slots[0], slots[1], slots[2], slots[3], ntok, red);
-    else
-      warp_tb<kQ1, 2>(tb, S.sel1, nullptr, limbs, lstride, kbase, slots[0], slots[1], slots[2], slots[3], ntok, red);
+    if (ntok <= 2) {
+      const uint8_t *bp[1];
+      b_planes<1>(limbs, lstride, slots, ntok, bp);
+      float acc[1][4] = {{0.f, 0.f, 0.f, 0.f}};
+      tb_q1<1>(tb, S.sel1, bp, kbase, acc);
+      store_partials<1>(acc, red);
+    } else {
+      const uint8_t *bp[2];
+      b_planes<2>(limbs, lstride, slots, ntok, bp);
+      float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+      tb_q1<2>(tb, S.sel1, bp, kbase, acc);
+      store_partials<2>(acc, red);
+    }
   }
 }
 
@@ -908,26 +922,25 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(FusedArgs a)
         }
       }
       float *red = S.red + (size_t)s * kCWarps * 64;
-      int nw;  // warps holding partials of this item
+      int nw, lst, kb;  // warps holding partials; limb stride and input offset of this warp
       if (inf.phase == 1) {
-        const int nkb = H / 256;  // <= 8: warp w takes input block w
-        nw = nkb;
-#ifdef REDLITE_TRACE
-        const long long c0 = clock64();
-#endif
-        if (warp < nkb)
-          warp_tile_block(qtype, stage + warp * tbb, S, S.limbs, lstrideX, warp * 256, slots, ntok, red + warp * 64);
-#ifdef REDLITE_TRACE
-        if (k < 4 && warp < 4) TRACEC(k * 4 + warp, (uint64_t)(clock64() - c0));
-#endif
+        nw = H / 256;  // <= 8: warp w takes input block w
+        lst = lstrideX;
+        kb = warp * 256;
       } else {
         const int nkb = F / 256, it = item_tiles_of(F);
         const int tiles = min(it, H / 16 - inf.tile * it);
         nw = tiles * nkb;  // <= 8: warp w takes tile w / nkb, input block w % nkb
-        if (warp < nw)
-          warp_tile_block(qtype, stage + warp * tbb, S, S.limbs, F + kLimbPad, (warp % nkb) * 256, slots, ntok,
-                          red + warp * 64);
+        lst = F + kLimbPad;
+        kb = (warp % nkb) * 256;
       }
+#ifdef REDLITE_TRACE
+      const long long c0 = clock64();
+#endif
+      if (warp < nw) warp_tile_block(qtype, stage + warp * tbb, S, S.limbs, lst, kb, slots, ntok, red + warp * 64);
+#ifdef REDLITE_TRACE
+      if (inf.phase == 1 && k < 4 && warp < 4) TRACEC(k * 4 + warp, (uint64_t)(clock64() - c0));
+#endif
       // the last consumer warp to finish reduces the item and frees the stage
       __syncwarp();
       int prev = 0;

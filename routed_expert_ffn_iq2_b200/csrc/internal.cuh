@@ -76,7 +76,11 @@ struct ActiveEntry {
   int expert;      // slot id, or -1 for the shared expert
   int pair_start;  // first pair of this expert in the sorted pair list
   int pair_count;  // tokens routed to it (0: skipped)
-  int tile_base;   // first work ticket of this expert (fused scheduler)
+  int gu_base;     // first gate/up work unit of this expert (tensor-core path)
+  int dn_base;     // first down work unit of this expert (tensor-core path)
+  int ffn;         // expert width
+  int qtype;       // weight format
+  int pad;
 };
 
 struct Pair {
@@ -92,7 +96,11 @@ struct Ctrl {
   int exit_count;      // CTAs that finished (the last one resets)
   int phase1_done;     // CTAs past the gate/up phase (fused decode kernel)
   int phase0_done;     // CTAs past the activation-conversion phase
-  int pad[58];
+  int n_gu_units;      // tensor-core path: gate/up work units
+  int n_dn_units;      // tensor-core path: down work units
+  int ticket_gu;       // next gate/up unit
+  int ticket_dn;       // next down unit
+  int pad[54];
 };
 static_assert(sizeof(Ctrl) == 256, "ctrl block is 256 bytes");
 
@@ -225,6 +233,7 @@ struct RouteArgs {
   int n_tokens, top_k, n_experts, hidden, max_ffn;
   const redlite_moe_expert *experts;
   bool has_shared;
+  int shared_ffn, shared_qtype;
   uint8_t *ws;
   WorkspaceLayout L;
   int32_t *status;
@@ -239,6 +248,7 @@ struct TileArgs {
   const uint8_t *grids;
   uint8_t *ws;
   WorkspaceLayout L;
+  int32_t *status;
 };
 
 constexpr int kRouteMaxExperts = 8192;
@@ -267,6 +277,11 @@ struct FusedArgs {
   int32_t *status;
 };
 bool fused_supported(int hidden, int max_ffn, int n_tokens, int top_k, int n_experts, bool has_shared);
+
+// Tensor-core (tcgen05) grouped path: tokens per work unit, and the launch.
+constexpr int kTcTokens = 256;
+bool tc_supported(int hidden, int max_ffn);
+cudaError_t launch_tc(const TileArgs &a, cudaStream_t stream);
 cudaError_t launch_fused(const FusedArgs &a, cudaStream_t stream);
 
 }  // namespace redlite

@@ -97,7 +97,7 @@ __global__ void __launch_bounds__(1024) route_kernel(RouteArgs a) {
   for (int e = e0; e < e1; ++e) {
     cursor[e] = pair_off;
     if (cnt[e]) {
-      active[act_off] = ActiveEntry{e, pair_off, cnt[e], 0};
+      active[act_off] = ActiveEntry{e, pair_off, cnt[e], 0, 0, 0, 0, 0};
       ++act_off;
     }
     pair_off += cnt[e];
@@ -112,16 +112,47 @@ __global__ void __launch_bounds__(1024) route_kernel(RouteArgs a) {
   int n_active = tot_active, n_pairs = tot_pairs;
   if (a.has_shared) {
     for (int t = threadIdx.x; t < a.n_tokens; t += blockDim.x) pairs[tot_pairs + t] = Pair{t, 1.0f};
-    if (threadIdx.x == 0) active[tot_active] = ActiveEntry{-1, tot_pairs, a.n_tokens, 0};
+    if (threadIdx.x == 0) active[tot_active] = ActiveEntry{-1, tot_pairs, a.n_tokens, 0, 0, 0, 0, 0};
     n_active += 1;
     n_pairs += a.n_tokens;
   }
   if (bad) atomicOr(&s_bad, bad);
   __syncthreads();
-  if (threadIdx.x == 0) {
-    ctrl->n_active = n_active;
-    ctrl->n_pairs = n_pairs;
-    if (s_bad) atomicOr(a.status, s_bad);
+  // work units of the tensor-core path: per expert (width / 128 row tiles) x
+  // (tokens / kTcTokens token tiles) for gate/up, (hidden / 128) x (same) for down
+  {
+    int carry_gu = 0, carry_dn = 0;
+    for (int i0 = 0; i0 < n_active; i0 += blockDim.x) {
+      const int i = i0 + threadIdx.x;
+      int cgu = 0, cdn = 0;
+      if (i < n_active) {
+        ActiveEntry &ae = active[i];
+        const bool sh = ae.expert < 0;
+        ae.ffn = sh ? a.shared_ffn : a.experts[ae.expert].ffn;
+        ae.qtype = sh ? a.shared_qtype : a.experts[ae.expert].qtype;
+        const int nt = (ae.pair_count + kTcTokens - 1) / kTcTokens;
+        cgu = (ae.ffn / 128) * nt;
+        cdn = (a.hidden / 128) * nt;
+      }
+      int tg, td;
+      const int og = block_exclusive_scan(cgu, scan_tmp, &tg);
+      const int od = block_exclusive_scan(cdn, scan_tmp, &td);
+      if (i < n_active) {
+        active[i].gu_base = carry_gu + og;
+        active[i].dn_base = carry_dn + od;
+      }
+      carry_gu += tg;
+      carry_dn += td;
+    }
+    if (threadIdx.x == 0) {
+      ctrl->n_active = n_active;
+      ctrl->n_pairs = n_pairs;
+      ctrl->n_gu_units = carry_gu;
+      ctrl->n_dn_units = carry_dn;
+      ctrl->ticket_gu = 0;
+      ctrl->ticket_dn = 0;
+      if (s_bad) atomicOr(a.status, s_bad);
+    }
   }
 }
 

@@ -198,3 +198,23 @@ def test_general_path_agrees_with_fast_path(P):
     general = _run(L, w.x, w.ids, w.weights)
     assert L.read_status() == 0
     assert _rel_err(fast, general) <= TOL_FP32
+
+
+def test_tensor_core_path_mixed_formats(P, oracle_lib):
+    """128 tokens x top-10 (1280 pairs): the bucketed tcgen05 path, IQ2 and IQ1
+    experts and the shared expert, bf16 operands with fp32 accumulation."""
+    w = fixtures.workload(4)
+    st = fixtures.Stream(991, 2)
+    logits = st.normal(128 * 512).reshape(128, 512)
+    ids, wt = fixtures.softmax_topk_routing(logits, 10)
+    x = fixtures.make_x(991, 128, 2048)
+    sel = sorted(set(ids.reshape(-1).tolist()))
+    L = P.layer_for_workload(w, experts=sel, max_tokens=128)
+    got = _run(L, x, ids, wt)
+    experts = [None] * 512
+    for e in sel:
+        experts[e] = w.expert(e)
+    ref = oracle_lib.moe_layer(x, ids, wt, experts, w.shared(), oracle_lib.expand_grid(1, w.grid_iq2),
+                               oracle_lib.expand_grid(2, w.grid_iq1))
+    assert L.read_status() == 0
+    assert _rel_err(got, ref) <= TOL_BF16
