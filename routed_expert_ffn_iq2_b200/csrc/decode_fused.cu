@@ -151,13 +151,15 @@ __device__ __forceinline__ void mma_k16(int32_t d[4], uint32_t a0, uint32_t a1, 
 // Optional timeline (build with -DREDLITE_TRACE): CTA c writes %globaltimer
 // stamps to the 32 words after the workspace layout's end, slot c * 32 + i.
 #ifdef REDLITE_TRACE
-#define TRACE(i)                                                                  \
-  do {                                                                            \
-    if (threadIdx.x == 0) {                                                       \
-      uint64_t t_;                                                                \
-      asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_));                      \
-      reinterpret_cast<uint64_t *>(a.ws + a.L.total)[blockIdx.x * 32 + (i)] = t_; \
-    }                                                                             \
+#define TRACE(i)                                                                            \
+  do {                                                                                      \
+    if (threadIdx.x == 0) {                                                                 \
+      uint64_t t_;                                                                          \
+      asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_));                                \
+      reinterpret_cast<uint64_t *>(a.ws + a.L.total)[blockIdx.x * 32 + (i)] = t_;           \
+      reinterpret_cast<uint64_t *>(a.ws + a.L.total)[148 * 48 + blockIdx.x * 32 + (i)] =    \
+          (uint64_t)clock64();                                                              \
+    }                                                                                       \
   } while (0)
 #define TRACEC(i, v)                                                                                 \
   do {                                                                                               \
@@ -553,14 +555,13 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(FusedArgs a)
   off += sizeof(float) * kCWarps * 4;
   __shared__ int s_n_inst, s_n1, s_n2, s_bad, s_scan[33];
   TRACE(0);
+  // the next layer call may start its own table setup on SMs this grid frees
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
   // ---- prologue part 1: every independent global load first
   int my_ids[3];
   float my_w[3];
   float4 xv[8];  // activation slots of the (<= 4) tokens when they are converted locally
-  if (tid < kCThreads && local_x)
-    load_slots(T, H, [&](int j, int i4) { return __ldcg(reinterpret_cast<const float4 *>(a.x + (size_t)j * H) + i4); },
-               xv);
   if (tid < kCThreads) {
     // selector tables with replication: thread tid fills words tid + 256 j of
     // each replicated table (consecutive lanes -> consecutive banks); the
@@ -568,12 +569,6 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(FusedArgs a)
     const uint32_t *g2 = reinterpret_cast<const uint32_t *>(a.grids + kGridQ2Sel);
     const uint32_t *gs = reinterpret_cast<const uint32_t *>(a.grids + kGridSign);
     const uint32_t *g1 = reinterpret_cast<const uint32_t *>(a.grids + kGridQ1Sel);
-#pragma unroll
-    for (int j = 0; j < 3; ++j) {
-      const int p = tid + kCThreads * j;
-      my_ids[j] = p < npairs ? __ldg(a.ids + p) : -1;
-      my_w[j] = p < npairs ? __ldg(a.weights + p) : 0.f;
-    }
     auto fill = [&](uint32_t *dst, const uint32_t *src, int words, int rep) {
       for (int j0 = 0; j0 < words; j0 += 16 * kCThreads) {
         uint32_t v[16];
@@ -592,7 +587,22 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(FusedArgs a)
     fill(S.sel2, g2, 512 * kRep2, kRep2);
     fill(S.sgn2, gs, 256 * kRep2, kRep2);
     fill(S.sel1, g1, 4096 * kRep1, kRep1);
-  } else if (lane == 0) {
+    // everything above reads only the expanded grids (set up once, before any
+    // layer call); the call's own inputs may come from the previous kernel
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+#pragma unroll
+    for (int j = 0; j < 3; ++j) {
+      const int p = tid + kCThreads * j;
+      my_ids[j] = p < npairs ? __ldcg(a.ids + p) : -1;
+      my_w[j] = p < npairs ? __ldcg(a.weights + p) : 0.f;
+    }
+    if (local_x)
+      load_slots(T, H, [&](int j, int i4) { return __ldcg(reinterpret_cast<const float4 *>(a.x + (size_t)j * H) + i4); },
+                 xv);
+  } else {
+    asm volatile("griddepcontrol.wait;" ::: "memory");
+  }
+  if (warp == kCWarps && lane == 0) {
     for (int s = 0; s < kRing; ++s) {
       mbar_init(&S.full[s], 1);
       mbar_init(&S.empty[s], 1);
@@ -901,21 +911,23 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(FusedArgs a)
             consumers_sync();
           }
         } else {
-          // h = SiLU(g) * u of each token of the chunk, then its limbs
-          consumers_sync();
+          // h = SiLU(g) * u of the chunk's tokens, then its limbs
+          consumers_sync();  // every warp is done with the previous limbs
           const int lstrideH = F + kLimbPad;
           uint8_t *dst[4];
 #pragma unroll
           for (int j = 0; j < 4; ++j) dst[j] = S.limbs + (size_t)j * 3 * lstrideH;
-          const float *gbase = gu + (size_t)pbase * 2 * a.max_ffn;
-          const int mf = a.max_ffn;
+          const float *grow = gu + (size_t)pbase * 2 * a.max_ffn;
+          const int mf2 = 2 * a.max_ffn, mf = a.max_ffn;
           float4 v[8];
           load_slots(
               ntok, F,
               [&](int j, int i4) {
-                const float4 g = __ldcg(reinterpret_cast<const float4 *>(gbase + (size_t)j * 2 * mf) + i4);
-                const float4 u = __ldcg(reinterpret_cast<const float4 *>(gbase + (size_t)j * 2 * mf + mf) + i4);
-                return make_float4(silu_mul(g.x, u.x), silu_mul(g.y, u.y), silu_mul(g.z, u.z), silu_mul(g.w, u.w));
+                const float *g = grow + (size_t)j * mf2;
+                const float4 gg = __ldcg(reinterpret_cast<const float4 *>(g) + i4);
+                const float4 uu = __ldcg(reinterpret_cast<const float4 *>(g + mf) + i4);
+                return make_float4(silu_mul(gg.x, uu.x), silu_mul(gg.y, uu.y), silu_mul(gg.z, uu.z),
+                                   silu_mul(gg.w, uu.w));
               },
               v);
           block_limbs(ntok, F, v, dst, lstrideH, S.wmax, S.tok_scale);
@@ -968,7 +980,8 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(FusedArgs a)
             float v = 0.f;
             for (int kb = 0; kb < nkb; ++kb) v += red[(tile * nkb + kb) * 64 + row * 4 + j];
             const int r = (inf.tile * it + tile) * 16 + row;
-            atomicAdd(a.out + (size_t)S.pair_tok[pbase + j] * H + r, S.pair_w[pbase + j] * (v * S.tok_scale[j]));
+            atomicAdd(a.out + (size_t)S.pair_tok[pbase + j] * H + r,
+                      S.pair_w[pbase + j] * (v * S.tok_scale[slots[j]]));
           }
         }
         __syncwarp();
@@ -1044,12 +1057,22 @@ cudaError_t launch_fused(const FusedArgs &a, cudaStream_t stream) {
   cfg.blockDim = dim3(kFThreads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = stream;
-  cudaLaunchAttribute attr[1];
+  cudaLaunchAttribute attr[2];
   attr[0].id = cudaLaunchAttributeCooperative;
   attr[0].val.cooperative = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
   cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  return cudaLaunchKernelEx(&cfg, decode_fused_kernel, a);
+  static bool pdl_ok = true;  // dependent launch lets a call's table setup overlap the previous call
+  cfg.numAttrs = pdl_ok ? 2 : 1;
+  e = cudaLaunchKernelEx(&cfg, decode_fused_kernel, a);
+  if (e != cudaSuccess && pdl_ok) {
+    (void)cudaGetLastError();
+    pdl_ok = false;
+    cfg.numAttrs = 1;
+    e = cudaLaunchKernelEx(&cfg, decode_fused_kernel, a);
+  }
+  return e;
 }
 
 }  // namespace redlite
