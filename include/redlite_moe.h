@@ -129,8 +129,10 @@ size_t redlite_moe_matrix_bytes(int32_t qtype, int64_t rows, int64_t k);
 size_t redlite_moe_workspace_bytes(int32_t hidden, int32_t n_experts, int32_t max_tokens, int32_t top_k,
                                    int32_t max_ffn);
 
-/* Zero the workspace's control words (call once after allocating it, and
- * after a call reported REDLITE_STATUS_TIMEOUT).  Enqueued on table->stream. */
+/* Zero the workspace (table->workspace_bytes): its control words and
+ * completion counters.  Call once after allocating it; layer calls leave it
+ * ready for the next call, a call that reported REDLITE_STATUS_TIMEOUT
+ * included.  Enqueued on table->stream. */
 int redlite_moe_workspace_reset(const redlite_moe_table *table);
 
 /* The routed layer ("Red Metal dev8", steps 4-6).

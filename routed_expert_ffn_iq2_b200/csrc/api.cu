@@ -61,8 +61,9 @@ static bool table_ok(const redlite_moe_table *t) {
 
 int redlite_moe_workspace_reset(const redlite_moe_table *t) {
   if (!t || !t->workspace) return REDLITE_EINVAL;
-  return cudaMemsetAsync(t->workspace, 0, sizeof(Ctrl), (cudaStream_t)t->stream) == cudaSuccess ? REDLITE_OK
-                                                                                                 : REDLITE_ECUDA;
+  return cudaMemsetAsync(t->workspace, 0, t->workspace_bytes, (cudaStream_t)t->stream) == cudaSuccess
+             ? REDLITE_OK
+             : REDLITE_ECUDA;
 }
 
 int redlite_moe_layer(const float *x, int32_t n_tokens, const int32_t *expert_ids, const float *router_weights,

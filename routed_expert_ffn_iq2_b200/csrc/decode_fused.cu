@@ -31,6 +31,8 @@
 // accumulation), the sub-block multiplier (2sc+1) is applied in int32 per
 // sub-block and the block scale d in fp32 per 256 weights.  The only
 // rounding is the activations' 2^-21 relative quantisation and fp32 sums.
+#include <stdio.h>
+
 #include "internal.cuh"
 
 namespace redlite {
@@ -46,7 +48,6 @@ constexpr int kTokChunk = 4;
 #endif
 constexpr int kRep2 = REDLITE_REP2;  // replicas of the IQ2 selector/sign tables (bank spread)
 constexpr int kRep1 = 2;   // replicas of the IQ1 selector table
-constexpr int kFusedMaxInst = kFusedMaxPairs + 2;
 constexpr int kLimbPad = 32;  // padding per limb plane (spreads shared-memory banks)
 constexpr uint32_t kSpinLimit = 1u << 24;
 
@@ -166,7 +167,31 @@ __device__ __forceinline__ void mma_k16(int32_t d[4], uint32_t a0, uint32_t a1, 
     if ((threadIdx.x & 31) == 0)                                                                     \
       reinterpret_cast<uint64_t *>(a.ws + a.L.total)[148 * 32 + (blockIdx.x * 16 + (i))] = (v);       \
   } while (0)
+#define TRACE_DECL long long tr_acc_[12] = {0}; long long tr_t_ = 0
+#define TRACE_T0() tr_t_ = clock64()
+#define TRACE_ADD(c, i, j)            \
+  do {                                \
+    const long long d_ = clock64() - tr_t_; \
+    if (c) tr_acc_[i] += d_;          \
+    else tr_acc_[j] += d_;            \
+  } while (0)
+#define TRACE_CNT(c, i, j) \
+  do {                     \
+    if (c) tr_acc_[i] += 1; \
+    else tr_acc_[j] += 1;   \
+  } while (0)
+#define TRACE_FLUSH()                                                                              \
+  do {                                                                                             \
+    if (threadIdx.x == 0)                                                                          \
+      for (int i_ = 0; i_ < 12; ++i_)                                                              \
+        reinterpret_cast<uint64_t *>(a.ws + a.L.total)[148 * 80 + blockIdx.x * 16 + i_] = tr_acc_[i_]; \
+  } while (0)
 #else
+#define TRACE_DECL
+#define TRACE_T0()
+#define TRACE_ADD(c, i, j)
+#define TRACE_CNT(c, i, j)
+#define TRACE_FLUSH()
 #define TRACE(i) \
   do {           \
   } while (0)
@@ -202,13 +227,14 @@ __device__ __forceinline__ void to_limbs(float v, float scale, int &l0, int &l1,
 // and 7 are zero.  Each lane gets, per token pair p, a pointer to the limb
 // plane it reads (nullptr: a zero column).  Limb planes are int8 vectors.
 template <int NP>
-__device__ __forceinline__ void b_planes(const uint8_t *limbs, int lstride, const int slots[4], int ntok,
+__device__ __forceinline__ void b_planes(const uint8_t *limbs, int lstride, int slot4, int ntok,
                                          const uint8_t *bp[NP]) {
   const int n = (threadIdx.x & 31) >> 2;
 #pragma unroll
   for (int p = 0; p < NP; ++p) {
     const int pos = 2 * p + n / 3;
-    bp[p] = (n < 6 && pos < ntok) ? limbs + (size_t)(slots[pos] * 3 + n % 3) * lstride : nullptr;
+    const int slot = (slot4 >> (2 * pos)) & 3;
+    bp[p] = (n < 6 && pos < ntok) ? limbs + (size_t)(slot * 3 + n % 3) * lstride : nullptr;
   }
 }
 
@@ -381,17 +407,17 @@ __device__ __forceinline__ void store_partials(const float acc[NP][4], float *re
 // call site so the table and stage pointers keep their shared-memory
 // provenance (shared loads, not generic loads).
 __device__ __forceinline__ void warp_tile_block(int qtype, const uint8_t *tb, const Smem &S, const uint8_t *limbs,
-                                                int lstride, int kbase, const int slots[4], int ntok, float *red) {
+                                                int lstride, int kbase, int slot4, int ntok, float *red) {
   if (qtype == kQ2) {
     if (ntok <= 2) {
       const uint8_t *bp[1];
-      b_planes<1>(limbs, lstride, slots, ntok, bp);
+      b_planes<1>(limbs, lstride, slot4, ntok, bp);
       float acc[1][4] = {{0.f, 0.f, 0.f, 0.f}};
       tb_q2<1>(tb, S.sel2, S.sgn2, bp, kbase, acc);
       store_partials<1>(acc, red);
     } else {
       const uint8_t *bp[2];
-      b_planes<2>(limbs, lstride, slots, ntok, bp);
+      b_planes<2>(limbs, lstride, slot4, ntok, bp);
       float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
       tb_q2<2>(tb, S.sel2, S.sgn2, bp, kbase, acc);
       store_partials<2>(acc, red);
@@ -399,13 +425,13 @@ __device__ __forceinline__ void warp_tile_block(int qtype, const uint8_t *tb, co
   } else {
     if (ntok <= 2) {
       const uint8_t *bp[1];
-      b_planes<1>(limbs, lstride, slots, ntok, bp);
+      b_planes<1>(limbs, lstride, slot4, ntok, bp);
       float acc[1][4] = {{0.f, 0.f, 0.f, 0.f}};
       tb_q1<1>(tb, S.sel1, bp, kbase, acc);
       store_partials<1>(acc, red);
     } else {
       const uint8_t *bp[2];
-      b_planes<2>(limbs, lstride, slots, ntok, bp);
+      b_planes<2>(limbs, lstride, slot4, ntok, bp);
       float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
       tb_q1<2>(tb, S.sel1, bp, kbase, acc);
       store_partials<2>(acc, red);
@@ -413,78 +439,77 @@ __device__ __forceinline__ void warp_tile_block(int qtype, const uint8_t *tb, co
   }
 }
 
-// Vectors are handled as float4 slots: consumer thread tid owns slot
-// g = tid + kCThreads * i (i < 8) of the concatenation of nvec vectors of
-// n floats (n a multiple of 4, nvec * n / 4 <= 8 * kCThreads).
-template <class Load>
-__device__ __forceinline__ void load_slots(int nvec, int n, Load load, float4 v[8]) {
-  const int per = n / 4, total = nvec * per;
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int g = threadIdx.x + kCThreads * i;
-    if (g < total) v[i] = load(g / per, g % per);
-  }
-}
-
-// Limbs of up to 4 vectors held in slots (see load_slots): vector j's limb
-// planes go to dst[j] + limb * lstride, scale_out[j] = 2^(e_j - 20) with
-// 2^e_j > max |vector j|.  Two consumer-only syncs (partial maxima).
-__device__ __noinline__ void block_limbs(int nvec, int n, const float4 v[8], uint8_t *const dst[4], int lstride,
-                                         float *wmax, float *scale_out) {
+// Limbs of up to 4 vectors of n floats (n a multiple of 4, n <= 2048) read
+// from global memory: vector j's limb planes go to dst + (3 j + limb) *
+// lstride, scale_out[j] = 2^(e_j - 20) with 2^e_j > max |vector j|.  With
+// up_off == 0 vector j is src + j * src_stride; otherwise it is SiLU(g) * u
+// with g = src + j * src_stride and u = g + up_off.  Consumer thread tid
+// holds float4 number tid + kCThreads * i (i < 2) of every vector.  Out of
+// line and compact: it runs a few times per call, and the kernel's hot loop
+// must stay in the instruction cache.  Two consumer-only syncs.
+__device__ __noinline__ void limbs_from_global(int nvec, int n, const float *src, size_t src_stride, int up_off,
+                                               uint8_t *dst, int lstride, float *wmax, float *scale_out) {
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int per = n / 4, total = nvec * per;
-  float m[4] = {0.f, 0.f, 0.f, 0.f};
+  const int per = n / 4;
+  float4 v[4][2];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int g = tid + kCThreads * i;
-    if (g < total) {
-      const float mm = fmaxf(fmaxf(fabsf(v[i].x), fabsf(v[i].y)), fmaxf(fabsf(v[i].z), fabsf(v[i].w)));
-      const int j = g / per;
+  for (int j = 0; j < 4; ++j)
 #pragma unroll
-      for (int jj = 0; jj < 4; ++jj)
-        if (jj == j) m[jj] = fmaxf(m[jj], mm);
+    for (int i = 0; i < 2; ++i) {
+      const int e4 = tid + kCThreads * i;
+      v[j][i] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (j < nvec && e4 < per) {
+        const float *g = src + (size_t)j * src_stride;
+        v[j][i] = __ldcg(reinterpret_cast<const float4 *>(g) + e4);
+        if (up_off) {
+          const float4 u = __ldcg(reinterpret_cast<const float4 *>(g + up_off) + e4);
+          v[j][i] = make_float4(silu_mul_fast(v[j][i].x, u.x), silu_mul_fast(v[j][i].y, u.y),
+                                silu_mul_fast(v[j][i].z, u.z), silu_mul_fast(v[j][i].w, u.w));
+        }
+      }
     }
-  }
 #pragma unroll
-  for (int jj = 0; jj < 4; ++jj) {
+  for (int j = 0; j < 4; ++j) {
+    float m = 0.f;
 #pragma unroll
-    for (int o = 16; o; o >>= 1) m[jj] = fmaxf(m[jj], __shfl_xor_sync(0xffffffffu, m[jj], o));
-    if (lane == 0) wmax[warp * 4 + jj] = m[jj];
+    for (int i = 0; i < 2; ++i)
+      m = fmaxf(m, fmaxf(fmaxf(fabsf(v[j][i].x), fabsf(v[j][i].y)), fmaxf(fabsf(v[j][i].z), fabsf(v[j][i].w))));
+#pragma unroll
+    for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (lane == 0) wmax[warp * 4 + j] = m;
   }
   consumers_sync();
-  float scale[4];
-#pragma unroll
-  for (int jj = 0; jj < 4; ++jj) {
+#pragma unroll 1
+  for (int j = 0; j < nvec; ++j) {
     float mm = 0.f;
 #pragma unroll
-    for (int w = 0; w < kCWarps; ++w) mm = fmaxf(mm, wmax[w * 4 + jj]);
+    for (int w = 0; w < kCWarps; ++w) mm = fmaxf(mm, wmax[w * 4 + j]);
     const int e = pow2_above(mm);
-    scale[jj] = pow2f(20 - e);
-    if (tid == 0 && jj < nvec) scale_out[jj] = pow2f(e - 20);
-  }
+    const float sc = pow2f(20 - e);
+    if (tid == 0) scale_out[j] = pow2f(e - 20);
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    const int g = tid + kCThreads * i;
-    if (g < total) {
-      const int j = g / per, e4 = g % per;
-      float sc = scale[0];
+    for (int i = 0; i < 2; ++i) {
+      const int e4 = tid + kCThreads * i;
+      if (e4 < per) {
+        float4 f = v[0][i];
 #pragma unroll
-      for (int jj = 1; jj < 4; ++jj)
-        if (jj == j) sc = scale[jj];
-      const float f[4] = {v[i].x, v[i].y, v[i].z, v[i].w};
-      uint32_t p0 = 0, p1 = 0, p2 = 0;
+        for (int jj = 1; jj < 4; ++jj)
+          if (jj == j) f = v[jj][i];
+        const float fc[4] = {f.x, f.y, f.z, f.w};
+        uint32_t p0 = 0, p1 = 0, p2 = 0;
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
-        int l0, l1, l2;
-        to_limbs(f[c], sc, l0, l1, l2);
-        p0 |= (uint32_t)(l0 & 0xFF) << (8 * c);
-        p1 |= (uint32_t)(l1 & 0xFF) << (8 * c);
-        p2 |= (uint32_t)(l2 & 0xFF) << (8 * c);
+        for (int c = 0; c < 4; ++c) {
+          int l0, l1, l2;
+          to_limbs(fc[c], sc, l0, l1, l2);
+          p0 |= (uint32_t)(l0 & 0xFF) << (8 * c);
+          p1 |= (uint32_t)(l1 & 0xFF) << (8 * c);
+          p2 |= (uint32_t)(l2 & 0xFF) << (8 * c);
+        }
+        uint8_t *d = dst + (size_t)j * 3 * lstride + 4 * e4;
+        *reinterpret_cast<uint32_t *>(d) = p0;
+        *reinterpret_cast<uint32_t *>(d + lstride) = p1;
+        *reinterpret_cast<uint32_t *>(d + 2 * lstride) = p2;
       }
-      uint8_t *d = dst[j] + 4 * e4;
-      *reinterpret_cast<uint32_t *>(d) = p0;
-      *reinterpret_cast<uint32_t *>(d + lstride) = p1;
-      *reinterpret_cast<uint32_t *>(d + 2 * lstride) = p2;
     }
   }
   consumers_sync();
@@ -558,177 +583,55 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(FusedArgs a)
   // the next layer call may start its own table setup on SMs this grid frees
   asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
 
-  // ---- prologue part 1: every independent global load first
+  // ---- prologue part 1: every independent global load first.  One thread
+  // starts bulk copies of the three selector tables (unreplicated) into the
+  // first bytes of their shared-memory regions; the consumers replicate them
+  // after the routing, while the first weight copies are in flight.
+  __shared__ uint64_t s_lut_bar;
+  if (tid == kCThreads) {
+    for (int s = 0; s < kRing; ++s) {
+      mbar_init(&S.full[s], 1);
+      mbar_init(&S.empty[s], 1);
+      S.done[s] = 0;
+    }
+    mbar_init(&s_lut_bar, 1);
+    mbar_fence_init();
+    s_bad = 0;
+    // the expanded grids are set up once, before any layer call: they may be
+    // read before the previous kernel of the stream has finished
+    mbar_expect_tx(&s_lut_bar, (512 + 256 + 4096) * 4);
+    bulk_g2s(S.sel2, a.grids + kGridQ2Sel, 512 * 4, &s_lut_bar);
+    bulk_g2s(S.sgn2, a.grids + kGridSign, 256 * 4, &s_lut_bar);
+    bulk_g2s(S.sel1, a.grids + kGridQ1Sel, 4096 * 4, &s_lut_bar);
+  }
+  // the call's own inputs may come from the previous kernel
+  asm volatile("griddepcontrol.wait;" ::: "memory");
   int my_ids[3];
   float my_w[3];
-  float4 xv[8];  // activation slots of the (<= 4) tokens when they are converted locally
+  uint4 my_d[3][2];  // slot-table entry of each of this thread's pairs
   if (tid < kCThreads) {
-    // selector tables with replication: thread tid fills words tid + 256 j of
-    // each replicated table (consecutive lanes -> consecutive banks); the
-    // source words are fetched in batches so their latencies overlap
-    const uint32_t *g2 = reinterpret_cast<const uint32_t *>(a.grids + kGridQ2Sel);
-    const uint32_t *gs = reinterpret_cast<const uint32_t *>(a.grids + kGridSign);
-    const uint32_t *g1 = reinterpret_cast<const uint32_t *>(a.grids + kGridQ1Sel);
-    auto fill = [&](uint32_t *dst, const uint32_t *src, int words, int rep) {
-      for (int j0 = 0; j0 < words; j0 += 16 * kCThreads) {
-        uint32_t v[16];
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const int w = j0 + tid + kCThreads * j;
-          v[j] = w < words ? __ldg(src + w / rep) : 0u;
-        }
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const int w = j0 + tid + kCThreads * j;
-          if (w < words) dst[w] = v[j];
-        }
-      }
-    };
-    fill(S.sel2, g2, 512 * kRep2, kRep2);
-    fill(S.sgn2, gs, 256 * kRep2, kRep2);
-    fill(S.sel1, g1, 4096 * kRep1, kRep1);
-    // everything above reads only the expanded grids (set up once, before any
-    // layer call); the call's own inputs may come from the previous kernel
-    asm volatile("griddepcontrol.wait;" ::: "memory");
 #pragma unroll
     for (int j = 0; j < 3; ++j) {
       const int p = tid + kCThreads * j;
       my_ids[j] = p < npairs ? __ldcg(a.ids + p) : -1;
       my_w[j] = p < npairs ? __ldcg(a.weights + p) : 0.f;
     }
-    if (local_x)
-      load_slots(T, H, [&](int j, int i4) { return __ldcg(reinterpret_cast<const float4 *>(a.x + (size_t)j * H) + i4); },
-                 xv);
-  } else {
-    asm volatile("griddepcontrol.wait;" ::: "memory");
-  }
-  if (warp == kCWarps && lane == 0) {
-    for (int s = 0; s < kRing; ++s) {
-      mbar_init(&S.full[s], 1);
-      mbar_init(&S.empty[s], 1);
-      S.done[s] = 0;
+    if (local_x)  // warm L2 for the conversion after the routing
+      for (int i = tid; i < T * H / 32; i += kCThreads) asm volatile("prefetch.global.L2 [%0];" ::"l"(a.x + 32 * i));
+#pragma unroll
+    for (int j = 0; j < 3; ++j) {
+      const int e = my_ids[j];
+      if (e >= 0 && e < E) {
+        const uint4 *d = reinterpret_cast<const uint4 *>(a.experts + e);
+        my_d[j][0] = __ldg(d);
+        my_d[j][1] = __ldg(d + 1);
+      }
     }
-    mbar_fence_init();
-    s_bad = 0;
   }
   TRACE(1);
 
-  // ---- bucketing: counts per expert in the ring (scratch before any copy)
-  int *cnt = reinterpret_cast<int *>(S.ring);  // [E]
-  int *ids_s = cnt + E;                        // [npairs]
-  float *w_s = reinterpret_cast<float *>(ids_s + npairs);
-  for (int e = tid; e < E; e += kFThreads) cnt[e] = 0;
-  __syncthreads();
-  int bad = 0;
-  if (tid < kCThreads) {
-#pragma unroll
-    for (int j = 0; j < 3; ++j) {
-      const int p = tid + kCThreads * j;
-      if (p >= npairs) continue;
-      const int e = my_ids[j];
-      ids_s[p] = e;
-      w_s[p] = my_w[j];
-      if (e < 0 || e >= E) {
-        bad |= REDLITE_STATUS_BAD_ID;
-        continue;
-      }
-      atomicAdd(&cnt[e], 1);
-    }
-  }
-  __syncthreads();
-  // active experts in ascending id: exclusive scans of (count > 0) and counts
-  int n_routed_pairs = 0;
-  {
-    const int per = (E + kCThreads - 1) / kCThreads;
-    const int e0 = tid < kCThreads ? tid * per : E, e1 = min(E, e0 + per);
-    int my_act = 0, my_pairs = 0;
-    for (int e = e0; e < e1; ++e) {
-      my_act += cnt[e] > 0;
-      my_pairs += cnt[e];
-    }
-    int incl_a = my_act, incl_p = my_pairs;
-#pragma unroll
-    for (int o = 1; o < 32; o <<= 1) {
-      const int ya = __shfl_up_sync(0xffffffffu, incl_a, o), yp = __shfl_up_sync(0xffffffffu, incl_p, o);
-      if (lane >= o) incl_a += ya, incl_p += yp;
-    }
-    if (lane == 31 && warp < kCWarps) s_scan[warp] = incl_a, s_scan[16 + warp] = incl_p;
-    __syncthreads();
-    if (tid == 0) {
-      int sa = 0, sp = 0;
-      for (int w = 0; w < kCWarps; ++w) {
-        const int ta = s_scan[w], tp = s_scan[16 + w];
-        s_scan[w] = sa, s_scan[16 + w] = sp;
-        sa += ta, sp += tp;
-      }
-      s_n_inst = sa;
-      s_scan[32] = sp;
-    }
-    __syncthreads();
-    if (tid < kCThreads) {
-      int act = s_scan[warp] + incl_a - my_act, pst = s_scan[16 + warp] + incl_p - my_pairs;
-      for (int e = e0; e < e1; ++e) {
-        if (cnt[e] > 0) {
-          Inst &I = S.inst[act];
-          I.qtype = e;  // expert id for now; descriptor below
-          I.pair_start = pst;
-          I.count = cnt[e];
-          cnt[e] = pst;  // becomes the running cursor of the stable fill
-          ++act;
-          pst += I.count;
-        }
-      }
-    }
-    __syncthreads();
-    n_routed_pairs = s_scan[32];
-  }
-  int n_inst = s_n_inst;
-  if (warp == kCWarps) {
-    // stable fill of the pair list (the producer warp, pairs in index order)
-    for (int p0 = 0; p0 < npairs; p0 += 32) {
-      const int p = p0 + lane;
-      const int e = p < npairs ? ids_s[p] : -1;
-      const bool ok = e >= 0 && e < E;
-      const unsigned m = __match_any_sync(0xffffffffu, ok ? e : -1);
-      if (ok) {
-        const int rank = __popc(m & ((1u << lane) - 1u));
-        const int pos = cnt[e] + rank;
-        S.pair_tok[pos] = p / K;
-        S.pair_w[pos] = w_s[p];
-      }
-      __syncwarp();
-      if (ok && (m & ((1u << lane) - 1u)) == 0) cnt[e] += __popc(m);
-      __syncwarp();
-    }
-  } else {
-    // descriptors (consumer threads, one instance each)
-    for (int u = tid; u < n_inst; u += kCThreads) {
-      Inst &I = S.inst[u];
-      const redlite_moe_expert d = a.experts[I.qtype];
-      if (fused_expert_ok(d, H, a.max_ffn)) {
-        I.gate = (const uint8_t *)d.gate, I.up = (const uint8_t *)d.up, I.down = (const uint8_t *)d.down;
-        I.qtype = d.qtype, I.ffn = d.ffn;
-      } else {
-        bad |= REDLITE_STATUS_BAD_EXPERT;
-        I.gate = I.up = I.down = nullptr;
-        I.qtype = kQ2, I.ffn = 256, I.count = 0;
-      }
-    }
-    if (a.has_shared) {
-      if (tid == 0) {
-        Inst &I = S.inst[n_inst];
-        I.gate = (const uint8_t *)a.shared.gate, I.up = (const uint8_t *)a.shared.up;
-        I.down = (const uint8_t *)a.shared.down, I.qtype = a.shared.qtype, I.ffn = a.shared.ffn;
-        I.pair_start = n_routed_pairs, I.count = T;
-      }
-      for (int t = tid; t < T; t += kCThreads) S.pair_tok[n_routed_pairs + t] = t, S.pair_w[n_routed_pairs + t] = 1.f;
-    }
-  }
-  if (a.has_shared) n_inst += 1;
-  if (bad) atomicOr(&s_bad, bad);
-  __syncthreads();
-  // work items per instance and their prefix sums (one warp; n_inst is small)
-  if (warp == 0) {
+  // work items per instance and their prefix sums (warp 0; n_inst is small)
+  auto item_prefix = [&](int n_inst) {
     int base1 = 0, base2 = 0;
     for (int u0 = 0; u0 < n_inst; u0 += 32) {
       const int u = u0 + lane;
@@ -751,13 +654,193 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(FusedArgs a)
       base2 += __shfl_sync(0xffffffffu, i2, 31);
     }
     if (lane == 0) {
-      s_n1 = base1, s_n2 = base2;
+      s_n_inst = n_inst, s_n1 = base1, s_n2 = base2;
       if (s_bad) atomicOr(a.status, s_bad);
     }
+  };
+  if (npairs <= 32) {
+    // ---- small call: warp 0 routes alone (lane p holds pair p), no block syncs
+    if (warp == 0) {
+      const bool inrange = lane < npairs;
+      const int e = inrange ? my_ids[0] : -1;
+      const bool ok = e >= 0 && e < E;
+      int bad = (inrange && !ok) ? REDLITE_STATUS_BAD_ID : 0;
+      const int key = ok ? e : 0x7fffffff;
+      int rank = 0;          // position of this pair in (expert, pair index) order
+      unsigned less = 0u;    // lanes whose expert id is smaller
+#pragma unroll 4
+      for (int q = 0; q < 32; ++q) {
+        const int kq = __shfl_sync(0xffffffffu, key, q);
+        rank += (kq < key) || (kq == key && q < lane);
+        less |= (unsigned)(kq < key) << q;
+      }
+      const unsigned same = __match_any_sync(0xffffffffu, key), lt = (1u << lane) - 1u;
+      const bool leader = ok && (same & lt) == 0;
+      const unsigned leaders = __ballot_sync(0xffffffffu, leader);
+      if (ok) {
+        S.pair_tok[rank] = lane / K;
+        S.pair_w[rank] = my_w[0];
+      }
+      if (leader) {
+        Inst &I = S.inst[__popc(leaders & less)];
+        redlite_moe_expert d;
+        memcpy(reinterpret_cast<uint8_t *>(&d), &my_d[0][0], 16);
+        memcpy(reinterpret_cast<uint8_t *>(&d) + 16, &my_d[0][1], 16);
+        if (fused_expert_ok(d, H, a.max_ffn)) {
+          I.gate = (const uint8_t *)d.gate, I.up = (const uint8_t *)d.up, I.down = (const uint8_t *)d.down;
+          I.qtype = d.qtype, I.ffn = d.ffn, I.count = __popc(same);
+        } else {
+          bad |= REDLITE_STATUS_BAD_EXPERT;
+          I.gate = I.up = I.down = nullptr;
+          I.qtype = kQ2, I.ffn = 256, I.count = 0;
+        }
+        I.pair_start = rank;
+      }
+      int n_inst = __popc(leaders);
+      const int n_routed_pairs = __popc(__ballot_sync(0xffffffffu, ok));
+      if (a.has_shared) {
+        if (lane == 0) {
+          Inst &I = S.inst[n_inst];
+          I.gate = (const uint8_t *)a.shared.gate, I.up = (const uint8_t *)a.shared.up;
+          I.down = (const uint8_t *)a.shared.down, I.qtype = a.shared.qtype, I.ffn = a.shared.ffn;
+          I.pair_start = n_routed_pairs, I.count = T;
+        }
+        if (lane < T) S.pair_tok[n_routed_pairs + lane] = lane, S.pair_w[n_routed_pairs + lane] = 1.f;
+        n_inst += 1;
+      }
+      bad = __reduce_or_sync(0xffffffffu, bad);
+      if (lane == 0) s_bad = bad;
+      __syncwarp();
+      item_prefix(n_inst);
+    }
+  } else {
+    // ---- bucketing: counts per expert in the ring (scratch before any copy)
+    uint4 *desc_s = reinterpret_cast<uint4 *>(S.ring);  // [npairs][2]: slot-table entries
+    int *cnt = reinterpret_cast<int *>(desc_s + 2 * npairs);  // [E]
+    int *first = cnt + E;                                     // [E]: lowest pair index
+    int *ids_s = first + E;                                   // [npairs]
+    float *w_s = reinterpret_cast<float *>(ids_s + npairs);
+    for (int e = tid; e < E; e += kFThreads) cnt[e] = 0, first[e] = 0x7fffffff;
+    __syncthreads();
+    int bad = 0;
+    if (tid < kCThreads) {
+#pragma unroll
+      for (int j = 0; j < 3; ++j) {
+        const int p = tid + kCThreads * j;
+        if (p >= npairs) continue;
+        const int e = my_ids[j];
+        ids_s[p] = e;
+        w_s[p] = my_w[j];
+        if (e < 0 || e >= E) {
+          bad |= REDLITE_STATUS_BAD_ID;
+          continue;
+        }
+        desc_s[2 * p] = my_d[j][0];
+        desc_s[2 * p + 1] = my_d[j][1];
+        atomicAdd(&cnt[e], 1);
+        atomicMin(&first[e], p);
+      }
+    }
+    __syncthreads();
+    // active experts in ascending id: exclusive scans of (count > 0) and counts
+    int n_routed_pairs = 0;
+    {
+      const int per = (E + kCThreads - 1) / kCThreads;
+      const int e0 = tid < kCThreads ? tid * per : E, e1 = min(E, e0 + per);
+      int my_act = 0, my_pairs = 0;
+      for (int e = e0; e < e1; ++e) {
+        my_act += cnt[e] > 0;
+        my_pairs += cnt[e];
+      }
+      int incl_a = my_act, incl_p = my_pairs;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        const int ya = __shfl_up_sync(0xffffffffu, incl_a, o), yp = __shfl_up_sync(0xffffffffu, incl_p, o);
+        if (lane >= o) incl_a += ya, incl_p += yp;
+      }
+      if (lane == 31 && warp < kCWarps) s_scan[warp] = incl_a, s_scan[16 + warp] = incl_p;
+      __syncthreads();
+      if (tid == 0) {
+        int sa = 0, sp = 0;
+        for (int w = 0; w < kCWarps; ++w) {
+          const int ta = s_scan[w], tp = s_scan[16 + w];
+          s_scan[w] = sa, s_scan[16 + w] = sp;
+          sa += ta, sp += tp;
+        }
+        s_n_inst = sa;
+        s_scan[32] = sp;
+      }
+      __syncthreads();
+      if (tid < kCThreads) {
+        int act = s_scan[warp] + incl_a - my_act, pst = s_scan[16 + warp] + incl_p - my_pairs;
+        for (int e = e0; e < e1; ++e) {
+          if (cnt[e] > 0) {
+            Inst &I = S.inst[act];
+            redlite_moe_expert d;
+            static_assert(sizeof(redlite_moe_expert) == 32, "slot-table entries are two 16-byte words");
+            const uint4 d0 = desc_s[2 * first[e]], d1 = desc_s[2 * first[e] + 1];
+            memcpy(reinterpret_cast<uint8_t *>(&d), &d0, 16);
+            memcpy(reinterpret_cast<uint8_t *>(&d) + 16, &d1, 16);
+            const int c = cnt[e];
+            if (fused_expert_ok(d, H, a.max_ffn)) {
+              I.gate = (const uint8_t *)d.gate, I.up = (const uint8_t *)d.up, I.down = (const uint8_t *)d.down;
+              I.qtype = d.qtype, I.ffn = d.ffn, I.count = c;
+            } else {
+              bad |= REDLITE_STATUS_BAD_EXPERT;
+              I.gate = I.up = I.down = nullptr;
+              I.qtype = kQ2, I.ffn = 256, I.count = 0;
+            }
+            I.pair_start = pst;
+            cnt[e] = pst;  // becomes the running cursor of the stable fill
+            ++act;
+            pst += c;
+          }
+        }
+      }
+      __syncthreads();
+      n_routed_pairs = s_scan[32];
+    }
+    int n_inst = s_n_inst;
+    if (warp == kCWarps) {
+      // stable fill of the pair list (the producer warp, pairs in index order)
+      for (int p0 = 0; p0 < npairs; p0 += 32) {
+        const int p = p0 + lane;
+        const int e = p < npairs ? ids_s[p] : -1;
+        const bool ok = e >= 0 && e < E;
+        const unsigned m = __match_any_sync(0xffffffffu, ok ? e : -1);
+        if (ok) {
+          const int rank = __popc(m & ((1u << lane) - 1u));
+          const int pos = cnt[e] + rank;
+          S.pair_tok[pos] = p / K;
+          S.pair_w[pos] = w_s[p];
+        }
+        __syncwarp();
+        if (ok && (m & ((1u << lane) - 1u)) == 0) cnt[e] += __popc(m);
+        __syncwarp();
+      }
+    } else {
+      if (a.has_shared) {
+        if (tid == 0) {
+          Inst &I = S.inst[n_inst];
+          I.gate = (const uint8_t *)a.shared.gate, I.up = (const uint8_t *)a.shared.up;
+          I.down = (const uint8_t *)a.shared.down, I.qtype = a.shared.qtype, I.ffn = a.shared.ffn;
+          I.pair_start = n_routed_pairs, I.count = T;
+        }
+        for (int t = tid; t < T; t += kCThreads) S.pair_tok[n_routed_pairs + t] = t, S.pair_w[n_routed_pairs + t] = 1.f;
+      }
+    }
+    if (a.has_shared) n_inst += 1;
+    if (bad) atomicOr(&s_bad, bad);
+    __syncthreads();
+    if (warp == 0) item_prefix(n_inst);
   }
+  // the ring's bucketing scratch is overwritten by bulk copies next
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
   __syncthreads();
   TRACE(2);
-  const int N1 = s_n1, N2 = s_n2;
+  const int n_inst = s_n_inst, N1 = s_n1, N2 = s_n2;
+  // gate/up items split evenly over the CTAs; down items in reverse CTA order
+  // (a CTA with one more gate/up item tends to get one fewer down item)
   const int b1 = (int)((int64_t)cta * N1 / G), e1i = (int)((int64_t)(cta + 1) * N1 / G);
   const int rc = G - 1 - cta;
   const int b2 = (int)((int64_t)rc * N2 / G), e2i = (int)((int64_t)(rc + 1) * N2 / G);
@@ -805,23 +888,40 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(FusedArgs a)
       }
     }
   } else {
+    // ---- consumers: replicate the selector tables (word w of a table with
+    // r replicas holds source word w / r; replicas spread lanes over banks)
+    {
+      static_assert(kRep2 == 16 && kRep1 == 2, "replication below assumes 16 / 2 replicas");
+      if (!mbar_wait(&s_lut_bar, 0) && lane == 0) atomicOr(a.status, REDLITE_STATUS_TIMEOUT);
+      TRACE(13);
+      uint32_t v2[2], vs, v1[16];
+#pragma unroll
+      for (int i = 0; i < 2; ++i) v2[i] = S.sel2[tid + kCThreads * i];
+      vs = S.sgn2[tid];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) v1[i] = S.sel1[tid + kCThreads * i];
+      consumers_sync();  // every source word is read before any is overwritten
+      const int rot = lane >> 1;  // lanes of one store wavefront cover distinct banks
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const int q = (r + rot) & 3;
+#pragma unroll
+        for (int i = 0; i < 2; ++i)
+          reinterpret_cast<uint4 *>(S.sel2)[(tid + kCThreads * i) * 4 + q] = make_uint4(v2[i], v2[i], v2[i], v2[i]);
+        reinterpret_cast<uint4 *>(S.sgn2)[tid * 4 + q] = make_uint4(vs, vs, vs, vs);
+      }
+#pragma unroll
+      for (int i = 0; i < 16; ++i) reinterpret_cast<uint2 *>(S.sel1)[tid + kCThreads * i] = make_uint2(v1[i], v1[i]);
+      consumers_sync();
+    }
     // ---- consumers: activations to limbs (locally, or phase 0 cooperative)
     if (local_x) {
-      uint8_t *dst[4];
-#pragma unroll
-      for (int j = 0; j < 4; ++j) dst[j] = S.limbs + (size_t)j * 3 * lstrideX;
       TRACE(12);
-      block_limbs(T, H, xv, dst, lstrideX, S.wmax, S.tok_scale);
+      limbs_from_global(T, H, a.x, (size_t)H, 0, S.limbs, lstrideX, S.wmax, S.tok_scale);
     } else {
-      for (int t = cta; t < T; t += G) {
-        uint8_t *dst[4];
-#pragma unroll
-        for (int j = 0; j < 4; ++j) dst[j] = glimbs + (size_t)t * 3 * lstrideX;
-        float4 v[8];
-        load_slots(1, H, [&](int, int i4) { return __ldcg(reinterpret_cast<const float4 *>(a.x + (size_t)t * H) + i4); },
-                   v);
-        block_limbs(1, H, v, dst, lstrideX, S.wmax, gscale + t);
-      }
+      for (int t = cta; t < T; t += G)
+        limbs_from_global(1, H, a.x + (size_t)t * H, 0, 0, glimbs + (size_t)t * 3 * lstrideX, lstrideX, S.wmax,
+                          gscale + t);
       consumers_sync();
       if (tid == 0) {
         __threadfence();
@@ -843,12 +943,13 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(FusedArgs a)
     // ---- main loop over this CTA's items
     int cur_inst = -1, cur_chunk = -1, cur_phase = 0;
     int ntok = 0;
-    int slots[kTokChunk] = {0, 0, 0, 0};  // limb slot of each token position of the chunk
+    int slot4 = 0xE4;  // limb slot of token position j of the chunk: bits 2j, 2j + 1
+    TRACE_DECL;
     for (int k = 0; k < my_items; ++k) {
       const int s = k % kRing;
       if (k == my1) {
         TRACE(4);
-        // end of phase 1: zero a slice of out, then the grid barrier
+        // end of the gate/up items: zero a slice of out, then the grid barrier
         const size_t total4 = (size_t)T * H / 4;
         const size_t z0 = total4 * cta / G, z1 = total4 * (cta + 1) / G;
         for (size_t i = z0 + tid; i < z1; i += kCThreads)
@@ -870,10 +971,14 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(FusedArgs a)
         consumers_sync();
         TRACE(5);
       }
+      TRACE_T0();
       if (!mbar_wait(&S.full[s], (uint32_t)((k / kRing) & 1))) {
         if (lane == 0) atomicOr(a.status, REDLITE_STATUS_TIMEOUT);
       }
       const ItemInfo inf = S.info[s];
+      TRACE_ADD(inf.phase == 1, 0, 1);
+      TRACE_CNT(inf.phase == 1, 8, 9);
+      TRACE_T0();
       const Inst &I = S.inst[inf.inst];
       const int qtype = I.qtype, F = I.ffn;
       const uint8_t *stage = S.ring + (size_t)s * kStageBytes;
@@ -882,12 +987,13 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(FusedArgs a)
       // (re)load the token chunk's limbs when the instance/chunk/phase changes
       if (inf.inst != cur_inst || inf.chunk != cur_chunk || inf.phase != cur_phase) {
         cur_inst = inf.inst, cur_chunk = inf.chunk, cur_phase = inf.phase;
+        TRACE_CNT(inf.phase == 1, 10, 11);
         ntok = min(kTokChunk, I.count - kTokChunk * inf.chunk);
-#pragma unroll
-        for (int j = 0; j < kTokChunk; ++j) slots[j] = j;
+        slot4 = 0xE4;
         if (inf.phase == 1) {
           if (local_x) {
-            for (int j = 0; j < ntok; ++j) slots[j] = S.pair_tok[pbase + j];  // limbs are indexed by token
+            slot4 = 0;  // limbs are indexed by token
+            for (int j = 0; j < ntok; ++j) slot4 |= S.pair_tok[pbase + j] << (2 * j);
           } else {
             consumers_sync();  // every warp is done with the previous chunk's limbs
             const int nvec = 3 * lstrideX / 16;  // <= 390 for H <= 2048
@@ -913,26 +1019,12 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(FusedArgs a)
         } else {
           // h = SiLU(g) * u of the chunk's tokens, then its limbs
           consumers_sync();  // every warp is done with the previous limbs
-          const int lstrideH = F + kLimbPad;
-          uint8_t *dst[4];
-#pragma unroll
-          for (int j = 0; j < 4; ++j) dst[j] = S.limbs + (size_t)j * 3 * lstrideH;
-          const float *grow = gu + (size_t)pbase * 2 * a.max_ffn;
-          const int mf2 = 2 * a.max_ffn, mf = a.max_ffn;
-          float4 v[8];
-          load_slots(
-              ntok, F,
-              [&](int j, int i4) {
-                const float *g = grow + (size_t)j * mf2;
-                const float4 gg = __ldcg(reinterpret_cast<const float4 *>(g) + i4);
-                const float4 uu = __ldcg(reinterpret_cast<const float4 *>(g + mf) + i4);
-                return make_float4(silu_mul(gg.x, uu.x), silu_mul(gg.y, uu.y), silu_mul(gg.z, uu.z),
-                                   silu_mul(gg.w, uu.w));
-              },
-              v);
-          block_limbs(ntok, F, v, dst, lstrideH, S.wmax, S.tok_scale);
+          limbs_from_global(ntok, F, gu + (size_t)pbase * 2 * a.max_ffn, (size_t)2 * a.max_ffn, a.max_ffn, S.limbs,
+                            F + kLimbPad, S.wmax, S.tok_scale);
         }
       }
+      TRACE_ADD(inf.phase == 1, 2, 3);
+      TRACE_T0();
       float *red = S.red + (size_t)s * kCWarps * 64;
       int nw, lst, kb;  // warps holding partials; limb stride and input offset of this warp
       if (inf.phase == 1) {
@@ -949,10 +1041,12 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(FusedArgs a)
 #ifdef REDLITE_TRACE
       const long long c0 = clock64();
 #endif
-      if (warp < nw) warp_tile_block(qtype, stage + warp * tbb, S, S.limbs, lst, kb, slots, ntok, red + warp * 64);
+      if (warp < nw) warp_tile_block(qtype, stage + warp * tbb, S, S.limbs, lst, kb, slot4, ntok, red + warp * 64);
 #ifdef REDLITE_TRACE
       if (inf.phase == 1 && k < 4 && warp < 4) TRACEC(k * 4 + warp, (uint64_t)(clock64() - c0));
 #endif
+      TRACE_ADD(inf.phase == 1, 4, 5);
+      TRACE_T0();
       // the last consumer warp to finish reduces the item and frees the stage
       __syncwarp();
       int prev = 0;
@@ -968,7 +1062,7 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(FusedArgs a)
             const int row = j2 & 15, j = j2 >> 4;
             float v = 0.f;
             for (int w = 0; w < nw; ++w) v += red[w * 64 + row * 4 + j];
-            const float sc = local_x ? S.tok_scale[slots[j]] : S.tok_scale[j];
+            const float sc = S.tok_scale[(slot4 >> (2 * j)) & 3];
             gu[(size_t)(pbase + j) * 2 * a.max_ffn + (size_t)inf.sub * a.max_ffn + inf.tile * 16 + row] = v * sc;
           }
         } else {
@@ -981,7 +1075,7 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(FusedArgs a)
             for (int kb = 0; kb < nkb; ++kb) v += red[(tile * nkb + kb) * 64 + row * 4 + j];
             const int r = (inf.tile * it + tile) * 16 + row;
             atomicAdd(a.out + (size_t)S.pair_tok[pbase + j] * H + r,
-                      S.pair_w[pbase + j] * (v * S.tok_scale[slots[j]]));
+                      S.pair_w[pbase + j] * (v * S.tok_scale[(slot4 >> (2 * j)) & 3]));
           }
         }
         __syncwarp();
@@ -990,9 +1084,12 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(FusedArgs a)
           mbar_arrive(&S.empty[s]);
         }
       }
+      TRACE_ADD(inf.phase == 1, 6, 7);
     }
+    TRACE(9);
+    TRACE_FLUSH();
     if (my1 == my_items) {
-      // no phase-2 items: still zero the slice and count at the barrier
+      // no down items: still zero the slice and count at the barrier
       const size_t total4 = (size_t)T * H / 4;
       const size_t z0 = total4 * cta / G, z1 = total4 * (cta + 1) / G;
       for (size_t i = z0 + tid; i < z1; i += kCThreads)
@@ -1037,8 +1134,8 @@ bool fused_supported(int hidden, int max_ffn, int n_tokens, int top_k, int n_exp
   if (hidden % 256 || hidden > 2048 || max_ffn % 256 || max_ffn > 2048) return false;
   if ((int64_t)n_tokens * top_k > kFusedMaxPairs) return false;
   if (has_shared && n_tokens > 64) return false;
-  // bucketing scratch (counts, ids, weights) lives in the ring
-  if ((size_t)n_experts * 4 + 8 * (size_t)kFusedMaxPairs > (size_t)kRing * kStageBytes) return false;
+  // bucketing scratch (slot-table entries, counts, first pairs, ids, weights) lives in the ring
+  if ((size_t)n_experts * 8 + 40 * (size_t)kFusedMaxPairs > (size_t)kRing * kStageBytes) return false;
   return fused_smem_bytes(hidden, max_ffn) <= 227 * 1024;
 }
 
@@ -1072,6 +1169,17 @@ cudaError_t launch_fused(const FusedArgs &a, cudaStream_t stream) {
     cfg.numAttrs = 1;
     e = cudaLaunchKernelEx(&cfg, decode_fused_kernel, a);
   }
+#ifdef REDLITE_DEBUG_LAUNCH
+  if (e != cudaSuccess) fprintf(stderr, "decode_fused_kernel launch: %s\n", cudaGetErrorString(e));
+  {
+    cudaFuncAttributes fa{};
+    cudaFuncGetAttributes(&fa, decode_fused_kernel);
+    int nb = -1;
+    cudaOccupancyMaxActiveBlocksPerMultiprocessor(&nb, decode_fused_kernel, kFThreads, smem);
+    fprintf(stderr, "regs %d maxThreads %d static smem %zu dyn %zu blocks/SM %d\n", fa.numRegs,
+            fa.maxThreadsPerBlock, fa.sharedSizeBytes, smem, nb);
+  }
+#endif
   return e;
 }
 

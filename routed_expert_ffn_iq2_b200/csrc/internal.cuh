@@ -94,7 +94,7 @@ struct Ctrl {
   int n_pairs;         // pairs in the sorted list
   int ticket;          // next work ticket
   int exit_count;      // CTAs that finished (the last one resets)
-  int phase1_done;     // CTAs past the gate/up phase (fused decode kernel)
+  int phase1_done;     // CTAs past the gate/up items (fused decode kernel)
   int phase0_done;     // CTAs past the activation-conversion phase
   int n_gu_units;      // tensor-core path: gate/up work units
   int n_dn_units;      // tensor-core path: down work units
@@ -111,6 +111,7 @@ struct WorkspaceLayout {
 
 // Largest (token, slot) pair count the fused decode kernel takes.
 constexpr int kFusedMaxPairs = 640;
+constexpr int kFusedMaxInst = kFusedMaxPairs + 2;  // selected experts + the shared expert, rounded up
 
 inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
@@ -128,7 +129,7 @@ inline WorkspaceLayout workspace_layout(int hidden, int n_experts, int max_token
   off = align256(off + sizeof(Pair) * (size_t)L.max_pairs);
   L.counts = off;
   off = align256(off + sizeof(int) * (size_t)(n_experts + 1));
-  L.done = off;  // per-active-expert completion counters (fused scheduler)
+  L.done = off;  // per-active-expert completion counters (reserved)
   off = align256(off + sizeof(int) * (size_t)L.max_active);
   L.h = off;
   off = align256(off + sizeof(float) * (size_t)L.max_pairs * (size_t)max_ffn);
@@ -218,6 +219,8 @@ __device__ __forceinline__ void decode_group_f32(const uint8_t *__restrict__ mat
 }
 
 __device__ __forceinline__ float silu_mul(float g, float u) { return g / (1.0f + __expf(-g)) * u; }
+// Same with the approximate divide (2 ulp; 0 once 1 + e^-g exceeds 2^126).
+__device__ __forceinline__ float silu_mul_fast(float g, float u) { return __fdividef(g, 1.0f + __expf(-g)) * u; }
 
 __device__ __forceinline__ float warp_sum(float v) {
 #pragma unroll
