@@ -11,6 +11,17 @@ namespace redlite {
 
 // One thread per (format, entry): writes the int8 values, the bf16 copies
 // the tensor-core path reads, and keeps the compact entry.
+// Byte-permute selectors that build weights 2w, 2w+1 of a grid entry (compact
+// 2-bit symbols c) as bf16 pairs from a table of three bf16 values.
+__device__ uint64_t bf16_pair_selectors(uint16_t c) {
+  uint64_t sel = 0;
+  for (int j = 0; j < 8; ++j) {
+    const uint64_t s = (c >> (2 * j)) & 3;
+    sel |= ((2 * s) | ((2 * s + 1) << 4)) << (8 * j);
+  }
+  return sel;
+}
+
 __global__ void expand_grids_kernel(const uint16_t *__restrict__ comp2, const uint16_t *__restrict__ comp1,
                                     uint8_t *__restrict__ grids) {
   const int t = blockIdx.x * blockDim.x + threadIdx.x;
@@ -29,6 +40,7 @@ __global__ void expand_grids_kernel(const uint16_t *__restrict__ comp2, const ui
     uint32_t sel = 0;
     for (int j = 0; j < 8; ++j) sel |= (uint32_t)((c >> (2 * j)) & 3) << (4 * j);
     reinterpret_cast<uint32_t *>(grids + kGridQ2Sel)[t] = sel;
+    reinterpret_cast<uint64_t *>(grids + kGridQ2Bsel)[t] = bf16_pair_selectors(c);
     if (t < 256) {
       uint32_t sg = 0;
       for (int j = 0; j < 8; ++j) sg |= (uint32_t)((t >> j) & 1) << (4 * j + 2);
@@ -52,6 +64,7 @@ __global__ void expand_grids_kernel(const uint16_t *__restrict__ comp2, const ui
     uint32_t sel = 0;
     for (int j = 0; j < 8; ++j) sel |= (uint32_t)((c >> (2 * j)) & 3) << (4 * j);
     reinterpret_cast<uint32_t *>(grids + kGridQ1Sel)[e] = sel;
+    reinterpret_cast<uint64_t *>(grids + kGridQ1Bsel)[e] = bf16_pair_selectors(c);
     reinterpret_cast<uint32_t *>(grids + kGridQ1Sel)[e + 2048] = sel | 0x44444444u;
   }
 }

@@ -6,176 +6,283 @@
 // every expert's gate/up and down projections run as dense contractions on
 // the 5th-generation tensor cores (tcgen05.mma, bf16 operands in shared
 // memory, fp32 accumulators in tensor memory).  Weights are decoded from the
-// packed blocks straight into 128-byte-swizzled bf16 tiles (each value is
-// exact in fp32; bf16 rounds it to nearest even); activations are rounded to
-// bf16 the same way.  Accumulation is fp32.
+// packed tile-blocks into 128-byte-swizzled bf16 tiles (each weight is exact
+// in fp32 and rounded to bf16, nearest even); activations are rounded to bf16
+// the same way.  Accumulation is fp32.
 //
-// Work unit (persistent CTAs, atomic tickets):
-//   gate/up  expert e, 128 output rows of gate and of up, up to 256 tokens:
-//            D_gate, D_up in TMEM [128 x N]; epilogue h = SiLU(g) * u (bf16)
-//            to the workspace, one row per (token, expert) pair;
-//   down     expert e, 128 output rows of down, up to 256 tokens: D in TMEM;
-//            epilogue out[token] += weight * D with fp32 atomics.
-// Inputs along K arrive in 64-wide chunks through two shared-memory stages:
-// all threads fill one stage while the tensor cores consume the other.
+// Work unit: (expert, 128 output rows, up to 128 of the expert's tokens).
+//   gate/up  A = the rows of gate and of up, B = the tokens' activations;
+//            D_gate, D_up in TMEM; epilogue h = SiLU(g) * u (bf16) per pair;
+//   down     A = the rows of down, B = the pairs' h; epilogue out += w * D
+//            with fp32 atomics.
+// One persistent CTA per SM takes units cta, cta + grid, ...; its warps:
+//   warp 0      one thread bulk-copies the packed tile-blocks of each
+//               256-input column of a unit (8 per matrix) into a 2-deep ring;
+//   warp 1      one thread issues the tcgen05.mma of every 64-input step and
+//               commits them to the step's slot and, per unit, to one of two
+//               accumulator buffers;
+//   warps 2-9   dequant warp w decodes tile-block w (rows 16w..16w+15) of
+//               each matrix into the A tiles of a 3-4 deep ring of steps and
+//               fetches rows 16w..16w+15 of B with cp.async;
+//   warps 10-13 the epilogue (TMEM -> registers -> h or out), overlapping
+//               the next unit's contraction.
 #include "internal.cuh"
+#include "layout.cuh"
 #include "ptx.cuh"
 
 namespace redlite {
+namespace {
 
-constexpr int kTcThreads = 256;
-constexpr int kKc = 64;                        // K chunk: one 128-byte swizzle row of bf16
-constexpr int kTileA = 128 * kKc * 2;          // 16 KB: 128 rows x 64 bf16
-constexpr int kTileB = kTcTokens * kKc * 2;    // 32 KB: 256 tokens x 64 bf16
+constexpr int kDqWarps = 8;
+constexpr int kEpWarps = 4;
+constexpr int kTcWarps = 2 + kDqWarps + kEpWarps;
+constexpr int kTcThreads = 32 * kTcWarps;  // 448
+constexpr int kTile = 128 * 64 * 2;        // 16 KB: 128 rows x 64 bf16
+constexpr int kPr = 2;                     // packed columns in flight
+constexpr int kMaxUnits = 128;             // unit records per pass
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kWaitLimit = 1u << 26;
 
-struct TcSmem {
-  uint8_t *stage[2];  // gate/up: A_gate | A_up | B ; down: A | B
-  int8_t *g2, *g1;    // expanded grids (int8)
-  int *tok;           // tokens of the current unit
-  float *wt;          // their router weights (down)
-  uint64_t *mma_done; // [2]
+template <bool DOWN>
+struct Cfg {
+  static constexpr int kMats = DOWN ? 1 : 2;
+  static constexpr int kAr = DOWN ? 4 : 3;                  // 64-input steps in flight
+  static constexpr int kStep = (kMats + 1) * kTile;         // A tiles, then the B tile
+  static constexpr int kPacked = kMats * 8 * kQ2TileBlock;  // one column, largest format
+  static constexpr uint32_t kBufCols = DOWN ? 128 : 256;    // TMEM columns per accumulator buffer
+};
+
+struct Unit {
+  const uint8_t *mat0, *mat1;  // gate, up (or down, unused)
+  int qtype, K, rt, p0, n_real, n_pad, pad0, pad1;
+};
+static_assert(sizeof(Unit) == 48, "unit records are 48 bytes");
+
+struct Bars {
+  uint64_t pfull[kPr], pempty[kPr], afull[4], aempty[4], accfull[2], accempty[2];
+};
+
+struct Smem {
+  uint8_t *ring, *packed;
+  const uint2 *sel2, *sel1;
+  Unit *units;
+  Bars *bars;
   uint32_t *taddr;
-  int *unit;
 };
 
-__device__ __forceinline__ uint32_t bf16x2_bits(float lo, float hi) {
-  __nv_bfloat162 b = __floats2bfloat162_rn(lo, hi);
-  return *reinterpret_cast<uint32_t *>(&b);
+template <bool DOWN>
+constexpr size_t smem_bytes() {
+  return 1024 + (size_t)Cfg<DOWN>::kAr * Cfg<DOWN>::kStep + (size_t)kPr * Cfg<DOWN>::kPacked + 512 * 8 + 2048 * 8 +
+         sizeof(Unit) * kMaxUnits + sizeof(Bars) + 16;
 }
 
-// 8 weights of group G of a resident matrix -> 8 bf16 (exact fp32 values
-// rounded to nearest even), read with the grid from shared memory.
-template <int QT>
-__device__ __forceinline__ uint4 group_bf16(const uint8_t *mat, int64_t k, int64_t G, const int8_t *grid) {
-  float w[8];
-  decode_group_f32<QT>(mat, k, true, G, grid, w);
-  return make_uint4(bf16x2_bits(w[0], w[1]), bf16x2_bits(w[2], w[3]), bf16x2_bits(w[4], w[5]),
-                    bf16x2_bits(w[6], w[7]));
+template <bool DOWN>
+__device__ __forceinline__ Smem carve(uint8_t *smem) {
+  Smem S;
+  uint8_t *p = reinterpret_cast<uint8_t *>(((uintptr_t)smem + 1023) & ~(uintptr_t)1023);  // swizzled tiles
+  S.ring = p;
+  p += (size_t)Cfg<DOWN>::kAr * Cfg<DOWN>::kStep;
+  S.packed = p;
+  p += (size_t)kPr * Cfg<DOWN>::kPacked;
+  S.sel2 = reinterpret_cast<const uint2 *>(p);
+  p += 512 * 8;
+  S.sel1 = reinterpret_cast<const uint2 *>(p);
+  p += 2048 * 8;
+  S.units = reinterpret_cast<Unit *>(p);
+  p += sizeof(Unit) * kMaxUnits;
+  S.bars = reinterpret_cast<Bars *>(p);
+  p += sizeof(Bars);
+  S.taddr = reinterpret_cast<uint32_t *>(p);
+  return S;
 }
 
-// Decode rows [row0, row0+128) x inputs [k0, k0+64) of a matrix with k inputs
-// into a swizzled bf16 tile (all threads; 1024 groups, 4 per thread).
-template <int QT>
-__device__ __forceinline__ void fill_weights(uint8_t *tile, const uint8_t *mat, int64_t k, int row0, int k0,
-                                             const int8_t *grid) {
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int g = threadIdx.x + kTcThreads * i;  // 0..1023
-    const int r = g >> 3, c8 = g & 7;
-    const int64_t G = ((int64_t)(row0 + r) * k + k0 + 8 * c8) >> 3;
-    *reinterpret_cast<uint4 *>(tile + ptx::sw128_offset(r, 8 * c8)) = group_bf16<QT>(mat, k, G, grid);
-  }
-}
-
-__device__ __forceinline__ void fill_weights_any(int qtype, uint8_t *tile, const uint8_t *mat, int64_t k, int row0,
-                                                 int k0, const TcSmem &S) {
-  if (qtype == kQ2)
-    fill_weights<kQ2>(tile, mat, k, row0, k0, S.g2);
-  else
-    fill_weights<kQ1>(tile, mat, k, row0, k0, S.g1);
-}
-
-// Token rows of B from fp32 activations (bf16-rounded); rows >= n_real are zero.
-__device__ __forceinline__ void fill_tokens_f32(uint8_t *tile, const float *x, int64_t hidden, int k0, int n_real,
-                                                int n_pad, const int *tok) {
-  for (int g = threadIdx.x; g < n_pad * 8; g += kTcThreads) {
-    const int j = g >> 3, c8 = g & 7;
-    uint4 v = make_uint4(0u, 0u, 0u, 0u);
-    if (j < n_real) {
-      const float4 *src = reinterpret_cast<const float4 *>(x + (size_t)tok[j] * hidden + k0 + 8 * c8);
-      const float4 a = __ldg(src), b = __ldg(src + 1);
-      v = make_uint4(bf16x2_bits(a.x, a.y), bf16x2_bits(a.z, a.w), bf16x2_bits(b.x, b.y), bf16x2_bits(b.z, b.w));
-    }
-    *reinterpret_cast<uint4 *>(tile + ptx::sw128_offset(j, 8 * c8)) = v;
-  }
-}
-
-// Token rows of B from bf16 rows of h (row stride ld elements); rows >= n_real zero.
-__device__ __forceinline__ void fill_tokens_bf16(uint8_t *tile, const __nv_bfloat16 *h, int64_t ld, int64_t row0,
-                                                 int k0, int n_real, int n_pad) {
-  for (int g = threadIdx.x; g < n_pad * 8; g += kTcThreads) {
-    const int j = g >> 3, c8 = g & 7;
-    uint4 v = make_uint4(0u, 0u, 0u, 0u);
-    if (j < n_real) v = __ldcg(reinterpret_cast<const uint4 *>(h + (row0 + j) * ld + k0 + 8 * c8));
-    *reinterpret_cast<uint4 *>(tile + ptx::sw128_offset(j, 8 * c8)) = v;
-  }
-}
-
-struct UnitInfo {
-  int inst, rt, n_real, n_pad, p0;
-};
-
-// Locate work unit j of one phase: the last active entry whose base <= j.
-__device__ __forceinline__ UnitInfo find_unit(const ActiveEntry *act, int n_active, int j, bool down, int hidden) {
+// Work unit j of a phase: the last active entry whose first unit is <= j.
+__device__ Unit make_unit(const TileArgs &a, const ActiveEntry *act, int n_active, int j, bool down) {
   int lo = 0, hi = n_active - 1;
   while (lo < hi) {
     const int mid = (lo + hi + 1) >> 1;
     if ((down ? act[mid].dn_base : act[mid].gu_base) <= j) lo = mid; else hi = mid - 1;
   }
-  const ActiveEntry &e = act[lo];
-  const int nrt = (down ? hidden : e.ffn) / 128;
+  const ActiveEntry e = act[lo];
+  const redlite_moe_expert ex = e.expert >= 0 ? a.experts[e.expert] : a.shared;
+  const int nrt = (down ? a.hidden : e.ffn) / 128;
   const int loc = j - (down ? e.dn_base : e.gu_base);
-  UnitInfo u;
-  u.inst = lo;
-  u.rt = loc % nrt;
   const int tt = loc / nrt;
+  Unit u;
+  u.mat0 = (const uint8_t *)(down ? ex.down : ex.gate);
+  u.mat1 = (const uint8_t *)(down ? nullptr : ex.up);
+  u.qtype = e.qtype;
+  u.K = down ? e.ffn : a.hidden;
+  u.rt = loc % nrt;
   u.p0 = e.pair_start + kTcTokens * tt;
   u.n_real = min(kTcTokens, e.pair_count - kTcTokens * tt);
   u.n_pad = (u.n_real + 15) & ~15;
+  u.pad0 = u.pad1 = 0;
   return u;
 }
 
-__device__ __forceinline__ void carve(uint8_t *smem, TcSmem &S, int stage_bytes) {
-  uintptr_t base = ((uintptr_t)smem + 1023) & ~(uintptr_t)1023;  // swizzled tiles need 1024-byte alignment
-  uint8_t *p = reinterpret_cast<uint8_t *>(base);
-  S.stage[0] = p;
-  S.stage[1] = p + stage_bytes;
-  p += 2 * stage_bytes;
-  S.g2 = reinterpret_cast<int8_t *>(p);
-  p += 512 * 8;
-  S.g1 = reinterpret_cast<int8_t *>(p);
-  p += 2048 * 8;
-  S.tok = reinterpret_cast<int *>(p);
-  p += sizeof(int) * kTcTokens;
-  S.wt = reinterpret_cast<float *>(p);
-  p += sizeof(float) * kTcTokens;
-  S.mma_done = reinterpret_cast<uint64_t *>(p);
-  p += 2 * sizeof(uint64_t);
-  S.taddr = reinterpret_cast<uint32_t *>(p);
-  p += 16;
-  S.unit = reinterpret_cast<int *>(p);
+__device__ __forceinline__ uint32_t bf16x2(float lo, float hi) {
+  uint32_t r;
+  asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
+  return r;
 }
 
-__device__ __forceinline__ const redlite_moe_expert expert_desc(const TileArgs &a, const ActiveEntry &e) {
-  return e.expert >= 0 ? a.experts[e.expert] : a.shared;
+__device__ __forceinline__ void cp_async16(void *dst, const void *src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(ptx::smem_u32(dst)), "l"(src) : "memory");
 }
 
-// One tensor-core kernel for both phases (DOWN selects the down projection).
+// --------------------------------------------------------------- dequant
+//
+// A lane builds the bf16 values of one (row, sub-block) as a table of three
+// entries (the scaled grid values of symbols 0, 1, 2) in two registers; the
+// byte-permute selectors of the weights' grid entry then pick a bf16 pair
+// per instruction.  IQ2_XS-style signs are flipped with one XOR per pair.
+
+// IQ2_XS-style tile-block fields of lane (q, t) (the resident layout's lane
+// order: rows q and q+8, groups 4c + t, field i = 2c + h).
+struct Q2Lane {
+  uint32_t qs[4], sg[4], qh, sc0, sc1;
+  float d0, d1;  // d / 8 of rows q and q+8
+};
+
+__device__ __forceinline__ Q2Lane load_q2(const uint8_t *tb, int lane) {
+  Q2Lane r;
+  const uint4 qs = *reinterpret_cast<const uint4 *>(tb + 32 * lane);
+  const uint4 sg = *reinterpret_cast<const uint4 *>(tb + 32 * lane + 16);
+  r.qs[0] = qs.x, r.qs[1] = qs.y, r.qs[2] = qs.z, r.qs[3] = qs.w;
+  r.sg[0] = sg.x, r.sg[1] = sg.y, r.sg[2] = sg.z, r.sg[3] = sg.w;
+  r.qh = *reinterpret_cast<const uint16_t *>(tb + 1024 + 2 * lane);
+  const int q = lane >> 2;
+  const uint2 sc = *reinterpret_cast<const uint2 *>(tb + 1088 + 8 * q);
+  r.sc0 = sc.x, r.sc1 = sc.y;
+  const uint32_t dw = *reinterpret_cast<const uint32_t *>(tb + 1152 + 4 * q);
+  r.d0 = __half2float(__ushort_as_half((unsigned short)(dw & 0xFFFFu))) * 0.125f;
+  r.d1 = __half2float(__ushort_as_half((unsigned short)(dw >> 16))) * 0.125f;
+  return r;
+}
+
+// Step s (inputs 64s..64s+63 of the column) of one IQ2 tile-block into rows
+// row0..row0+15 of the swizzled A tile: fields i = 4s + 2 c2 + h.
+__device__ __forceinline__ void dequant_q2(const Q2Lane &L, int s, uint8_t *A, int row0, const uint2 *sel2,
+                                           int lane) {
+  const int q = lane >> 2, t = lane & 3;
+  const uint32_t qw = s == 0 ? L.qs[0] : s == 1 ? L.qs[1] : s == 2 ? L.qs[2] : L.qs[3];
+  const uint32_t sw = s == 0 ? L.sg[0] : s == 1 ? L.sg[1] : s == 2 ? L.sg[2] : L.sg[3];
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    const int c2 = j ^ (q & 1);  // odd rows take the other half first: conflict-free stores
+    const int c = 2 * s + c2;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int f = 2 * c2 + h;
+      const uint32_t qsb = (qw >> (8 * f)) & 0xFFu, sgb = (sw >> (8 * f)) & 0xFFu;
+      const uint32_t idx = qsb | (((L.qh >> (4 * s + f)) & 1u) << 8);
+      const uint2 sel = sel2[idx];
+      const uint32_t nib = ((h ? L.sc1 : L.sc0) >> (4 * c)) & 15u;
+      const float sc = (h ? L.d1 : L.d0) * (float)(2 * nib + 1);
+      const uint32_t t0 = bf16x2(sc * 8.f, sc * 25.f), t1 = bf16x2(sc * 43.f, 0.f);
+      // sign bits 2w, 2w+1 -> bit 15, 31 of pair w: (b * (2^15 + 2^30)) & 0x80008000
+      uint4 v;
+      v.x = __byte_perm(t0, t1, sel.x) ^ ((sgb * 0x40008000u) & 0x80008000u);
+      v.y = __byte_perm(t0, t1, sel.x >> 16) ^ (((sgb >> 2) * 0x40008000u) & 0x80008000u);
+      v.z = __byte_perm(t0, t1, sel.y) ^ (((sgb >> 4) * 0x40008000u) & 0x80008000u);
+      v.w = __byte_perm(t0, t1, sel.y >> 16) ^ (((sgb >> 6) * 0x40008000u) & 0x80008000u);
+      *reinterpret_cast<uint4 *>(A + ptx::sw128_offset(row0 + q + 8 * h, 32 * c2 + 8 * t)) = v;
+    }
+  }
+}
+
+// IQ1_M-style tile-block fields of lane (q, t): pair p = t >> 1 (groups
+// 2 sb + p of rows q and q+8, field i = 2 sb + h); half = t & 1 takes
+// sub-blocks 4S + 2 half + {0, 1} of step S.
+struct Q1Lane {
+  uint32_t qs[4], nb[4];
+  uint64_t row0, row1;  // 16 x 3-bit sub-block scales of rows q and q+8
+  float d0, d1;
+};
+
+__device__ __forceinline__ Q1Lane load_q1(const uint8_t *tb, int lane) {
+  Q1Lane r;
+  const int q = lane >> 2, p = (lane >> 1) & 1, half = lane & 1;
+  const uint8_t *pb = tb + 48 * (2 * q + p);
+  const uint4 qa = *reinterpret_cast<const uint4 *>(pb), qb = *reinterpret_cast<const uint4 *>(pb + 16);
+  const uint4 nb = *reinterpret_cast<const uint4 *>(pb + 32);
+  // qs word 2S + half holds fields 8S + 4 half .. + 3 of step S
+  r.qs[0] = half ? qa.y : qa.x;
+  r.qs[1] = half ? qa.w : qa.z;
+  r.qs[2] = half ? qb.y : qb.x;
+  r.qs[3] = half ? qb.w : qb.z;
+  r.nb[0] = nb.x, r.nb[1] = nb.y, r.nb[2] = nb.z, r.nb[3] = nb.w;
+  const uint32_t *scp = reinterpret_cast<const uint32_t *>(tb + 768 + 12 * q);
+  const uint32_t s0 = scp[0], s1 = scp[1], s2 = scp[2];
+  r.row0 = (uint64_t)s0 | ((uint64_t)(s1 & 0xFFFFu) << 32);
+  r.row1 = (uint64_t)(s1 >> 16) | ((uint64_t)s2 << 16);
+  const uint32_t dw = *reinterpret_cast<const uint32_t *>(tb + 864 + 4 * q);
+  r.d0 = __half2float(__ushort_as_half((unsigned short)(dw & 0xFFFFu)));
+  r.d1 = __half2float(__ushort_as_half((unsigned short)(dw >> 16)));
+  return r;
+}
+
+__device__ __forceinline__ void dequant_q1(const Q1Lane &L, int S, uint8_t *A, int row0, const uint2 *sel1,
+                                           int lane) {
+  const int q = lane >> 2, p = (lane >> 1) & 1, half = lane & 1;
+  const uint32_t qw = S == 0 ? L.qs[0] : S == 1 ? L.qs[1] : S == 2 ? L.qs[2] : L.qs[3];
+  const uint32_t nw = S == 0 ? L.nb[0] : S == 1 ? L.nb[1] : S == 2 ? L.nb[2] : L.nb[3];
+  const uint32_t nb16 = half ? (nw >> 16) : (nw & 0xFFFFu);
+#pragma unroll
+  for (int j = 0; j < 2; ++j) {
+    const int s2 = j ^ (q & 1);            // odd rows take the other sub-block first: conflict-free stores
+    const int sb = 4 * S + 2 * half + s2;  // sub-block of 16 inputs within the column
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int f = 2 * s2 + h;
+      const uint32_t qsb = (qw >> (8 * f)) & 0xFFu;
+      const uint32_t nib = (nb16 >> (4 * f)) & 15u;
+      const uint2 sel = sel1[qsb | ((nib & 7u) << 8)];
+      const uint32_t sc3 = (uint32_t)(((h ? L.row1 : L.row0) >> (3 * sb)) & 7u);
+      const float sc = (h ? L.d1 : L.d0) * (float)(2 * sc3 + 1);
+      const float dl = (nib & 8u) ? -0.125f : 0.125f;
+      const uint32_t t0 = bf16x2(sc * (dl - 1.f), sc * dl), t1 = bf16x2(sc * (dl + 1.f), 0.f);
+      uint4 v;
+      v.x = __byte_perm(t0, t1, sel.x);
+      v.y = __byte_perm(t0, t1, sel.x >> 16);
+      v.z = __byte_perm(t0, t1, sel.y);
+      v.w = __byte_perm(t0, t1, sel.y >> 16);
+      *reinterpret_cast<uint4 *>(A + ptx::sw128_offset(row0 + q + 8 * h, 16 * (2 * half + s2) + 8 * p)) = v;
+    }
+  }
+}
+
+// --------------------------------------------------------------- the kernel
+
 template <bool DOWN>
-__global__ void __launch_bounds__(kTcThreads, 1) grouped_tc_kernel(TileArgs a) {
+__global__ void __maxnreg__(128) grouped_tc_kernel(TileArgs a) {
+  using C = Cfg<DOWN>;
   extern __shared__ uint8_t smem[];
-  constexpr int kStageBytes = (DOWN ? 1 : 2) * kTileA + kTileB;
-  constexpr uint32_t kCols = DOWN ? 256 : 512;  // TMEM columns: D (and D_up at +256)
-  TcSmem S;
-  carve(smem, S, kStageBytes);
+  const Smem S = carve<DOWN>(smem);
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int G = gridDim.x, cta = blockIdx.x;
   const int H = a.hidden;
   Ctrl *ctrl = reinterpret_cast<Ctrl *>(a.ws + a.L.ctrl);
   const ActiveEntry *act = reinterpret_cast<const ActiveEntry *>(a.ws + a.L.active);
   const Pair *pairs = reinterpret_cast<const Pair *>(a.ws + a.L.pairs);
   __nv_bfloat16 *hbuf = reinterpret_cast<__nv_bfloat16 *>(a.ws + a.L.h);
+  const __nv_bfloat16 *xb = reinterpret_cast<const __nv_bfloat16 *>(a.ws + a.L.xb);
+  Bars &B = *S.bars;
 
-  // expanded grids into shared memory
-  for (int i = tid; i < (512 * 8 + 2048 * 8) / 16; i += kTcThreads)
-    reinterpret_cast<uint4 *>(S.g2)[i] = __ldg(reinterpret_cast<const uint4 *>(a.grids + kGridQ2Vals) + i);
-  if (warp == 0) {
-    ptx::tmem_alloc(S.taddr, kCols);
-    ptx::tmem_relinquish();
-  }
+  // selector tables, barriers, TMEM
+  for (int i = tid; i < (512 + 2048) * 8 / 16; i += kTcThreads)
+    reinterpret_cast<uint4 *>(const_cast<uint2 *>(S.sel2))[i] =
+        __ldg(reinterpret_cast<const uint4 *>(a.grids + kGridQ2Bsel) + i);
   if (tid == 0) {
-    ptx::mbar_init(&S.mma_done[0], 1);
-    ptx::mbar_init(&S.mma_done[1], 1);
+    for (int i = 0; i < kPr; ++i) ptx::mbar_init(&B.pfull[i], 1), ptx::mbar_init(&B.pempty[i], kDqWarps);
+    for (int i = 0; i < C::kAr; ++i) ptx::mbar_init(&B.afull[i], kDqWarps), ptx::mbar_init(&B.aempty[i], 1);
+    for (int i = 0; i < 2; ++i) ptx::mbar_init(&B.accfull[i], 1), ptx::mbar_init(&B.accempty[i], kEpWarps);
     ptx::mbar_fence_init();
+  }
+  if (warp == 0) {
+    ptx::tmem_alloc(S.taddr, kTmemCols);
+    ptx::tmem_relinquish();
   }
   ptx::tc_fence_before();
   __syncthreads();
@@ -183,127 +290,212 @@ __global__ void __launch_bounds__(kTcThreads, 1) grouped_tc_kernel(TileArgs a) {
   const uint32_t tmem = *S.taddr;
   const int n_active = ctrl->n_active;
   const int n_units = DOWN ? ctrl->n_dn_units : ctrl->n_gu_units;
-  uint32_t waits[2] = {0u, 0u};  // completed phases consumed per stage
-  bool timed_out = false;
+  const int my_total = n_units > cta ? (n_units - cta + G - 1) / G : 0;
+  bool bad = false;
+  // per-role pipeline positions (they carry over between passes)
+  uint32_t col = 0, step = 0, ucount = 0;
 
-  for (;;) {
-    if (tid == 0) *S.unit = atomicAdd(DOWN ? &ctrl->ticket_dn : &ctrl->ticket_gu, 1);
+  for (int base = 0; base < my_total; base += kMaxUnits) {
+    const int n_this = min(kMaxUnits, my_total - base);
+    __syncthreads();  // every role is done with the previous pass's records
+    for (int i = tid; i < n_this; i += kTcThreads) S.units[i] = make_unit(a, act, n_active, cta + (base + i) * G, DOWN);
     __syncthreads();
-    const int j = *S.unit;
-    if (j >= n_units || timed_out) break;
-    const UnitInfo U = find_unit(act, n_active, j, DOWN, H);
-    const ActiveEntry &E = act[U.inst];
-    const redlite_moe_expert ex = expert_desc(a, E);
-    for (int i = tid; i < U.n_real; i += kTcThreads) {
-      const Pair pr = pairs[U.p0 + i];
-      S.tok[i] = pr.token;
-      S.wt[i] = pr.weight;
-    }
-    __syncthreads();
-    const int K = DOWN ? E.ffn : H;
-    const int nk = K / kKc;
-    const uint32_t idesc = ptx::idesc_bf16_f32(128, U.n_pad);
-    for (int kc = 0; kc < nk; ++kc) {
-      const int st = kc & 1;
-      if (kc >= 2) {  // the mma of chunk kc - 2 used this stage
-        if (!ptx::mbar_wait(&S.mma_done[st], waits[st] & 1u)) timed_out = true;
-        ++waits[st];
+
+    if (warp == 0) {
+      // ---- producer: packed tile-blocks, one 256-input column per ring slot
+      if (lane == 0) {
+        for (int u = 0; u < n_this; ++u) {
+          const Unit U = S.units[u];
+          const int tbb = tile_block_bytes(U.qtype), nkb = U.K / 256;
+          for (int kb = 0; kb < nkb; ++kb, ++col) {
+            const int ps = col % kPr;
+            if (col >= (uint32_t)kPr && !ptx::mbar_wait(&B.pempty[ps], ((col / kPr) - 1) & 1u, kWaitLimit)) bad = true;
+            ptx::mbar_expect_tx(&B.pfull[ps], (uint32_t)(C::kMats * 8 * tbb));
+            uint8_t *dst = S.packed + (size_t)ps * C::kPacked;
+#pragma unroll
+            for (int m = 0; m < C::kMats; ++m) {
+              const uint8_t *mat = m ? U.mat1 : U.mat0;
+              for (int i = 0; i < 8; ++i)
+                ptx::bulk_g2s(dst + (m * 8 + i) * tbb, mat + ((size_t)(8 * U.rt + i) * nkb + kb) * tbb, tbb,
+                              &B.pfull[ps]);
+            }
+          }
+        }
       }
-      uint8_t *A0 = S.stage[st];
-      if (DOWN) {
-        fill_weights_any(E.qtype, A0, (const uint8_t *)ex.down, E.ffn, 128 * U.rt, kKc * kc, S);
-        fill_tokens_bf16(A0 + kTileA, hbuf, a.max_ffn, U.p0, kKc * kc, U.n_real, U.n_pad);
-      } else {
-        fill_weights_any(E.qtype, A0, (const uint8_t *)ex.gate, H, 128 * U.rt, kKc * kc, S);
-        fill_weights_any(E.qtype, A0 + kTileA, (const uint8_t *)ex.up, H, 128 * U.rt, kKc * kc, S);
-        fill_tokens_f32(A0 + 2 * kTileA, a.x, H, kKc * kc, U.n_real, U.n_pad, S.tok);
+    } else if (warp == 1) {
+      // ---- tensor-core issue (one thread)
+      if (lane == 0) {
+        for (int u = 0; u < n_this; ++u, ++ucount) {
+          const Unit U = S.units[u];
+          const int buf = ucount & 1;
+          if (ucount >= 2 && !ptx::mbar_wait(&B.accempty[buf], ((ucount >> 1) - 1) & 1u, kWaitLimit)) bad = true;
+          ptx::tc_fence_after();
+          const uint32_t d = tmem + buf * C::kBufCols;
+          const uint32_t idesc = ptx::idesc_bf16_f32(128, U.n_pad);
+          const int nsteps = U.K / 64;
+          for (int k = 0; k < nsteps; ++k, ++step) {
+            const int as = step % C::kAr;
+            if (!ptx::mbar_wait(&B.afull[as], (step / C::kAr) & 1u, kWaitLimit)) bad = true;
+            ptx::tc_fence_after();
+            const uint32_t a0 = ptx::smem_u32(S.ring + (size_t)as * C::kStep);
+            const uint32_t b0 = a0 + C::kMats * kTile;
+#pragma unroll
+            for (int ks = 0; ks < 4; ++ks) {
+              const bool acc = k > 0 || ks > 0;
+              ptx::umma_bf16(d, ptx::sdesc_k_sw128(a0 + 32 * ks), ptx::sdesc_k_sw128(b0 + 32 * ks), idesc, acc);
+              if (!DOWN)
+                ptx::umma_bf16(d + 128, ptx::sdesc_k_sw128(a0 + kTile + 32 * ks), ptx::sdesc_k_sw128(b0 + 32 * ks),
+                               idesc, acc);
+            }
+            ptx::umma_commit(&B.aempty[as]);  // the slot is free once these have read it
+          }
+          ptx::umma_commit(&B.accfull[buf]);
+        }
       }
-      ptx::fence_proxy_async_smem();
-      __syncthreads();
-      if (tid == 0) {
+    } else if (warp < 2 + kDqWarps) {
+      // ---- dequant warps: A tiles (and this warp's 16 rows of B)
+      const int w = warp - 2;
+      for (int u = 0; u < n_this; ++u) {
+        const Unit U = S.units[u];
+        const int nkb = U.K / 256;
+        // B rows 16w + (lane >> 3) + 4i, 16-byte chunk lane & 7 of each step
+        const __nv_bfloat16 *brow[4];
+        int nb = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int j = 16 * w + (lane >> 3) + 4 * i;
+          const int jj = min(j, U.n_real - 1);  // pad rows read a real row; their results are dropped
+          if (j < U.n_pad) nb = i + 1;
+          brow[i] = DOWN ? hbuf + (size_t)(U.p0 + jj) * a.max_ffn : xb + (size_t)pairs[U.p0 + jj].token * H;
+        }
+        const int tbb = tile_block_bytes(U.qtype);
+        for (int kb = 0; kb < nkb; ++kb, ++col) {
+          const int ps = col % kPr;
+          if (!ptx::mbar_wait(&B.pfull[ps], (col / kPr) & 1u, kWaitLimit)) bad = true;
+          const uint8_t *pk = S.packed + (size_t)ps * C::kPacked;
+          Q2Lane l2[C::kMats];
+          Q1Lane l1[C::kMats];
+          if (U.qtype == kQ2) {
+#pragma unroll
+            for (int m = 0; m < C::kMats; ++m) l2[m] = load_q2(pk + (m * 8 + w) * tbb, lane);
+          } else {
+#pragma unroll
+            for (int m = 0; m < C::kMats; ++m) l1[m] = load_q1(pk + (m * 8 + w) * tbb, lane);
+          }
+          __syncwarp();
+          if (lane == 0) ptx::mbar_arrive(&B.pempty[ps]);
+#pragma unroll 1
+          for (int s = 0; s < 4; ++s, ++step) {
+            const int as = step % C::kAr;
+            if (step >= (uint32_t)C::kAr && !ptx::mbar_wait(&B.aempty[as], ((step / C::kAr) - 1) & 1u, kWaitLimit))
+              bad = true;
+            uint8_t *stg = S.ring + (size_t)as * C::kStep;
+            const int k0 = 256 * kb + 64 * s + 8 * (lane & 7);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              if (i < nb)
+                cp_async16(stg + C::kMats * kTile + ptx::sw128_offset(16 * w + (lane >> 3) + 4 * i, 8 * (lane & 7)),
+                           brow[i] + k0);
+            asm volatile("cp.async.commit_group;" ::: "memory");
+            if (U.qtype == kQ2) {
+#pragma unroll
+              for (int m = 0; m < C::kMats; ++m) dequant_q2(l2[m], s, stg + m * kTile, 16 * w, S.sel2, lane);
+            } else {
+#pragma unroll
+              for (int m = 0; m < C::kMats; ++m) dequant_q1(l1[m], s, stg + m * kTile, 16 * w, S.sel1, lane);
+            }
+            asm volatile("cp.async.wait_group 0;" ::: "memory");
+            ptx::fence_proxy_async_smem();  // generic-proxy writes -> the tensor cores
+            __syncwarp();
+            if (lane == 0) ptx::mbar_arrive(&B.afull[as]);
+          }
+        }
+      }
+    } else {
+      // ---- epilogue: warp reads TMEM lanes 32 (warp % 4) .. + 31 (= tile rows)
+      const int lq = warp & 3, row = 32 * lq + lane;
+      for (int u = 0; u < n_this; ++u, ++ucount) {
+        const Unit U = S.units[u];
+        const int buf = ucount & 1;
+        if (!ptx::mbar_wait(&B.accfull[buf], (ucount >> 1) & 1u, kWaitLimit)) bad = true;
         ptx::tc_fence_after();
-        const uint32_t a0 = ptx::smem_u32(A0);
-        const uint32_t b0 = a0 + (DOWN ? 1 : 2) * kTileA;
-#pragma unroll
-        for (int ks = 0; ks < kKc / 16; ++ks) {
-          const bool acc = kc > 0 || ks > 0;
-          ptx::umma_bf16(tmem, ptx::sdesc_k_sw128(a0 + 32 * ks), ptx::sdesc_k_sw128(b0 + 32 * ks), idesc, acc);
-          if (!DOWN)
-            ptx::umma_bf16(tmem + 256, ptx::sdesc_k_sw128(a0 + kTileA + 32 * ks), ptx::sdesc_k_sw128(b0 + 32 * ks),
-                           idesc, acc);
-        }
-        ptx::umma_commit(&S.mma_done[st]);
-      }
-    }
-    // drain the last two chunks' commits (they cover every mma of the unit)
-    for (int kc = (nk >= 2 ? nk - 2 : 0); kc < nk; ++kc) {
-      const int st = kc & 1;
-      if (!ptx::mbar_wait(&S.mma_done[st], waits[st] & 1u)) timed_out = true;
-      ++waits[st];
-    }
-    ptx::tc_fence_after();
-    // epilogue: warp w reads TMEM lanes 32 (w % 4) .. (rows), column chunks of 16
-    const int lg = warp & 3, half = warp >> 2;
-    const int row = 32 * lg + lane;
-    for (int c0 = 16 * half; c0 < U.n_pad; c0 += 32) {
-      uint32_t d0[16];
-      ptx::tmem_ld16(tmem + ((uint32_t)(32 * lg) << 16) + (uint32_t)c0, d0);
-      if (DOWN) {
-        ptx::tmem_wait_ld();
+        const uint32_t d = tmem + buf * C::kBufCols + ((uint32_t)(32 * lq) << 16);
         const int r = 128 * U.rt + row;
+        for (int c0 = 0; c0 < U.n_pad; c0 += 16) {
+          uint32_t d0[16];
+          ptx::tmem_ld16(d + (uint32_t)c0, d0);
+          if (DOWN) {
+            ptx::tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int jj = c0 + i;
-          if (jj < U.n_real) atomicAdd(a.out + (size_t)S.tok[jj] * H + r, S.wt[jj] * __uint_as_float(d0[i]));
-        }
-      } else {
-        uint32_t d1[16];
-        ptx::tmem_ld16(tmem + 256 + ((uint32_t)(32 * lg) << 16) + (uint32_t)c0, d1);
-        ptx::tmem_wait_ld();
-        const int col = 128 * U.rt + row;  // position within the expert's width
+            for (int i = 0; i < 16; ++i) {
+              const int jj = c0 + i;
+              if (jj < U.n_real) {
+                const Pair pr = pairs[U.p0 + jj];
+                atomicAdd(a.out + (size_t)pr.token * H + r, pr.weight * __uint_as_float(d0[i]));
+              }
+            }
+          } else {
+            uint32_t d1[16];
+            ptx::tmem_ld16(d + 128 + (uint32_t)c0, d1);
+            ptx::tmem_wait_ld();
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int jj = c0 + i;
-          if (jj < U.n_real)
-            hbuf[(size_t)(U.p0 + jj) * a.max_ffn + col] =
-                __float2bfloat16_rn(silu_mul(__uint_as_float(d0[i]), __uint_as_float(d1[i])));
+            for (int i = 0; i < 16; ++i) {
+              const int jj = c0 + i;
+              if (jj < U.n_real)
+                hbuf[(size_t)(U.p0 + jj) * a.max_ffn + r] =
+                    __float2bfloat16_rn(silu_mul(__uint_as_float(d0[i]), __uint_as_float(d1[i])));
+            }
+          }
         }
+        ptx::tc_fence_before();
+        __syncwarp();
+        if (lane == 0) ptx::mbar_arrive(&B.accempty[buf]);
       }
     }
-    ptx::tc_fence_before();
-    timed_out = __syncthreads_or(timed_out);  // TMEM read and tokens consumed before the next unit
   }
-  if (timed_out && lane == 0) atomicOr(a.status, REDLITE_STATUS_TIMEOUT);
+  if (bad) atomicOr(a.status, REDLITE_STATUS_TIMEOUT);
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
-  if (warp == 0) ptx::tmem_dealloc(tmem, kCols);
+  if (warp == 0) ptx::tmem_dealloc(tmem, kTmemCols);
 }
 
-static size_t tc_smem_bytes(bool down) {
-  const size_t stage = (down ? 1 : 2) * (size_t)kTileA + kTileB;
-  return 1024 + 2 * stage + 512 * 8 + 2048 * 8 + 2 * sizeof(int) * kTcTokens + 2 * sizeof(uint64_t) + 16 + 16;
+// Activations to bf16 (round to nearest even), 8 per thread.
+__global__ void to_bf16_kernel(const float *__restrict__ x, __nv_bfloat16 *__restrict__ xb, int64_t n8) {
+  const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  if (i >= n8) return;
+  const float4 v0 = __ldg(reinterpret_cast<const float4 *>(x) + 2 * i);
+  const float4 v1 = __ldg(reinterpret_cast<const float4 *>(x) + 2 * i + 1);
+  reinterpret_cast<uint4 *>(xb)[i] =
+      make_uint4(bf16x2(v0.x, v0.y), bf16x2(v0.z, v0.w), bf16x2(v1.x, v1.y), bf16x2(v1.z, v1.w));
 }
 
-bool tc_supported(int hidden, int max_ffn) {
-  return hidden % 256 == 0 && max_ffn % 256 == 0;
-}
+}  // namespace
+
+bool tc_supported(int hidden, int max_ffn) { return hidden % 256 == 0 && max_ffn % 256 == 0; }
 
 cudaError_t launch_tc(const TileArgs &a, cudaStream_t stream) {
+  static_assert(smem_bytes<false>() <= 227 * 1024 && smem_bytes<true>() <= 227 * 1024, "shared memory");
   int dev = 0, sms = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   e = cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return e;
-  const size_t s_gu = tc_smem_bytes(false), s_dn = tc_smem_bytes(true);
-  e = cudaFuncSetAttribute(grouped_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s_gu);
+  e = cudaFuncSetAttribute(grouped_tc_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem_bytes<false>());
   if (e != cudaSuccess) return e;
-  e = cudaFuncSetAttribute(grouped_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)s_dn);
+  e = cudaFuncSetAttribute(grouped_tc_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           (int)smem_bytes<true>());
   if (e != cudaSuccess) return e;
-  grouped_tc_kernel<false><<<sms, kTcThreads, s_gu, stream>>>(a);
+  const int64_t n8 = (int64_t)a.n_tokens * a.hidden / 8;
+  to_bf16_kernel<<<(unsigned)((n8 + 255) / 256), 256, 0, stream>>>(
+      a.x, reinterpret_cast<__nv_bfloat16 *>(a.ws + a.L.xb), n8);
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
-  grouped_tc_kernel<true><<<sms, kTcThreads, s_dn, stream>>>(a);
+  grouped_tc_kernel<false><<<sms, kTcThreads, smem_bytes<false>(), stream>>>(a);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  grouped_tc_kernel<true><<<sms, kTcThreads, smem_bytes<true>(), stream>>>(a);
   return cudaGetLastError();
 }
 

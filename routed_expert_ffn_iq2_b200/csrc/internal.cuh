@@ -37,6 +37,10 @@ constexpr int kQ1GridEntries = 2048;
 //   kGridSign   : u32 [256]   nibble j bit 2 = sign bit j of a sign byte
 //   kGridQ1Sel  : u32 [4096]  index e = idx | delta_bit << 11: nibble j =
 //                 symbol j of grid entry idx | delta_bit << 2
+//   kGridQ2Bsel : u64 [512], kGridQ1Bsel : u64 [2048]  bf16-pair selectors:
+//                 bits 16w..16w+15 select weights 2w, 2w+1 as the byte pairs
+//                 (2 s, 2 s + 1) of a table of three bf16 values indexed by
+//                 the weights' symbols s
 // A selector nibble picks one byte of a constant 8-byte table (see the
 // decode kernels), so two byte-permutes turn a selector into eight signed
 // int8 weights.
@@ -49,7 +53,9 @@ constexpr size_t kGridQ1Comp = kGridQ2Comp + 512 * 2;
 constexpr size_t kGridQ2Sel = kGridQ1Comp + 2048 * 2;
 constexpr size_t kGridSign = kGridQ2Sel + 512 * 4;
 constexpr size_t kGridQ1Sel = kGridSign + 256 * 4;
-constexpr size_t kGridBytes = kGridQ1Sel + 4096 * 4;
+constexpr size_t kGridQ2Bsel = kGridQ1Sel + 4096 * 4;
+constexpr size_t kGridQ1Bsel = kGridQ2Bsel + 512 * 8;
+constexpr size_t kGridBytes = kGridQ1Bsel + 2048 * 8;
 
 inline __host__ __device__ int block_bytes(int qtype) {
   return qtype == kQ2 ? kQ2BlockBytes : (qtype == kQ1 ? kQ1BlockBytes : 0);
@@ -105,7 +111,7 @@ struct Ctrl {
 static_assert(sizeof(Ctrl) == 256, "ctrl block is 256 bytes");
 
 struct WorkspaceLayout {
-  size_t ctrl, active, pairs, counts, done, h, gu, limbs, exps, total;
+  size_t ctrl, active, pairs, counts, done, h, xb, gu, limbs, exps, total;
   int max_active, max_pairs;
 };
 
@@ -133,6 +139,8 @@ inline WorkspaceLayout workspace_layout(int hidden, int n_experts, int max_token
   off = align256(off + sizeof(int) * (size_t)L.max_active);
   L.h = off;
   off = align256(off + sizeof(float) * (size_t)L.max_pairs * (size_t)max_ffn);
+  L.xb = off;  // tensor-core path: the call's activations as bf16 [tokens][hidden]
+  off = align256(off + 2 * (size_t)max_tokens * (size_t)hidden);
   // fused decode kernel: gate/up results per pair, activation limbs per token
   const int64_t ft = std::min<int64_t>(max_tokens, kFusedMaxPairs / (top_k > 0 ? top_k : 1));
   const int64_t fpairs = ft * top_k + ft;
@@ -282,7 +290,7 @@ struct FusedArgs {
 bool fused_supported(int hidden, int max_ffn, int n_tokens, int top_k, int n_experts, bool has_shared);
 
 // Tensor-core (tcgen05) grouped path: tokens per work unit, and the launch.
-constexpr int kTcTokens = 256;
+constexpr int kTcTokens = 128;
 bool tc_supported(int hidden, int max_ffn);
 cudaError_t launch_tc(const TileArgs &a, cudaStream_t stream);
 cudaError_t launch_fused(const FusedArgs &a, cudaStream_t stream);
