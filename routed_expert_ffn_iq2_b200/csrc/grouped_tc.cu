@@ -22,8 +22,9 @@
 //               commits them to the step's slot and, per unit, to one of two
 //               accumulator buffers;
 //   warps 2-9   dequant warp w decodes tile-block w (rows 16w..16w+15) of
-//               each matrix into the A tiles of a 3-4 deep ring of steps and
-//               fetches rows 16w..16w+15 of B with cp.async;
+//               each matrix into the A tiles of a ring of 64-input steps (3
+//               deep for gate/up, 5 for down) and
+//               fetches rows 16w..16w+15 of B with cp.async, a step ahead;
 //   warps 10-13 the epilogue (TMEM -> registers -> h or out), overlapping
 //               the next unit's contraction.
 #include "internal.cuh"
@@ -43,10 +44,31 @@ constexpr int kMaxUnits = 128;             // unit records per pass
 constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kWaitLimit = 1u << 26;
 
+// Optional per-warp cycle counters (build with -DREDLITE_TC_TRACE): CTA c,
+// warp w adds to 8 words at the end of the workspace layout, slot (c * 16 + w) * 8.
+#ifdef REDLITE_TC_TRACE
+#define TC_T0() const long long tc_t0_ = clock64()
+#define TC_ADD(i) tc_acc_[i] += clock64() - tc_t0_
+#define TC_DECL long long tc_acc_[8] = {0, 0, 0, 0, 0, 0, 0, 0}; const long long tc_start_ = clock64()
+#define TC_FLUSH()                                                                                   \
+  do {                                                                                               \
+    tc_acc_[7] = clock64() - tc_start_;                                                              \
+    if (lane == 0)                                                                                   \
+      for (int i_ = 0; i_ < 8; ++i_)                                                                 \
+        reinterpret_cast<long long *>(a.ws + a.L.total)[((size_t)(DOWN * 148 + blockIdx.x) * 16 + warp) * 8 + i_] += \
+            tc_acc_[i_];                                                                             \
+  } while (0)
+#else
+#define TC_T0()
+#define TC_ADD(i)
+#define TC_DECL
+#define TC_FLUSH()
+#endif
+
 template <bool DOWN>
 struct Cfg {
   static constexpr int kMats = DOWN ? 1 : 2;
-  static constexpr int kAr = DOWN ? 4 : 3;                  // 64-input steps in flight
+  static constexpr int kAr = DOWN ? 5 : 3;                  // 64-input steps in flight
   static constexpr int kStep = (kMats + 1) * kTile;         // A tiles, then the B tile
   static constexpr int kPacked = kMats * 8 * kQ2TileBlock;  // one column, largest format
   static constexpr uint32_t kBufCols = DOWN ? 128 : 256;    // TMEM columns per accumulator buffer
@@ -59,7 +81,7 @@ struct Unit {
 static_assert(sizeof(Unit) == 48, "unit records are 48 bytes");
 
 struct Bars {
-  uint64_t pfull[kPr], pempty[kPr], afull[4], aempty[4], accfull[2], accempty[2];
+  uint64_t pfull[kPr], pempty[kPr], afull[8], aempty[8], accfull[2], accempty[2];
 };
 
 struct Smem {
@@ -145,17 +167,17 @@ struct Q2Lane {
   float d0, d1;  // d / 8 of rows q and q+8
 };
 
-__device__ __forceinline__ Q2Lane load_q2(const uint8_t *tb, int lane) {
+__device__ __forceinline__ Q2Lane load_q2(uint32_t tb, int lane) {
   Q2Lane r;
-  const uint4 qs = *reinterpret_cast<const uint4 *>(tb + 32 * lane);
-  const uint4 sg = *reinterpret_cast<const uint4 *>(tb + 32 * lane + 16);
+  const uint4 qs = ptx::lds128(tb + 32 * lane);
+  const uint4 sg = ptx::lds128(tb + 32 * lane + 16);
   r.qs[0] = qs.x, r.qs[1] = qs.y, r.qs[2] = qs.z, r.qs[3] = qs.w;
   r.sg[0] = sg.x, r.sg[1] = sg.y, r.sg[2] = sg.z, r.sg[3] = sg.w;
-  r.qh = *reinterpret_cast<const uint16_t *>(tb + 1024 + 2 * lane);
+  r.qh = ptx::lds16(tb + 1024 + 2 * lane);
   const int q = lane >> 2;
-  const uint2 sc = *reinterpret_cast<const uint2 *>(tb + 1088 + 8 * q);
+  const uint2 sc = ptx::lds64(tb + 1088 + 8 * q);
   r.sc0 = sc.x, r.sc1 = sc.y;
-  const uint32_t dw = *reinterpret_cast<const uint32_t *>(tb + 1152 + 4 * q);
+  const uint32_t dw = ptx::lds32(tb + 1152 + 4 * q);
   r.d0 = __half2float(__ushort_as_half((unsigned short)(dw & 0xFFFFu))) * 0.125f;
   r.d1 = __half2float(__ushort_as_half((unsigned short)(dw >> 16))) * 0.125f;
   return r;
@@ -163,7 +185,7 @@ __device__ __forceinline__ Q2Lane load_q2(const uint8_t *tb, int lane) {
 
 // Step s (inputs 64s..64s+63 of the column) of one IQ2 tile-block into rows
 // row0..row0+15 of the swizzled A tile: fields i = 4s + 2 c2 + h.
-__device__ __forceinline__ void dequant_q2(const Q2Lane &L, int s, uint8_t *A, int row0, const uint2 *sel2,
+__device__ __forceinline__ void dequant_q2(const Q2Lane &L, int s, uint32_t A, int row0, uint32_t sel2,
                                            int lane) {
   const int q = lane >> 2, t = lane & 3;
   const uint32_t qw = s == 0 ? L.qs[0] : s == 1 ? L.qs[1] : s == 2 ? L.qs[2] : L.qs[3];
@@ -177,7 +199,7 @@ __device__ __forceinline__ void dequant_q2(const Q2Lane &L, int s, uint8_t *A, i
       const int f = 2 * c2 + h;
       const uint32_t qsb = (qw >> (8 * f)) & 0xFFu, sgb = (sw >> (8 * f)) & 0xFFu;
       const uint32_t idx = qsb | (((L.qh >> (4 * s + f)) & 1u) << 8);
-      const uint2 sel = sel2[idx];
+      const uint2 sel = ptx::lds64_const(sel2 + 8 * idx);
       const uint32_t nib = ((h ? L.sc1 : L.sc0) >> (4 * c)) & 15u;
       const float sc = (h ? L.d1 : L.d0) * (float)(2 * nib + 1);
       const uint32_t t0 = bf16x2(sc * 8.f, sc * 25.f), t1 = bf16x2(sc * 43.f, 0.f);
@@ -187,7 +209,7 @@ __device__ __forceinline__ void dequant_q2(const Q2Lane &L, int s, uint8_t *A, i
       v.y = __byte_perm(t0, t1, sel.x >> 16) ^ (((sgb >> 2) * 0x40008000u) & 0x80008000u);
       v.z = __byte_perm(t0, t1, sel.y) ^ (((sgb >> 4) * 0x40008000u) & 0x80008000u);
       v.w = __byte_perm(t0, t1, sel.y >> 16) ^ (((sgb >> 6) * 0x40008000u) & 0x80008000u);
-      *reinterpret_cast<uint4 *>(A + ptx::sw128_offset(row0 + q + 8 * h, 32 * c2 + 8 * t)) = v;
+      ptx::sts128(A + ptx::sw128_offset(row0 + q + 8 * h, 32 * c2 + 8 * t), v);
     }
   }
 }
@@ -201,29 +223,29 @@ struct Q1Lane {
   float d0, d1;
 };
 
-__device__ __forceinline__ Q1Lane load_q1(const uint8_t *tb, int lane) {
+__device__ __forceinline__ Q1Lane load_q1(uint32_t tb, int lane) {
   Q1Lane r;
   const int q = lane >> 2, p = (lane >> 1) & 1, half = lane & 1;
-  const uint8_t *pb = tb + 48 * (2 * q + p);
-  const uint4 qa = *reinterpret_cast<const uint4 *>(pb), qb = *reinterpret_cast<const uint4 *>(pb + 16);
-  const uint4 nb = *reinterpret_cast<const uint4 *>(pb + 32);
+  const uint32_t pb = tb + 48 * (2 * q + p);
+  const uint4 qa = ptx::lds128(pb), qb = ptx::lds128(pb + 16);
+  const uint4 nb = ptx::lds128(pb + 32);
   // qs word 2S + half holds fields 8S + 4 half .. + 3 of step S
   r.qs[0] = half ? qa.y : qa.x;
   r.qs[1] = half ? qa.w : qa.z;
   r.qs[2] = half ? qb.y : qb.x;
   r.qs[3] = half ? qb.w : qb.z;
   r.nb[0] = nb.x, r.nb[1] = nb.y, r.nb[2] = nb.z, r.nb[3] = nb.w;
-  const uint32_t *scp = reinterpret_cast<const uint32_t *>(tb + 768 + 12 * q);
-  const uint32_t s0 = scp[0], s1 = scp[1], s2 = scp[2];
+  const uint32_t s0 = ptx::lds32(tb + 768 + 12 * q), s1 = ptx::lds32(tb + 772 + 12 * q),
+                 s2 = ptx::lds32(tb + 776 + 12 * q);
   r.row0 = (uint64_t)s0 | ((uint64_t)(s1 & 0xFFFFu) << 32);
   r.row1 = (uint64_t)(s1 >> 16) | ((uint64_t)s2 << 16);
-  const uint32_t dw = *reinterpret_cast<const uint32_t *>(tb + 864 + 4 * q);
+  const uint32_t dw = ptx::lds32(tb + 864 + 4 * q);
   r.d0 = __half2float(__ushort_as_half((unsigned short)(dw & 0xFFFFu)));
   r.d1 = __half2float(__ushort_as_half((unsigned short)(dw >> 16)));
   return r;
 }
 
-__device__ __forceinline__ void dequant_q1(const Q1Lane &L, int S, uint8_t *A, int row0, const uint2 *sel1,
+__device__ __forceinline__ void dequant_q1(const Q1Lane &L, int S, uint32_t A, int row0, uint32_t sel1,
                                            int lane) {
   const int q = lane >> 2, p = (lane >> 1) & 1, half = lane & 1;
   const uint32_t qw = S == 0 ? L.qs[0] : S == 1 ? L.qs[1] : S == 2 ? L.qs[2] : L.qs[3];
@@ -238,7 +260,7 @@ __device__ __forceinline__ void dequant_q1(const Q1Lane &L, int S, uint8_t *A, i
       const int f = 2 * s2 + h;
       const uint32_t qsb = (qw >> (8 * f)) & 0xFFu;
       const uint32_t nib = (nb16 >> (4 * f)) & 15u;
-      const uint2 sel = sel1[qsb | ((nib & 7u) << 8)];
+      const uint2 sel = ptx::lds64_const(sel1 + 8 * (qsb | ((nib & 7u) << 8)));
       const uint32_t sc3 = (uint32_t)(((h ? L.row1 : L.row0) >> (3 * sb)) & 7u);
       const float sc = (h ? L.d1 : L.d0) * (float)(2 * sc3 + 1);
       const float dl = (nib & 8u) ? -0.125f : 0.125f;
@@ -248,7 +270,7 @@ __device__ __forceinline__ void dequant_q1(const Q1Lane &L, int S, uint8_t *A, i
       v.y = __byte_perm(t0, t1, sel.x >> 16);
       v.z = __byte_perm(t0, t1, sel.y);
       v.w = __byte_perm(t0, t1, sel.y >> 16);
-      *reinterpret_cast<uint4 *>(A + ptx::sw128_offset(row0 + q + 8 * h, 16 * (2 * half + s2) + 8 * p)) = v;
+      ptx::sts128(A + ptx::sw128_offset(row0 + q + 8 * h, 16 * (2 * half + s2) + 8 * p), v);
     }
   }
 }
@@ -292,6 +314,7 @@ __global__ void __maxnreg__(128) grouped_tc_kernel(TileArgs a) {
   const int n_units = DOWN ? ctrl->n_dn_units : ctrl->n_gu_units;
   const int my_total = n_units > cta ? (n_units - cta + G - 1) / G : 0;
   bool bad = false;
+  TC_DECL;
   // per-role pipeline positions (they carry over between passes)
   uint32_t col = 0, step = 0, ucount = 0;
 
@@ -309,7 +332,12 @@ __global__ void __maxnreg__(128) grouped_tc_kernel(TileArgs a) {
           const int tbb = tile_block_bytes(U.qtype), nkb = U.K / 256;
           for (int kb = 0; kb < nkb; ++kb, ++col) {
             const int ps = col % kPr;
-            if (col >= (uint32_t)kPr && !ptx::mbar_wait(&B.pempty[ps], ((col / kPr) - 1) & 1u, kWaitLimit)) bad = true;
+            {
+              TC_T0();
+              if (col >= (uint32_t)kPr && !ptx::mbar_wait(&B.pempty[ps], ((col / kPr) - 1) & 1u, kWaitLimit))
+                bad = true;
+              TC_ADD(0);
+            }
             ptx::mbar_expect_tx(&B.pfull[ps], (uint32_t)(C::kMats * 8 * tbb));
             uint8_t *dst = S.packed + (size_t)ps * C::kPacked;
 #pragma unroll
@@ -328,14 +356,22 @@ __global__ void __maxnreg__(128) grouped_tc_kernel(TileArgs a) {
         for (int u = 0; u < n_this; ++u, ++ucount) {
           const Unit U = S.units[u];
           const int buf = ucount & 1;
-          if (ucount >= 2 && !ptx::mbar_wait(&B.accempty[buf], ((ucount >> 1) - 1) & 1u, kWaitLimit)) bad = true;
+          {
+            TC_T0();
+            if (ucount >= 2 && !ptx::mbar_wait(&B.accempty[buf], ((ucount >> 1) - 1) & 1u, kWaitLimit)) bad = true;
+            TC_ADD(0);
+          }
           ptx::tc_fence_after();
           const uint32_t d = tmem + buf * C::kBufCols;
           const uint32_t idesc = ptx::idesc_bf16_f32(128, U.n_pad);
           const int nsteps = U.K / 64;
           for (int k = 0; k < nsteps; ++k, ++step) {
             const int as = step % C::kAr;
-            if (!ptx::mbar_wait(&B.afull[as], (step / C::kAr) & 1u, kWaitLimit)) bad = true;
+            {
+              TC_T0();
+              if (!ptx::mbar_wait(&B.afull[as], (step / C::kAr) & 1u, kWaitLimit)) bad = true;
+              TC_ADD(1);
+            }
             ptx::tc_fence_after();
             const uint32_t a0 = ptx::smem_u32(S.ring + (size_t)as * C::kStep);
             const uint32_t b0 = a0 + C::kMats * kTile;
@@ -355,6 +391,7 @@ __global__ void __maxnreg__(128) grouped_tc_kernel(TileArgs a) {
     } else if (warp < 2 + kDqWarps) {
       // ---- dequant warps: A tiles (and this warp's 16 rows of B)
       const int w = warp - 2;
+      const uint32_t sel2a = ptx::smem_u32(S.sel2), sel1a = ptx::smem_u32(S.sel1);
       for (int u = 0; u < n_this; ++u) {
         const Unit U = S.units[u];
         const int nkb = U.K / 256;
@@ -368,11 +405,33 @@ __global__ void __maxnreg__(128) grouped_tc_kernel(TileArgs a) {
           if (j < U.n_pad) nb = i + 1;
           brow[i] = DOWN ? hbuf + (size_t)(U.p0 + jj) * a.max_ffn : xb + (size_t)pairs[U.p0 + jj].token * H;
         }
-        const int tbb = tile_block_bytes(U.qtype);
+        const int tbb = tile_block_bytes(U.qtype), nsteps = 4 * nkb;
+        // B rows of local step n into ring slot `as`, as one cp.async group;
+        // issued a step ahead so the copies overlap the decode of the step before
+        auto fetch_b = [&](int n, uint32_t gstep) {
+          const int as = gstep % C::kAr;
+          {
+            TC_T0();
+            if (gstep >= (uint32_t)C::kAr && !ptx::mbar_wait(&B.aempty[as], ((gstep / C::kAr) - 1) & 1u, kWaitLimit))
+              bad = true;
+            TC_ADD(1);
+          }
+          uint8_t *bt = S.ring + (size_t)as * C::kStep + C::kMats * kTile;
+          const int k0 = 64 * n + 8 * (lane & 7);
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            if (i < nb) cp_async16(bt + ptx::sw128_offset(16 * w + (lane >> 3) + 4 * i, 8 * (lane & 7)), brow[i] + k0);
+          asm volatile("cp.async.commit_group;" ::: "memory");
+        };
+        fetch_b(0, step);
         for (int kb = 0; kb < nkb; ++kb, ++col) {
           const int ps = col % kPr;
-          if (!ptx::mbar_wait(&B.pfull[ps], (col / kPr) & 1u, kWaitLimit)) bad = true;
-          const uint8_t *pk = S.packed + (size_t)ps * C::kPacked;
+          {
+            TC_T0();
+            if (!ptx::mbar_wait(&B.pfull[ps], (col / kPr) & 1u, kWaitLimit)) bad = true;
+            TC_ADD(0);
+          }
+          const uint32_t pk = ptx::smem_u32(S.packed) + ps * C::kPacked;
           Q2Lane l2[C::kMats];
           Q1Lane l1[C::kMats];
           if (U.qtype == kQ2) {
@@ -386,25 +445,24 @@ __global__ void __maxnreg__(128) grouped_tc_kernel(TileArgs a) {
           if (lane == 0) ptx::mbar_arrive(&B.pempty[ps]);
 #pragma unroll 1
           for (int s = 0; s < 4; ++s, ++step) {
-            const int as = step % C::kAr;
-            if (step >= (uint32_t)C::kAr && !ptx::mbar_wait(&B.aempty[as], ((step / C::kAr) - 1) & 1u, kWaitLimit))
-              bad = true;
-            uint8_t *stg = S.ring + (size_t)as * C::kStep;
-            const int k0 = 256 * kb + 64 * s + 8 * (lane & 7);
-#pragma unroll
-            for (int i = 0; i < 4; ++i)
-              if (i < nb)
-                cp_async16(stg + C::kMats * kTile + ptx::sw128_offset(16 * w + (lane >> 3) + 4 * i, 8 * (lane & 7)),
-                           brow[i] + k0);
-            asm volatile("cp.async.commit_group;" ::: "memory");
+            const int n = 4 * kb + s, as = step % C::kAr;
+            const bool more = n + 1 < nsteps;
+            if (more) fetch_b(n + 1, step + 1);
+            const uint32_t stg = ptx::smem_u32(S.ring) + as * C::kStep;
+            TC_T0();
             if (U.qtype == kQ2) {
 #pragma unroll
-              for (int m = 0; m < C::kMats; ++m) dequant_q2(l2[m], s, stg + m * kTile, 16 * w, S.sel2, lane);
+              for (int m = 0; m < C::kMats; ++m) dequant_q2(l2[m], s, stg + m * kTile, 16 * w, sel2a, lane);
             } else {
 #pragma unroll
-              for (int m = 0; m < C::kMats; ++m) dequant_q1(l1[m], s, stg + m * kTile, 16 * w, S.sel1, lane);
+              for (int m = 0; m < C::kMats; ++m) dequant_q1(l1[m], s, stg + m * kTile, 16 * w, sel1a, lane);
             }
-            asm volatile("cp.async.wait_group 0;" ::: "memory");
+            TC_ADD(2);
+            // this step's B rows landed (the next step's may still be in flight)
+            if (more)
+              asm volatile("cp.async.wait_group 1;" ::: "memory");
+            else
+              asm volatile("cp.async.wait_group 0;" ::: "memory");
             ptx::fence_proxy_async_smem();  // generic-proxy writes -> the tensor cores
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(&B.afull[as]);
@@ -417,22 +475,30 @@ __global__ void __maxnreg__(128) grouped_tc_kernel(TileArgs a) {
       for (int u = 0; u < n_this; ++u, ++ucount) {
         const Unit U = S.units[u];
         const int buf = ucount & 1;
-        if (!ptx::mbar_wait(&B.accfull[buf], (ucount >> 1) & 1u, kWaitLimit)) bad = true;
+        {
+          TC_T0();
+          if (!ptx::mbar_wait(&B.accfull[buf], (ucount >> 1) & 1u, kWaitLimit)) bad = true;
+          TC_ADD(0);
+        }
         ptx::tc_fence_after();
         const uint32_t d = tmem + buf * C::kBufCols + ((uint32_t)(32 * lq) << 16);
         const int r = 128 * U.rt + row;
+        Pair pl = {0, 0.f};  // down: pair c0 - (c0 % 32) + lane of the unit, broadcast by shuffles
         for (int c0 = 0; c0 < U.n_pad; c0 += 16) {
           uint32_t d0[16];
           ptx::tmem_ld16(d + (uint32_t)c0, d0);
           if (DOWN) {
+            if ((c0 & 31) == 0) {
+              const int jl = c0 + lane;
+              if (jl < U.n_real) pl = pairs[U.p0 + jl];
+            }
             ptx::tmem_wait_ld();
 #pragma unroll
             for (int i = 0; i < 16; ++i) {
-              const int jj = c0 + i;
-              if (jj < U.n_real) {
-                const Pair pr = pairs[U.p0 + jj];
-                atomicAdd(a.out + (size_t)pr.token * H + r, pr.weight * __uint_as_float(d0[i]));
-              }
+              const int src = (c0 & 16) + i;
+              const int tok = __shfl_sync(0xffffffffu, pl.token, src);
+              const float wgt = __shfl_sync(0xffffffffu, pl.weight, src);
+              if (c0 + i < U.n_real) atomicAdd(a.out + (size_t)tok * H + r, wgt * __uint_as_float(d0[i]));
             }
           } else {
             uint32_t d1[16];
@@ -454,6 +520,7 @@ __global__ void __maxnreg__(128) grouped_tc_kernel(TileArgs a) {
     }
   }
   if (bad) atomicOr(a.status, REDLITE_STATUS_TIMEOUT);
+  TC_FLUSH();
   ptx::tc_fence_before();
   __syncthreads();
   ptx::tc_fence_after();
