@@ -45,7 +45,7 @@ constexpr uint32_t kTmemCols = 512;
 constexpr uint32_t kWaitLimit = 1u << 26;
 
 // Optional per-warp cycle counters (build with -DREDLITE_TC_TRACE): CTA c,
-// warp w adds to 8 words at the end of the workspace layout, slot (c * 16 + w) * 8.
+// warp w adds to 8 words at the end of the workspace layout, slot (c * 32 + w) * 8.
 #ifdef REDLITE_TC_TRACE
 #define TC_T0() const long long tc_t0_ = clock64()
 #define TC_ADD(i) tc_acc_[i] += clock64() - tc_t0_
@@ -55,7 +55,7 @@ constexpr uint32_t kWaitLimit = 1u << 26;
     tc_acc_[7] = clock64() - tc_start_;                                                              \
     if (lane == 0)                                                                                   \
       for (int i_ = 0; i_ < 8; ++i_)                                                                 \
-        reinterpret_cast<long long *>(a.ws + a.L.total)[((size_t)(DOWN * 148 + blockIdx.x) * 16 + warp) * 8 + i_] += \
+        reinterpret_cast<long long *>(a.ws + a.L.total)[((size_t)(DOWN * 148 + blockIdx.x) * 32 + warp) * 8 + i_] += \
             tc_acc_[i_];                                                                             \
   } while (0)
 #else
@@ -143,6 +143,9 @@ __device__ Unit make_unit(const TileArgs &a, const ActiveEntry *act, int n_activ
   return u;
 }
 
+// (float)(2 n + 1) for 0 <= n < 2^22, exactly, without a conversion instruction.
+__device__ __forceinline__ float odd_f(uint32_t n) { return __uint_as_float(0x4B000001u + 2 * n) - 8388608.f; }
+
 __device__ __forceinline__ uint32_t bf16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
@@ -201,14 +204,15 @@ __device__ __forceinline__ void dequant_q2(const Q2Lane &L, int s, uint32_t A, i
       const uint32_t idx = qsb | (((L.qh >> (4 * s + f)) & 1u) << 8);
       const uint2 sel = ptx::lds64_const(sel2 + 8 * idx);
       const uint32_t nib = ((h ? L.sc1 : L.sc0) >> (4 * c)) & 15u;
-      const float sc = (h ? L.d1 : L.d0) * (float)(2 * nib + 1);
+      const float sc = (h ? L.d1 : L.d0) * odd_f(nib);
       const uint32_t t0 = bf16x2(sc * 8.f, sc * 25.f), t1 = bf16x2(sc * 43.f, 0.f);
-      // sign bits 2w, 2w+1 -> bit 15, 31 of pair w: (b * (2^15 + 2^30)) & 0x80008000
+      // sign bits 2w, 2w+1 -> bits 15, 31 of pair w: b * (2^(15-2w) + 2^(30-2w)), masked
+      // (the two shifted copies of b never overlap, so no carries)
       uint4 v;
       v.x = __byte_perm(t0, t1, sel.x) ^ ((sgb * 0x40008000u) & 0x80008000u);
-      v.y = __byte_perm(t0, t1, sel.x >> 16) ^ (((sgb >> 2) * 0x40008000u) & 0x80008000u);
-      v.z = __byte_perm(t0, t1, sel.y) ^ (((sgb >> 4) * 0x40008000u) & 0x80008000u);
-      v.w = __byte_perm(t0, t1, sel.y >> 16) ^ (((sgb >> 6) * 0x40008000u) & 0x80008000u);
+      v.y = __byte_perm(t0, t1, sel.x >> 16) ^ ((sgb * 0x10002000u) & 0x80008000u);
+      v.z = __byte_perm(t0, t1, sel.y) ^ ((sgb * 0x04000800u) & 0x80008000u);
+      v.w = __byte_perm(t0, t1, sel.y >> 16) ^ ((sgb * 0x01000200u) & 0x80008000u);
       ptx::sts128(A + ptx::sw128_offset(row0 + q + 8 * h, 32 * c2 + 8 * t), v);
     }
   }
@@ -262,7 +266,7 @@ __device__ __forceinline__ void dequant_q1(const Q1Lane &L, int S, uint32_t A, i
       const uint32_t nib = (nb16 >> (4 * f)) & 15u;
       const uint2 sel = ptx::lds64_const(sel1 + 8 * (qsb | ((nib & 7u) << 8)));
       const uint32_t sc3 = (uint32_t)(((h ? L.row1 : L.row0) >> (3 * sb)) & 7u);
-      const float sc = (h ? L.d1 : L.d0) * (float)(2 * sc3 + 1);
+      const float sc = (h ? L.d1 : L.d0) * odd_f(sc3);
       const float dl = (nib & 8u) ? -0.125f : 0.125f;
       const uint32_t t0 = bf16x2(sc * (dl - 1.f), sc * dl), t1 = bf16x2(sc * (dl + 1.f), 0.f);
       uint4 v;
@@ -374,14 +378,20 @@ __global__ void __maxnreg__(128) grouped_tc_kernel(TileArgs a) {
             }
             ptx::tc_fence_after();
             const uint32_t a0 = ptx::smem_u32(S.ring + (size_t)as * C::kStep);
-            const uint32_t b0 = a0 + C::kMats * kTile;
+            // descriptors of the step's tiles; 16 more inputs = 32 bytes = 2 in the start-address field
+            const uint64_t da = ptx::sdesc_k_sw128(a0), du = da + (kTile >> 4),
+                           db = ptx::sdesc_k_sw128(a0 + C::kMats * kTile);
+            if (k == 0) {
+              ptx::umma_bf16(d, da, db, idesc, false);
+              if (!DOWN) ptx::umma_bf16(d + 128, du, db, idesc, false);
+            } else {
+              ptx::umma_bf16_acc(d, da, db, idesc);
+              if (!DOWN) ptx::umma_bf16_acc(d + 128, du, db, idesc);
+            }
 #pragma unroll
-            for (int ks = 0; ks < 4; ++ks) {
-              const bool acc = k > 0 || ks > 0;
-              ptx::umma_bf16(d, ptx::sdesc_k_sw128(a0 + 32 * ks), ptx::sdesc_k_sw128(b0 + 32 * ks), idesc, acc);
-              if (!DOWN)
-                ptx::umma_bf16(d + 128, ptx::sdesc_k_sw128(a0 + kTile + 32 * ks), ptx::sdesc_k_sw128(b0 + 32 * ks),
-                               idesc, acc);
+            for (int ks = 1; ks < 4; ++ks) {
+              ptx::umma_bf16_acc(d, da + 2 * ks, db + 2 * ks, idesc);
+              if (!DOWN) ptx::umma_bf16_acc(d + 128, du + 2 * ks, db + 2 * ks, idesc);
             }
             ptx::umma_commit(&B.aempty[as]);  // the slot is free once these have read it
           }
