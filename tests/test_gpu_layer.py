@@ -218,3 +218,63 @@ def test_tensor_core_path_mixed_formats(P, oracle_lib):
                                oracle_lib.expand_grid(2, w.grid_iq1))
     assert L.read_status() == 0
     assert _rel_err(got, ref) <= TOL_BF16
+
+
+def _bf16_rne(a):
+    """Round finite values to bf16 (nearest even), returned as float64."""
+    u = np.asarray(a, np.float32).view(np.uint32).astype(np.uint64)
+    r = ((u + 0x7FFF + ((u >> 16) & 1)) >> 16) << 16
+    return r.astype(np.uint32).view(np.float32).astype(np.float64)
+
+
+def test_bf16_rounding_helper_matches_oracle(oracle_lib):
+    v = fixtures.make_x(77, 4, 256).reshape(-1) * np.float32(37.0)
+    want = oracle_lib.float_to_bf16(v).astype(np.uint32) << 16
+    assert np.array_equal(_bf16_rne(v).astype(np.float32).view(np.uint32), want)
+
+
+def test_tensor_core_path_matches_bf16_operand_reference(P, oracle_lib):
+    """72 tokens x top-10 from a pool of 12 experts (6 per format) plus the
+    shared expert: the tcgen05 path against the oracle's exact weights with
+    the path's own roundings applied (weights, activations and h to bf16,
+    nearest even).  What remains is fp32 accumulation order and rare bf16
+    ties in h, so the bar is 1e-3 of max|ref| -- tight enough that a wrong
+    sub-block scale, sign or selector shows."""
+    w = fixtures.workload(4)
+    q = np.asarray(w.qtypes)
+    pool = [int(e) for e in np.nonzero(q == 1)[0][:6]] + [int(e) for e in np.nonzero(q == 2)[0][:6]]
+    T, K, H = 72, 10, w.hidden
+    st = fixtures.Stream(4242, 9)
+    ids = np.zeros((T, K), np.int32)
+    for t in range(T):
+        perm = np.argsort(st.uniform(len(pool)))
+        ids[t] = np.array(pool)[perm[:K]]
+    wt = st.uniform(T * K).reshape(T, K).astype(np.float32) + np.float32(0.05)
+    wt = (wt / wt.sum(axis=1, keepdims=True)).astype(np.float32)
+    x = fixtures.make_x(4242, T, H)
+    L = P.layer_for_workload(w, experts=pool, max_tokens=T)
+    got = _run(L, x, ids, wt)
+    assert L.read_status() == 0
+
+    grids = {1: oracle_lib.expand_grid(1, w.grid_iq2), 2: oracle_lib.expand_grid(2, w.grid_iq1)}
+    xb = _bf16_rne(x)
+    ref = np.zeros((T, H))
+
+    def run_expert(ex, toks, scale):
+        F = ex.ffn
+        wg = _bf16_rne(oracle_lib.dequant_matrix(ex.qtype, ex.gate, F, H, grids[ex.qtype]))
+        wu = _bf16_rne(oracle_lib.dequant_matrix(ex.qtype, ex.up, F, H, grids[ex.qtype]))
+        wd = _bf16_rne(oracle_lib.dequant_matrix(ex.qtype, ex.down, H, F, grids[ex.qtype]))
+        g = xb[toks] @ wg.T
+        u = xb[toks] @ wu.T
+        h = _bf16_rne(g / (1.0 + np.exp(-g)) * u)
+        ref[toks] += scale[:, None] * (h @ wd.T)
+
+    for e in pool:
+        tt, kk = np.nonzero(ids == e)
+        if len(tt):
+            run_expert(w.expert(e), tt, wt[tt, kk].astype(np.float64))
+    sh = w.shared()
+    if sh is not None:
+        run_expert(sh, np.arange(T), np.ones(T))
+    assert _rel_err(got, ref) <= 1e-3
