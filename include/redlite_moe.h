@@ -145,7 +145,8 @@ int redlite_moe_workspace_reset(const redlite_moe_table *table);
  *   shared_expert  host struct with device matrix pointers, or NULL
  *   out            device [n_tokens, hidden] fp32, overwritten (not accumulated into)
  * Enqueued on expert_table->stream; x, ids, weights and out must not be
- * written by other work until it completes.  Two calls that share a
+ * written by other work until it completes, and out must not overlap x,
+ * ids or weights.  Two calls that share a
  * workspace must be ordered on one stream.  Decode-sized calls run one
  * fused kernel; calls with many tokens per expert run the bucketed
  * tensor-core path (bf16 operands, fp32 accumulation). */

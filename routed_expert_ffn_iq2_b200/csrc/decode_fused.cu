@@ -515,6 +515,41 @@ __device__ __noinline__ void limbs_from_global(int nvec, int n, const float *src
   consumers_sync();
 }
 
+// Replicate the selector tables in place (word w of a table with r replicas
+// holds source word w / r; replicas spread lanes over banks): NT threads,
+// t = 0..NT-1, named barrier BAR.  Every source word is read before any is
+// overwritten.
+template <int NT, int BAR>
+__device__ __forceinline__ void replicate_tables(const Smem &S, int t) {
+  static_assert(kRep2 == 16 && kRep1 == 2, "replication below assumes 16 / 2 replicas");
+  constexpr int N2 = (512 + NT - 1) / NT, NS = (256 + NT - 1) / NT, N1 = (4096 + NT - 1) / NT;
+  uint32_t v2[N2], vs[NS], v1[N1];
+#pragma unroll
+  for (int i = 0; i < N2; ++i) v2[i] = t + NT * i < 512 ? S.sel2[t + NT * i] : 0u;
+#pragma unroll
+  for (int i = 0; i < NS; ++i) vs[i] = t + NT * i < 256 ? S.sgn2[t + NT * i] : 0u;
+#pragma unroll
+  for (int i = 0; i < N1; ++i) v1[i] = t + NT * i < 4096 ? S.sel1[t + NT * i] : 0u;
+  asm volatile("bar.sync %0, %1;" ::"n"(BAR), "n"(NT) : "memory");
+  const int rot = (t & 31) >> 1;  // lanes of one store wavefront cover distinct banks
+#pragma unroll
+  for (int r = 0; r < 4; ++r) {
+    const int q = (r + rot) & 3;
+#pragma unroll
+    for (int i = 0; i < N2; ++i)
+      if (t + NT * i < 512)
+        reinterpret_cast<uint4 *>(S.sel2)[(t + NT * i) * 4 + q] = make_uint4(v2[i], v2[i], v2[i], v2[i]);
+#pragma unroll
+    for (int i = 0; i < NS; ++i)
+      if (t + NT * i < 256)
+        reinterpret_cast<uint4 *>(S.sgn2)[(t + NT * i) * 4 + q] = make_uint4(vs[i], vs[i], vs[i], vs[i]);
+  }
+#pragma unroll
+  for (int i = 0; i < N1; ++i)
+    if (t + NT * i < 4096) reinterpret_cast<uint2 *>(S.sel1)[t + NT * i] = make_uint2(v1[i], v1[i]);
+  asm volatile("bar.sync %0, %1;" ::"n"(BAR), "n"(NT) : "memory");
+}
+
 // ------------------------------------------------------------------ the kernel
 
 __device__ bool fused_expert_ok(const redlite_moe_expert &e, int hidden, int max_ffn) {
@@ -526,8 +561,8 @@ __device__ bool fused_expert_ok(const redlite_moe_expert &e, int hidden, int max
 }
 
 __device__ __forceinline__ int item_tiles_of(int ffn) {
-  const int nkb = ffn / 256;
-  return nkb >= 8 ? 1 : 8 / nkb;
+  const int nkb = ffn >> 8;  // 8 / nkb tiles per item, nibble table for nkb = 1..7
+  return nkb >= 8 ? 1 : (int)((0x1112248u >> (4 * (nkb - 1))) & 15u);
 }
 
 __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(FusedArgs a) {
@@ -712,6 +747,11 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(FusedArgs a)
       if (lane == 0) s_bad = bad;
       __syncwarp();
       item_prefix(n_inst);
+    } else if (warp < kCWarps) {
+      // the other consumer warps replicate the selector tables meanwhile
+      if (!mbar_wait(&s_lut_bar, 0) && lane == 0) atomicOr(a.status, REDLITE_STATUS_TIMEOUT);
+      TRACE(13);
+      replicate_tables<kCThreads - 32, 2>(S, tid - 32);
     }
   } else {
     // ---- bucketing: counts per expert in the ring (scratch before any copy)
@@ -841,9 +881,10 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(FusedArgs a)
   const int n_inst = s_n_inst, N1 = s_n1, N2 = s_n2;
   // gate/up items split evenly over the CTAs; down items in reverse CTA order
   // (a CTA with one more gate/up item tends to get one fewer down item)
-  const int b1 = (int)((int64_t)cta * N1 / G), e1i = (int)((int64_t)(cta + 1) * N1 / G);
+  const unsigned uG = (unsigned)G, uN1 = (unsigned)N1, uN2 = (unsigned)N2;  // products < 2^31
+  const int b1 = (int)(cta * uN1 / uG), e1i = (int)((cta + 1) * uN1 / uG);
   const int rc = G - 1 - cta;
-  const int b2 = (int)((int64_t)rc * N2 / G), e2i = (int)((int64_t)(rc + 1) * N2 / G);
+  const int b2 = (int)(rc * uN2 / uG), e2i = (int)((rc + 1) * uN2 / uG);
   const int my1 = e1i - b1, my2 = e2i - b2, my_items = my1 + my2;
 
   // ---- producer warp: streams this CTA's items through the ring
@@ -888,31 +929,20 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(FusedArgs a)
       }
     }
   } else {
-    // ---- consumers: replicate the selector tables (word w of a table with
-    // r replicas holds source word w / r; replicas spread lanes over banks)
+    // ---- consumers: zero this CTA's slice of out (the down items add into
+    // it after the grid barrier; out does not overlap the inputs)
     {
-      static_assert(kRep2 == 16 && kRep1 == 2, "replication below assumes 16 / 2 replicas");
+      const unsigned total4 = (unsigned)(T * H / 4);
+      const unsigned z0 = cta * total4 / uG, z1 = (cta + 1) * total4 / uG;
+      for (unsigned i = z0 + tid; i < z1; i += kCThreads)
+        reinterpret_cast<float4 *>(a.out)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    // ---- consumers: replicate the selector tables (small calls did it while
+    // warp 0 routed)
+    if (npairs > 32) {
       if (!mbar_wait(&s_lut_bar, 0) && lane == 0) atomicOr(a.status, REDLITE_STATUS_TIMEOUT);
       TRACE(13);
-      uint32_t v2[2], vs, v1[16];
-#pragma unroll
-      for (int i = 0; i < 2; ++i) v2[i] = S.sel2[tid + kCThreads * i];
-      vs = S.sgn2[tid];
-#pragma unroll
-      for (int i = 0; i < 16; ++i) v1[i] = S.sel1[tid + kCThreads * i];
-      consumers_sync();  // every source word is read before any is overwritten
-      const int rot = lane >> 1;  // lanes of one store wavefront cover distinct banks
-#pragma unroll
-      for (int r = 0; r < 4; ++r) {
-        const int q = (r + rot) & 3;
-#pragma unroll
-        for (int i = 0; i < 2; ++i)
-          reinterpret_cast<uint4 *>(S.sel2)[(tid + kCThreads * i) * 4 + q] = make_uint4(v2[i], v2[i], v2[i], v2[i]);
-        reinterpret_cast<uint4 *>(S.sgn2)[tid * 4 + q] = make_uint4(vs, vs, vs, vs);
-      }
-#pragma unroll
-      for (int i = 0; i < 16; ++i) reinterpret_cast<uint2 *>(S.sel1)[tid + kCThreads * i] = make_uint2(v1[i], v1[i]);
-      consumers_sync();
+      replicate_tables<kCThreads, 1>(S, tid);
     }
     // ---- consumers: activations to limbs (locally, or phase 0 cooperative)
     if (local_x) {
@@ -949,15 +979,16 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(FusedArgs a)
       const int s = k % kRing;
       if (k == my1) {
         TRACE(4);
-        // end of the gate/up items: zero a slice of out, then the grid barrier
-        const size_t total4 = (size_t)T * H / 4;
-        const size_t z0 = total4 * cta / G, z1 = total4 * (cta + 1) / G;
-        for (size_t i = z0 + tid; i < z1; i += kCThreads)
-          reinterpret_cast<float4 *>(a.out)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-        consumers_sync();
+        // grid barrier: every CTA has written its g/u (it arrived when its
+        // last gate/up item was reduced) and zeroed its slice of out
+        if (my1 == 0) {
+          consumers_sync();  // this CTA's zero stores precede the arrival
+          if (tid == 0) {
+            __threadfence();
+            atomicAdd(&ctrl->phase1_done, 1);
+          }
+        }
         if (tid == 0) {
-          __threadfence();
-          atomicAdd(&ctrl->phase1_done, 1);
           uint32_t it = 0;
           while (ld_acquire(&ctrl->phase1_done) < G) {
             if (++it > kSpinLimit) {
@@ -1032,11 +1063,11 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(FusedArgs a)
         lst = lstrideX;
         kb = warp * 256;
       } else {
-        const int nkb = F / 256, it = item_tiles_of(F);
+        const int nkb = F >> 8, it = item_tiles_of(F);
         const int tiles = min(it, H / 16 - inf.tile * it);
         nw = tiles * nkb;  // <= 8: warp w takes tile w / nkb, input block w % nkb
         lst = F + kLimbPad;
-        kb = (warp % nkb) * 256;
+        kb = ((nkb & (nkb - 1)) == 0 ? (warp & (nkb - 1)) : warp % nkb) * 256;
       }
 #ifdef REDLITE_TRACE
       const long long c0 = clock64();
@@ -1065,17 +1096,29 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(FusedArgs a)
             const float sc = S.tok_scale[(slot4 >> (2 * j)) & 3];
             gu[(size_t)(pbase + j) * 2 * a.max_ffn + (size_t)inf.sub * a.max_ffn + inf.tile * 16 + row] = v * sc;
           }
+          if (k == my1 - 1) {
+            // this CTA's last gate/up item: arrive at the grid barrier (the
+            // fence is cumulative over the warp's and, through the earlier
+            // block barriers, the CTA's stores)
+            __syncwarp();
+            if (lane == 0) {
+              __threadfence();
+              atomicAdd(&ctrl->phase1_done, 1);
+            }
+          }
         } else {
-          const int nkb = F / 256, it = item_tiles_of(F);
-          const int tiles = nw / nkb;
-          for (int j2 = lane; j2 < tiles * 16 * ntok; j2 += 32) {
-            const int j = j2 % ntok, rt = j2 / ntok;
-            const int tile = rt >> 4, row = rt & 15;
-            float v = 0.f;
-            for (int kb = 0; kb < nkb; ++kb) v += red[(tile * nkb + kb) * 64 + row * 4 + j];
-            const int r = (inf.tile * it + tile) * 16 + row;
-            atomicAdd(a.out + (size_t)S.pair_tok[pbase + j] * H + r,
-                      S.pair_w[pbase + j] * (v * S.tok_scale[(slot4 >> (2 * j)) & 3]));
+          const int nkb = F >> 8, it = item_tiles_of(F);
+          const int tiles = min(it, H / 16 - inf.tile * it);
+          const int r0 = inf.tile * it * 16;
+          for (int j = 0; j < ntok; ++j) {
+            float *orow = a.out + (size_t)S.pair_tok[pbase + j] * H + r0;
+            const float wj = S.pair_w[pbase + j] * S.tok_scale[(slot4 >> (2 * j)) & 3];
+            for (int rt = lane; rt < tiles * 16; rt += 32) {  // rt = 16 tile + row
+              const float *rp = red + (rt >> 4) * nkb * 64 + (rt & 15) * 4 + j;
+              float v = 0.f;
+              for (int kb = 0; kb < nkb; ++kb) v += rp[kb * 64];
+              atomicAdd(orow + rt, wj * v);
+            }
           }
         }
         __syncwarp();
@@ -1088,12 +1131,8 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(FusedArgs a)
     }
     TRACE(9);
     TRACE_FLUSH();
-    if (my1 == my_items) {
-      // no down items: still zero the slice and count at the barrier
-      const size_t total4 = (size_t)T * H / 4;
-      const size_t z0 = total4 * cta / G, z1 = total4 * (cta + 1) / G;
-      for (size_t i = z0 + tid; i < z1; i += kCThreads)
-        reinterpret_cast<float4 *>(a.out)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+    if (my_items == 0) {
+      // no items at all: still count at the barrier (the zero stores first)
       consumers_sync();
       if (tid == 0) {
         __threadfence();
