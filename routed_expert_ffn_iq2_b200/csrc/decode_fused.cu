@@ -444,19 +444,21 @@ __device__ __forceinline__ void warp_tile_block(int qtype, const uint8_t *tb, co
 // lstride, scale_out[j] = 2^(e_j - 20) with 2^e_j > max |vector j|.  With
 // up_off == 0 vector j is src + j * src_stride; otherwise it is SiLU(g) * u
 // with g = src + j * src_stride and u = g + up_off.  Consumer thread tid
-// holds float4 number tid + kCThreads * i (i < 2) of every vector.  Out of
+// holds float4 number t + nt * i (i < 3) of every vector.  Out of
 // line and compact: it runs a few times per call, and the kernel's hot loop
-// must stay in the instruction cache.  Two consumer-only syncs.
+// must stay in the instruction cache.  Threads t = 0..nt-1 (nt >= 176, a
+// multiple of 32) take part, with two syncs on named barrier `bar`.
 __device__ __noinline__ void limbs_from_global(int nvec, int n, const float *src, size_t src_stride, int up_off,
-                                               uint8_t *dst, int lstride, float *wmax, float *scale_out) {
-  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+                                               uint8_t *dst, int lstride, float *wmax, float *scale_out, int t,
+                                               int nt, int bar) {
+  const int warp = t >> 5, lane = t & 31;
   const int per = n / 4;
-  float4 v[4][2];
+  float4 v[4][3];
 #pragma unroll
   for (int j = 0; j < 4; ++j)
 #pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      const int e4 = tid + kCThreads * i;
+    for (int i = 0; i < 3; ++i) {
+      const int e4 = t + nt * i;
       v[j][i] = make_float4(0.f, 0.f, 0.f, 0.f);
       if (j < nvec && e4 < per) {
         const float *g = src + (size_t)j * src_stride;
@@ -472,24 +474,26 @@ __device__ __noinline__ void limbs_from_global(int nvec, int n, const float *src
   for (int j = 0; j < 4; ++j) {
     float m = 0.f;
 #pragma unroll
-    for (int i = 0; i < 2; ++i)
+    for (int i = 0; i < 3; ++i)
       m = fmaxf(m, fmaxf(fmaxf(fabsf(v[j][i].x), fabsf(v[j][i].y)), fmaxf(fabsf(v[j][i].z), fabsf(v[j][i].w))));
 #pragma unroll
     for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
     if (lane == 0) wmax[warp * 4 + j] = m;
   }
-  consumers_sync();
+  asm volatile("bar.sync %0, %1;" ::"r"(bar), "r"(nt) : "memory");
+  const int nw = nt >> 5;
 #pragma unroll 1
   for (int j = 0; j < nvec; ++j) {
     float mm = 0.f;
 #pragma unroll
-    for (int w = 0; w < kCWarps; ++w) mm = fmaxf(mm, wmax[w * 4 + j]);
+    for (int w = 0; w < kCWarps; ++w)
+      if (w < nw) mm = fmaxf(mm, wmax[w * 4 + j]);
     const int e = pow2_above(mm);
     const float sc = pow2f(20 - e);
-    if (tid == 0) scale_out[j] = pow2f(e - 20);
+    if (t == 0) scale_out[j] = pow2f(e - 20);
 #pragma unroll
-    for (int i = 0; i < 2; ++i) {
-      const int e4 = tid + kCThreads * i;
+    for (int i = 0; i < 3; ++i) {
+      const int e4 = t + nt * i;
       if (e4 < per) {
         float4 f = v[0][i];
 #pragma unroll
@@ -512,7 +516,7 @@ __device__ __noinline__ void limbs_from_global(int nvec, int n, const float *src
       }
     }
   }
-  consumers_sync();
+  asm volatile("bar.sync %0, %1;" ::"r"(bar), "r"(nt) : "memory");
 }
 
 // Replicate the selector tables in place (word w of a table with r replicas
@@ -639,6 +643,7 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(FusedArgs a)
     bulk_g2s(S.sgn2, a.grids + kGridSign, 256 * 4, &s_lut_bar);
     bulk_g2s(S.sel1, a.grids + kGridQ1Sel, 4096 * 4, &s_lut_bar);
   }
+  __syncthreads();  // the mbarriers are initialised before anyone waits on them
   // the call's own inputs may come from the previous kernel
   asm volatile("griddepcontrol.wait;" ::: "memory");
   int my_ids[3];
@@ -747,11 +752,19 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(FusedArgs a)
       if (lane == 0) s_bad = bad;
       __syncwarp();
       item_prefix(n_inst);
+      TRACE(2);
+      asm volatile("bar.arrive 3, %0;" ::"n"(64) : "memory");  // the routing is published to the producer
     } else if (warp < kCWarps) {
-      // the other consumer warps replicate the selector tables meanwhile
+      // meanwhile the other consumer warps replicate the selector tables and
+      // turn the (<= 4) tokens' activations into limbs
       if (!mbar_wait(&s_lut_bar, 0) && lane == 0) atomicOr(a.status, REDLITE_STATUS_TIMEOUT);
       TRACE(13);
       replicate_tables<kCThreads - 32, 2>(S, tid - 32);
+      if (local_x)
+        limbs_from_global(T, H, a.x, (size_t)H, 0, S.limbs, lstrideX, S.wmax, S.tok_scale, tid - 32, kCThreads - 32,
+                          2);
+    } else {
+      asm volatile("bar.sync 3, %0;" ::"n"(64) : "memory");  // the producer waits for the routing only
     }
   } else {
     // ---- bucketing: counts per expert in the ring (scratch before any copy)
@@ -873,22 +886,29 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(FusedArgs a)
     if (bad) atomicOr(&s_bad, bad);
     __syncthreads();
     if (warp == 0) item_prefix(n_inst);
+    // the ring's bucketing scratch is overwritten by bulk copies next
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+    __syncthreads();
+    TRACE(2);
   }
-  // the ring's bucketing scratch is overwritten by bulk copies next
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-  __syncthreads();
-  TRACE(2);
-  const int n_inst = s_n_inst, N1 = s_n1, N2 = s_n2;
   // gate/up items split evenly over the CTAs; down items in reverse CTA order
-  // (a CTA with one more gate/up item tends to get one fewer down item)
-  const unsigned uG = (unsigned)G, uN1 = (unsigned)N1, uN2 = (unsigned)N2;  // products < 2^31
-  const int b1 = (int)(cta * uN1 / uG), e1i = (int)((cta + 1) * uN1 / uG);
-  const int rc = G - 1 - cta;
-  const int b2 = (int)(rc * uN2 / uG), e2i = (int)((rc + 1) * uN2 / uG);
-  const int my1 = e1i - b1, my2 = e2i - b2, my_items = my1 + my2;
+  // (a CTA with one more gate/up item tends to get one fewer down item).
+  // Read once the routing is visible to the reading thread.
+  const unsigned uG = (unsigned)G;
+  int n_inst = 0, N1 = 0, N2 = 0, b1 = 0, b2 = 0, my1 = 0, my_items = 0;
+  auto load_split = [&]() {
+    n_inst = s_n_inst, N1 = s_n1, N2 = s_n2;
+    const unsigned uN1 = (unsigned)N1, uN2 = (unsigned)N2;  // products < 2^31
+    b1 = (int)(cta * uN1 / uG);
+    const int e1i = (int)((cta + 1) * uN1 / uG), rc = G - 1 - cta;
+    b2 = (int)(rc * uN2 / uG);
+    const int e2i = (int)((rc + 1) * uN2 / uG);
+    my1 = e1i - b1, my_items = my1 + (e2i - b2);
+  };
 
   // ---- producer warp: streams this CTA's items through the ring
   if (warp == kCWarps) {
+    load_split();
     if (lane == 0) {
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // generic writes before bulk copies
       for (int k = 0; k < my_items; ++k) {
@@ -947,11 +967,12 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(FusedArgs a)
     // ---- consumers: activations to limbs (locally, or phase 0 cooperative)
     if (local_x) {
       TRACE(12);
-      limbs_from_global(T, H, a.x, (size_t)H, 0, S.limbs, lstrideX, S.wmax, S.tok_scale);
+      if (npairs > 32)
+        limbs_from_global(T, H, a.x, (size_t)H, 0, S.limbs, lstrideX, S.wmax, S.tok_scale, tid, kCThreads, 1);
     } else {
       for (int t = cta; t < T; t += G)
         limbs_from_global(1, H, a.x + (size_t)t * H, 0, 0, glimbs + (size_t)t * 3 * lstrideX, lstrideX, S.wmax,
-                          gscale + t);
+                          gscale + t, tid, kCThreads, 1);
       consumers_sync();
       if (tid == 0) {
         __threadfence();
@@ -968,6 +989,8 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(FusedArgs a)
       }
       consumers_sync();
     }
+    consumers_sync();  // small calls: warp 0's routing and the other warps' limbs are done
+    load_split();
     TRACE(3);
 
     // ---- main loop over this CTA's items
@@ -1051,7 +1074,7 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(FusedArgs a)
           // h = SiLU(g) * u of the chunk's tokens, then its limbs
           consumers_sync();  // every warp is done with the previous limbs
           limbs_from_global(ntok, F, gu + (size_t)pbase * 2 * a.max_ffn, (size_t)2 * a.max_ffn, a.max_ffn, S.limbs,
-                            F + kLimbPad, S.wmax, S.tok_scale);
+                            F + kLimbPad, S.wmax, S.tok_scale, tid, kCThreads, 1);
         }
       }
       TRACE_ADD(inf.phase == 1, 2, 3);
