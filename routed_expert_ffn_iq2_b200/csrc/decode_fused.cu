@@ -51,6 +51,7 @@ constexpr int kRep1 = 2;   // replicas of the IQ1 selector table
 constexpr int kLimbPad = 32;  // padding per limb plane (spreads shared-memory banks)
 constexpr uint32_t kSpinLimit = 1u << 24;
 
+
 // 8-byte tables the selector nibbles index: IQ2 +8,+25,+43,0,-8,-25,-43,0;
 // IQ1 (delta +1/8) -7,1,9,0 and (delta -1/8) -9,-1,7,0, all scaled by 8.
 constexpr uint32_t kQ2Pos = 0x002B1908u, kQ2Neg = 0x00D5E7F8u;
@@ -130,6 +131,29 @@ __device__ __forceinline__ int ld_acquire(const int *p) {
   int v;
   asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
   return v;
+}
+
+constexpr uint64_t kGridWaitNs = 1000000000ull;  // a grid-wide wait gives up after 1 s
+
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+// Spin until *counter >= target; false (and the TIMEOUT status bit) if that
+// takes longer than kGridWaitNs.  One thread per CTA calls it.
+__device__ __noinline__ bool wait_count(const int *counter, int target, int32_t *status) {
+  const uint64_t t_end = global_ns() + kGridWaitNs;
+  while (ld_acquire(counter) < target) {
+    if (global_ns() > t_end) {
+      atomicOr(status, REDLITE_STATUS_TIMEOUT);
+      return false;
+    }
+    __nanosleep(32);
+  }
+  __threadfence();
+  return true;
 }
 
 // named barrier over the consumer warps only
@@ -977,15 +1001,7 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(FusedArgs a)
       if (tid == 0) {
         __threadfence();
         atomicAdd(&ctrl->phase0_done, 1);
-        uint32_t it = 0;
-        while (ld_acquire(&ctrl->phase0_done) < G) {
-          if (++it > kSpinLimit) {
-            atomicOr(a.status, REDLITE_STATUS_TIMEOUT);
-            break;
-          }
-          __nanosleep(64);
-        }
-        __threadfence();
+        wait_count(&ctrl->phase0_done, G, a.status);
       }
       consumers_sync();
     }
@@ -1011,17 +1027,7 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(FusedArgs a)
             atomicAdd(&ctrl->phase1_done, 1);
           }
         }
-        if (tid == 0) {
-          uint32_t it = 0;
-          while (ld_acquire(&ctrl->phase1_done) < G) {
-            if (++it > kSpinLimit) {
-              atomicOr(a.status, REDLITE_STATUS_TIMEOUT);
-              break;
-            }
-            __nanosleep(32);
-          }
-          __threadfence();
-        }
+        if (tid == 0) wait_count(&ctrl->phase1_done, G, a.status);
         consumers_sync();
         TRACE(5);
       }

@@ -278,3 +278,23 @@ def test_tensor_core_path_matches_bf16_operand_reference(P, oracle_lib):
     if sh is not None:
         run_expert(sh, np.arange(T), np.ones(T))
     assert _rel_err(got, ref) <= 1e-3
+
+
+def test_grid_wait_gives_up_and_reports(P):
+    """A grid-wide wait that can never be met (the gate/up barrier counter is
+    corrupted from the host) gives up after its time limit, sets
+    REDLITE_STATUS_TIMEOUT, and leaves the context and the workspace usable:
+    the next call returns the right result with a clean status."""
+    w = fixtures.workload(2)
+    L = P.layer_for_workload(w)
+    ref = _run(L, w.x, w.ids, w.weights)
+    assert L.read_status() == 0
+    ctrl = L.workspace.view(torch.int32)
+    ctrl[4] = -(1 << 30)  # control word 4: CTAs past their gate/up items
+    torch.cuda.synchronize()
+    _run(L, w.x, w.ids, w.weights)
+    assert L.read_status() & P.REDLITE_STATUS_TIMEOUT
+    L.clear_status()
+    again = _run(L, w.x, w.ids, w.weights)
+    assert L.read_status() == 0
+    assert _rel_err(again, ref) <= 1e-6
