@@ -88,6 +88,36 @@ struct Smem {
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
 
+// Shared-memory loads by 32-bit shared address (never generic).  The
+// volatile forms read data that other threads or the bulk copies write (kept
+// in program order); the plain form reads the selector tables, which nobody
+// writes after the setup.
+__device__ __forceinline__ uint32_t lds_b32(uint32_t a) {
+  uint32_t v;
+  asm volatile("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ uint32_t lds_table(uint32_t a) {
+  uint32_t v;
+  asm("ld.shared.b32 %0, [%1];" : "=r"(v) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ uint32_t lds_b16(uint32_t a) {
+  uint16_t v;
+  asm volatile("ld.shared.b16 %0, [%1];" : "=h"(v) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ uint2 lds_v2(uint32_t a) {
+  uint2 v;
+  asm volatile("ld.shared.v2.b32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "r"(a));
+  return v;
+}
+__device__ __forceinline__ uint4 lds_v4(uint32_t a) {
+  uint4 v;
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w) : "r"(a));
+  return v;
+}
+
 __device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
   asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
 }
@@ -248,17 +278,19 @@ __device__ __forceinline__ void to_limbs(float v, float scale, int &l0, int &l1,
 //
 // Column n of the mma B operand (n = lane >> 2 of the lane holding it) is
 // limb n % 3 of token position 2p + n / 3 of the chunk (n < 6); columns 6
-// and 7 are zero.  Each lane gets, per token pair p, a pointer to the limb
-// plane it reads (nullptr: a zero column).  Limb planes are int8 vectors.
+// and 7 are zero.  Each lane gets, per token pair p, the shared address of
+// the limb plane it reads and whether its column is used.  Limb planes are
+// int8 vectors.
 template <int NP>
-__device__ __forceinline__ void b_planes(const uint8_t *limbs, int lstride, int slot4, int ntok,
-                                         const uint8_t *bp[NP]) {
+__device__ __forceinline__ void b_planes(uint32_t limbs, int lstride, int slot4, int ntok, uint32_t bp[NP],
+                                         bool bv[NP]) {
   const int n = (threadIdx.x & 31) >> 2;
 #pragma unroll
   for (int p = 0; p < NP; ++p) {
     const int pos = 2 * p + n / 3;
     const int slot = (slot4 >> (2 * pos)) & 3;
-    bp[p] = (n < 6 && pos < ntok) ? limbs + (size_t)(slot * 3 + n % 3) * lstride : nullptr;
+    bv[p] = n < 6 && pos < ntok;
+    bp[p] = limbs + (uint32_t)((slot * 3 + n % 3) * lstride);
   }
 }
 
@@ -270,19 +302,16 @@ __device__ __forceinline__ void b_planes(const uint8_t *limbs, int lstride, int 
 // two multiply-adds for the table offsets (entry stride 64 bytes = 16
 // replicas), two table loads, one OR, two byte permutes and one shift.
 template <int NP>
-__device__ __forceinline__ void tb_q2(const uint8_t *__restrict__ tb, const uint32_t *__restrict__ sel2,
-                                      const uint32_t *__restrict__ sgn2, const uint8_t *const bp[NP], int kbase,
-                                      float acc[NP][4]) {
+__device__ __forceinline__ void tb_q2(uint32_t tb, uint32_t g2, uint32_t gs, const uint32_t bp[NP],
+                                      const bool bv[NP], int kbase, float acc[NP][4]) {
   static_assert(kRep2 == 16, "table offsets below assume 16 replicas (64-byte entries)");
   const int lane = threadIdx.x & 31, q = lane >> 2, t = lane & 3;
   const uint32_t r4 = (uint32_t)(lane & 15) << 2;
-  const uint8_t *g2 = reinterpret_cast<const uint8_t *>(sel2);
-  const uint8_t *gs = reinterpret_cast<const uint8_t *>(sgn2);
-  const uint4 qs = *reinterpret_cast<const uint4 *>(tb + 32 * lane);
-  const uint4 sg = *reinterpret_cast<const uint4 *>(tb + 32 * lane + 16);
-  const uint32_t qh14 = (uint32_t)(*reinterpret_cast<const uint16_t *>(tb + 1024 + 2 * lane)) << 14;
-  const uint2 scw = *reinterpret_cast<const uint2 *>(tb + 1088 + 8 * q);
-  const uint32_t dw = *reinterpret_cast<const uint32_t *>(tb + 1152 + 4 * q);
+  const uint4 qs = lds_v4(tb + 32 * lane);
+  const uint4 sg = lds_v4(tb + 32 * lane + 16);
+  const uint32_t qh14 = lds_b16(tb + 1024 + 2 * lane) << 14;
+  const uint2 scw = lds_v2(tb + 1088 + 8 * q);
+  const uint32_t dw = lds_b32(tb + 1152 + 4 * q);
   const uint32_t qsw[4] = {qs.x, qs.y, qs.z, qs.w};
   const uint32_t sgw[4] = {sg.x, sg.y, sg.z, sg.w};
   uint32_t sel[16];  // field i = 2c + h
@@ -293,14 +322,14 @@ __device__ __forceinline__ void tb_q2(const uint8_t *__restrict__ tb, const uint
     const uint32_t hi = ((qh14 >> i) & 0x4000u) | r4;  // index bit 8, times 64, plus replica
     const uint32_t go = qsb * 64u + hi;
     const uint32_t so = sgb * 64u + r4;
-    sel[i] = *reinterpret_cast<const uint32_t *>(g2 + go) | *reinterpret_cast<const uint32_t *>(gs + so);
+    sel[i] = lds_table(g2 + go) | lds_table(gs + so);
   }
   uint2 b[NP][8];
 #pragma unroll
   for (int p = 0; p < NP; ++p)
 #pragma unroll
     for (int c = 0; c < 8; ++c)
-      b[p][c] = bp[p] ? *reinterpret_cast<const uint2 *>(bp[p] + kbase + 32 * c + 8 * t) : make_uint2(0u, 0u);
+      b[p][c] = bv[p] ? lds_v2(bp[p] + kbase + 32 * c + 8 * t) : make_uint2(0u, 0u);
   // sub-block multipliers 2sc+1 as bytes: chunk c is byte c >> 1 of the even
   // (c even) or odd (c odd) nibble word of its row
   const uint32_t me0 = ((scw.x & 0x0F0F0F0Fu) << 1) | 0x01010101u, mo0 = ((scw.x >> 3) & 0x1E1E1E1Eu) | 0x01010101u;
@@ -340,18 +369,17 @@ __device__ __forceinline__ void tb_q2(const uint8_t *__restrict__ tb, const uint
 // IQ1_M-style tile-block: one k16 mma per 16-weight sub-block; lane t holds
 // weights 4t..4t+3 of the sub-block (half of group 2s + (t >> 1)).
 template <int NP>
-__device__ __forceinline__ void tb_q1(const uint8_t *__restrict__ tb, const uint32_t *__restrict__ sel1,
-                                      const uint8_t *const bp[NP], int kbase, float acc[NP][4]) {
+__device__ __forceinline__ void tb_q1(uint32_t tb, uint32_t sel1, const uint32_t bp[NP], const bool bv[NP],
+                                      int kbase, float acc[NP][4]) {
   const int lane = threadIdx.x & 31, q = lane >> 2, t = lane & 3, r = lane & (kRep1 - 1);
-  const uint8_t *pb = tb + 48 * (2 * q + (t >> 1));
-  const uint4 qa = *reinterpret_cast<const uint4 *>(pb);
-  const uint4 qb = *reinterpret_cast<const uint4 *>(pb + 16);
-  const uint4 nb = *reinterpret_cast<const uint4 *>(pb + 32);
-  const uint32_t *scp = reinterpret_cast<const uint32_t *>(tb + 768 + 12 * q);
-  const uint32_t s0 = scp[0], s1 = scp[1], s2 = scp[2];
+  const uint32_t pb = tb + 48 * (2 * q + (t >> 1));
+  const uint4 qa = lds_v4(pb);
+  const uint4 qb = lds_v4(pb + 16);
+  const uint4 nb = lds_v4(pb + 32);
+  const uint32_t s0 = lds_b32(tb + 768 + 12 * q), s1 = lds_b32(tb + 772 + 12 * q), s2 = lds_b32(tb + 776 + 12 * q);
   const uint64_t row0 = (uint64_t)s0 | ((uint64_t)(s1 & 0xFFFFu) << 32);
   const uint64_t row1 = (uint64_t)(s1 >> 16) | ((uint64_t)s2 << 16);
-  const uint32_t dw = *reinterpret_cast<const uint32_t *>(tb + 864 + 4 * q);
+  const uint32_t dw = lds_b32(tb + 864 + 4 * q);
   const int hshift = 16 * (t & 1);
   const uint32_t qsw[8] = {qa.x, qa.y, qa.z, qa.w, qb.x, qb.y, qb.z, qb.w};
   const uint32_t nbw[4] = {nb.x, nb.y, nb.z, nb.w};
@@ -360,13 +388,13 @@ __device__ __forceinline__ void tb_q1(const uint8_t *__restrict__ tb, const uint
   for (int i = 0; i < 32; ++i) {
     const uint32_t qsb = (qsw[i >> 2] >> (8 * (i & 3))) & 0xFFu;
     const uint32_t nib = (nbw[i >> 3] >> (4 * (i & 7))) & 0xFu;
-    sel[i] = sel1[(qsb | (nib << 8)) * kRep1 + r] >> hshift;
+    sel[i] = lds_table(sel1 + 4 * ((qsb | (nib << 8)) * kRep1 + r)) >> hshift;
   }
   uint32_t b[NP][16];
 #pragma unroll
   for (int p = 0; p < NP; ++p)
 #pragma unroll
-    for (int s = 0; s < 16; ++s) b[p][s] = bp[p] ? *reinterpret_cast<const uint32_t *>(bp[p] + kbase + 16 * s + 4 * t) : 0u;
+    for (int s = 0; s < 16; ++s) b[p][s] = bv[p] ? lds_b32(bp[p] + kbase + 16 * s + 4 * t) : 0u;
   int32_t cb[NP][4];
 #pragma unroll
   for (int p = 0; p < NP; ++p) cb[p][0] = cb[p][1] = cb[p][2] = cb[p][3] = 0;
@@ -428,36 +456,42 @@ __device__ __forceinline__ void store_partials(const float acc[NP][4], float *re
 
 // One tile-block of either format for 1-2 (NP = 1) or 3-4 (NP = 2) token
 // positions; the warp's partials go to red (16 x 4 floats).  Inlined at one
-// call site so the table and stage pointers keep their shared-memory
-// provenance (shared loads, not generic loads).
-__device__ __forceinline__ void warp_tile_block(int qtype, const uint8_t *tb, const Smem &S, const uint8_t *limbs,
+// call site.
+__device__ __forceinline__ void warp_tile_block(int qtype, const uint8_t *tb_p, const Smem &S, const uint8_t *limbs_p,
                                                 int lstride, int kbase, int slot4, int ntok, float *red) {
+  const uint32_t tb = smem_u32(tb_p), limbs = smem_u32(limbs_p);
   if (qtype == kQ2) {
+    const uint32_t g2 = smem_u32(S.sel2), gs = smem_u32(S.sgn2);
     if (ntok <= 2) {
-      const uint8_t *bp[1];
-      b_planes<1>(limbs, lstride, slot4, ntok, bp);
+      uint32_t bp[1];
+      bool bv[1];
+      b_planes<1>(limbs, lstride, slot4, ntok, bp, bv);
       float acc[1][4] = {{0.f, 0.f, 0.f, 0.f}};
-      tb_q2<1>(tb, S.sel2, S.sgn2, bp, kbase, acc);
+      tb_q2<1>(tb, g2, gs, bp, bv, kbase, acc);
       store_partials<1>(acc, red);
     } else {
-      const uint8_t *bp[2];
-      b_planes<2>(limbs, lstride, slot4, ntok, bp);
+      uint32_t bp[2];
+      bool bv[2];
+      b_planes<2>(limbs, lstride, slot4, ntok, bp, bv);
       float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-      tb_q2<2>(tb, S.sel2, S.sgn2, bp, kbase, acc);
+      tb_q2<2>(tb, g2, gs, bp, bv, kbase, acc);
       store_partials<2>(acc, red);
     }
   } else {
+    const uint32_t g1 = smem_u32(S.sel1);
     if (ntok <= 2) {
-      const uint8_t *bp[1];
-      b_planes<1>(limbs, lstride, slot4, ntok, bp);
+      uint32_t bp[1];
+      bool bv[1];
+      b_planes<1>(limbs, lstride, slot4, ntok, bp, bv);
       float acc[1][4] = {{0.f, 0.f, 0.f, 0.f}};
-      tb_q1<1>(tb, S.sel1, bp, kbase, acc);
+      tb_q1<1>(tb, g1, bp, bv, kbase, acc);
       store_partials<1>(acc, red);
     } else {
-      const uint8_t *bp[2];
-      b_planes<2>(limbs, lstride, slot4, ntok, bp);
+      uint32_t bp[2];
+      bool bv[2];
+      b_planes<2>(limbs, lstride, slot4, ntok, bp, bv);
       float acc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
-      tb_q1<2>(tb, S.sel1, bp, kbase, acc);
+      tb_q1<2>(tb, g1, bp, bv, kbase, acc);
       store_partials<2>(acc, red);
     }
   }
