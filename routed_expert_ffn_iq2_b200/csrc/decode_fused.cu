@@ -78,7 +78,7 @@ struct Smem {
   int *pair_tok;
   float *pair_w;
   uint64_t *full, *empty;
-  int *done;  // per stage: consumer warps finished
+  uint64_t *pdone;  // per stage: all consumer warps' partials are in red (mbarrier, 8 arrivals)
   ItemInfo *info;
   float *tok_scale;  // per token slot: 2^(e - 20)
   float *wmax;       // [kCWarps][4] partial maxima
@@ -171,6 +171,13 @@ __device__ __forceinline__ uint64_t global_ns() {
   return t;
 }
 
+// counter += 1 with release semantics at GPU scope: every write that
+// happens before it (this thread's, and through block barriers or warp syncs
+// the block's) is visible to a thread that acquires the new value.
+__device__ __forceinline__ void arrive_release(int *counter) {
+  asm volatile("red.release.gpu.global.add.s32 [%0], 1;" ::"l"(counter) : "memory");
+}
+
 // Spin until *counter >= target; false (and the TIMEOUT status bit) if that
 // takes longer than kGridWaitNs.  One thread per CTA calls it.
 __device__ __noinline__ bool wait_count(const int *counter, int target, int32_t *status) {
@@ -182,8 +189,7 @@ __device__ __noinline__ bool wait_count(const int *counter, int target, int32_t 
     }
     __nanosleep(32);
   }
-  __threadfence();
-  return true;
+  return true;  // the acquiring load orders what follows
 }
 
 // named barrier over the consumer warps only
@@ -667,8 +673,8 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(FusedArgs a)
   off += sizeof(uint64_t) * kRing;
   S.empty = reinterpret_cast<uint64_t *>(smem + off);
   off += sizeof(uint64_t) * kRing;
-  S.done = reinterpret_cast<int *>(smem + off);
-  off += sizeof(int) * kRing;
+  S.pdone = reinterpret_cast<uint64_t *>(smem + off);
+  off += sizeof(uint64_t) * kRing;
   S.info = reinterpret_cast<ItemInfo *>(smem + off);
   off += sizeof(ItemInfo) * kRing;
   S.tok_scale = reinterpret_cast<float *>(smem + off);
@@ -689,7 +695,7 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(FusedArgs a)
     for (int s = 0; s < kRing; ++s) {
       mbar_init(&S.full[s], 1);
       mbar_init(&S.empty[s], 1);
-      S.done[s] = 0;
+      mbar_init(&S.pdone[s], kCWarps);
     }
     mbar_init(&s_lut_bar, 1);
     mbar_fence_init();
@@ -813,14 +819,15 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(FusedArgs a)
       TRACE(2);
       asm volatile("bar.arrive 3, %0;" ::"n"(64) : "memory");  // the routing is published to the producer
     } else if (warp < kCWarps) {
-      // meanwhile the other consumer warps replicate the selector tables and
-      // turn the (<= 4) tokens' activations into limbs
-      if (!mbar_wait(&s_lut_bar, 0) && lane == 0) atomicOr(a.status, REDLITE_STATUS_TIMEOUT);
-      TRACE(13);
-      replicate_tables<kCThreads - 32, 2>(S, tid - 32);
+      // meanwhile the other consumer warps turn the (<= 4) tokens'
+      // activations into limbs and then (the bulk copy has had time to land)
+      // replicate the selector tables
       if (local_x)
         limbs_from_global(T, H, a.x, (size_t)H, 0, S.limbs, lstrideX, S.wmax, S.tok_scale, tid - 32, kCThreads - 32,
                           2);
+      if (!mbar_wait(&s_lut_bar, 0) && lane == 0) atomicOr(a.status, REDLITE_STATUS_TIMEOUT);
+      TRACE(13);
+      replicate_tables<kCThreads - 32, 2>(S, tid - 32);
     } else {
       asm volatile("bar.sync 3, %0;" ::"n"(64) : "memory");  // the producer waits for the routing only
     }
@@ -1033,8 +1040,7 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(FusedArgs a)
                           gscale + t, tid, kCThreads, 1);
       consumers_sync();
       if (tid == 0) {
-        __threadfence();
-        atomicAdd(&ctrl->phase0_done, 1);
+        arrive_release(&ctrl->phase0_done);
         wait_count(&ctrl->phase0_done, G, a.status);
       }
       consumers_sync();
@@ -1057,8 +1063,7 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(FusedArgs a)
         if (my1 == 0) {
           consumers_sync();  // this CTA's zero stores precede the arrival
           if (tid == 0) {
-            __threadfence();
-            atomicAdd(&ctrl->phase1_done, 1);
+            arrive_release(&ctrl->phase1_done);
           }
         }
         if (tid == 0) wait_count(&ctrl->phase1_done, G, a.status);
@@ -1137,20 +1142,17 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(FusedArgs a)
 #endif
       if (warp < nw) warp_tile_block(qtype, stage + warp * tbb, S, S.limbs, lst, kb, slot4, ntok, red + warp * 64);
 #ifdef REDLITE_TRACE
-      if (inf.phase == 1 && k < 4 && warp < 4) TRACEC(k * 4 + warp, (uint64_t)(clock64() - c0));
+      const long long tr_tb = clock64();
 #endif
       TRACE_ADD(inf.phase == 1, 4, 5);
       TRACE_T0();
-      // the last consumer warp to finish reduces the item and frees the stage
+      // every warp announces its partials; warp k % 8 reduces the item once
+      // all are in and frees the stage (the other warps move on at once)
       __syncwarp();
-      int prev = 0;
-      if (lane == 0) {
-        __threadfence_block();
-        prev = atomicAdd(&S.done[s], 1);
-      }
-      prev = __shfl_sync(0xffffffffu, prev, 0);
-      if (prev == kCWarps - 1) {
-        __threadfence_block();
+      if (lane == 0) mbar_arrive(&S.pdone[s]);
+      if (warp == k % kCWarps) {
+        if (!mbar_wait(&S.pdone[s], (uint32_t)((k / kRing) & 1)) && lane == 0)
+          atomicOr(a.status, REDLITE_STATUS_TIMEOUT);
         if (inf.phase == 1) {
           for (int j2 = lane; j2 < 16 * ntok; j2 += 32) {
             const int row = j2 & 15, j = j2 >> 4;
@@ -1161,12 +1163,11 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(FusedArgs a)
           }
           if (k == my1 - 1) {
             // this CTA's last gate/up item: arrive at the grid barrier (the
-            // fence is cumulative over the warp's and, through the earlier
+            // release is cumulative over the warp's and, through the earlier
             // block barriers, the CTA's stores)
             __syncwarp();
             if (lane == 0) {
-              __threadfence();
-              atomicAdd(&ctrl->phase1_done, 1);
+              arrive_release(&ctrl->phase1_done);
             }
           }
         } else {
@@ -1185,12 +1186,17 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(FusedArgs a)
           }
         }
         __syncwarp();
-        if (lane == 0) {
-          S.done[s] = 0;
-          mbar_arrive(&S.empty[s]);
-        }
+        if (lane == 0) mbar_arrive(&S.empty[s]);
       }
       TRACE_ADD(inf.phase == 1, 6, 7);
+#ifdef REDLITE_TRACE
+      if (warp == 0 && k < 5) {  // tile-block start and end, item end (warp 0)
+        TRACEC(k * 3, (uint64_t)c0);
+        TRACEC(k * 3 + 1, (uint64_t)tr_tb);
+        TRACEC(k * 3 + 2, (uint64_t)clock64());
+      }
+      if (warp == 0 && k == 0) TRACEC(15, (uint64_t)my1);
+#endif
     }
     TRACE(9);
     TRACE_FLUSH();
@@ -1198,8 +1204,7 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(FusedArgs a)
       // no items at all: still count at the barrier (the zero stores first)
       consumers_sync();
       if (tid == 0) {
-        __threadfence();
-        atomicAdd(&ctrl->phase1_done, 1);
+        arrive_release(&ctrl->phase1_done);
       }
     }
   }
@@ -1227,7 +1232,7 @@ size_t fused_smem_bytes(int hidden, int max_ffn) {
   off = (off + 15) & ~size_t(15);
   off += sizeof(Inst) * kFusedMaxInst;
   off += 2 * sizeof(int) * (kFusedMaxPairs + 64);
-  off += 2 * sizeof(uint64_t) * kRing + sizeof(int) * kRing + sizeof(ItemInfo) * kRing;
+  off += 3 * sizeof(uint64_t) * kRing + sizeof(ItemInfo) * kRing;
   off += sizeof(float) * kTokChunk + sizeof(float) * kCWarps * 4;
   return off + 64;
 }
