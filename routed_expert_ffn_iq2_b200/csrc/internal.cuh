@@ -111,11 +111,12 @@ struct Ctrl {
 static_assert(sizeof(Ctrl) == 256, "ctrl block is 256 bytes");
 
 struct WorkspaceLayout {
-  size_t ctrl, active, pairs, counts, done, h, xb, gu, limbs, exps, total;
+  size_t ctrl, active, pairs, counts, hist, h, xb, gu, limbs, exps, total;
   int max_active, max_pairs;
 };
 
 // Largest (token, slot) pair count the fused decode kernel takes.
+constexpr int kRouteBlocks = 32;  // bucketing: blocks that count and place pairs
 constexpr int kFusedMaxPairs = 640;
 constexpr int kFusedMaxInst = kFusedMaxPairs + 2;  // selected experts + the shared expert, rounded up
 
@@ -135,8 +136,8 @@ inline WorkspaceLayout workspace_layout(int hidden, int n_experts, int max_token
   off = align256(off + sizeof(Pair) * (size_t)L.max_pairs);
   L.counts = off;
   off = align256(off + sizeof(int) * (size_t)(n_experts + 1));
-  L.done = off;  // per-active-expert completion counters (reserved)
-  off = align256(off + sizeof(int) * (size_t)L.max_active);
+  L.hist = off;  // bucketing: per (expert, block) pair counts, then offsets
+  off = align256(off + sizeof(int) * (size_t)kRouteBlocks * (size_t)n_experts);
   L.h = off;
   off = align256(off + sizeof(float) * (size_t)L.max_pairs * (size_t)max_ffn);
   L.xb = off;  // tensor-core path: the call's activations as bf16 [tokens][hidden]

@@ -52,7 +52,7 @@ WorkspaceLayout noalloc_layout(int hidden, int n_tokens, int top_k, int max_ffn)
   off = align256(off + (size_t)n_tokens * 3 * (size_t)(hidden + 32));
   L.exps = off;
   off = align256(off + sizeof(int) * (size_t)(n_tokens + 1));
-  L.active = L.pairs = L.counts = L.done = L.h = L.xb = off;
+  L.active = L.pairs = L.counts = L.hist = L.h = L.xb = off;
   L.total = off;
   L.max_pairs = (int)pairs;
   L.max_active = 0;

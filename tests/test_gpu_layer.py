@@ -233,6 +233,30 @@ def test_bf16_rounding_helper_matches_oracle(oracle_lib):
     assert np.array_equal(_bf16_rne(v).astype(np.float32).view(np.uint32), want)
 
 
+def test_tensor_core_path_is_repeatable(P):
+    """Three calls of the tcgen05 path on the same inputs agree up to the order
+    of the fp32 atomic additions into out (a few ulp): a read of a shared-memory
+    stage before its copies or its decode landed shows as a large difference.
+    96 tokens x top-10 over a pool of 16 experts (~60 tokens each) + shared."""
+    w = fixtures.workload(4)
+    q = np.asarray(w.qtypes)
+    pool = [int(e) for e in np.nonzero(q == 1)[0][:8]] + [int(e) for e in np.nonzero(q == 2)[0][:8]]
+    T, K = 96, 10
+    st = fixtures.Stream(5150, 3)
+    ids = np.zeros((T, K), np.int32)
+    for t in range(T):
+        ids[t] = np.array(pool)[np.argsort(st.uniform(len(pool)))[:K]]
+    wt = st.uniform(T * K).reshape(T, K).astype(np.float32) + np.float32(0.05)
+    wt = (wt / wt.sum(axis=1, keepdims=True)).astype(np.float32)
+    x = fixtures.make_x(5150, T, w.hidden)
+    L = P.layer_for_workload(w, experts=pool, max_tokens=T)
+    outs = [_run(L, x, ids, wt) for _ in range(3)]
+    assert L.read_status() == 0
+    scale = np.abs(outs[0]).max()
+    for o in outs[1:]:
+        assert np.abs(o - outs[0]).max() <= 1e-5 * scale
+
+
 def test_tensor_core_path_matches_bf16_operand_reference(P, oracle_lib):
     """72 tokens x top-10 from a pool of 12 experts (6 per format) plus the
     shared expert: the tcgen05 path against the oracle's exact weights with
