@@ -23,13 +23,10 @@
 //               accumulator buffers;
 //   warps 2-9   dequant warp w decodes tile-block w (rows 16w..16w+15) of
 //               each matrix into the A tiles of a ring of 64-input steps (3
-//               deep for gate/up, 5 for down);
+//               deep for gate/up, 5 for down) and
+//               fetches rows 16w..16w+15 of B with cp.async, a step ahead;
 //   warps 10-13 the epilogue (TMEM -> registers -> h or out), overlapping
-//               the next unit's contraction;
-//   warps 14-15 copy the B rows of every step (the unit's activations, x
-//               as bf16 or h) with cp.async; the copies' completion arrives
-//               on the step's barrier, so the tensor cores wait for both the
-//               decoded A tiles and the B rows.
+//               the next unit's contraction.
 #include "internal.cuh"
 #include "layout.cuh"
 #include "ptx.cuh"
@@ -39,10 +36,8 @@ namespace {
 
 constexpr int kDqWarps = 8;
 constexpr int kEpWarps = 4;
-constexpr int kLoadWarp = 2 + kDqWarps + kEpWarps;  // first of the B-row warps
-constexpr int kLoadWarps = 2;
-constexpr int kTcWarps = kLoadWarp + kLoadWarps;
-constexpr int kTcThreads = 32 * kTcWarps;  // 512
+constexpr int kTcWarps = 2 + kDqWarps + kEpWarps;
+constexpr int kTcThreads = 32 * kTcWarps;  // 448
 constexpr int kTile = 128 * 64 * 2;        // 16 KB: 128 rows x 64 bf16
 constexpr int kPr = 2;                     // packed columns in flight
 constexpr int kMaxUnits = 128;             // unit records per pass
@@ -76,7 +71,6 @@ struct Cfg {
   static constexpr int kStep = (kMats + 1) * kTile;         // A tiles, then the B tile
   static constexpr int kPacked = kMats * 8 * kQ2TileBlock;  // one column, largest format
   static constexpr uint32_t kBufCols = DOWN ? 128 : 256;    // TMEM columns per accumulator buffer
-  static constexpr uint32_t kBufs = 512 / kBufCols;         // accumulator buffers (all of TMEM)
 };
 
 struct Unit {
@@ -86,7 +80,7 @@ struct Unit {
 static_assert(sizeof(Unit) == 48, "unit records are 48 bytes");
 
 struct Bars {
-  uint64_t pfull[kPr], pempty[kPr], afull[8], aempty[8], accfull[4], accempty[4];
+  uint64_t pfull[kPr], pempty[kPr], afull[8], aempty[8], accfull[2], accempty[2];
 };
 
 struct Smem {
@@ -192,10 +186,7 @@ __device__ __forceinline__ Q2Lane load_q2(uint32_t tb, int lane) {
 }
 
 // Step s (inputs 64s..64s+63 of the column) of one IQ2 tile-block into rows
-// row0..row0+15 of the swizzled A tile: fields i = 4s + 2 c2 + h.  `lane` is
-// the layout lane (q, t); the warp runs it on thread q + 8 t, so the eight
-// threads of each quarter-warp store to eight different rows' swizzled
-// chunks (no bank conflicts) with the same field order.
+// row0..row0+15 of the swizzled A tile: fields i = 4s + 2 c2 + h.
 __device__ __forceinline__ void dequant_q2(const Q2Lane &L, int s, uint32_t A, int row0, uint32_t sel2,
                                            int lane) {
   const int q = lane >> 2, t = lane & 3;
@@ -203,7 +194,7 @@ __device__ __forceinline__ void dequant_q2(const Q2Lane &L, int s, uint32_t A, i
   const uint32_t sw = s == 0 ? L.sg[0] : s == 1 ? L.sg[1] : s == 2 ? L.sg[2] : L.sg[3];
 #pragma unroll
   for (int j = 0; j < 2; ++j) {
-    const int c2 = j;
+    const int c2 = j ^ (q & 1);  // odd rows take the other half first: conflict-free stores
     const int c = 2 * s + c2;
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
@@ -231,7 +222,7 @@ __device__ __forceinline__ void dequant_q2(const Q2Lane &L, int s, uint32_t A, i
 // sub-blocks 4S + 2 half + {0, 1} of step S.
 struct Q1Lane {
   uint32_t qs[4], nb[4];
-  uint64_t row0, row1;  // 3-bit sub-block scales of rows q and q+8, from sub-block 2 half
+  uint64_t row0, row1;  // 16 x 3-bit sub-block scales of rows q and q+8
   float d0, d1;
 };
 
@@ -246,17 +237,11 @@ __device__ __forceinline__ Q1Lane load_q1(uint32_t tb, int lane) {
   r.qs[1] = half ? qa.w : qa.z;
   r.qs[2] = half ? qb.y : qb.x;
   r.qs[3] = half ? qb.w : qb.z;
-  // nibble word of step S: this lane's half of it
-  r.nb[0] = half ? nb.x >> 16 : nb.x & 0xFFFFu;
-  r.nb[1] = half ? nb.y >> 16 : nb.y & 0xFFFFu;
-  r.nb[2] = half ? nb.z >> 16 : nb.z & 0xFFFFu;
-  r.nb[3] = half ? nb.w >> 16 : nb.w & 0xFFFFu;
+  r.nb[0] = nb.x, r.nb[1] = nb.y, r.nb[2] = nb.z, r.nb[3] = nb.w;
   const uint32_t s0 = ptx::lds32(tb + 768 + 12 * q), s1 = ptx::lds32(tb + 772 + 12 * q),
                  s2 = ptx::lds32(tb + 776 + 12 * q);
   r.row0 = (uint64_t)s0 | ((uint64_t)(s1 & 0xFFFFu) << 32);
   r.row1 = (uint64_t)(s1 >> 16) | ((uint64_t)s2 << 16);
-  r.row0 >>= 6 * half;  // this lane's sub-blocks are 4S + 2 half + {0, 1}
-  r.row1 >>= 6 * half;
   const uint32_t dw = ptx::lds32(tb + 864 + 4 * q);
   r.d0 = __half2float(__ushort_as_half((unsigned short)(dw & 0xFFFFu)));
   r.d1 = __half2float(__ushort_as_half((unsigned short)(dw >> 16)));
@@ -267,11 +252,12 @@ __device__ __forceinline__ void dequant_q1(const Q1Lane &L, int S, uint32_t A, i
                                            int lane) {
   const int q = lane >> 2, p = (lane >> 1) & 1, half = lane & 1;
   const uint32_t qw = S == 0 ? L.qs[0] : S == 1 ? L.qs[1] : S == 2 ? L.qs[2] : L.qs[3];
-  const uint32_t nb16 = S == 0 ? L.nb[0] : S == 1 ? L.nb[1] : S == 2 ? L.nb[2] : L.nb[3];
+  const uint32_t nw = S == 0 ? L.nb[0] : S == 1 ? L.nb[1] : S == 2 ? L.nb[2] : L.nb[3];
+  const uint32_t nb16 = half ? (nw >> 16) : (nw & 0xFFFFu);
 #pragma unroll
   for (int j = 0; j < 2; ++j) {
-    const int s2 = j;
-    const int sb = 4 * S + s2;  // sub-block 4 S + 2 half + s2 of the column, relative to the lane's first
+    const int s2 = j ^ (q & 1);            // odd rows take the other sub-block first: conflict-free stores
+    const int sb = 4 * S + 2 * half + s2;  // sub-block of 16 inputs within the column
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       const int f = 2 * s2 + h;
@@ -315,8 +301,8 @@ __global__ void __maxnreg__(128) grouped_tc_kernel(TileArgs a) {
         __ldg(reinterpret_cast<const uint4 *>(a.grids + kGridQ2Bsel) + i);
   if (tid == 0) {
     for (int i = 0; i < kPr; ++i) ptx::mbar_init(&B.pfull[i], 1), ptx::mbar_init(&B.pempty[i], kDqWarps);
-    for (int i = 0; i < C::kAr; ++i) ptx::mbar_init(&B.afull[i], kDqWarps + 32 * kLoadWarps), ptx::mbar_init(&B.aempty[i], 1);
-    for (uint32_t i = 0; i < C::kBufs; ++i) ptx::mbar_init(&B.accfull[i], 1), ptx::mbar_init(&B.accempty[i], kEpWarps);
+    for (int i = 0; i < C::kAr; ++i) ptx::mbar_init(&B.afull[i], kDqWarps), ptx::mbar_init(&B.aempty[i], 1);
+    for (int i = 0; i < 2; ++i) ptx::mbar_init(&B.accfull[i], 1), ptx::mbar_init(&B.accempty[i], kEpWarps);
     ptx::mbar_fence_init();
   }
   if (warp == 0) {
@@ -372,11 +358,10 @@ __global__ void __maxnreg__(128) grouped_tc_kernel(TileArgs a) {
       if (lane == 0) {
         for (int u = 0; u < n_this; ++u, ++ucount) {
           const Unit U = S.units[u];
-          const uint32_t buf = ucount % C::kBufs;
+          const int buf = ucount & 1;
           {
             TC_T0();
-            if (ucount >= C::kBufs && !ptx::mbar_wait_suspend(&B.accempty[buf], ((ucount / C::kBufs) - 1) & 1u))
-              bad = true;
+            if (ucount >= 2 && !ptx::mbar_wait_suspend(&B.accempty[buf], ((ucount >> 1) - 1) & 1u)) bad = true;
             TC_ADD(0);
           }
           ptx::tc_fence_after();
@@ -391,9 +376,6 @@ __global__ void __maxnreg__(128) grouped_tc_kernel(TileArgs a) {
               TC_ADD(1);
             }
             ptx::tc_fence_after();
-            // the B rows were written by cp.async (generic proxy): order them before the
-            // tensor cores' reads (async proxy); without it stale rows were read at times
-            ptx::fence_proxy_async_smem();
             const uint32_t a0 = ptx::smem_u32(S.ring + (size_t)as * C::kStep);
             // descriptors of the step's tiles; 16 more inputs = 32 bytes = 2 in the start-address field
             const uint64_t da = ptx::sdesc_k_sw128(a0), du = da + (kTile >> 4),
@@ -416,14 +398,41 @@ __global__ void __maxnreg__(128) grouped_tc_kernel(TileArgs a) {
         }
       }
     } else if (warp < 2 + kDqWarps) {
-      // ---- dequant warps: A tiles
+      // ---- dequant warps: A tiles (and this warp's 16 rows of B)
       const int w = warp - 2;
-      const int ll = ((lane & 7) << 2) | (lane >> 3);  // the layout lane this thread decodes
       const uint32_t sel2a = ptx::smem_u32(S.sel2), sel1a = ptx::smem_u32(S.sel1);
       for (int u = 0; u < n_this; ++u) {
         const Unit U = S.units[u];
         const int nkb = U.K / 256;
-        const int tbb = tile_block_bytes(U.qtype);
+        // B rows 16w + (lane >> 3) + 4i, 16-byte chunk lane & 7 of each step
+        const __nv_bfloat16 *brow[4];
+        int nb = 0;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int j = 16 * w + (lane >> 3) + 4 * i;
+          const int jj = min(j, U.n_real - 1);  // pad rows read a real row; their results are dropped
+          if (j < U.n_pad) nb = i + 1;
+          brow[i] = DOWN ? hbuf + (size_t)(U.p0 + jj) * a.max_ffn : xb + (size_t)pairs[U.p0 + jj].token * H;
+        }
+        const int tbb = tile_block_bytes(U.qtype), nsteps = 4 * nkb;
+        // B rows of local step n into ring slot `as`, as one cp.async group;
+        // issued a step ahead so the copies overlap the decode of the step before
+        auto fetch_b = [&](int n, uint32_t gstep) {
+          const int as = gstep % C::kAr;
+          {
+            TC_T0();
+            if (gstep >= (uint32_t)C::kAr && !ptx::mbar_wait_suspend(&B.aempty[as], ((gstep / C::kAr) - 1) & 1u))
+              bad = true;
+            TC_ADD(1);
+          }
+          uint8_t *bt = S.ring + (size_t)as * C::kStep + C::kMats * kTile;
+          const int k0 = 64 * n + 8 * (lane & 7);
+#pragma unroll
+          for (int i = 0; i < 4; ++i)
+            if (i < nb) cp_async16(bt + ptx::sw128_offset(16 * w + (lane >> 3) + 4 * i, 8 * (lane & 7)), brow[i] + k0);
+          asm volatile("cp.async.commit_group;" ::: "memory");
+        };
+        fetch_b(0, step);
         for (int kb = 0; kb < nkb; ++kb, ++col) {
           const int ps = col % kPr;
           {
@@ -436,72 +445,37 @@ __global__ void __maxnreg__(128) grouped_tc_kernel(TileArgs a) {
           Q1Lane l1[C::kMats];
           if (U.qtype == kQ2) {
 #pragma unroll
-            for (int m = 0; m < C::kMats; ++m) l2[m] = load_q2(pk + (m * 8 + w) * tbb, ll);
+            for (int m = 0; m < C::kMats; ++m) l2[m] = load_q2(pk + (m * 8 + w) * tbb, lane);
           } else {
 #pragma unroll
-            for (int m = 0; m < C::kMats; ++m) l1[m] = load_q1(pk + (m * 8 + w) * tbb, ll);
+            for (int m = 0; m < C::kMats; ++m) l1[m] = load_q1(pk + (m * 8 + w) * tbb, lane);
           }
           __syncwarp();
           if (lane == 0) ptx::mbar_arrive(&B.pempty[ps]);
 #pragma unroll
           for (int s = 0; s < 4; ++s, ++step) {
-            const int as = step % C::kAr;
-            {
-              TC_T0();
-              if (step >= (uint32_t)C::kAr && !ptx::mbar_wait_suspend(&B.aempty[as], ((step / C::kAr) - 1) & 1u))
-                bad = true;
-              TC_ADD(1);
-            }
+            const int n = 4 * kb + s, as = step % C::kAr;
+            const bool more = n + 1 < nsteps;
+            if (more) fetch_b(n + 1, step + 1);
             const uint32_t stg = ptx::smem_u32(S.ring) + as * C::kStep;
             TC_T0();
             if (U.qtype == kQ2) {
 #pragma unroll
-              for (int m = 0; m < C::kMats; ++m) dequant_q2(l2[m], s, stg + m * kTile, 16 * w, sel2a, ll);
+              for (int m = 0; m < C::kMats; ++m) dequant_q2(l2[m], s, stg + m * kTile, 16 * w, sel2a, lane);
             } else {
 #pragma unroll
-              for (int m = 0; m < C::kMats; ++m) dequant_q1(l1[m], s, stg + m * kTile, 16 * w, sel1a, ll);
+              for (int m = 0; m < C::kMats; ++m) dequant_q1(l1[m], s, stg + m * kTile, 16 * w, sel1a, lane);
             }
             TC_ADD(2);
+            // this step's B rows landed (the next step's may still be in flight)
+            if (more)
+              asm volatile("cp.async.wait_group 1;" ::: "memory");
+            else
+              asm volatile("cp.async.wait_group 0;" ::: "memory");
             ptx::fence_proxy_async_smem();  // generic-proxy writes -> the tensor cores
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(&B.afull[as]);
           }
-        }
-      }
-    } else if (warp >= kLoadWarp) {
-      // ---- B rows of every step: thread lt copies 16-byte chunk lt & 7 of
-      // rows (lt >> 3) + 8 i, i < 16 (row & 7 is the thread's own, so its
-      // swizzled position within a row is fixed)
-      const int lt = tid - 32 * kLoadWarp, ch = lt & 7, r8 = lt >> 3;
-      const __nv_bfloat16 *bsrc = DOWN ? hbuf : xb;
-      const size_t bstride = DOWN ? (size_t)a.max_ffn : (size_t)H;
-      const uint32_t dst0 = (uint32_t)(r8 * 128 + ((ch ^ r8) << 4));
-      static_assert(kTcTokens == 128 && kLoadWarps == 2, "16 rows per loader thread");
-      for (int u = 0; u < n_this; ++u) {
-        const Unit U = S.units[u];
-        size_t off[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int jj = min(r8 + 8 * i, U.n_real - 1);  // pad rows read a real row; their results are dropped
-          off[i] = (size_t)(DOWN ? U.p0 + jj : pairs[U.p0 + jj].token) * bstride + 8 * ch;
-        }
-        const int nsteps = U.K / 64;
-        for (int n = 0; n < nsteps; ++n, ++step) {
-          const int as = step % C::kAr;
-          {
-            TC_T0();
-            if (step >= (uint32_t)C::kAr && !ptx::mbar_wait_suspend(&B.aempty[as], ((step / C::kAr) - 1) & 1u))
-              bad = true;
-            TC_ADD(1);
-          }
-          uint8_t *bt = S.ring + (size_t)as * C::kStep + C::kMats * kTile + dst0;
-          const __nv_bfloat16 *src = bsrc + 64 * n;
-#pragma unroll
-          for (int i = 0; i < 16; ++i)
-            if (r8 + 8 * i < U.n_pad) cp_async16(bt + 1024 * i, src + off[i]);
-          // arrives on the step's barrier once this thread's copies have landed
-          asm volatile("cp.async.mbarrier.arrive.noinc.shared::cta.b64 [%0];" ::"r"(ptx::smem_u32(&B.afull[as]))
-                       : "memory");
         }
       }
     } else {
@@ -509,18 +483,10 @@ __global__ void __maxnreg__(128) grouped_tc_kernel(TileArgs a) {
       const int lq = warp & 3, row = 32 * lq + lane;
       for (int u = 0; u < n_this; ++u, ++ucount) {
         const Unit U = S.units[u];
-        const uint32_t buf = ucount % C::kBufs;
-        Pair pk[4];  // down: pairs lane + 32 k of the unit, loaded before the wait
-        if (DOWN) {
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const int jl = 32 * k + lane;
-            pk[k] = jl < U.n_real ? pairs[U.p0 + jl] : Pair{0, 0.f};
-          }
-        }
+        const int buf = ucount & 1;
         {
           TC_T0();
-          if (!ptx::mbar_wait_suspend(&B.accfull[buf], (ucount / C::kBufs) & 1u)) bad = true;
+          if (!ptx::mbar_wait_suspend(&B.accfull[buf], (ucount >> 1) & 1u)) bad = true;
           TC_ADD(0);
         }
         ptx::tc_fence_after();
@@ -532,8 +498,8 @@ __global__ void __maxnreg__(128) grouped_tc_kernel(TileArgs a) {
           ptx::tmem_ld16(d + (uint32_t)c0, d0);
           if (DOWN) {
             if ((c0 & 31) == 0) {
-              const int k = c0 >> 5;
-              pl = k == 0 ? pk[0] : k == 1 ? pk[1] : k == 2 ? pk[2] : pk[3];
+              const int jl = c0 + lane;
+              if (jl < U.n_real) pl = pairs[U.p0 + jl];
             }
             ptx::tmem_wait_ld();
 #pragma unroll
