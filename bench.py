@@ -375,7 +375,7 @@ def main():
             ach = mean_bytes / per_step_s / 1e9
             peak = peaks["hbm_gbs"]
             roof = {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak,
-                    "traffic": _traffic("decode" if P.cfg in (2, 3) else "batched"),
+                    "traffic": _traffic({2: "decode", 3: "decode_iq1"}.get(P.cfg, "batched")),
                     "peak_kind": f"{peaks['src']} HBM copy"}
         line = {
             "metric": METRIC, "value": tok_s, "unit": "tokens/s", "n_gpus": world, "steps": steps,

@@ -192,10 +192,11 @@ def redlite_moe_upload_experts(hidden: int, ids, host_experts, pool: torch.Tenso
 
 def launches_per_call(n_tokens: int, top_k: int, has_shared: bool, fast: bool = True) -> int:
     """Kernels one redlite_moe_layer call enqueues: the fused decode kernel for
-    decode-sized calls on tiled tables; otherwise bucketing, then gate/up and
-    down (tensor-core kernels on tiled tables, CUDA-core tiles otherwise)."""
+    decode-sized calls on tiled tables; otherwise bucketing (count, plan,
+    scatter), then on tiled tables the bf16 conversion of x and the gate/up and
+    down tensor-core kernels, else the gate/up and down CUDA-core tiles."""
     if n_tokens == 0:
         return 0
     if fast and n_tokens * top_k <= 640 and (not has_shared or n_tokens <= 64):
         return 1
-    return 3
+    return 6 if fast else 5
