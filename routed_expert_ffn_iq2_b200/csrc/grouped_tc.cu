@@ -186,7 +186,10 @@ __device__ __forceinline__ Q2Lane load_q2(uint32_t tb, int lane) {
 }
 
 // Step s (inputs 64s..64s+63 of the column) of one IQ2 tile-block into rows
-// row0..row0+15 of the swizzled A tile: fields i = 4s + 2 c2 + h.
+// row0..row0+15 of the swizzled A tile: fields i = 4s + 2 c2 + h.  `lane` is
+// the layout lane (q, t); the warp runs it on thread q + 8 t, so the eight
+// threads of a quarter-warp store to eight different rows (conflict-free
+// 128-bit stores in the swizzled tile) with a field order fixed at compile time.
 __device__ __forceinline__ void dequant_q2(const Q2Lane &L, int s, uint32_t A, int row0, uint32_t sel2,
                                            int lane) {
   const int q = lane >> 2, t = lane & 3;
@@ -194,7 +197,7 @@ __device__ __forceinline__ void dequant_q2(const Q2Lane &L, int s, uint32_t A, i
   const uint32_t sw = s == 0 ? L.sg[0] : s == 1 ? L.sg[1] : s == 2 ? L.sg[2] : L.sg[3];
 #pragma unroll
   for (int j = 0; j < 2; ++j) {
-    const int c2 = j ^ (q & 1);  // odd rows take the other half first: conflict-free stores
+    const int c2 = j;
     const int c = 2 * s + c2;
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
@@ -222,7 +225,7 @@ __device__ __forceinline__ void dequant_q2(const Q2Lane &L, int s, uint32_t A, i
 // sub-blocks 4S + 2 half + {0, 1} of step S.
 struct Q1Lane {
   uint32_t qs[4], nb[4];
-  uint64_t row0, row1;  // 16 x 3-bit sub-block scales of rows q and q+8
+  uint64_t row0, row1;  // 3-bit sub-block scales of rows q and q+8, from sub-block 2 half
   float d0, d1;
 };
 
@@ -237,11 +240,17 @@ __device__ __forceinline__ Q1Lane load_q1(uint32_t tb, int lane) {
   r.qs[1] = half ? qa.w : qa.z;
   r.qs[2] = half ? qb.y : qb.x;
   r.qs[3] = half ? qb.w : qb.z;
-  r.nb[0] = nb.x, r.nb[1] = nb.y, r.nb[2] = nb.z, r.nb[3] = nb.w;
+  // nibble word of step S: this lane's half of it
+  r.nb[0] = half ? nb.x >> 16 : nb.x & 0xFFFFu;
+  r.nb[1] = half ? nb.y >> 16 : nb.y & 0xFFFFu;
+  r.nb[2] = half ? nb.z >> 16 : nb.z & 0xFFFFu;
+  r.nb[3] = half ? nb.w >> 16 : nb.w & 0xFFFFu;
   const uint32_t s0 = ptx::lds32(tb + 768 + 12 * q), s1 = ptx::lds32(tb + 772 + 12 * q),
                  s2 = ptx::lds32(tb + 776 + 12 * q);
   r.row0 = (uint64_t)s0 | ((uint64_t)(s1 & 0xFFFFu) << 32);
   r.row1 = (uint64_t)(s1 >> 16) | ((uint64_t)s2 << 16);
+  r.row0 >>= 6 * half;  // this lane's sub-blocks are 4 S + 2 half + {0, 1}
+  r.row1 >>= 6 * half;
   const uint32_t dw = ptx::lds32(tb + 864 + 4 * q);
   r.d0 = __half2float(__ushort_as_half((unsigned short)(dw & 0xFFFFu)));
   r.d1 = __half2float(__ushort_as_half((unsigned short)(dw >> 16)));
@@ -252,12 +261,11 @@ __device__ __forceinline__ void dequant_q1(const Q1Lane &L, int S, uint32_t A, i
                                            int lane) {
   const int q = lane >> 2, p = (lane >> 1) & 1, half = lane & 1;
   const uint32_t qw = S == 0 ? L.qs[0] : S == 1 ? L.qs[1] : S == 2 ? L.qs[2] : L.qs[3];
-  const uint32_t nw = S == 0 ? L.nb[0] : S == 1 ? L.nb[1] : S == 2 ? L.nb[2] : L.nb[3];
-  const uint32_t nb16 = half ? (nw >> 16) : (nw & 0xFFFFu);
+  const uint32_t nb16 = S == 0 ? L.nb[0] : S == 1 ? L.nb[1] : S == 2 ? L.nb[2] : L.nb[3];
 #pragma unroll
   for (int j = 0; j < 2; ++j) {
-    const int s2 = j ^ (q & 1);            // odd rows take the other sub-block first: conflict-free stores
-    const int sb = 4 * S + 2 * half + s2;  // sub-block of 16 inputs within the column
+    const int s2 = j;
+    const int sb = 4 * S + s2;  // sub-block 4 S + 2 half + s2, counted from the lane's first
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       const int f = 2 * s2 + h;
@@ -400,6 +408,7 @@ __global__ void __maxnreg__(128) grouped_tc_kernel(TileArgs a) {
     } else if (warp < 2 + kDqWarps) {
       // ---- dequant warps: A tiles (and this warp's 16 rows of B)
       const int w = warp - 2;
+      const int ll = ((lane & 7) << 2) | (lane >> 3);  // the layout lane this thread decodes
       const uint32_t sel2a = ptx::smem_u32(S.sel2), sel1a = ptx::smem_u32(S.sel1);
       for (int u = 0; u < n_this; ++u) {
         const Unit U = S.units[u];
@@ -445,10 +454,10 @@ __global__ void __maxnreg__(128) grouped_tc_kernel(TileArgs a) {
           Q1Lane l1[C::kMats];
           if (U.qtype == kQ2) {
 #pragma unroll
-            for (int m = 0; m < C::kMats; ++m) l2[m] = load_q2(pk + (m * 8 + w) * tbb, lane);
+            for (int m = 0; m < C::kMats; ++m) l2[m] = load_q2(pk + (m * 8 + w) * tbb, ll);
           } else {
 #pragma unroll
-            for (int m = 0; m < C::kMats; ++m) l1[m] = load_q1(pk + (m * 8 + w) * tbb, lane);
+            for (int m = 0; m < C::kMats; ++m) l1[m] = load_q1(pk + (m * 8 + w) * tbb, ll);
           }
           __syncwarp();
           if (lane == 0) ptx::mbar_arrive(&B.pempty[ps]);
@@ -461,10 +470,10 @@ __global__ void __maxnreg__(128) grouped_tc_kernel(TileArgs a) {
             TC_T0();
             if (U.qtype == kQ2) {
 #pragma unroll
-              for (int m = 0; m < C::kMats; ++m) dequant_q2(l2[m], s, stg + m * kTile, 16 * w, sel2a, lane);
+              for (int m = 0; m < C::kMats; ++m) dequant_q2(l2[m], s, stg + m * kTile, 16 * w, sel2a, ll);
             } else {
 #pragma unroll
-              for (int m = 0; m < C::kMats; ++m) dequant_q1(l1[m], s, stg + m * kTile, 16 * w, sel1a, lane);
+              for (int m = 0; m < C::kMats; ++m) dequant_q1(l1[m], s, stg + m * kTile, 16 * w, sel1a, ll);
             }
             TC_ADD(2);
             // this step's B rows landed (the next step's may still be in flight)
