@@ -137,6 +137,35 @@ def test_missing_expert_reported(P):
     assert L.read_status() & P.REDLITE_STATUS_BAD_EXPERT
 
 
+def test_bad_and_missing_ids_on_bucketed_paths(P):
+    """Invalid ids and a never-uploaded slot in a 128-token call, on the
+    bucketed tensor-core path and on the general CUDA-core path: both are
+    reported in the status word and their pairs contribute nothing (the same
+    call with those slots' weights set to 0 agrees up to summation order)."""
+    w = fixtures.workload(4)
+    st = fixtures.Stream(991, 2)
+    logits = st.normal(128 * 512).reshape(128, 512)
+    ids, wt = fixtures.softmax_topk_routing(logits, 10)
+    x = fixtures.make_x(991, 128, 2048)
+    sel = sorted(set(ids.reshape(-1).tolist()))
+    missing = next(e for e in range(512) if e not in set(sel))
+    bad = ids.copy()
+    bad[0, 2], bad[5, 7], bad[9, 0] = 512, -3, missing
+    w0 = wt.copy()
+    w0[0, 2] = w0[5, 7] = w0[9, 0] = 0
+    L = P.layer_for_workload(w, experts=sel, max_tokens=128)
+    for general in (False, True):
+        if general:
+            L.table.min_ffn = 0  # unknown widths: the general CUDA-core path runs
+        got = _run(L, x, bad, wt)
+        status = L.read_status()
+        assert status & P.REDLITE_STATUS_BAD_ID and status & P.REDLITE_STATUS_BAD_EXPERT
+        L.clear_status()
+        ref = _run(L, x, ids, w0)
+        assert L.read_status() == 0
+        assert np.abs(got - ref).max() <= 1e-5 * np.abs(ref).max()
+
+
 def test_max_topk_and_ragged_shapes(P, oracle_lib):
     """top_k = 16, hidden 768, ffn 128 (down rows of half a block), a shared expert of width 256,
     7 tokens (ragged against the 4-token passes)."""
