@@ -83,6 +83,24 @@ class ClockSampler:
 _NOT_IN = {k: ("grouped_tc.cu", "route.cu", "tiles_simt.cu") for k in ("decode", "decode_iq1", "batched")}
 
 
+def pack_inputs(x, ids, weights):
+    """One call's inputs (x fp32 [T, H], ids int32 [T, k], weights fp32 [T, k])
+    as one byte array, in that order, so that a step moves them host -> device
+    with a single copy; x starts the array (16-byte aligned with the buffer)
+    and each part's size is a multiple of 4 bytes."""
+    parts = [np.ascontiguousarray(a).view(np.uint8).reshape(-1) for a in (x, ids, weights)]
+    return np.concatenate(parts)
+
+
+def input_views(buf, T, H, k):
+    """Typed views (x, ids, weights) of a torch uint8 tensor made by pack_inputs."""
+    import torch
+
+    nx, ni = 4 * T * H, 4 * T * k
+    return (buf[:nx].view(torch.float32).view(T, H), buf[nx:nx + ni].view(torch.int32).view(T, k),
+            buf[nx + ni:nx + 2 * ni].view(torch.float32).view(T, k))
+
+
 def _source_sha(exclude=()):
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "routed_expert_ffn_iq2_b200", "csrc")
@@ -257,9 +275,12 @@ def main():
     if sh is not None:
         R._native._check(L.set_shared(sh), "set_shared")
 
-    dx = [torch.from_numpy(np.ascontiguousarray(s[0])).to(dev) for s in P.sets]
-    di = [torch.from_numpy(np.ascontiguousarray(s[1])).to(dev) for s in P.sets]
-    dw = [torch.from_numpy(np.ascontiguousarray(s[2])).to(dev) for s in P.sets]
+    # each set's inputs live in one device buffer (x, ids, weights), so the
+    # end-to-end leg below copies them host -> device in one transfer
+    packed = [pack_inputs(*s[:3]) for s in P.sets]
+    dbuf = [torch.from_numpy(pk).to(dev) for pk in packed]
+    views = [input_views(b, s[0].shape[0], w.hidden, w.top_k) for b, s in zip(dbuf, P.sets)]
+    dx, di, dw = [v[0] for v in views], [v[1] for v in views], [v[2] for v in views]
     do = [torch.empty((s[0].shape[0], w.hidden), dtype=torch.float32, device=dev) for s in P.sets]
     nsets = len(P.sets)
 
@@ -318,20 +339,16 @@ def main():
     del graph
 
     # end-to-end through the public call with host buffers (pinned), per step:
-    # H2D of x, ids, weights; the layer; D2H of out.
+    # H2D of the step's x, ids and weights (one packed transfer); the layer; D2H of out.
     e2e = None
     if not args.no_e2e:
-        hx = [torch.from_numpy(np.ascontiguousarray(s[0])).pin_memory() for s in P.sets]
-        hi = [torch.from_numpy(np.ascontiguousarray(s[1])).pin_memory() for s in P.sets]
-        hw = [torch.from_numpy(np.ascontiguousarray(s[2])).pin_memory() for s in P.sets]
+        hbuf = [torch.from_numpy(pk).pin_memory() for pk in packed]
         ho = [torch.empty((s[0].shape[0], w.hidden), dtype=torch.float32).pin_memory() for s in P.sets]
         e_steps = min(steps, 2000 if nsets > 1 else steps)
 
         def e2e_step(i):
             j = i % nsets
-            dx[j].copy_(hx[j], non_blocking=True)
-            di[j].copy_(hi[j], non_blocking=True)
-            dw[j].copy_(hw[j], non_blocking=True)
+            dbuf[j].copy_(hbuf[j], non_blocking=True)
             call(j)
             ho[j].copy_(do[j], non_blocking=True)
 
@@ -353,7 +370,7 @@ def main():
             t = torch.tensor([ems], device=dev)
             dist.all_reduce(t, op=dist.ReduceOp.MAX)
             ems = float(t.item())
-        h2d = hx[0].nbytes + hi[0].nbytes + hw[0].nbytes
+        h2d = hbuf[0].nbytes
         e2e = {"value": world * e_steps * P.tokens_per_step / (ems / 1e3), "unit": "tokens/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(ho[0].nbytes), "steps": e_steps}
 

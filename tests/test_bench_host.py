@@ -1,0 +1,36 @@
+"""Host-side helpers of bench.py: the packed per-step input buffer that the
+end-to-end leg copies host -> device in one transfer."""
+import importlib.util
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import fixtures
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def bench():
+    spec = importlib.util.spec_from_file_location("bench_host", os.path.join(ROOT, "bench.py"))
+    m = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(m)
+    return m
+
+
+@pytest.mark.parametrize("T,H,k", [(1, 2048, 10), (64, 2048, 10), (7, 768, 16), (1, 256, 4)])
+def test_packed_inputs_round_trip(bench, T, H, k):
+    x = fixtures.make_x(31, T, H)
+    st = fixtures.Stream(31, 5)
+    ids = st.randint(T * k, 512).astype(np.int32).reshape(T, k)
+    wt = st.uniform(T * k).astype(np.float32).reshape(T, k)
+    pk = bench.pack_inputs(x, ids, wt)
+    assert pk.dtype == np.uint8 and pk.nbytes == x.nbytes + ids.nbytes + wt.nbytes
+    vx, vi, vw = bench.input_views(torch.from_numpy(pk), T, H, k)
+    assert vx.dtype == torch.float32 and vi.dtype == torch.int32 and vw.dtype == torch.float32
+    assert vx.is_contiguous() and vi.is_contiguous() and vw.is_contiguous()
+    assert np.array_equal(vx.numpy(), x) and np.array_equal(vi.numpy(), ids) and np.array_equal(vw.numpy(), wt)
+    # x leads the buffer; ids and weights start on 4-byte boundaries
+    assert vi.data_ptr() - vx.data_ptr() == x.nbytes and (vw.data_ptr() - vx.data_ptr()) % 4 == 0
