@@ -83,6 +83,23 @@ class ClockSampler:
 _NOT_IN = {k: ("grouped_tc.cu", "route.cu", "tiles_simt.cu") for k in ("decode", "decode_iq1", "batched")}
 
 
+def max_over_ranks(ms, world, device=None):
+    """The slowest rank's time; every rank calls this at the same points."""
+    if world <= 1:
+        return ms
+    import torch
+    import torch.distributed as dist
+
+    t = torch.tensor([ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_rate(world, steps, tokens_per_step, ms):
+    """Whole-job tokens/s: all ranks' tokens over the slowest rank's time (ms)."""
+    return world * steps * tokens_per_step / (ms / 1e3)
+
+
 def pack_inputs(x, ids, weights):
     """One call's inputs (x fp32 [T, H], ids int32 [T, k], weights fp32 [T, k])
     as one byte array, in that order, so that a step moves them host -> device
@@ -328,13 +345,7 @@ def main():
     torch.cuda.synchronize()
     barrier()
     clocks = clk.stop()
-    ms = ev0.elapsed_time(ev1)
-    if world > 1:
-        import torch.distributed as dist
-
-        t = torch.tensor([ms], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms = float(t.item())
+    ms = max_over_ranks(ev0.elapsed_time(ev1), world, dev)
     launches_per_call = R.launches_per_call(dx[0].shape[0], w.top_k, sh is not None)
     del graph
 
@@ -363,15 +374,9 @@ def main():
         e1.record(stream)
         e1.synchronize()
         barrier()
-        ems = e0.elapsed_time(e1)
-        if world > 1:
-            import torch.distributed as dist
-
-            t = torch.tensor([ems], device=dev)
-            dist.all_reduce(t, op=dist.ReduceOp.MAX)
-            ems = float(t.item())
+        ems = max_over_ranks(e0.elapsed_time(e1), world, dev)
         h2d = hbuf[0].nbytes
-        e2e = {"value": world * e_steps * P.tokens_per_step / (ems / 1e3), "unit": "tokens/s",
+        e2e = {"value": job_rate(world, e_steps, P.tokens_per_step, ems), "unit": "tokens/s",
                "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(ho[0].nbytes), "steps": e_steps}
 
     if L.read_status() != 0:
@@ -388,7 +393,7 @@ def main():
         per_step_s = sec / steps
         mean_bytes = float(np.mean([P.step_bytes[i % nsets] for i in range(G)]))
         mean_flops = float(np.mean([P.step_flops[i % nsets] for i in range(G)]))
-        tok_s = world * steps * P.tokens_per_step / sec
+        tok_s = job_rate(world, steps, P.tokens_per_step, ms)
         if P.cfg == 5:
             ach = mean_flops / per_step_s / 1e12
             peak = peaks["bf16_tflops_sustained"]
