@@ -15,7 +15,7 @@
 // expert, and the shared expert as a last active entry that owns every
 // token with weight 1.  Invalid ids (outside [0, n_experts)) and selected
 // slots without usable matrices are reported in the status word and their
-// pairs are dropped ("the offending pair contributes nothing").  Within an
+// pairs are dropped, so such a pair contributes nothing.  Within an
 // expert the order of its pairs is not fixed.
 #include <climits>
 
