@@ -256,6 +256,29 @@ def _bf16_rne(a):
     return r.astype(np.uint32).view(np.float32).astype(np.float64)
 
 
+def test_tensor_core_tile_boundaries(P, oracle_lib):
+    """257 tokens all routed to the same three experts (top-3, one IQ2_XS-style,
+    two IQ1_M-style) plus the shared expert: 771 pairs take the tcgen05 path and
+    every expert's pairs span token tiles of 128, 128 and 1."""
+    w = fixtures.workload(4)
+    q = np.asarray(w.qtypes)
+    sel = [int(np.nonzero(q == 1)[0][0]), int(np.nonzero(q == 2)[0][0]), int(np.nonzero(q == 2)[0][1])]
+    T = 257
+    ids = np.tile(np.array(sel, np.int32), (T, 1))
+    st = fixtures.Stream(257, 4)
+    wt = (st.uniform(T * 3).reshape(T, 3) + 0.1).astype(np.float32)
+    x = fixtures.make_x(257, T, w.hidden)
+    L = P.layer_for_workload(w, experts=sel, max_tokens=T)
+    got = _run(L, x, ids, wt)
+    experts = [None] * 512
+    for e in sel:
+        experts[e] = w.expert(e)
+    ref = oracle_lib.moe_layer(x, ids, wt, experts, w.shared(), oracle_lib.expand_grid(1, w.grid_iq2),
+                               oracle_lib.expand_grid(2, w.grid_iq1))
+    assert L.read_status() == 0
+    assert _rel_err(got, ref) <= TOL_BF16
+
+
 def test_bf16_rounding_helper_matches_oracle(oracle_lib):
     v = fixtures.make_x(77, 4, 256).reshape(-1) * np.float32(37.0)
     want = oracle_lib.float_to_bf16(v).astype(np.uint32) << 16
