@@ -11,14 +11,6 @@ using namespace redlite;
 
 static bool aligned16(const void *p) { return ((uintptr_t)p & 15) == 0; }
 
-static bool host_expert_ok(const redlite_moe_expert *e, int hidden, int max_ffn) {
-  if (!e || !e->gate || !e->up || !e->down) return false;
-  if (e->qtype != kQ2 && e->qtype != kQ1) return false;
-  if (e->ffn <= 0 || e->ffn > max_ffn) return false;
-  if (!aligned16(e->gate) || !aligned16(e->up) || !aligned16(e->down)) return false;
-  return shape_ok(e->ffn, hidden) && shape_ok(hidden, e->ffn);
-}
-
 extern "C" {
 
 size_t redlite_moe_grids_bytes(void) { return kGridBytes; }
@@ -74,7 +66,11 @@ int redlite_moe_layer(const float *x, int32_t n_tokens, const int32_t *expert_id
   if (n_tokens == 0) return REDLITE_OK;
   if (!x || !expert_ids || !router_weights || !out) return REDLITE_EINVAL;
   if (!aligned16(x) || !aligned16(out)) return REDLITE_EINVAL;
-  if (shared && !host_expert_ok(shared, t->hidden, t->max_ffn)) return REDLITE_EINVAL;
+  // min_ffn >= 256 declares every slot tiled: the fast kernels then run, and
+  // the shared expert must be one they can read (selected slots are checked
+  // on the device and reported in the status word)
+  const bool tiled = t->min_ffn >= 256;
+  if (shared && !shared_ok(*shared, t, tiled)) return REDLITE_EINVAL;
   // the largest top_k this workspace can hold for n_tokens
   WorkspaceLayout L = workspace_layout(t->hidden, t->n_experts, n_tokens, top_k, t->max_ffn);
   WorkspaceLayout Lmax = workspace_layout(t->hidden, t->n_experts, t->max_tokens, top_k, t->max_ffn);
@@ -83,7 +79,7 @@ int redlite_moe_layer(const float *x, int32_t n_tokens, const int32_t *expert_id
   cudaStream_t s = (cudaStream_t)t->stream;
   uint8_t *ws = (uint8_t *)t->workspace;
 
-  if (t->min_ffn >= 256 && fused_supported(t->hidden, t->max_ffn, n_tokens, top_k, t->n_experts, shared != nullptr)) {
+  if (tiled && fused_supported(t->hidden, t->max_ffn, n_tokens, top_k, t->n_experts, shared != nullptr)) {
     FusedArgs fa{};
     fa.x = x;
     fa.ids = expert_ids;
@@ -104,8 +100,10 @@ int redlite_moe_layer(const float *x, int32_t n_tokens, const int32_t *expert_id
     return launch_fused(fa, s) == cudaSuccess ? REDLITE_OK : REDLITE_ECUDA;
   }
   if (cudaMemsetAsync(out, 0, sizeof(float) * (size_t)n_tokens * t->hidden, s) != cudaSuccess) return REDLITE_ECUDA;
+  const bool tc = tiled && tc_supported(t->hidden, t->max_ffn);
   RouteArgs ra{expert_ids, router_weights, n_tokens, top_k, t->n_experts, t->hidden, t->max_ffn,
-               t->experts, shared != nullptr, shared ? shared->ffn : 0, shared ? shared->qtype : 0, ws, L, t->status};
+               t->experts, shared != nullptr, shared ? shared->ffn : 0, shared ? shared->qtype : 0, tc, ws, L,
+               t->status};
   if (launch_route(ra, s) != cudaSuccess) return REDLITE_ECUDA;
   TileArgs ta{};
   ta.x = x;
@@ -119,7 +117,7 @@ int redlite_moe_layer(const float *x, int32_t n_tokens, const int32_t *expert_id
   ta.ws = ws;
   ta.L = L;
   ta.status = t->status;
-  if (t->min_ffn >= 256 && tc_supported(t->hidden, t->max_ffn))
+  if (tc)
     return launch_tc(ta, s) == cudaSuccess ? REDLITE_OK : REDLITE_ECUDA;
   const int64_t routed = (int64_t)n_tokens * top_k;
   const int max_active = (int)((routed < t->n_experts ? routed : t->n_experts) + (shared ? 1 : 0));

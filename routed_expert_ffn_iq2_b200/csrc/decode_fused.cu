@@ -620,12 +620,19 @@ __device__ __forceinline__ void replicate_tables(const Smem &S, int t) {
 
 // ------------------------------------------------------------------ the kernel
 
-__device__ bool fused_expert_ok(const redlite_moe_expert &e, int hidden, int max_ffn) {
-  if (!e.gate || !e.up || !e.down) return false;
-  if (e.qtype != kQ2 && e.qtype != kQ1) return false;
-  if (e.ffn <= 0 || e.ffn > max_ffn || e.ffn % 256) return false;
-  if (((uintptr_t)e.gate | (uintptr_t)e.up | (uintptr_t)e.down) & 15) return false;
-  return shape_ok(e.ffn, hidden) && shape_ok(hidden, e.ffn);
+// The shared expert's instance (every token, weight 1), or an empty one with
+// the BAD_EXPERT bit if its descriptor is not one this kernel can read.
+__device__ void set_shared_inst(Inst &I, const FusedArgs &a, int pair_start, int &bad) {
+  I.pair_start = pair_start;
+  if (expert_ok(a.shared, a.hidden, a.max_ffn, true)) {
+    I.gate = (const uint8_t *)a.shared.gate, I.up = (const uint8_t *)a.shared.up;
+    I.down = (const uint8_t *)a.shared.down, I.qtype = a.shared.qtype, I.ffn = a.shared.ffn;
+    I.count = a.n_tokens;
+  } else {
+    bad |= REDLITE_STATUS_BAD_EXPERT;
+    I.gate = I.up = I.down = nullptr;
+    I.qtype = kQ2, I.ffn = 256, I.count = 0;
+  }
 }
 
 __device__ __forceinline__ int item_tiles_of(int ffn) {
@@ -790,7 +797,7 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(FusedArgs a)
         redlite_moe_expert d;
         memcpy(reinterpret_cast<uint8_t *>(&d), &my_d[0][0], 16);
         memcpy(reinterpret_cast<uint8_t *>(&d) + 16, &my_d[0][1], 16);
-        if (fused_expert_ok(d, H, a.max_ffn)) {
+        if (expert_ok(d, H, a.max_ffn, true)) {
           I.gate = (const uint8_t *)d.gate, I.up = (const uint8_t *)d.up, I.down = (const uint8_t *)d.down;
           I.qtype = d.qtype, I.ffn = d.ffn, I.count = __popc(same);
         } else {
@@ -803,12 +810,7 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(FusedArgs a)
       int n_inst = __popc(leaders);
       const int n_routed_pairs = __popc(__ballot_sync(0xffffffffu, ok));
       if (a.has_shared) {
-        if (lane == 0) {
-          Inst &I = S.inst[n_inst];
-          I.gate = (const uint8_t *)a.shared.gate, I.up = (const uint8_t *)a.shared.up;
-          I.down = (const uint8_t *)a.shared.down, I.qtype = a.shared.qtype, I.ffn = a.shared.ffn;
-          I.pair_start = n_routed_pairs, I.count = T;
-        }
+        if (lane == 0) set_shared_inst(S.inst[n_inst], a, n_routed_pairs, bad);
         if (lane < T) S.pair_tok[n_routed_pairs + lane] = lane, S.pair_w[n_routed_pairs + lane] = 1.f;
         n_inst += 1;
       }
@@ -900,7 +902,7 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(FusedArgs a)
             memcpy(reinterpret_cast<uint8_t *>(&d), &d0, 16);
             memcpy(reinterpret_cast<uint8_t *>(&d) + 16, &d1, 16);
             const int c = cnt[e];
-            if (fused_expert_ok(d, H, a.max_ffn)) {
+            if (expert_ok(d, H, a.max_ffn, true)) {
               I.gate = (const uint8_t *)d.gate, I.up = (const uint8_t *)d.up, I.down = (const uint8_t *)d.down;
               I.qtype = d.qtype, I.ffn = d.ffn, I.count = c;
             } else {
@@ -938,12 +940,7 @@ __global__ void __launch_bounds__(kFThreads, 1) decode_fused_kernel(FusedArgs a)
       }
     } else {
       if (a.has_shared) {
-        if (tid == 0) {
-          Inst &I = S.inst[n_inst];
-          I.gate = (const uint8_t *)a.shared.gate, I.up = (const uint8_t *)a.shared.up;
-          I.down = (const uint8_t *)a.shared.down, I.qtype = a.shared.qtype, I.ffn = a.shared.ffn;
-          I.pair_start = n_routed_pairs, I.count = T;
-        }
+        if (tid == 0) set_shared_inst(S.inst[n_inst], a, n_routed_pairs, bad);
         for (int t = tid; t < T; t += kCThreads) S.pair_tok[n_routed_pairs + t] = t, S.pair_w[n_routed_pairs + t] = 1.f;
       }
     }

@@ -75,6 +75,21 @@ inline __host__ __device__ size_t matrix_bytes(int qtype, int64_t rows, int64_t 
   return (size_t)(rows * k / kBlockWeights) * block_bytes(qtype);
 }
 
+// Whether a slot descriptor can be used by a layer kernel: three non-null,
+// 16-byte aligned matrices of a known format whose shapes the packed layout
+// takes, 0 < ffn <= max_ffn.  The fast kernels (fused decode, tensor-core
+// tiles) read every matrix in the tiled resident layout, so on their path the
+// width must also be a multiple of 256.  Used on the host for the shared
+// expert and on the device for every selected slot.
+inline __host__ __device__ bool expert_ok(const redlite_moe_expert &e, int hidden, int max_ffn, bool tiled_path) {
+  if (!e.gate || !e.up || !e.down) return false;
+  if (e.qtype != kQ2 && e.qtype != kQ1) return false;
+  if (e.ffn <= 0 || e.ffn > max_ffn) return false;
+  if (((uintptr_t)e.gate | (uintptr_t)e.up | (uintptr_t)e.down) & 15) return false;
+  if (tiled_path && (e.ffn % kBlockWeights || hidden % kBlockWeights)) return false;
+  return shape_ok(e.ffn, hidden) && shape_ok(hidden, e.ffn);
+}
+
 // ---------------------------------------------------------------- workspace
 // Control words, the active-expert list, the token pairs sorted by expert
 // and the per-pair hidden activations h.  Sizes depend on the table limits.
@@ -153,6 +168,13 @@ inline WorkspaceLayout workspace_layout(int hidden, int n_experts, int max_token
   off = align256(off + sizeof(int) * (size_t)(ft + 1));
   L.total = off;
   return L;
+}
+
+// The shared expert of a layer call, checked on the host: a usable slot
+// descriptor (expert_ok) whose width is at least the table's declared
+// min_ffn; on the tiled path (min_ffn >= 256) a multiple of 256.
+inline bool shared_ok(const redlite_moe_expert &e, const redlite_moe_table *t, bool tiled_path) {
+  return expert_ok(e, t->hidden, t->max_ffn, tiled_path) && e.ffn >= t->min_ffn;
 }
 
 // ---------------------------------------------------------------- device helpers
@@ -246,6 +268,7 @@ struct RouteArgs {
   const redlite_moe_expert *experts;
   bool has_shared;
   int shared_ffn, shared_qtype;
+  bool tiled_path;  // the tensor-core kernels follow: slots must have the tiled layout
   uint8_t *ws;
   WorkspaceLayout L;
   int32_t *status;

@@ -73,7 +73,9 @@ extern "C" int redlite_moe_layer_noalloc(const float *x, int32_t n_tokens, const
   if (n_tokens == 0) return REDLITE_OK;
   if (!x || !expert_ids || !router_weights || !out) return REDLITE_EINVAL;
   if ((((uintptr_t)x) | ((uintptr_t)out)) & 15) return REDLITE_EINVAL;
-  if (shared && (!shared->gate || !shared->up || !shared->down || shared->ffn > t->max_ffn)) return REDLITE_EINVAL;
+  // the fused kernel reads the shared expert in the tiled layout: check it as
+  // redlite_moe_layer does on that path
+  if (shared && !shared_ok(*shared, t, true)) return REDLITE_EINVAL;
   // only the fused decode kernel runs here
   if (t->min_ffn < 256 || !fused_supported(t->hidden, t->max_ffn, n_tokens, top_k, t->n_experts, shared != nullptr))
     return REDLITE_EUNSUPPORTED;

@@ -23,14 +23,6 @@
 
 namespace redlite {
 
-__device__ bool expert_usable(const redlite_moe_expert &e, int hidden, int max_ffn) {
-  if (!e.gate || !e.up || !e.down) return false;
-  if (e.qtype != kQ2 && e.qtype != kQ1) return false;
-  if (e.ffn <= 0 || e.ffn > max_ffn) return false;
-  if (((uintptr_t)e.gate | (uintptr_t)e.up | (uintptr_t)e.down) & 15) return false;
-  return shape_ok(e.ffn, hidden) && shape_ok(hidden, e.ffn);
-}
-
 // Block-wide exclusive scan of one int per thread (blockDim.x == 1024).
 __device__ int block_exclusive_scan(int v, int *smem32, int *total) {
   const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
@@ -130,7 +122,7 @@ __global__ void __launch_bounds__(1024) route_plan_kernel(RouteArgs a, int nb) {
   int bad = 0;
   // drop experts whose slot is unusable
   for (int e = threadIdx.x; e < E; e += blockDim.x) {
-    if (cnt[e] && !expert_usable(a.experts[e], a.hidden, a.max_ffn)) {
+    if (cnt[e] && !expert_ok(a.experts[e], a.hidden, a.max_ffn, a.tiled_path)) {
       cnt[e] = 0;
       bad |= REDLITE_STATUS_BAD_EXPERT;
     }

@@ -100,3 +100,57 @@ def test_dequant_rejects_on_host(native):
     assert L.redlite_moe_dequant(3, p, 1, 256, p, p, None, None) == native.REDLITE_EINVAL
     assert L.redlite_moe_dequant(1, p, 1, 300, p, p, None, None) == native.REDLITE_EUNSUPPORTED
     assert L.redlite_moe_dequant(1, p, 1, 256, p, None, None, None) == native.REDLITE_EINVAL
+
+
+def _shared_cases(native):
+    """Shared-expert descriptors no layer kernel may be handed, each with why."""
+    E = native.redlite_moe_expert
+    return [
+        (E(3, 512, 0x1000, 0x2000, 0x3000), "unknown qtype"),
+        (E(1, 0, 0x1000, 0x2000, 0x3000), "zero width"),
+        (E(1, -256, 0x1000, 0x2000, 0x3000), "negative width"),
+        (E(1, 1024, 0x1000, 0x2000, 0x3000), "wider than max_ffn"),
+        (E(1, 512, 0x1004, 0x2000, 0x3000), "gate not 16-byte aligned"),
+        (E(2, 512, 0x1000, 0x2008, 0x3000), "up not 16-byte aligned"),
+        (E(1, 512, 0x1000, 0x2000, 0x3001), "down not 16-byte aligned"),
+        (E(1, 512, 0x1000, None, 0x3000), "null up"),
+        (E(1, 48, 0x1000, 0x2000, 0x3000), "width the packed layout does not take"),
+    ]
+
+
+def test_layer_rejects_bad_shared_expert_on_both_paths(native):
+    """Every malformed shared expert returns EINVAL before any device work,
+    whichever path the table selects; on the tiled path (min_ffn >= 256) a
+    width that is not a multiple of 256, or below the declared min_ffn, is
+    malformed too."""
+    L = native.lib()
+    p = ctypes.c_void_p(0x10000)
+    for min_ffn in (0, 256):
+        t = native.redlite_moe_table(2048, 512, 512, 64, min_ffn, 0, 0x1000, 0x2000, 0x3000, 1 << 30, 0x4000, None)
+        for sh, why in _shared_cases(native):
+            rc = L.redlite_moe_layer(p, 1, p, p, 10, ctypes.byref(t), ctypes.byref(sh), p)
+            assert rc == native.REDLITE_EINVAL, (min_ffn, why, rc)
+    t = native.redlite_moe_table(2048, 512, 512, 64, 512, 0, 0x1000, 0x2000, 0x3000, 1 << 30, 0x4000, None)
+    for sh in (native.redlite_moe_expert(1, 128, 0x1000, 0x2000, 0x3000),   # valid shape, not tiled
+               native.redlite_moe_expert(1, 256, 0x1000, 0x2000, 0x3000)):  # below the declared min_ffn
+        assert L.redlite_moe_layer(p, 1, p, p, 10, ctypes.byref(t), ctypes.byref(sh), p) == native.REDLITE_EINVAL
+
+
+def test_no_alloc_rejects_on_host(native):
+    """The allocation-free entry point validates the shared expert like the
+    fused path of redlite_moe_layer, and refuses a call whose scratch does not
+    fit its fixed array with ENOMEM before it touches the device (without a
+    GPU any device call would return ECUDA instead)."""
+    L = native.lib()
+    p = ctypes.c_void_p(0x10000)
+    t = native.redlite_moe_table(2048, 512, 512, 64, 512, 0, 0x1000, 0x2000, 0x3000, 0, 0x4000, None)
+    for sh, why in _shared_cases(native) + [(native.redlite_moe_expert(1, 128, 0x1000, 0x2000, 0x3000), "not tiled")]:
+        rc = L.redlite_moe_layer_noalloc(p, 1, p, p, 10, ctypes.byref(t), ctypes.byref(sh), p)
+        assert rc == native.REDLITE_EINVAL, (why, rc)
+    # 64 tokens x top-10 + shared at width 2048: 704 pairs x 2 x 2048 fp32 gate/up values > 4 MiB
+    big = native.redlite_moe_table(2048, 512, 2048, 64, 2048, 0, 0x1000, 0x2000, 0x3000, 0, 0x4000, None)
+    sh = native.redlite_moe_expert(1, 2048, 0x1000, 0x2000, 0x3000)
+    assert L.redlite_moe_layer_noalloc(p, 64, p, p, 10, ctypes.byref(big), ctypes.byref(sh), p) == native.REDLITE_ENOMEM
+    # widths the fused kernel does not take
+    t1 = native.redlite_moe_table(256, 16, 64, 1, 64, 0, 0x1000, 0x2000, 0x3000, 0, 0x4000, None)
+    assert L.redlite_moe_layer_noalloc(p, 1, p, p, 4, ctypes.byref(t1), None, p) == native.REDLITE_EUNSUPPORTED

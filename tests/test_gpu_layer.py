@@ -374,3 +374,26 @@ def test_grid_wait_gives_up_and_reports(P):
     again = _run(L, w.x, w.ids, w.weights)
     assert L.read_status() == 0
     assert _rel_err(again, ref) <= 1e-6
+
+
+@pytest.mark.parametrize("T", [1, 200])
+def test_overstated_min_ffn_is_reported_not_read(P, T):
+    """A table that declares min_ffn = 256 while its slots hold width-128
+    experts (interchange layout, not tiled): the fast kernels (fused decode at
+    T = 1, bucketed tensor-core path at T = 200) check every selected slot,
+    report REDLITE_STATUS_BAD_EXPERT and read nothing from it, so every pair
+    is dropped and out is all zeros."""
+    H, E, F, k = 512, 8, 128, 4
+    seed = 515
+    g2, g1 = fixtures.make_grid(seed, 1), fixtures.make_grid(seed, 2)
+    experts = [fixtures.make_expert(seed, 1 + (e % 2), H, F, e) for e in range(E)]
+    L = P.MoeLayer(H, E, 256, T, k, g2, g1, pool_bytes=(E + 1) * fixtures.expert_bytes(1, H, 256) + 4096)
+    assert L.upload(list(range(E)), experts) == 0
+    L.table.min_ffn = 256  # overstated: the slots are 128 wide
+    st = fixtures.Stream(seed, 5)
+    ids = st.randint(T * k, E).astype(np.int32).reshape(T, k)
+    wt = (0.1 + st.uniform(T * k)).astype(np.float32).reshape(T, k)
+    x = fixtures.make_x(seed, T, H)
+    got = _run(L, x, ids, wt)
+    assert L.read_status() & P.REDLITE_STATUS_BAD_EXPERT
+    assert np.all(got == 0.0)

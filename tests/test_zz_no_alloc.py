@@ -56,3 +56,31 @@ def test_no_alloc_rejects_what_it_cannot_take(P):
     out = torch.empty_like(x)
     rc = P.redlite_moe_layer_noalloc(x, 1, ids, wt, w.top_k, L.table, None, out)
     assert rc == P.REDLITE_EUNSUPPORTED
+
+
+def test_no_alloc_refusals_leave_out_untouched(P):
+    """Calls the fixed scratch array cannot serve, and malformed shared
+    experts, are refused on the host before anything is enqueued: out keeps
+    its contents and the status word stays clear."""
+    import copy
+
+    w = fixtures.workload(4)  # 64 tokens x top-10 + shared expert
+    L = P.layer_for_workload(w)
+    x = torch.from_numpy(w.x).cuda()
+    ids = torch.from_numpy(w.ids).cuda()
+    wt = torch.from_numpy(w.weights).cuda()
+    out = torch.full_like(x, 3.5)
+    # declared max_ffn 2048: 704 pairs x 2 x 2048 fp32 gate/up values do not fit 4 MiB
+    big = copy.copy(L.table)
+    big.max_ffn = 2048
+    rc = P.redlite_moe_layer_noalloc(x, x.shape[0], ids, wt, w.top_k, big, L.shared, out)
+    assert rc == P.REDLITE_ENOMEM
+    bad = P.redlite_moe_expert(L.shared.qtype, L.shared.ffn, L.shared.gate + 8, L.shared.up, L.shared.down)
+    rc = P.redlite_moe_layer_noalloc(x, x.shape[0], ids, wt, w.top_k, L.table, bad, out)
+    assert rc == P.REDLITE_EINVAL
+    bad = P.redlite_moe_expert(7, L.shared.ffn, L.shared.gate, L.shared.up, L.shared.down)
+    rc = P.redlite_moe_layer_noalloc(x, x.shape[0], ids, wt, w.top_k, L.table, bad, out)
+    assert rc == P.REDLITE_EINVAL
+    torch.cuda.synchronize()
+    assert bool((out == 3.5).all())
+    assert L.read_status() == 0
