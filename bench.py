@@ -1,13 +1,19 @@
 """Benchmark of the routed top-k MoE layer (one JSON line on rank 0).
 
-Default workload: the Qwen3-Next-shaped decode layer with IQ2_XS-style
+Headline workload: the Qwen3-Next-shaped decode layer with IQ2_XS-style
 experts (hidden 2048, 512 experts of width 512, top-10, one token per call).
-A step is one layer call over one token.  All 512 experts are resident; the
-steps cycle through 48 pairwise-disjoint top-10 sets (480 experts, 436 MB of
-packed weights, far above the 126 MB L2), so every step streams its experts
-from HBM.  Steps are issued as CUDA-graph replays of the C-ABI call.
+All selected experts are resident; the calls cycle through 48 pairwise-disjoint
+top-10 sets (480 experts, 436 MB of packed weights, far above the 126 MB L2), so
+every call streams its experts from HBM.  Calls are issued as CUDA-graph
+replays of the C-ABI call.
 
-  python bench.py [--gpus N] [--steps K] [--warmup W] [--config 2..5]
+A step is a fixed number of graph replays (`calls_per_step` layer calls:
+50 passes over the 48 decode sets, 50 batched-decode calls, 10 prefill calls),
+so `--steps K` times exactly K steps.  On one GPU the line also carries a
+`workloads` map with the other workloads (IQ1_M-style cold decode, batched
+decode, prefill), each measured the same way.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config 2..5] [--workloads 3,4,5|none]
   python bench.py --impl reference ...   # the fp64 CPU oracle, timed on host cores
 
 Multi-GPU (torchrun): every rank runs an independent replica (the layer has no
@@ -17,6 +23,7 @@ exchange step); value = all ranks' tokens / the slowest rank's device time.
 from __future__ import annotations
 
 import argparse
+import datetime
 import hashlib
 import json
 import os
@@ -35,7 +42,14 @@ import fixtures  # noqa: E402
 
 METRIC = "routed-MoE-layer tokens/sec on 1 B200; achieved HBM GB/s vs ~8 TB/s peak"
 N_SETS = 48
-GRAPH_CYCLES = 5  # graph = GRAPH_CYCLES * N_SETS calls for the decode workloads
+# calls captured in one CUDA graph, and graph replays per step
+GRAPH_CALLS = {2: 240, 3: 240, 4: 10, 5: 10}
+REPLAYS_PER_STEP = {2: 10, 3: 10, 4: 5, 5: 1}
+DTYPE = {2: "f32", 3: "f32", 4: "f32", 5: "bf16"}
+
+
+def calls_per_step(cfg: int) -> int:
+    return GRAPH_CALLS[cfg] * REPLAYS_PER_STEP[cfg]
 
 
 def _peaks():
@@ -48,13 +62,17 @@ def _peaks():
 
 
 class ClockSampler:
-    QUERY = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    """nvidia-smi samples every 100 ms; only samples taken inside the timed
+    window (host timestamps) are summarised, unless the window saw none."""
+
+    QUERY = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, index: int):
         self.index = index
         self.proc = None
+        self.window = None
 
     def start(self):
         try:
@@ -64,23 +82,44 @@ class ClockSampler:
         except OSError:
             self.proc = None
 
+    def mark(self, t0: float, t1: float):
+        self.window = (t0, t1)
+
+    @staticmethod
+    def summarise(rows, window=None):
+        def ts(r):
+            try:
+                return datetime.datetime.strptime(r[0].strip(), "%Y/%m/%d %H:%M:%S.%f").timestamp()
+            except ValueError:
+                return None
+
+        inside = [r for r in rows if window and ts(r) is not None and window[0] <= ts(r) <= window[1]]
+        use = inside if inside else rows
+
+        def num(v):
+            v = v.strip()
+            return float(v) if v.replace(".", "", 1).isdigit() else None
+
+        sm = [num(r[2]) for r in use if num(r[2]) is not None]
+        mx = [num(r[3]) for r in use if num(r[3]) is not None]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in use for i in range(4) if "Active" in r[6 + i] and "Not" not in r[6 + i]})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
+                "reasons": reasons, "samples": len(use), "samples_in_window": len(inside)}
+
     def stop(self):
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
         self.proc.terminate()
         out, _ = self.proc.communicate(timeout=10)
-        rows = [r.split(",") for r in out.strip().splitlines() if r.count(",") >= 8]
-        sm = [float(r[1]) for r in rows if r[1].strip().replace(".", "").isdigit()]
-        mx = [float(r[2]) for r in rows if r[2].strip().replace(".", "").isdigit()]
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        reasons = sorted({names[i] for r in rows for i in range(4) if "Active" in r[5 + i] and "Not" not in r[5 + i]})
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(mx) if mx else None,
-                "reasons": reasons, "samples": len(rows)}
+        rows = [r.split(",") for r in out.strip().splitlines() if r.count(",") >= 9]
+        return self.summarise(rows, self.window)
 
 
 # Source files that do not go into a kernel's translation unit: a change there
 # leaves the counters taken for that kernel valid.
 _NOT_IN = {k: ("grouped_tc.cu", "route.cu", "tiles_simt.cu") for k in ("decode", "decode_iq1", "batched")}
+_NOT_IN["prefill"] = ("decode_fused.cu", "noalloc.cu", "tiles_simt.cu")
 
 
 def max_over_ranks(ms, world, device=None):
@@ -139,11 +178,31 @@ def _traffic(kernel_key: str):
     return d.get("dram_bytes_per_launch")
 
 
+def layer_for_workload(w, experts=None, max_tokens=None, extra_pool: int = 0, device: str = "cuda"):
+    """A MoeLayer holding the experts of a fixtures.Workload (by default the
+    selected ones) and its shared expert, uploaded through the C ABI."""
+    import routed_expert_ffn_iq2_b200 as R
+
+    ids = w.selected() if experts is None else list(experts)
+    per = max(fixtures.expert_bytes(q, w.hidden, w.ffn) for q in (1, 2)) + 64
+    sh = w.shared()
+    pool = per * len(ids) + (sh.nbytes + 64 if sh is not None else 0) + extra_pool
+    max_ffn = max(w.ffn, w.shared_ffn if sh is not None else 0)
+    L = R.MoeLayer(w.hidden, w.n_experts, max_ffn, max_tokens or w.n_tokens, w.top_k, w.grid_iq2, w.grid_iq1, pool,
+                   device=device)
+    for i in range(0, len(ids), 32):
+        chunk = ids[i:i + 32]
+        R._native._check(L.upload(chunk, [w.expert(e) for e in chunk]), "upload")
+    if sh is not None:
+        R._native._check(L.set_shared(sh), "set_shared")
+    return L
+
+
 # ------------------------------------------------------------------ workloads
 
 
 class Problem:
-    """Per-config inputs: `sets` of (x [T,H], ids [T,k], weights [T,k]) cycled by the steps."""
+    """Per-config inputs: `sets` of (x [T,H], ids [T,k], weights [T,k]) cycled by the calls."""
 
     def __init__(self, cfg: int):
         self.cfg = cfg
@@ -163,9 +222,9 @@ class Problem:
         else:
             raise SystemExit("bench supports --config 2..5 (config 1 is a parity case)")
         w = self.w
-        self.tokens_per_step = self.sets[0][0].shape[0]
-        self.step_bytes = []
-        self.step_flops = []
+        self.tokens_per_call = self.sets[0][0].shape[0]
+        self.call_bytes = []
+        self.call_flops = []
         sh = w.shared()
         for x, ids, _ in self.sets:
             uniq = sorted(set(ids.reshape(-1).tolist()))
@@ -173,9 +232,9 @@ class Problem:
             if sh is not None:
                 b += sh.nbytes
             b += x.nbytes * 2 + ids.nbytes * 2  # x in, out back, ids and weights in
-            self.step_bytes.append(b)
+            self.call_bytes.append(b)
             pairs = ids.size + (x.shape[0] if sh is not None else 0)
-            self.step_flops.append(2.0 * 3 * w.hidden * w.ffn * pairs)
+            self.call_flops.append(2.0 * 3 * w.hidden * w.ffn * pairs)
 
     def name(self):
         return self.w.name
@@ -194,7 +253,7 @@ def _oracle_step(oracle, P: Problem, i: int, cache):
 
 
 def cpu_oracle_rate(P: Problem, budget_s: float, max_steps: int):
-    """Time the fp64 oracle as it stands on the host cores: steps/s (tokens/s)."""
+    """Time the fp64 oracle as it stands on the host cores: layer calls/s as tokens/s."""
     import oracle
 
     cores = oracle.set_threads(0)
@@ -220,75 +279,49 @@ def cpu_oracle_rate(P: Problem, budget_s: float, max_steps: int):
     return toks / dt, cores, sample
 
 
-# ------------------------------------------------------------------ main
+def roofline(P: Problem, per_call_s: float, peaks):
+    """Achieved rate of one call against the measured peak (bytes or FLOPs per call / call time)."""
+    n = len(P.sets)
+    G = GRAPH_CALLS[P.cfg]
+    mean_bytes = float(np.mean([P.call_bytes[i % n] for i in range(G)]))
+    mean_flops = float(np.mean([P.call_flops[i % n] for i in range(G)]))
+    if P.cfg == 5:
+        ach = mean_flops / per_call_s / 1e12
+        peak = peaks["bf16_tflops_sustained"]
+        return {"bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s", "frac": ach / peak,
+                "traffic": _traffic("prefill"), "peak_kind": f"{peaks['src']} bf16 sustained",
+                "flops_per_call": mean_flops}, mean_bytes
+    ach = mean_bytes / per_call_s / 1e9
+    peak = peaks["hbm_gbs"]
+    return {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak,
+            "traffic": _traffic({2: "decode", 3: "decode_iq1"}.get(P.cfg, "batched")),
+            "peak_kind": f"{peaks['src']} HBM copy", "bytes_per_call": mean_bytes}, mean_bytes
 
 
-def main():
-    ap = argparse.ArgumentParser()
-    ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=0)
-    ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--config", type=int, default=2)
-    ap.add_argument("--impl", default="native", choices=["native", "reference"])
-    ap.add_argument("--cpu-budget", type=float, default=12.0)
-    ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--no-e2e", action="store_true")
-    args = ap.parse_args()
+# ------------------------------------------------------------------ one workload on the GPU
 
-    rank = int(os.environ.get("RANK", "0"))
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
 
-    if args.impl == "reference":
-        if rank != 0:
-            return
-        P = Problem(args.config)
-        rate, cores, sample = cpu_oracle_rate(P, args.cpu_budget, max_steps=max(args.steps, 1) * 48)
-        peaks = _peaks()
-        line = {
-            "impl": "reference", "metric": METRIC, "value": rate, "unit": "tokens/s", "n_gpus": args.gpus,
-            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * P.tokens_per_step / rate,
-            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": P.name(), "tokens_per_step": P.tokens_per_step},
-            "cpu_baseline": {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
-            "e2e": {"value": rate, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
-            "peaks_src": peaks["src"],
-        }
-        print(json.dumps(line), flush=True)
-        return
-
+def measure(cfg: int, steps: int, warmup: int, world: int, rank: int, local: int, dev, e2e_on: bool,
+            cpu_budget: float = 0.0):
+    """Time `steps` steps of workload `cfg` (max over ranks) and its end-to-end leg."""
     import torch
 
-    torch.cuda.set_device(local)
-    dev = torch.device("cuda", local)
-    if world > 1:
-        import datetime
-
-        import torch.distributed as dist
-
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
-
-    from routed_expert_ffn_iq2_b200 import build as B
-
-    B.build()
     import routed_expert_ffn_iq2_b200 as R
 
-    P = Problem(args.config)
+    P = Problem(cfg)
     w = P.w
     stream = torch.cuda.Stream(dev)
     torch.cuda.set_stream(stream)
     per = max(fixtures.expert_bytes(q, w.hidden, w.ffn) for q in (1, 2)) + 64
     sh = w.shared()
     pool = per * len(P.resident) + (sh.nbytes + 64 if sh is not None else 0)
-    max_tok = P.tokens_per_step
-    L = R.MoeLayer(w.hidden, w.n_experts, max(w.ffn, w.shared_ffn), max_tok, w.top_k, w.grid_iq2, w.grid_iq1,
-                   pool, device=str(dev), stream=stream)
+    L = R.MoeLayer(w.hidden, w.n_experts, max(w.ffn, w.shared_ffn), P.tokens_per_call, w.top_k, w.grid_iq2,
+                   w.grid_iq1, pool, device=str(dev), stream=stream)
     for i in range(0, len(P.resident), 32):
         chunk = P.resident[i:i + 32]
         R._native._check(L.upload(chunk, [w.expert(e) for e in chunk]), "upload")
-        if rank != 0:
-            for e in chunk:
-                w._experts.pop(e, None)
+        for e in chunk:  # host copies are no longer needed
+            w._experts.pop(e, None)
     if sh is not None:
         R._native._check(L.set_shared(sh), "set_shared")
 
@@ -307,19 +340,15 @@ def main():
         if rc != 0:
             raise RuntimeError(f"redlite_moe_layer rc={rc}")
 
-    # graph of G calls
-    G = GRAPH_CYCLES * nsets if nsets > 1 else 10
-    steps = args.steps if args.steps > 0 else (G * 800 if nsets > 1 else (200 if P.cfg == 4 else 30))
-    steps = ((steps + G - 1) // G) * G
-    for i in range(max(args.warmup, 3)):
+    G, reps = GRAPH_CALLS[cfg], REPLAYS_PER_STEP[cfg]
+    for i in range(3):
         call(i)
     stream.synchronize()
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph, stream=stream):
         for i in range(G):
             call(i)
-    reps_w = max(1, (max(args.warmup, 3) + G - 1) // G)
-    for _ in range(reps_w):
+    for _ in range(max(warmup, 3) * reps):
         graph.replay()
     stream.synchronize()
     if L.read_status() != 0:
@@ -332,96 +361,168 @@ def main():
             dist.barrier()
 
     clk = ClockSampler(local)
+    clk.start()
+    time.sleep(0.25)  # nvidia-smi is up before the timed window opens
     barrier()
     torch.cuda.synchronize()
-    clk.start()
-    time.sleep(0.3)
     ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0 = time.time()
     ev0.record(stream)
-    for _ in range(steps // G):
+    for _ in range(steps * reps):
         graph.replay()
     ev1.record(stream)
     ev1.synchronize()
+    t1 = time.time()
     torch.cuda.synchronize()
     barrier()
+    time.sleep(0.15)
+    clk.mark(t0, t1)
     clocks = clk.stop()
     ms = max_over_ranks(ev0.elapsed_time(ev1), world, dev)
+    cps = calls_per_step(cfg)
     launches_per_call = R.launches_per_call(dx[0].shape[0], w.top_k, sh is not None)
     del graph
 
-    # end-to-end through the public call with host buffers (pinned), per step:
-    # H2D of the step's x, ids and weights (one packed transfer); the layer; D2H of out.
+    # end-to-end through the public call with host buffers (pinned), per call:
+    # H2D of the call's x, ids and weights (one packed transfer); the layer; D2H of out.
     e2e = None
-    if not args.no_e2e:
+    if e2e_on:
         hbuf = [torch.from_numpy(pk).pin_memory() for pk in packed]
         ho = [torch.empty((s[0].shape[0], w.hidden), dtype=torch.float32).pin_memory() for s in P.sets]
-        e_steps = min(steps, 2000 if nsets > 1 else steps)
+        e_calls = min(steps * cps, 2400 if nsets > 1 else steps * cps)
 
-        def e2e_step(i):
+        def e2e_call(i):
             j = i % nsets
             dbuf[j].copy_(hbuf[j], non_blocking=True)
             call(j)
             ho[j].copy_(do[j], non_blocking=True)
 
         for i in range(3):
-            e2e_step(i)
+            e2e_call(i)
         stream.synchronize()
         barrier()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         e0.record(stream)
-        for i in range(e_steps):
-            e2e_step(i)
+        for i in range(e_calls):
+            e2e_call(i)
         e1.record(stream)
         e1.synchronize()
         barrier()
         ems = max_over_ranks(e0.elapsed_time(e1), world, dev)
-        h2d = hbuf[0].nbytes
-        e2e = {"value": job_rate(world, e_steps, P.tokens_per_step, ems), "unit": "tokens/s",
-               "h2d_bytes_per_step": int(h2d), "d2h_bytes_per_step": int(ho[0].nbytes), "steps": e_steps}
+        e2e = {"value": job_rate(world, e_calls, P.tokens_per_call, ems), "unit": "tokens/s",
+               "h2d_bytes_per_step": int(hbuf[0].nbytes) * cps, "d2h_bytes_per_step": int(ho[0].nbytes) * cps,
+               "calls": e_calls}
 
-    if L.read_status() != 0:
-        raise RuntimeError(f"device status {L.read_status()}")
+    status = L.read_status()
+    if status != 0:
+        raise RuntimeError(f"device status {status}")
+    del L, dbuf, do
+    torch.cuda.empty_cache()
 
     cpu = None
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        rate, cores, sample = cpu_oracle_rate(P, args.cpu_budget, max_steps=10 ** 6)
+    if rank == 0 and world == 1 and cpu_budget > 0:
+        rate, cores, sample = cpu_oracle_rate(P, cpu_budget, max_steps=10 ** 6)
         cpu = {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample}
 
-    if rank == 0:
+    peaks = _peaks()
+    per_call_s = ms / 1e3 / (steps * cps)
+    roof, mean_bytes = roofline(P, per_call_s, peaks)
+    tokens_per_step = cps * P.tokens_per_call
+    return {
+        "workload": P.name(),
+        "value": job_rate(world, steps, tokens_per_step, ms), "unit": "tokens/s",
+        "ms_per_step": ms / steps, "steps": steps, "calls_per_step": cps, "tokens_per_step": tokens_per_step,
+        "us_per_call": per_call_s * 1e6, "dtype": DTYPE[cfg],
+        "weight_gbs": mean_bytes / per_call_s / 1e9,
+        "roofline": roof, "e2e": e2e, "clocks": clocks, "cpu_baseline": cpu,
+        "gpu_launches": launches_per_call * steps * cps,
+        "l2": ("inputs larger than L2: calls cycle 48 disjoint top-10 sets over 480 resident experts (436 MB)"
+               if nsets > 1 else f"inputs larger than L2 (expert bytes per call {mean_bytes / 1e6:.0f} MB)"),
+        "issue": f"CUDA graph of {G} layer calls, {reps} replays per step",
+    }
+
+
+# ------------------------------------------------------------------ main
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--config", type=int, default=2)
+    ap.add_argument("--workloads", default="3,4,5", help="other workloads on one GPU, or 'none'")
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--cpu-budget", type=float, default=12.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    args = ap.parse_args()
+    steps = max(1, args.steps)
+
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        if rank != 0:
+            return
+        P = Problem(args.config)
+        rate, cores, sample = cpu_oracle_rate(P, args.cpu_budget, max_steps=max(args.steps, 1) * 48)
         peaks = _peaks()
-        sec = ms / 1e3
-        per_step_s = sec / steps
-        mean_bytes = float(np.mean([P.step_bytes[i % nsets] for i in range(G)]))
-        mean_flops = float(np.mean([P.step_flops[i % nsets] for i in range(G)]))
-        tok_s = job_rate(world, steps, P.tokens_per_step, ms)
-        if P.cfg == 5:
-            ach = mean_flops / per_step_s / 1e12
-            peak = peaks["bf16_tflops_sustained"]
-            roof = {"bound": "tensor", "achieved": ach, "peak": peak, "unit": "TFLOP/s", "frac": ach / peak,
-                    "traffic": _traffic("prefill"), "peak_kind": f"{peaks['src']} bf16 sustained"}
-        else:
-            ach = mean_bytes / per_step_s / 1e9
-            peak = peaks["hbm_gbs"]
-            roof = {"bound": "hbm", "achieved": ach, "peak": peak, "unit": "GB/s", "frac": ach / peak,
-                    "traffic": _traffic({2: "decode", 3: "decode_iq1"}.get(P.cfg, "batched")),
-                    "peak_kind": f"{peaks['src']} HBM copy"}
         line = {
-            "metric": METRIC, "value": tok_s, "unit": "tokens/s", "n_gpus": world, "steps": steps,
-            "warmup": args.warmup, "ms_per_step": ms / steps, "higher_is_better": True, "scaling": "weak",
-            "vs_baseline": None, "dtype": "f32" if P.cfg != 5 else "bf16", "data": "synthetic",
-            "config": {"workload": P.name(), "tokens_per_step": P.tokens_per_step,
-                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
-                       "l2": ("inputs larger than L2: steps cycle 48 disjoint top-10 sets over 480 resident "
-                              "experts (436 MB)" if nsets > 1 else "inputs larger than L2 (expert bytes per step "
-                              f"{mean_bytes / 1e6:.0f} MB)"),
-                       "issue": f"CUDA graph of {G} layer calls, replayed"},
-            "weight_gbs": mean_bytes / per_step_s / 1e9,
-            "roofline": roof,
-            "cpu_baseline": cpu,
-            "e2e": e2e,
-            "gpu_launches": launches_per_call * steps,
-            "clocks": clocks,
+            "impl": "reference", "metric": METRIC, "value": rate, "unit": "tokens/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * P.tokens_per_call / rate,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": P.name(), "tokens_per_step": P.tokens_per_call},
+            "cpu_baseline": {"value": rate, "unit": "tokens/s", "cores": cores, "kind": "oracle", "sample": sample},
+            "e2e": {"value": rate, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+            "peaks_src": peaks["src"],
         }
+        print(json.dumps(line), flush=True)
+        return
+
+    import torch
+
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+    if world > 1:
+        import torch.distributed as dist
+
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120), device_id=dev)
+
+    from routed_expert_ffn_iq2_b200 import build as B
+
+    B.build()
+
+    head = measure(args.config, steps, args.warmup, world, rank, local, dev, not args.no_e2e,
+                   cpu_budget=0.0 if args.no_cpu_baseline else args.cpu_budget)
+    others = {}
+    if world == 1 and args.workloads != "none":
+        for c in [int(v) for v in args.workloads.split(",") if v.strip()]:
+            if c != args.config:
+                r = measure(c, steps, args.warmup, world, rank, local, dev, not args.no_e2e)
+                r.pop("cpu_baseline", None)
+                others[str(c)] = r
+
+    if rank == 0:
+        line = {
+            "metric": METRIC, "value": head["value"], "unit": "tokens/s", "n_gpus": world, "steps": steps,
+            "warmup": args.warmup, "ms_per_step": head["ms_per_step"], "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": head["dtype"], "data": "synthetic",
+            "config": {"workload": head["workload"], "tokens_per_step": head["tokens_per_step"],
+                       "calls_per_step": head["calls_per_step"],
+                       "parallelism": f"replicas x{world}" if world > 1 else "single GPU",
+                       "l2": head["l2"], "issue": head["issue"]},
+            "us_per_call": head["us_per_call"],
+            "weight_gbs": head["weight_gbs"],
+            "roofline": head["roofline"],
+            "cpu_baseline": head["cpu_baseline"],
+            "e2e": head["e2e"],
+            "gpu_launches": head["gpu_launches"],
+            "clocks": head["clocks"],
+        }
+        if others:
+            line["workloads"] = others
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist

@@ -32,4 +32,4 @@ from ._native import (  # noqa: F401
     redlite_moe_workspace_bytes,
     redlite_moe_workspace_reset,
 )
-from .layer import MoeLayer, layer_for_workload  # noqa: F401
+from .layer import MoeLayer  # noqa: F401

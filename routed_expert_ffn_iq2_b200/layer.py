@@ -75,23 +75,3 @@ class MoeLayer:
     def clear_status(self):
         self.status.zero_()
 
-
-def layer_for_workload(w, experts: Optional[Sequence[int]] = None, max_tokens: Optional[int] = None,
-                       extra_pool: int = 0, device: str = "cuda") -> MoeLayer:
-    """A MoeLayer holding the experts of a fixtures.Workload (by default the selected ones)."""
-    import fixtures
-
-    ids = w.selected() if experts is None else list(experts)
-    per = fixtures.expert_bytes(int(w.qtypes[0]), w.hidden, w.ffn) + 64
-    per = max(per, max(fixtures.expert_bytes(q, w.hidden, w.ffn) for q in (1, 2)) + 64)
-    sh = w.shared()
-    pool = per * len(ids) + (sh.nbytes + 64 if sh is not None else 0) + extra_pool
-    max_ffn = max(w.ffn, w.shared_ffn if sh is not None else 0)
-    L = MoeLayer(w.hidden, w.n_experts, max_ffn, max_tokens or w.n_tokens, w.top_k, w.grid_iq2, w.grid_iq1, pool,
-                 device=device)
-    for i in range(0, len(ids), 32):
-        chunk = ids[i:i + 32]
-        N._check(L.upload(chunk, [w.expert(e) for e in chunk]), "upload")
-    if sh is not None:
-        N._check(L.set_shared(sh), "set_shared")
-    return L

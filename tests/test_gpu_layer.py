@@ -8,6 +8,7 @@ import pytest
 import torch
 
 import fixtures
+from bench import layer_for_workload
 
 pytestmark = pytest.mark.gpu
 
@@ -42,7 +43,7 @@ def _rel_err(got, ref):
 @pytest.mark.parametrize("cfg", [1, 2, 3])
 def test_decode_workloads(P, oracle_lib, cfg):
     w = fixtures.workload(cfg)
-    L = P.layer_for_workload(w)
+    L = layer_for_workload(w)
     got = _run(L, w.x, w.ids, w.weights)
     ref = oracle_lib.workload_layer(w)
     assert L.read_status() == 0
@@ -52,14 +53,14 @@ def test_decode_workloads(P, oracle_lib, cfg):
 def test_cold_upload_counters(P):
     """A cold top-10 selection makes 10 experts resident with 30 matrix copies."""
     w = fixtures.workload(3)
-    L = P.layer_for_workload(w)
+    L = layer_for_workload(w)
     assert (L.counters.loads, L.counters.copies) == (10, 30)
     assert L.counters.bytes == 10 * fixtures.expert_bytes(2, 2048, 512)
 
 
 def test_batched_decode_workload(P, oracle_lib):
     w = fixtures.workload(4)
-    L = P.layer_for_workload(w)
+    L = layer_for_workload(w)
     got = _run(L, w.x, w.ids, w.weights)
     ref = oracle_lib.workload_layer(w)
     assert L.read_status() == 0
@@ -68,7 +69,7 @@ def test_batched_decode_workload(P, oracle_lib):
 
 def test_prefill_small(P, oracle_lib):
     w = fixtures.workload(5, n_tokens=192)
-    L = P.layer_for_workload(w)
+    L = layer_for_workload(w)
     got = _run(L, w.x, w.ids, w.weights)
     ref = oracle_lib.workload_layer(w)
     assert L.read_status() == 0
@@ -77,7 +78,7 @@ def test_prefill_small(P, oracle_lib):
 
 def test_prefill_full_sampled(P, oracle_lib):
     w = fixtures.workload(5)
-    L = P.layer_for_workload(w)
+    L = layer_for_workload(w)
     got = _run(L, w.x, w.ids, w.weights)
     sample = np.arange(0, 4096, 173)
     ref = oracle_lib.workload_layer(w, tokens=sample)
@@ -88,7 +89,7 @@ def test_prefill_full_sampled(P, oracle_lib):
 
 def test_slot_order_and_zero_weight(P):
     w = fixtures.workload(2)
-    L = P.layer_for_workload(w)
+    L = layer_for_workload(w)
     base = _run(L, w.x, w.ids, w.weights)
     perm = np.array([3, 9, 0, 5, 1, 8, 2, 7, 4, 6])
     permuted = _run(L, w.x, w.ids[:, perm], w.weights[:, perm])
@@ -102,7 +103,7 @@ def test_slot_order_and_zero_weight(P):
 
 def test_aliased_ids_equal_single_expert(P):
     w = fixtures.workload(2)
-    L = P.layer_for_workload(w)
+    L = layer_for_workload(w)
     e = int(w.ids[0, 0])
     ids = np.full((1, 4), e, np.int32)
     wt = np.array([[0.125, 0.25, 0.375, 0.25]], np.float32)
@@ -113,7 +114,7 @@ def test_aliased_ids_equal_single_expert(P):
 
 def test_bad_ids_reported_and_skipped(P, oracle_lib):
     w = fixtures.workload(2)
-    L = P.layer_for_workload(w)
+    L = layer_for_workload(w)
     ids = w.ids.copy()
     ids[0, 2] = 512
     ids[0, 6] = -3
@@ -129,7 +130,7 @@ def test_bad_ids_reported_and_skipped(P, oracle_lib):
 
 def test_missing_expert_reported(P):
     w = fixtures.workload(2)
-    L = P.layer_for_workload(w)
+    L = layer_for_workload(w)
     ids = w.ids.copy()
     free = next(e for e in range(512) if e not in set(w.ids[0].tolist()))
     ids[0, 0] = free  # slot never uploaded: null matrices
@@ -153,7 +154,7 @@ def test_bad_and_missing_ids_on_bucketed_paths(P):
     bad[0, 2], bad[5, 7], bad[9, 0] = 512, -3, missing
     w0 = wt.copy()
     w0[0, 2] = w0[5, 7] = w0[9, 0] = 0
-    L = P.layer_for_workload(w, experts=sel, max_tokens=128)
+    L = layer_for_workload(w, experts=sel, max_tokens=128)
     for general in (False, True):
         if general:
             L.table.min_ffn = 0  # unknown widths: the general CUDA-core path runs
@@ -190,7 +191,7 @@ def test_max_topk_and_ragged_shapes(P, oracle_lib):
 
 def test_zero_tokens_noop(P):
     w = fixtures.workload(1)
-    L = P.layer_for_workload(w)
+    L = layer_for_workload(w)
     out = torch.full((1, 256), 7.0, device="cuda")
     e = torch.zeros((1, 4), dtype=torch.int32, device="cuda")
     rc = P.redlite_moe_layer(out, 0, e, out, 4, L.table, None, out)
@@ -200,7 +201,7 @@ def test_zero_tokens_noop(P):
 
 def test_repeat_calls_reuse_workspace(P):
     w = fixtures.workload(2)
-    L = P.layer_for_workload(w)
+    L = layer_for_workload(w)
     a = _run(L, w.x, w.ids, w.weights)
     for _ in range(3):
         b = _run(L, w.x, w.ids, w.weights)
@@ -212,7 +213,7 @@ def test_batched_token_counts(P, oracle_lib, T):
     """Mixed-format batched decode with the shared expert at several token
     counts: local activation limbs (T <= 4) and the cooperative conversion."""
     w = fixtures.workload(4, n_tokens=T)
-    L = P.layer_for_workload(w)
+    L = layer_for_workload(w)
     got = _run(L, w.x, w.ids, w.weights)
     ref = oracle_lib.workload_layer(w)
     assert L.read_status() == 0
@@ -221,7 +222,7 @@ def test_batched_token_counts(P, oracle_lib, T):
 
 def test_general_path_agrees_with_fast_path(P):
     w = fixtures.workload(4, n_tokens=9)
-    L = P.layer_for_workload(w)
+    L = layer_for_workload(w)
     fast = _run(L, w.x, w.ids, w.weights)
     L.table.min_ffn = 0  # unknown widths: the general CUDA-core path runs
     general = _run(L, w.x, w.ids, w.weights)
@@ -238,7 +239,7 @@ def test_tensor_core_path_mixed_formats(P, oracle_lib):
     ids, wt = fixtures.softmax_topk_routing(logits, 10)
     x = fixtures.make_x(991, 128, 2048)
     sel = sorted(set(ids.reshape(-1).tolist()))
-    L = P.layer_for_workload(w, experts=sel, max_tokens=128)
+    L = layer_for_workload(w, experts=sel, max_tokens=128)
     got = _run(L, x, ids, wt)
     experts = [None] * 512
     for e in sel:
@@ -268,7 +269,7 @@ def test_tensor_core_tile_boundaries(P, oracle_lib):
     st = fixtures.Stream(257, 4)
     wt = (st.uniform(T * 3).reshape(T, 3) + 0.1).astype(np.float32)
     x = fixtures.make_x(257, T, w.hidden)
-    L = P.layer_for_workload(w, experts=sel, max_tokens=T)
+    L = layer_for_workload(w, experts=sel, max_tokens=T)
     got = _run(L, x, ids, wt)
     experts = [None] * 512
     for e in sel:
@@ -301,7 +302,7 @@ def test_tensor_core_path_is_repeatable(P):
     wt = st.uniform(T * K).reshape(T, K).astype(np.float32) + np.float32(0.05)
     wt = (wt / wt.sum(axis=1, keepdims=True)).astype(np.float32)
     x = fixtures.make_x(5150, T, w.hidden)
-    L = P.layer_for_workload(w, experts=pool, max_tokens=T)
+    L = layer_for_workload(w, experts=pool, max_tokens=T)
     outs = [_run(L, x, ids, wt) for _ in range(8)]
     assert L.read_status() == 0
     scale = np.abs(outs[0]).max()
@@ -328,7 +329,7 @@ def test_tensor_core_path_matches_bf16_operand_reference(P, oracle_lib):
     wt = st.uniform(T * K).reshape(T, K).astype(np.float32) + np.float32(0.05)
     wt = (wt / wt.sum(axis=1, keepdims=True)).astype(np.float32)
     x = fixtures.make_x(4242, T, H)
-    L = P.layer_for_workload(w, experts=pool, max_tokens=T)
+    L = layer_for_workload(w, experts=pool, max_tokens=T)
     got = _run(L, x, ids, wt)
     assert L.read_status() == 0
 
@@ -362,7 +363,7 @@ def test_grid_wait_gives_up_and_reports(P):
     REDLITE_STATUS_TIMEOUT, and leaves the context and the workspace usable:
     the next call returns the right result with a clean status."""
     w = fixtures.workload(2)
-    L = P.layer_for_workload(w)
+    L = layer_for_workload(w)
     ref = _run(L, w.x, w.ids, w.weights)
     assert L.read_status() == 0
     ctrl = L.workspace.view(torch.int32)

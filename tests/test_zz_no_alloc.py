@@ -10,6 +10,7 @@ import pytest
 import torch
 
 import fixtures
+from bench import layer_for_workload
 
 pytestmark = pytest.mark.gpu
 
@@ -29,7 +30,7 @@ def P():
 @pytest.mark.parametrize("cfg,T", [(2, None), (4, 9)])
 def test_no_alloc_matches_workspace_entry_point(P, cfg, T):
     w = fixtures.workload(cfg, n_tokens=T) if T else fixtures.workload(cfg)
-    L = P.layer_for_workload(w)
+    L = layer_for_workload(w)
     x = torch.from_numpy(w.x).cuda()
     ids = torch.from_numpy(w.ids).cuda()
     wt = torch.from_numpy(w.weights).cuda()
@@ -49,7 +50,7 @@ def test_no_alloc_matches_workspace_entry_point(P, cfg, T):
 
 def test_no_alloc_rejects_what_it_cannot_take(P):
     w = fixtures.workload(1)  # expert width 64: not a fused-kernel shape
-    L = P.layer_for_workload(w)
+    L = layer_for_workload(w)
     x = torch.from_numpy(w.x).cuda()
     ids = torch.from_numpy(w.ids).cuda()
     wt = torch.from_numpy(w.weights).cuda()
@@ -65,7 +66,7 @@ def test_no_alloc_refusals_leave_out_untouched(P):
     import copy
 
     w = fixtures.workload(4)  # 64 tokens x top-10 + shared expert
-    L = P.layer_for_workload(w)
+    L = layer_for_workload(w)
     x = torch.from_numpy(w.x).cuda()
     ids = torch.from_numpy(w.ids).cuda()
     wt = torch.from_numpy(w.weights).cuda()
