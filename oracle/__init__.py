@@ -73,6 +73,13 @@ def lib():
             ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
         ]
         L.oracle_set_threads.argtypes = [ctypes.c_int]
+        L.oracle_route_topk.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_void_p,
+                                        ctypes.c_void_p]
+        L.oracle_moe_block.argtypes = [
+            ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_void_p, ctypes.c_double, ctypes.c_void_p,
+            ctypes.c_int, ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+            ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+        ]
         _lib = L
     return _lib
 
@@ -179,3 +186,38 @@ def workload_layer(w, tokens: Optional[Sequence[int]] = None):
         x, ids, wt = x[tokens], ids[tokens], wt[tokens]
     return moe_layer(x, ids, wt, experts, w.shared(), expand_grid(QTYPE_IQ2XS, w.grid_iq2),
                      expand_grid(QTYPE_IQ1M, w.grid_iq1))
+
+
+def route_topk(logits, top_k: int):
+    """The oracle router: (ids int32 [T, k], weights float64 [T, k]) from float logits [T, E]."""
+    lg = np.ascontiguousarray(logits, dtype=np.float32)
+    T, E = lg.shape
+    ids = np.zeros((T, top_k), dtype=np.int32)
+    w = np.zeros((T, top_k), dtype=np.float64)
+    rc = lib().oracle_route_topk(_ptr(lg), T, E, top_k, _ptr(ids), _ptr(w))
+    if rc != OK:
+        raise ValueError(f"oracle_route_topk failed ({rc})")
+    return ids, w
+
+
+def moe_block(h, gamma, eps: float, router_w, top_k: int, experts: Sequence, shared=None, grid_iq2=None,
+              grid_iq1=None, return_routing: bool = False):
+    """The oracle block out = h + layer(RMSNorm(h)) with its own routing; float64 [T, H]
+    (and the routing ids / weights when asked)."""
+    h = np.ascontiguousarray(h, dtype=np.float32)
+    T, H = h.shape
+    g = np.ascontiguousarray(gamma, dtype=np.float32)
+    rw = np.ascontiguousarray(router_w, dtype=np.float32)
+    E = rw.shape[0]
+    es = ExpertSet(experts)
+    sh = ExpertSet([shared]) if shared is not None else None
+    g2 = None if grid_iq2 is None else np.ascontiguousarray(grid_iq2, dtype=np.int8)
+    g1 = None if grid_iq1 is None else np.ascontiguousarray(grid_iq1, dtype=np.int8)
+    out = np.zeros((T, H), dtype=np.float64)
+    ids = np.zeros((T, top_k), dtype=np.int32)
+    w = np.zeros((T, top_k), dtype=np.float64)
+    rc = lib().oracle_moe_block(_ptr(h), T, H, _ptr(g), float(eps), _ptr(rw), E, top_k, es.ptr,
+                                sh.ptr if sh is not None else None, _ptr(g2), _ptr(g1), _ptr(out), _ptr(ids), _ptr(w))
+    if rc < 0:
+        raise ValueError(f"oracle_moe_block failed ({rc})")
+    return (out, ids, w) if return_routing else out

@@ -246,6 +246,142 @@ int oracle_moe_layer(const float *x, int n_tokens, int hidden, const int32_t *id
   return skipped ? ORACLE_SKIPPED_PAIRS : ORACLE_OK;
 }
 
+/* ------------------------------------------------------------------ router
+ * The step that feeds the layer its expert ids and router weights.  The
+ * pages name it as the milestone after the routed layer ("Red Metal dev8",
+ * section "Field validation": router-network integration and real token
+ * router outputs; "Red Lite dev10", section "What dev10 does not yet claim":
+ * connect the actual router output to the top-k path) without stating its
+ * arithmetic.  Reading (the router of the Qwen3-Next layers the pages run,
+ * and the recipe of the batched-decode workload): per token,
+ *   1. p = softmax(logits) over the n_experts logits (the largest logit is
+ *      subtracted before exp; exp is libm's, in double);
+ *   2. the top_k experts by p, in descending order of p, equal p going to
+ *      the lower id first;
+ *   3. their probabilities renormalised to sum 1: w_j = p_j / sum of the
+ *      selected p. */
+static void route_token(const double *lg, int n_experts, int top_k, double *p, char *taken, int32_t *ids,
+                        double *w) {
+  /* step 1: softmax */
+  double m = lg[0];
+  for (int e = 1; e < n_experts; ++e)
+    if (lg[e] > m) m = lg[e];
+  double sum = 0.0;
+  for (int e = 0; e < n_experts; ++e) {
+    p[e] = exp(lg[e] - m);
+    sum += p[e];
+  }
+  for (int e = 0; e < n_experts; ++e) p[e] /= sum;
+  /* step 2: top_k by probability, one at a time; only a strictly larger p
+   * replaces the current choice, so equal p keep the lower id */
+  memset(taken, 0, (size_t)n_experts);
+  double sel = 0.0;
+  for (int j = 0; j < top_k; ++j) {
+    int best = -1;
+    for (int e = 0; e < n_experts; ++e)
+      if (!taken[e] && (best < 0 || p[e] > p[best])) best = e;
+    taken[best] = 1;
+    ids[j] = best;
+    w[j] = p[best];
+    sel += p[best];
+  }
+  /* step 3: renormalise over the selected experts */
+  for (int j = 0; j < top_k; ++j) w[j] /= sel;
+}
+
+/* ids: [n_tokens, top_k]; weights: [n_tokens, top_k] doubles. */
+int oracle_route_topk(const float *logits, int n_tokens, int n_experts, int top_k, int32_t *ids,
+                      double *weights) {
+  if (n_tokens < 0 || n_experts <= 0 || top_k <= 0 || top_k > n_experts) return ORACLE_EINVAL;
+  if (n_tokens == 0) return ORACLE_OK;
+  if (!logits || !ids || !weights) return ORACLE_EINVAL;
+  double *lg = (double *)malloc(sizeof(double) * n_experts);
+  double *p = (double *)malloc(sizeof(double) * n_experts);
+  char *taken = (char *)malloc((size_t)n_experts);
+  for (int t = 0; t < n_tokens; ++t) {
+    for (int e = 0; e < n_experts; ++e) lg[e] = (double)logits[(int64_t)t * n_experts + e];
+    route_token(lg, n_experts, top_k, p, taken, ids + (int64_t)t * top_k, weights + (int64_t)t * top_k);
+  }
+  free(lg);
+  free(p);
+  free(taken);
+  return ORACLE_OK;
+}
+
+/* ------------------------------------------------------------------ block
+ * The composition around the layer ("Red Lite dev16 -- complete
+ * full-attention parity", block composition paragraph: the attention
+ * residual, the post-attention RMSNorm, the routed top-10 MoE plus shared
+ * expert, and the final residual).  For every token, h being the hidden
+ * state after the attention residual:
+ *   1. xn = RMSNorm(h): xn_i = gamma_i * h_i / sqrt(mean_j(h_j^2) + eps)
+ *      (reading: the plain RMSNorm with a multiplicative weight);
+ *   2. logits = W_r xn (router matrix [n_experts, hidden]);
+ *   3. ids, weights = the router above applied to the logits;
+ *   4. y = the routed layer of xn with those ids and weights, plus the
+ *      shared expert with weight 1 (oracle_moe_layer's definition);
+ *   5. out = h + y.
+ * Every step is in double: xn and the logits are not rounded to float.
+ * ids_out, weights_out (optional): the routing chosen in step 3. */
+int oracle_moe_block(const float *h, int n_tokens, int hidden, const float *gamma, double eps,
+                     const float *router_w, int n_experts, int top_k, const oracle_expert *experts,
+                     const oracle_expert *shared, const int8_t *grid_iq2, const int8_t *grid_iq1, double *out,
+                     int32_t *ids_out, double *weights_out) {
+  if (n_tokens < 0 || hidden <= 0 || n_experts <= 0 || top_k <= 0 || top_k > n_experts || eps < 0.0)
+    return ORACLE_EINVAL;
+  if (n_tokens == 0) return ORACLE_OK;
+  if (!h || !gamma || !router_w || !experts || !out) return ORACLE_EINVAL;
+  if (shared && !expert_ok(shared, hidden, grid_iq2, grid_iq1)) return ORACLE_EINVAL;
+  int skipped = 0;
+#pragma omp parallel for schedule(dynamic, 1) reduction(| : skipped)
+  for (int t = 0; t < n_tokens; ++t) {
+    const float *ht = h + (int64_t)t * hidden;
+    double *xn = (double *)malloc(sizeof(double) * hidden);
+    double *lg = (double *)malloc(sizeof(double) * n_experts);
+    double *p = (double *)malloc(sizeof(double) * n_experts);
+    char *taken = (char *)malloc((size_t)n_experts);
+    int32_t *ids = (int32_t *)malloc(sizeof(int32_t) * top_k);
+    double *w = (double *)malloc(sizeof(double) * top_k);
+    double *acc = out + (int64_t)t * hidden;
+    /* step 1 */
+    double ss = 0.0;
+    for (int i = 0; i < hidden; ++i) ss += (double)ht[i] * (double)ht[i];
+    const double inv = 1.0 / sqrt(ss / hidden + eps);
+    for (int i = 0; i < hidden; ++i) xn[i] = (double)gamma[i] * (double)ht[i] * inv;
+    /* step 2 */
+    for (int e = 0; e < n_experts; ++e) {
+      double s = 0.0;
+      for (int i = 0; i < hidden; ++i) s += (double)router_w[(int64_t)e * hidden + i] * xn[i];
+      lg[e] = s;
+    }
+    /* step 3 */
+    route_token(lg, n_experts, top_k, p, taken, ids, w);
+    /* step 4 (as in oracle_moe_layer, with xn in double) */
+    for (int r = 0; r < hidden; ++r) acc[r] = 0.0;
+    for (int s = 0; s < top_k; ++s) {
+      if (!expert_ok(&experts[ids[s]], hidden, grid_iq2, grid_iq1)) {
+        skipped = 1;
+        continue;
+      }
+      expert_ffn_accumulate(&experts[ids[s]], hidden, xn, grid_iq2, grid_iq1, w[s], acc, 0);
+    }
+    if (shared) expert_ffn_accumulate(shared, hidden, xn, grid_iq2, grid_iq1, 1.0, acc, 0);
+    /* step 5 */
+    for (int i = 0; i < hidden; ++i) acc[i] += (double)ht[i];
+    for (int j = 0; j < top_k; ++j) {
+      if (ids_out) ids_out[(int64_t)t * top_k + j] = ids[j];
+      if (weights_out) weights_out[(int64_t)t * top_k + j] = w[j];
+    }
+    free(xn);
+    free(lg);
+    free(p);
+    free(taken);
+    free(ids);
+    free(w);
+  }
+  return skipped ? ORACLE_SKIPPED_PAIRS : ORACLE_OK;
+}
+
 int oracle_set_threads(int n) {
 #ifdef _OPENMP
   if (n > 0) omp_set_num_threads(n);

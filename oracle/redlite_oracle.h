@@ -15,7 +15,10 @@
  *     optional shared expert with weight 1
  *       ("Red Metal dev8 -- resident routed top-k layer", steps 1-6;
  *        "Red Lite dev16 -- complete full-attention parity", the block
- *        composition paragraph: routed top-10 MoE plus shared expert).
+ *        composition paragraph: routed top-10 MoE plus shared expert);
+ *   - the router that feeds the layer (softmax, top-k, renormalisation) and
+ *     the block around it (RMSNorm, router, layer, residual), the steps the
+ *     pages name as the next milestones.
  *
  * Parity status: every function here is pinned by tests that do not call
  * back into this library (hand-computed golden blocks, closed forms,
@@ -76,6 +79,23 @@ int oracle_moe_layer(const float *x, int n_tokens, int hidden, const int32_t *id
                      const float *weights, int top_k, int n_experts,
                      const oracle_expert *experts, const oracle_expert *shared,
                      const int8_t *grid_iq2, const int8_t *grid_iq1, double *out);
+
+/* The router: per token softmax over the n_experts float logits (fp64),
+ * the top_k experts by probability in descending order (ties to the lower
+ * id), their probabilities renormalised to sum 1.  ids, weights:
+ * [n_tokens, top_k] (int32, double). */
+int oracle_route_topk(const float *logits, int n_tokens, int n_experts, int top_k, int32_t *ids,
+                      double *weights);
+
+/* The post-attention block around the layer: out = h + layer(RMSNorm(h)),
+ * RMSNorm with weight gamma [hidden] and eps, routed by the router above on
+ * logits = router_w [n_experts, hidden] times the normalised state, plus
+ * the optional shared expert; all in double.  ids_out / weights_out
+ * ([n_tokens, top_k], optional) receive the routing. */
+int oracle_moe_block(const float *h, int n_tokens, int hidden, const float *gamma, double eps,
+                     const float *router_w, int n_experts, int top_k, const oracle_expert *experts,
+                     const oracle_expert *shared, const int8_t *grid_iq2, const int8_t *grid_iq1, double *out,
+                     int32_t *ids_out, double *weights_out);
 
 /* Threads used by oracle_moe_layer (OpenMP build); returns the value in force. */
 int oracle_set_threads(int n);
