@@ -79,7 +79,7 @@ int redlite_moe_layer(const float *x, int32_t n_tokens, const int32_t *expert_id
   cudaStream_t s = (cudaStream_t)t->stream;
   uint8_t *ws = (uint8_t *)t->workspace;
 
-  if (tiled && fused_supported(t->hidden, t->max_ffn, n_tokens, top_k, t->n_experts, shared != nullptr)) {
+  if (tiled && fused_supported(t->hidden, t->max_ffn, n_tokens, top_k, t->n_experts, shared != nullptr, device_sms())) {
     FusedArgs fa{};
     fa.x = x;
     fa.ids = expert_ids;

@@ -202,19 +202,21 @@ __device__ __forceinline__ void dequant_q2(const Q2Lane &L, int s, uint32_t A, i
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
       const int f = 2 * c2 + h;
-      const uint32_t qsb = (qw >> (8 * f)) & 0xFFu, sgb = (sw >> (8 * f)) & 0xFFu;
+      // sign word s holds bit j of field 4s + f at bit 4j + f
+      const uint32_t qsb = (qw >> (8 * f)) & 0xFFu, sgz = (sw >> f) & 0x11111111u;
       const uint32_t idx = qsb | (((L.qh >> (4 * s + f)) & 1u) << 8);
       const uint2 sel = ptx::lds64_const(sel2 + 8 * idx);
       const uint32_t nib = ((h ? L.sc1 : L.sc0) >> (4 * c)) & 15u;
       const float sc = (h ? L.d1 : L.d0) * odd_f(nib);
       const uint32_t t0 = bf16x2(sc * 8.f, sc * 25.f), t1 = bf16x2(sc * 43.f, 0.f);
-      // sign bits 2w, 2w+1 -> bits 15, 31 of pair w: b * (2^(15-2w) + 2^(30-2w)), masked
-      // (the two shifted copies of b never overlap, so no carries)
+      // sign bits 2w, 2w+1 sit at bits 0 and 4 of byte w of sgz: that byte
+      // times 2^15 + 2^27 puts them at bits 15 and 31 of pair w (masked; the
+      // two shifted copies never overlap, so no carries)
       uint4 v;
-      v.x = __byte_perm(t0, t1, sel.x) ^ ((sgb * 0x40008000u) & 0x80008000u);
-      v.y = __byte_perm(t0, t1, sel.x >> 16) ^ ((sgb * 0x10002000u) & 0x80008000u);
-      v.z = __byte_perm(t0, t1, sel.y) ^ ((sgb * 0x04000800u) & 0x80008000u);
-      v.w = __byte_perm(t0, t1, sel.y >> 16) ^ ((sgb * 0x01000200u) & 0x80008000u);
+      v.x = __byte_perm(t0, t1, sel.x) ^ ((__byte_perm(sgz, 0u, 0x4440u) * 0x08008000u) & 0x80008000u);
+      v.y = __byte_perm(t0, t1, sel.x >> 16) ^ ((__byte_perm(sgz, 0u, 0x4441u) * 0x08008000u) & 0x80008000u);
+      v.z = __byte_perm(t0, t1, sel.y) ^ ((__byte_perm(sgz, 0u, 0x4442u) * 0x08008000u) & 0x80008000u);
+      v.w = __byte_perm(t0, t1, sel.y >> 16) ^ ((__byte_perm(sgz, 0u, 0x4443u) * 0x08008000u) & 0x80008000u);
       ptx::sts128(A + ptx::sw128_offset(row0 + q + 8 * h, 32 * c2 + 8 * t), v);
     }
   }

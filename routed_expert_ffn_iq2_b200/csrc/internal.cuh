@@ -202,7 +202,10 @@ __device__ __forceinline__ void decode_group_f32(const uint8_t *__restrict__ mat
       const Q2Loc o = q2_loc(rr, g);
       idx = tb[o.qs] | (((ld_u16(tb + o.qh_word) >> o.qh_bit) & 1) << 8);
       sc = (tb[o.scales + (g >> 3)] >> (4 * ((g >> 2) & 1))) & 15;
-      s = tb[o.sign];
+      const uint32_t sw = (uint32_t)tb[o.sign_word] | ((uint32_t)tb[o.sign_word + 1] << 8) |
+                          ((uint32_t)tb[o.sign_word + 2] << 16) | ((uint32_t)tb[o.sign_word + 3] << 24);
+#pragma unroll
+      for (int j = 0; j < 8; ++j) s |= ((sw >> (4 * j + o.sign_shift)) & 1u) << j;
       d = fp16_bits_to_float(ld_u16(tb + o.d));
     } else {
       const Q1Loc o = q1_loc(rr, g);
@@ -311,7 +314,10 @@ struct FusedArgs {
   WorkspaceLayout L;
   int32_t *status;
 };
-bool fused_supported(int hidden, int max_ffn, int n_tokens, int top_k, int n_experts, bool has_shared);
+// Whether the fused decode kernel takes a call; sms: the device's SM count
+// (0 if unknown: a B200's 148 is assumed).
+bool fused_supported(int hidden, int max_ffn, int n_tokens, int top_k, int n_experts, bool has_shared, int sms);
+int device_sms();
 
 // Tensor-core (tcgen05) grouped path: tokens per work unit, and the launch.
 constexpr int kTcTokens = 128;

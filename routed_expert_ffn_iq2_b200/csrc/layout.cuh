@@ -15,7 +15,10 @@
 // IQ2_XS-style tile-block (1184 bytes).  Lane L handles groups g = 4c + t
 // (c = 0..7) of rows q (h = 0) and q+8 (h = 1); field index i = 2c + h.
 //   [32L + i]        qs[g] of row q+8h
-//   [32L + 16 + i]   signs[g] of row q+8h
+//   [32L + 16 + 4w]  u32 sign word w (w = 0..3): bit 4j + m = sign bit j of
+//                    field i = 4w + m (bit j of signs[g] of row q+8h), so
+//                    shifting word w left by 2 - m puts the sign of weight j
+//                    at bit 4j + 2 of every nibble
 //   [1024 + 2L]      u16: bit i = index bit 8 of that group
 //   [1088 + 8q]      scales[0..3] of row q, then scales[0..3] of row q+8
 //   [1152 + 4q]      d of row q, then d of row q+8
@@ -49,14 +52,15 @@ inline __host__ __device__ int64_t tile_block_offset(int qtype, int64_t k, int64
 
 // Field offsets of (row-in-tile rr, group g) inside an IQ2 tile-block.
 struct Q2Loc {
-  int qs, sign, qh_word, qh_bit, scales, d;
+  int qs, sign_word, sign_shift, qh_word, qh_bit, scales, d;
 };
 inline __host__ __device__ Q2Loc q2_loc(int rr, int g) {
   const int q = rr & 7, h = rr >> 3, c = g >> 2, t = g & 3;
   const int L = 4 * q + t, i = 2 * c + h;
   Q2Loc o;
   o.qs = 32 * L + i;
-  o.sign = 32 * L + 16 + i;
+  o.sign_word = 32 * L + 16 + 4 * (i >> 2);
+  o.sign_shift = i & 3;
   o.qh_word = 1024 + 2 * L;
   o.qh_bit = i;
   o.scales = 1088 + 8 * q + 4 * h;

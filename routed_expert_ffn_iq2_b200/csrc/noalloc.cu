@@ -77,7 +77,7 @@ extern "C" int redlite_moe_layer_noalloc(const float *x, int32_t n_tokens, const
   // redlite_moe_layer does on that path
   if (shared && !shared_ok(*shared, t, true)) return REDLITE_EINVAL;
   // only the fused decode kernel runs here
-  if (t->min_ffn < 256 || !fused_supported(t->hidden, t->max_ffn, n_tokens, top_k, t->n_experts, shared != nullptr))
+  if (t->min_ffn < 256 || !fused_supported(t->hidden, t->max_ffn, n_tokens, top_k, t->n_experts, shared != nullptr, device_sms()))
     return REDLITE_EUNSUPPORTED;
   const WorkspaceLayout L = noalloc_layout(t->hidden, n_tokens, top_k, t->max_ffn);
   if (L.total > kNoAllocScratchBytes) return REDLITE_ENOMEM;

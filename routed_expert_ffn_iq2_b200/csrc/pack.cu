@@ -14,7 +14,10 @@ static void pack_tile_block_q2(const uint8_t *src, int64_t k, int64_t r0, int64_
     for (int g = 0; g < 32; ++g) {
       const Q2Loc o = q2_loc(rr, g);
       tb[o.qs] = b[6 + g];
-      tb[o.sign] = b[42 + g];
+      for (int j = 0; j < 8; ++j) {  // sign bit j -> bit 4j + m of the field's sign word
+        const int bit = 4 * j + o.sign_shift;
+        tb[o.sign_word + (bit >> 3)] |= (uint8_t)(((b[42 + g] >> j) & 1) << (bit & 7));
+      }
       const int hb = (b[38 + (g >> 3)] >> (g & 7)) & 1;
       uint16_t w = (uint16_t)(tb[o.qh_word] | (tb[o.qh_word + 1] << 8));
       w |= (uint16_t)(hb << o.qh_bit);

@@ -39,7 +39,8 @@ def test_iq2_tile_fields(P, rows, k):
             for g in range(32):
                 L, i = 4 * q + (g & 3), 2 * (g >> 2) + h
                 assert tb[32 * L + i] == blk[6 + g]
-                assert tb[32 * L + 16 + i] == blk[42 + g]
+                sw = int.from_bytes(bytes(tb[32 * L + 16 + 4 * (i // 4):32 * L + 20 + 4 * (i // 4)]), "little")
+                assert sum(((sw >> (4 * j + i % 4)) & 1) << j for j in range(8)) == blk[42 + g]
                 qh = int(tb[1024 + 2 * L]) | (int(tb[1025 + 2 * L]) << 8)
                 assert (qh >> i) & 1 == (blk[38 + g // 8] >> (g % 8)) & 1
             assert bytes(tb[1088 + 8 * q + 4 * h:1088 + 8 * q + 4 * h + 4]) == bytes(blk[2:6])

@@ -63,8 +63,6 @@ def test_no_alloc_refusals_leave_out_untouched(P):
     """Calls the fixed scratch array cannot serve, and malformed shared
     experts, are refused on the host before anything is enqueued: out keeps
     its contents and the status word stays clear."""
-    import copy
-
     w = fixtures.workload(4)  # 64 tokens x top-10 + shared expert
     L = layer_for_workload(w)
     x = torch.from_numpy(w.x).cuda()
@@ -72,7 +70,7 @@ def test_no_alloc_refusals_leave_out_untouched(P):
     wt = torch.from_numpy(w.weights).cuda()
     out = torch.full_like(x, 3.5)
     # declared max_ffn 2048: 704 pairs x 2 x 2048 fp32 gate/up values do not fit 4 MiB
-    big = copy.copy(L.table)
+    big = P.redlite_moe_table.from_buffer_copy(bytes(L.table))
     big.max_ffn = 2048
     rc = P.redlite_moe_layer_noalloc(x, x.shape[0], ids, wt, w.top_k, big, L.shared, out)
     assert rc == P.REDLITE_ENOMEM
