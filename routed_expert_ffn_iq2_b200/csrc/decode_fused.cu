@@ -42,8 +42,8 @@ namespace redlite {
 
 constexpr int kCWarps = 16;                // warps per CTA (all consume)
 constexpr int kCThreads = 32 * kCWarps;    // 512
-constexpr int kRing = 4;                   // bulk-copy stages per warp
-constexpr int kStageBytes = kQ2TileBlock;  // 1184 >= kQ1TileBlock
+constexpr int kRing = 4;                   // item stages in flight
+constexpr int kStageBytes = kQ2TileBlock;  // per warp and stage: 1184 >= kQ1TileBlock
 constexpr int kLimbPadW = 32;              // padding per limb plane (spreads shared-memory banks)
 constexpr int kRedSlots = 6;               // reduction slots (items in flight)
 constexpr int kRedLag = 2;                 // an item is reduced this many items after its own
@@ -96,13 +96,14 @@ __device__ __forceinline__ int groups_of(int rows, int nkb, int phase) {
 struct Smem {
   uint32_t *sel2, *sel1;
   uint32_t *items;  // [kMaxItems] this CTA's item list
-  uint8_t *ring;   // [kCWarps][kRing][kStageBytes]
+  uint8_t *ring;   // [kRing][kCWarps][kStageBytes]: stage s holds item k = s mod kRing
+  int *left;       // [kRing]: warps not yet done with the stage's item
   float *red;      // [kRedSlots][kCWarps][kRedFloats]
   uint8_t *wlimbs;  // [kCWarps][2 positions][3 limbs][kWPlane]: each warp's input slice
   Inst *inst;
   int *pair_tok;
   float *pair_w;
-  uint64_t *full;    // [kCWarps][kRing]: stage landed
+  uint64_t *full;    // [kRing]: stage landed
   uint64_t *rfull;   // [kRedSlots]: all warps' partials are in
   uint64_t *rfree;   // [kRedSlots]: the reducer is done with the slot
 };
@@ -251,10 +252,10 @@ __device__ __forceinline__ void to_limbs(float v, float scale, int &l0, int &l1,
 #ifdef REDLITE_TRACE
 #define TR_DECL long long tr_[10] = {0}; long long tr0_ = clock64()
 #define TR(i) do { const long long t_ = clock64(); tr_[i] += t_ - tr0_; tr0_ = t_; } while (0)
-#define TR_STAMP(i) do { if (threadIdx.x == 0) { uint64_t g_; asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(g_)); \
-    reinterpret_cast<uint64_t *>(a.ws + a.L.total)[blockIdx.x * 16 + (i)] = g_; } } while (0)
+#define TR_STAMP(i) do { if ((threadIdx.x & 31) == 0) { uint64_t g_; asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(g_)); \
+    reinterpret_cast<uint64_t *>(a.ws + a.L.total)[blockIdx.x * 32 + (i)] = g_; } } while (0)
 #define TR_FLUSH() do { if (lane == 0) for (int i_ = 0; i_ < 10; ++i_) \
-    reinterpret_cast<uint64_t *>(a.ws + a.L.total)[4096 + (blockIdx.x * 16 + warp) * 10 + i_] = tr_[i_]; } while (0)
+    reinterpret_cast<uint64_t *>(a.ws + a.L.total)[8192 + (blockIdx.x * 16 + warp) * 10 + i_] = tr_[i_]; } while (0)
 #else
 #define TR_DECL
 #define TR(i)
@@ -372,16 +373,15 @@ __device__ __forceinline__ void tb_q1(uint32_t tb, uint32_t sel1, uint32_t bp, b
   acc[3] += d1 * (float)cb[3];
 }
 
-// Combine the limb columns of each token position, apply the positions'
-// limb scales sc0, sc1 and store this warp's partial sums to
-// red[2 * row + position] (16 rows x 2 positions).
-__device__ __forceinline__ void store_partials(const float acc[4], float sc0, float sc1, float *red) {
-  const int lane = threadIdx.x & 31, q = lane >> 2, t = lane & 3;
+// Combine the limb columns of each token position: v = (row q, pos 0),
+// (row q, pos 1), (row q+8, pos 0), (row q+8, pos 1), complete in lanes
+// with t = lane & 3 = 0.
+__device__ __forceinline__ void quad_rows(const float acc[4], float v[4]) {
+  const int t = threadIdx.x & 3;
   const int n0 = 2 * t, n1 = 2 * t + 1;
   const float f0 = n0 < 6 ? (n0 % 3 == 0 ? 16384.f : (n0 % 3 == 1 ? 128.f : 1.f)) : 0.f;
   const float f1 = n1 < 6 ? (n1 % 3 == 0 ? 16384.f : (n1 % 3 == 1 ? 128.f : 1.f)) : 0.f;
   const int m0 = n0 / 3, m1 = n1 / 3;  // token position of the column (2 = none)
-  float v[4];  // (row q, pos 0), (row q, pos 1), (row q+8, pos 0), (row q+8, pos 1)
   v[0] = (m0 == 0 ? f0 * acc[0] : 0.f) + (m1 == 0 ? f1 * acc[1] : 0.f);
   v[1] = (m0 == 1 ? f0 * acc[0] : 0.f) + (m1 == 1 ? f1 * acc[1] : 0.f);
   v[2] = (m0 == 0 ? f0 * acc[2] : 0.f) + (m1 == 0 ? f1 * acc[3] : 0.f);
@@ -391,6 +391,14 @@ __device__ __forceinline__ void store_partials(const float acc[4], float sc0, fl
     v[j] += __shfl_xor_sync(0xffffffffu, v[j], 1);
     v[j] += __shfl_xor_sync(0xffffffffu, v[j], 2);
   }
+}
+
+// Store this warp's partial sums, scaled by the positions' limb scales sc0,
+// sc1, to red[2 * row + position] (16 rows x 2 positions).
+__device__ __forceinline__ void store_partials(const float acc[4], float sc0, float sc1, float *red) {
+  const int lane = threadIdx.x & 31, q = lane >> 2, t = lane & 3;
+  float v[4];
+  quad_rows(acc, v);
   if (t == 0) {
     *reinterpret_cast<float2 *>(red + 2 * q) = make_float2(v[0] * sc0, v[1] * sc1);
     *reinterpret_cast<float2 *>(red + 2 * (q + 8)) = make_float2(v[2] * sc0, v[3] * sc1);
@@ -431,11 +439,14 @@ __device__ __noinline__ float warp_slice_limbs(const float *src, bool coherent, 
 }
 
 // Replicate the selector tables in place (word w of a table with r replicas
-// holds source word w / r; replicas spread lanes over banks): NT threads,
-// t = 0..NT-1, named barrier BAR.  Every source word is read before any is
-// overwritten.
-template <int NT, int BAR>
-__device__ __forceinline__ void replicate_tables(const Smem &S, int t) {
+// holds source word w / r; replicas spread lanes over banks): warps 1..15
+// (t = 0..479), named barrier 2.  Every source word is read before any is
+// overwritten.  Out of line: it runs once per call.
+__device__ __noinline__ void replicate_tables(uint32_t *sel2, uint32_t *sel1, int t) {
+  constexpr int NT = 480, BAR = 2;
+  struct {
+    uint32_t *sel2, *sel1;
+  } S{sel2, sel1};
   static_assert(kRep2 == 16 && kRep1 == 2, "replication below assumes 16 / 2 replicas");
   constexpr int N2 = (512 + NT - 1) / NT, N1 = (4096 + NT - 1) / NT;
   uint32_t v2[N2], v1[N1];
@@ -494,7 +505,9 @@ __global__ void __launch_bounds__(kCThreads, 1) decode_fused_kernel(FusedArgs a)
   S.pair_w = reinterpret_cast<float *>(smem + off);
   off += sizeof(float) * (kFusedMaxPairs + 64);
   S.full = reinterpret_cast<uint64_t *>(smem + off);
-  off += sizeof(uint64_t) * kCWarps * kRing;
+  off += sizeof(uint64_t) * kRing;
+  S.left = reinterpret_cast<int *>(smem + off);
+  off += sizeof(int) * kRing;
   S.rfull = reinterpret_cast<uint64_t *>(smem + off);
   off += sizeof(uint64_t) * kRedSlots;
   S.rfree = reinterpret_cast<uint64_t *>(smem + off);
@@ -509,7 +522,10 @@ __global__ void __launch_bounds__(kCThreads, 1) decode_fused_kernel(FusedArgs a)
   // One thread starts bulk copies of the two selector tables (unreplicated)
   // into the first bytes of their shared-memory regions; they are replicated
   // after the routing has been read.
-  if (tid < kCWarps * kRing) mbar_init(&S.full[tid], 1);
+  if (tid < kRing) {
+    mbar_init(&S.full[tid], 1);
+    S.left[tid] = kCWarps;
+  }
   if (tid < kRedSlots) {
     mbar_init(&S.rfull[tid], kCWarps);
     mbar_init(&S.rfree[tid], 1);
@@ -538,6 +554,7 @@ __global__ void __launch_bounds__(kCThreads, 1) decode_fused_kernel(FusedArgs a)
     my_ids[j] = p < npairs ? __ldcg(a.ids + p) : -1;
     my_w[j] = p < npairs ? __ldcg(a.weights + p) : 0.f;
   }
+  TR_STAMP(8);
   if (T <= 4)  // warm L2 for the warps' activation slices
     for (int i = tid; i < T * H / 32; i += kCThreads) asm volatile("prefetch.global.L2 [%0];" ::"l"(a.x + 32 * i));
 #pragma unroll
@@ -630,10 +647,13 @@ __global__ void __launch_bounds__(kCThreads, 1) decode_fused_kernel(FusedArgs a)
       if (lane == 0) s_bad = bad;
       __syncwarp();
       item_prefix(n_inst);
+      TR_STAMP(9);
     } else {
       // meanwhile the other warps replicate the selector tables
       mbar_wait(&s_lut_bar, 0, a.status);
-      replicate_tables<kCThreads - 32, 2>(S, tid - 32);
+      if (warp == 1) TR_STAMP(10);
+      replicate_tables(S.sel2, S.sel1, tid - 32);
+      if (warp == 1) TR_STAMP(11);
     }
   } else {
     // ---- bucketing: counts per expert in the rings (scratch before any copy)
@@ -737,120 +757,146 @@ __global__ void __launch_bounds__(kCThreads, 1) decode_fused_kernel(FusedArgs a)
     if (warp == 0) item_prefix(n_inst);
     // replicate the selector tables (the bucketing scratch in the rings is
     // not touched)
-    mbar_wait(&s_lut_bar, 0, a.status);
-    replicate_tables<kCThreads, 2>(S, tid);
+    if (warp > 0) {
+      mbar_wait(&s_lut_bar, 0, a.status);
+      replicate_tables(S.sel2, S.sel1, tid - 32);
+    }
   }
-  __syncthreads();
+  TR_STAMP(16);
 
   // ---- the item split: gate/up items evenly over the CTAs, down items in
   // reverse CTA order (a CTA with one more gate/up item tends to get one
-  // fewer down item); this CTA's items listed once
-  const int n_inst = s_n_inst, N1 = s_n1, N2 = s_n2;
-  const unsigned uG = (unsigned)G, uN1 = (unsigned)N1, uN2 = (unsigned)N2;  // products < 2^31
-  // (the host keeps every CTA's list within kMaxItems; the clamps only
-  // guard the shared-memory list)
-  const int b1 = (int)(cta * uN1 / uG), my1 = min(kMaxItems, (int)((cta + 1) * uN1 / uG) - b1);
-  const int rc = G - 1 - cta;
-  const int b2 = (int)(rc * uN2 / uG), my2 = min(kMaxItems - my1, (int)((rc + 1) * uN2 / uG) - b2);
-  const int my_items = my1 + my2;
-  for (int k = tid; k < my_items; k += kCThreads) {
-    const int phase = k < my1 ? 1 : 2;
-    const int j = phase == 1 ? b1 + k : b2 + (k - my1);
-    int lo = 0, hi = n_inst - 1;  // last instance whose base <= j
-    while (lo < hi) {
-      const int mid = (lo + hi + 1) >> 1;
-      if ((phase == 1 ? S.inst[mid].p1_base : S.inst[mid].p2_base) <= j) lo = mid; else hi = mid - 1;
-    }
-    const Inst &I = S.inst[lo];
-    const int ng = phase == 1 ? I.ng1 : I.ng2;
-    const int loc = j - (phase == 1 ? I.p1_base : I.p2_base);
-    S.items[k] = item_word(lo, loc / ng, loc % ng, phase);
-  }
-
-  // ---- zero this CTA's slice of out (the down items add into it after the
-  // grid barrier; out does not overlap the inputs)
-  {
-    const unsigned total4 = (unsigned)(T * H / 4);
-    const unsigned z0 = cta * total4 / uG, z1 = (cta + 1) * total4 / uG;
-    for (unsigned i = z0 + tid; i < z1; i += kCThreads)
-      reinterpret_cast<float4 *>(a.out)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-  }
-  // the rings' bucketing scratch is overwritten by bulk copies next
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-  __syncthreads();
-  TR_STAMP(1);
-  TR_DECL;
-
-  // this warp's place in an item: phase 1 takes matrix p1_sub (gate, up),
-  // tile p1_off of the item's tiles and input block p1_kb; phase 2 items of
-  // an expert with ffn / 256 = nkb have byte nkb - 1 of p2tab = tile offset
-  // (bits 0-3), input block (4-6) and whether this warp has a tile-block (7)
-  const int p1_r = warp & 7, p1_sub = warp >> 3;
-  const int p1_off = p1_r / nkbH, p1_kb = p1_r % nkbH;
-  const bool p1_ok = p1_r < it1 * nkbH;
-  uint64_t p2tab = 0;
+  // fewer down item).  (The host keeps every CTA's list within kMaxItems;
+  // the clamps only guard the shared-memory list.)
+  auto split = [&](int &b1, int &my1, int &b2, int &my2) {
+    const unsigned uG = (unsigned)G, uN1 = (unsigned)s_n1, uN2 = (unsigned)s_n2;  // products < 2^31
+    b1 = (int)(cta * uN1 / uG);
+    my1 = min(kMaxItems, (int)((cta + 1) * uN1 / uG) - b1);
+    const int rc = G - 1 - cta;
+    b2 = (int)(rc * uN2 / uG);
+    my2 = min(kMaxItems - my1, (int)((rc + 1) * uN2 / uG) - b2);
+  };
+  // warp wi's place in an item, packed: phase 1 (bits 0-3 tile offset,
+  // 4-6 input block, 7 has a tile-block, 8 matrix: gate 0 / up 1); phase 2
+  // items of an expert with ffn / 256 = nkb: byte nkb - 1 of p2 = tile
+  // offset (bits 0-3), input block (4-6), has a tile-block (7)
+  auto warp_place = [&](int wi, uint32_t &p1, uint64_t &p2) {
+    const int r = wi & 7;
+    p1 = (uint32_t)(r / nkbH) | ((uint32_t)(r % nkbH) << 4) | (r < it1 * nkbH ? 128u : 0u) | ((uint32_t)(wi >> 3) << 8);
+    p2 = 0;
 #pragma unroll
-  for (int nkb = 1; nkb <= 8; ++nkb) {
-    const uint64_t okb = warp < it2_of(nkb) * nkb ? 128u : 0u;
-    p2tab |= ((uint64_t)(warp / nkb) | ((uint64_t)(warp % nkb) << 4) | okb) << (8 * (nkb - 1));
-  }
-  // this warp's tile-block of item word w: source address and bytes (0: none)
-  auto tile_of = [&](uint32_t w, const uint8_t *&src, int &kb) -> uint32_t {
+    for (int nkb = 1; nkb <= 8; ++nkb) {
+      const uint64_t okb = wi < it2_of(nkb) * nkb ? 128u : 0u;
+      p2 |= ((uint64_t)(wi / nkb) | ((uint64_t)(wi % nkb) << 4) | okb) << (8 * (nkb - 1));
+    }
+  };
+  // a warp's tile-block of item word w: source, bytes (0: none), input
+  // block and tile
+  auto tile_of = [&](uint32_t p1, uint64_t p2, uint32_t w, const uint8_t *&src, int &kb, int &tile) -> uint32_t {
     const Inst &I = S.inst[item_inst(w)];
     const int tbb = tile_block_bytes(I.qtype);
     if (item_phase(w) == 1) {
-      const int tile = item_grp(w) * it1 + p1_off;
-      if (!p1_ok || tile >= I.ffn / 16) return 0;
-      kb = p1_kb;
-      src = (p1_sub ? I.up : I.gate) + (size_t)(tile * nkbH + p1_kb) * tbb;
+      tile = item_grp(w) * it1 + (int)(p1 & 15u);
+      kb = (int)((p1 >> 4) & 7u);
+      if (!(p1 & 128u) || tile >= I.ffn / 16) return 0;
+      src = ((p1 >> 8) ? I.up : I.gate) + (size_t)(tile * nkbH + kb) * tbb;
     } else {
       const int nkb = I.ffn >> 8;
-      const uint32_t e = (uint32_t)(p2tab >> (8 * (nkb - 1))) & 0xFFu;
-      const int tile = item_grp(w) * it2_of(nkb) + (int)(e & 15u);
+      const uint32_t e = (uint32_t)(p2 >> (8 * (nkb - 1))) & 0xFFu;
+      tile = item_grp(w) * it2_of(nkb) + (int)(e & 15u);
       kb = (int)((e >> 4) & 7u);
       if (!(e & 128u) || tile >= H / 16) return 0;
       src = I.down + (size_t)(tile * nkb + kb) * tbb;
     }
     return (uint32_t)tbb;
   };
-  // lane 0: start the copy of this warp's tile-block of item k into stage
-  // k % kRing; an item with no tile-block for this warp completes the
-  // stage's phase at once (every stage advances one phase per item)
-  uint8_t *my_ring = S.ring + (size_t)warp * kRing * kStageBytes;
-  uint64_t *my_full = S.full + warp * kRing;
+  // copy item k into stage k % kRing: its gate and up tiles (phase 1,
+  // tile-blocks of warps 0..7 and 8..15) or its down tiles (phase 2), each
+  // contiguous in the resident layout; one thread
   auto issue = [&](int k) {
     const int s = k % kRing;
-    const uint8_t *src = nullptr;
-    int kb = 0;
-    const uint32_t bytes = tile_of(S.items[k], src, kb);
-    if (bytes) {
-      mbar_expect_tx(&my_full[s], bytes);
-      bulk_g2s(my_ring + (size_t)s * kStageBytes, src, bytes, &my_full[s]);
+    const uint32_t w = S.items[k];
+    const Inst &I = S.inst[item_inst(w)];
+    const int tbb = tile_block_bytes(I.qtype);
+    uint8_t *dst = S.ring + (size_t)s * kCWarps * kStageBytes;
+    if (item_phase(w) == 1) {
+      const int t0 = item_grp(w) * it1, nt = min(it1, I.ffn / 16 - t0);
+      const uint32_t bytes = (uint32_t)(nt * nkbH * tbb);
+      const size_t off0 = (size_t)t0 * nkbH * tbb;
+      mbar_expect_tx(&S.full[s], 2 * bytes);
+      bulk_g2s(dst, I.gate + off0, bytes, &S.full[s]);
+      bulk_g2s(dst + 8 * kStageBytes, I.up + off0, bytes, &S.full[s]);
     } else {
-      mbar_arrive(&my_full[s]);
+      const int nkb = I.ffn >> 8, it = it2_of(nkb);
+      const int t0 = item_grp(w) * it, nt = min(it, H / 16 - t0);
+      const uint32_t bytes = (uint32_t)(nt * nkb * tbb);
+      mbar_expect_tx(&S.full[s], bytes);
+      bulk_g2s(dst, I.down + (size_t)t0 * nkb * tbb, bytes, &S.full[s]);
     }
   };
-  // ---- fill this warp's ring
-  if (lane == 0)
-    for (int k = 0; k < kRing && k < my_items; ++k) issue(k);
 
-  // The reducer of item j (warp j mod 16) adds the item's partials once all
-  // warps have stored them: h = SiLU(g) * u for phase 1, out += weight * y
-  // for phase 2.  Reductions run kRedLag items late, so the reducer rarely
-  // waits for a slower warp; rj is the next item this warp considers.
+  if (warp == 0) {
+    // ---- warp 0: this CTA's item list, then the first kRing copies of
+    // every warp (the weights start streaming as soon as the routing is
+    // known)
+    __syncwarp();
+    int b1, my1, b2, my2;
+    split(b1, my1, b2, my2);
+    const int n_inst = s_n_inst;
+    for (int k = lane; k < my1 + my2; k += 32) {
+      const int phase = k < my1 ? 1 : 2;
+      const int j = phase == 1 ? b1 + k : b2 + (k - my1);
+      int lo = 0, hi = n_inst - 1;  // last instance whose base <= j
+      while (lo < hi) {
+        const int mid = (lo + hi + 1) >> 1;
+        if ((phase == 1 ? S.inst[mid].p1_base : S.inst[mid].p2_base) <= j) lo = mid; else hi = mid - 1;
+      }
+      const Inst &I = S.inst[lo];
+      const int ng = phase == 1 ? I.ng1 : I.ng2;
+      const int loc = j - (phase == 1 ? I.p1_base : I.p2_base);
+      S.items[k] = item_word(lo, loc / ng, loc % ng, phase);
+    }
+    __syncwarp();
+    if (lane < min(kRing, my1 + my2)) {
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // the rings were bucketing scratch
+      issue(lane);
+    }
+  } else {
+    // ---- the other warps zero this CTA's slice of out (the down items
+    // add into it after the grid barrier; out does not overlap the inputs)
+    const unsigned total4 = (unsigned)(T * H / 4);
+    const unsigned z0 = cta * total4 / (unsigned)G, z1 = (cta + 1) * total4 / (unsigned)G;
+    for (unsigned i = z0 + tid - 32; i < z1; i += kCThreads - 32)
+      reinterpret_cast<float4 *>(a.out)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  uint32_t my_p1;
+  uint64_t my_p2;
+  warp_place(warp, my_p1, my_p2);
+  __syncthreads();  // the item list and the replicated tables are visible
+  int b1, my1, b2, my2;
+  split(b1, my1, b2, my2);
+  const int my_items = my1 + my2;
+  TR_STAMP(1);
+  TR_DECL;
+
+  // The reducer of phase-1 item j (warp j mod 16) adds the item's partials
+  // once all warps have stored them and writes h = SiLU(g) * u for its rows.
+  // Reductions run kRedLag items late, so the reducer rarely waits for a
+  // slower warp; rj is the next item this warp considers.
   int rj = 0;
-  auto reduce_item = [&](int j) {
-    const uint32_t w = S.items[j];
-    const Inst &I = S.inst[item_inst(w)];
-    const int chunk = item_chunk(w), grp = item_grp(w);
-    const int ntok = min(kTokChunk, I.count - kTokChunk * chunk);
-    const int pbase = I.pair_start + kTokChunk * chunk;
-    const int r = j % kRedSlots;
-    const float *red = S.red + (size_t)r * kCWarps * kRedFloats;
-    mbar_wait(&S.rfull[r], (uint32_t)((j / kRedSlots) & 1), a.status);
-    TR(8);
-    const int pos = lane & 1;  // lane = 2 * row + position
-    if (item_phase(w) == 1) {
+  auto reduce_until = [&](int upto) {
+    for (; rj < upto; ++rj) {
+      if (rj % kCWarps != warp) continue;
+      const uint32_t w = S.items[rj];
+      const Inst &I = S.inst[item_inst(w)];
+      const int chunk = item_chunk(w), grp = item_grp(w);
+      const int ntok = min(kTokChunk, I.count - kTokChunk * chunk);
+      const int pbase = I.pair_start + kTokChunk * chunk;
+      const int r = rj % kRedSlots;
+      const float *red = S.red + (size_t)r * kCWarps * kRedFloats;
+      mbar_wait(&S.rfull[r], (uint32_t)((rj / kRedSlots) & 1), a.status);
+      TR(8);
+      const int pos = lane & 1;  // lane = 2 * row + position
       for (int ti = 0; ti < it1; ++ti) {
         const int tile = grp * it1 + ti;
         if (tile >= I.ffn / 16) break;
@@ -862,26 +908,10 @@ __global__ void __launch_bounds__(kCThreads, 1) decode_fused_kernel(FusedArgs a)
         if (pos < ntok)
           __stcg(hbuf + (size_t)(pbase + pos) * a.max_ffn + tile * 16 + (lane >> 1), silu_mul(g, u));
       }
-    } else {
-      const int nkb = I.ffn >> 8, it = it2_of(nkb);
-      const float wj = pos < ntok ? S.pair_w[pbase + pos] : 0.f;
-      float *orow = a.out + (size_t)(pos < ntok ? S.pair_tok[pbase + pos] : 0) * H;
-      for (int ti = 0; ti < it; ++ti) {
-        const int tile = grp * it + ti;
-        if (tile >= H / 16) break;
-        float y = 0.f;
-        for (int kb = 0; kb < nkb; ++kb) y += red[(ti * nkb + kb) * kRedFloats + lane];
-        if (pos < ntok) atomicAdd(orow + tile * 16 + (lane >> 1), wj * y);
-      }
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&S.rfree[r]);
+      TR(9);
     }
-    __syncwarp();
-    if (lane == 0) mbar_arrive(&S.rfree[r]);
-    TR(9);
-  };
-  // reduce this warp's items below `upto`
-  auto reduce_until = [&](int upto) {
-    for (; rj < upto; ++rj)
-      if (rj % kCWarps == warp) reduce_item(rj);
   };
 
   // ---- main loop over this CTA's items
@@ -899,7 +929,6 @@ __global__ void __launch_bounds__(kCThreads, 1) decode_fused_kernel(FusedArgs a)
       // grid barrier: every CTA has written its h rows and zeroed its slice
       // of out (all of this CTA's phase-1 reductions are done once every
       // warp has reduced its items below my1 and reached this point)
-      reduce_until(my1);
       TR(0);
       TR_STAMP(3);
       all_sync();
@@ -916,16 +945,16 @@ __global__ void __launch_bounds__(kCThreads, 1) decode_fused_kernel(FusedArgs a)
     const int s = k % kRing;
     const uint32_t w = S.items[k];
     const Inst &I = S.inst[item_inst(w)];
+    const int chunk = item_chunk(w), phase = item_phase(w);
+    const int ntok = min(kTokChunk, I.count - kTokChunk * chunk);
+    const int pbase = I.pair_start + kTokChunk * chunk;
     // ---- this warp's tile-block
     const uint8_t *src = nullptr;
-    int kb = 0;
-    const uint32_t bytes = tile_of(w, src, kb);
+    int kb = 0, tile = 0;
+    const uint32_t bytes = tile_of(my_p1, my_p2, w, src, kb, tile);
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
     TR(0);
     if (bytes) {
-      const int chunk = item_chunk(w), phase = item_phase(w);
-      const int ntok = min(kTokChunk, I.count - kTokChunk * chunk);
-      const int pbase = I.pair_start + kTokChunk * chunk;
       const uint32_t key = (w & ~(255u << 19)) | ((uint32_t)kb << 28);
       if (key != lim_key) {
         // limbs of the item's token positions, this warp's 256 inputs
@@ -938,25 +967,63 @@ __global__ void __launch_bounds__(kCThreads, 1) decode_fused_kernel(FusedArgs a)
         }
         TR(2);
       }
+    }
+    // every warp waits for the stage, also one without a tile-block in it:
+    // its refill must not start before all have seen this item's copy land
+    mbar_wait(&S.full[s], (uint32_t)((k / kRing) & 1), a.status);
+    if (bytes) {
       const bool bv = ncol < 6 && cpos < ntok;
-      mbar_wait(&my_full[s], (uint32_t)((k / kRing) & 1), a.status);
+      if (warp == 0 && k == 0) TR_STAMP(12);
+      if (warp == 0 && k == my1) TR_STAMP(14);
       TR(3);
-      const uint32_t tb = smem_u32(my_ring + (size_t)s * kStageBytes);
+      // this warp's tile-block in the stage (phase 1: gate part, then up
+      // part from slot 8; phase 2: down tiles from slot 0), tile-blocks at
+      // their own size
+      const int tbb = tile_block_bytes(I.qtype);
+      const uint32_t tb = smem_u32(S.ring + (size_t)s * kCWarps * kStageBytes) +
+                          (uint32_t)(phase == 1 ? (warp >> 3) * 8 * kStageBytes + (warp & 7) * tbb : warp * tbb);
       if (I.qtype == kQ2)
         tb_q2(tb, g2, bp, bv, acc);
       else
         tb_q1(tb, g1, bp, bv, acc);
+      if (warp == 0 && k == 0) TR_STAMP(13);
+      if (warp == 0 && k == my1) TR_STAMP(15);
       TR(4);
     }
-    // refill the stage with this warp's tile-block of item k + kRing (all
-    // lanes are done reading it)
+    // the last warp done with the stage refills it with item k + kRing
     __syncwarp();
-    if (lane == 0 && k + kRing < my_items) {
-      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      issue(k + kRing);
+    if (lane == 0 && atomicSub(&S.left[s], 1) == 1) {
+      S.left[s] = kCWarps;
+      if (k + kRing < my_items) {
+        asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+        issue(k + kRing);
+      }
+    }
+    if (phase == 2) {
+      // ---- down: this warp's rows go straight into out (fp32 atomics),
+      // scaled by the router weight and the slice's limb scale
+      if (bytes) {
+        float v[4];
+        quad_rows(acc, v);
+        if ((lane & 3) == 0) {
+          const int q = lane >> 2, row = tile * 16 + q;
+          float *o0 = a.out + (size_t)S.pair_tok[pbase] * H + row;
+          const float w0 = S.pair_w[pbase] * sc0;
+          atomicAdd(o0, w0 * v[0]);
+          atomicAdd(o0 + 8, w0 * v[2]);
+          if (ntok > 1) {
+            float *o1 = a.out + (size_t)S.pair_tok[pbase + 1] * H + row;
+            const float w1 = S.pair_w[pbase + 1] * sc1;
+            atomicAdd(o1, w1 * v[1]);
+            atomicAdd(o1 + 8, w1 * v[3]);
+          }
+        }
+      }
+      TR(7);
+      continue;
     }
     TR(5);
-    // ---- partial sums into the item's reduction slot
+    // ---- gate/up: partial sums into the item's reduction slot
     const int r = k % kRedSlots;
     float *red = S.red + (size_t)r * kCWarps * kRedFloats;
     if (k >= kRedSlots) mbar_wait(&S.rfree[r], (uint32_t)(((k / kRedSlots) - 1) & 1), a.status);
@@ -965,15 +1032,16 @@ __global__ void __launch_bounds__(kCThreads, 1) decode_fused_kernel(FusedArgs a)
     __syncwarp();
     if (lane == 0) mbar_arrive(&S.rfull[r]);
     TR(7);
-    // ---- reductions of earlier items
-    reduce_until(min(k + 1 - kRedLag, my1 > k ? my1 : my_items));
+    // ---- reductions of earlier items (all of them at the end of the phase)
+    reduce_until(k + 1 == my1 ? my1 : k + 1 - kRedLag);
     TR(0);
   }
-  reduce_until(my_items);
+  TR_STAMP(22);
   TR_FLUSH();
   TR_STAMP(6);
   // ---- exit: the last CTA resets the counters for the next call
   __syncthreads();
+  TR_STAMP(23);
   if (tid == 0) {
     __threadfence();
     const int prev = atomicAdd(&ctrl->exit_count, 1);
@@ -994,7 +1062,7 @@ size_t fused_smem_bytes(int hidden, int max_ffn) {
   off += sizeof(Inst) * kFusedMaxInst;
   off += sizeof(uint32_t) * kMaxItems;
   off += 2 * sizeof(int) * (kFusedMaxPairs + 64);
-  off += sizeof(uint64_t) * (kCWarps * kRing + 2 * kRedSlots);
+  off += sizeof(uint64_t) * (kRing + 2 * kRedSlots) + sizeof(int) * kRing;
   return off + 64;
 }
 
