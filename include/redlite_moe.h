@@ -70,7 +70,8 @@ enum {
   REDLITE_EINVAL = -1,       /* null pointer, bad size, bad enum, bad grid symbol */
   REDLITE_EUNSUPPORTED = -2, /* shape outside what the kernels support */
   REDLITE_ENOMEM = -3,       /* caller-provided workspace or pool too small */
-  REDLITE_ECUDA = -4         /* a CUDA call or kernel launch failed */
+  REDLITE_ECUDA = -4,        /* a CUDA call or kernel launch failed */
+  REDLITE_EAGAIN = -5        /* every slot the pool could evict is in flight: retry after work completes */
 };
 
 /* Bits ORed into the device status word. */
@@ -154,6 +155,51 @@ int redlite_moe_layer(const float *x, int32_t n_tokens, const int32_t *expert_id
                       int32_t top_k, const redlite_moe_table *expert_table, const redlite_moe_expert *shared_expert,
                       float *out);
 
+/* The router that feeds the layer ("Red Metal dev8", section "Field
+ * validation": router-network integration is the milestone after the
+ * routed layer; "Red Lite dev10", section "What dev10 does not yet claim":
+ * connect the router output to the top-k path).  Per token: softmax over
+ * the n_experts logits, the top_k experts by probability (equal
+ * probabilities: lower id first), their probabilities renormalised to sum
+ * 1 -- the expert_ids / router_weights a layer call takes.
+ *   logits          device [n_tokens, n_experts] fp32, finite
+ *   n_tokens        >= 0 (0 returns REDLITE_OK and enqueues nothing)
+ *   n_experts       1 .. 1024
+ *   top_k           1 .. min(16, n_experts)
+ *   expert_ids      device [n_tokens, top_k] int32, written in descending
+ *                   order of probability
+ *   router_weights  device [n_tokens, top_k] fp32, written
+ * Ranks on the logits (the same order as the probabilities); the weights
+ * are exp(l - max) / sum over the selection in fp32.  Enqueued on stream;
+ * REDLITE_EINVAL for a size out of range or a null pointer. */
+int redlite_moe_route_topk(const float *logits, int32_t n_tokens, int32_t n_experts, int32_t top_k,
+                           int32_t *expert_ids, float *router_weights, void *stream);
+
+/* The post-attention block around the layer ("Red Lite dev16 -- complete
+ * full-attention parity", block composition paragraph: attention residual,
+ * post-attention RMSNorm, routed top-10 MoE plus shared expert, final
+ * residual).  Per token, h being the hidden state after the attention
+ * residual:
+ *   xn = norm_weight * h / sqrt(mean(h^2) + eps)      (RMSNorm)
+ *   ids, weights = redlite_moe_route_topk(router_w xn, top_k)
+ *   out = h + redlite_moe_layer(xn, ids, weights)       (incl. shared expert)
+ *   h            device [n_tokens, hidden] fp32
+ *   n_tokens     0 .. table->max_tokens
+ *   norm_weight  device [hidden] fp32; eps >= 0
+ *   router_w     device [n_experts, hidden] fp32 (the router's matrix)
+ *   top_k        1 .. min(16, n_experts); n_experts <= 1024
+ *   out          device [n_tokens, hidden] fp32; may be h itself (in place)
+ *   scratch      device, >= redlite_moe_block_scratch_bytes(hidden,
+ *                n_experts, table->max_tokens, top_k) bytes, caller-owned;
+ *                holds the normalised state, logits, ids and weights
+ * All pointers 16-byte aligned.  Enqueued on table->stream; the layer's
+ * checks, paths and status word as redlite_moe_layer.  REDLITE_ENOMEM if
+ * the scratch is too small. */
+size_t redlite_moe_block_scratch_bytes(int32_t hidden, int32_t n_experts, int32_t max_tokens, int32_t top_k);
+int redlite_moe_block(const float *h, int32_t n_tokens, const float *norm_weight, float eps, const float *router_w,
+                      int32_t top_k, const redlite_moe_table *expert_table, const redlite_moe_expert *shared_expert,
+                      float *out, void *scratch, size_t scratch_bytes);
+
 /* The layer for callers that cannot allocate device memory.  Some callers
  * have no way to call cudaMalloc for the workspace: for example a plugin
  * running inside a host application that owns the whole device-memory
@@ -223,6 +269,80 @@ int redlite_moe_upload_experts(int32_t hidden, const int32_t *ids, const redlite
                                void *pool, size_t pool_bytes, size_t pool_offset, redlite_moe_expert *table_dev,
                                int32_t n_experts, void *stream, redlite_moe_upload_counters *counters,
                                size_t *pool_end);
+
+/* ---------------------------------------------------------------- slot pool
+ * The bounded, top-k-aware LRU pool of expert slots ("Red Metal dev8",
+ * steps 1-3: the hard-bounded LRU makes every selected expert resident,
+ * selected experts are protected from eviction while the remaining misses
+ * are filled, every selected slot is pinned for the work that uses it;
+ * "Red Lite dev9 -- native runtime foundation", section "Native selftest":
+ * hard capacity enforcement, LRU hit/miss/eviction, protection of the
+ * current top-k during acquire_many, in-flight slot protection).
+ * The pool is a host object; it owns no device memory.  Not thread-safe:
+ * one host thread drives a pool. */
+typedef struct redlite_moe_pool redlite_moe_pool;
+
+typedef struct {
+  int64_t loads;     /* misses filled */
+  int64_t hits;      /* selected experts already resident */
+  int64_t evictions; /* resident experts replaced */
+  int64_t copies;    /* host->device matrix copies (3 per load) */
+  int64_t bytes;     /* packed bytes copied */
+} redlite_moe_pool_counters;
+
+/* A pool of `capacity` slots for experts 0..n_experts-1 (all empty).
+ * NULL for a bad size or if host memory runs out. */
+redlite_moe_pool *redlite_moe_pool_create(int32_t n_experts, int32_t capacity);
+void redlite_moe_pool_destroy(redlite_moe_pool *pool);
+
+/* The policy step (host only, no device work): make ids[0..n) resident.
+ *   pass 1: every selected expert already resident is a hit: its slot is
+ *           refreshed (most recently used) and protected;
+ *   pass 2: each miss, in order, takes the lowest free slot, else the least
+ *           recently used slot that is neither protected (selected in this
+ *           call) nor pinned by a call still in flight; a repeated id shares
+ *           its first occurrence's slot;
+ *   then every selected slot is pinned under a new token.
+ * Outputs per id: slot_of[i], miss[i] (1 if it must be filled), evicted[i]
+ * (the expert whose slot it took, or -1).  REDLITE_ENOMEM if the distinct
+ * ids exceed the capacity; REDLITE_EAGAIN if a miss finds no slot because
+ * the others are in flight (nothing changes then); REDLITE_EINVAL for an id
+ * outside [0, n_experts). */
+int redlite_moe_pool_plan(redlite_moe_pool *pool, const int32_t *ids, int32_t n, int32_t *slot_of, int32_t *evicted,
+                          uint8_t *miss, int64_t *token);
+
+/* Unpin a token's slots now (the caller knows the work using them is done). */
+int redlite_moe_pool_complete(redlite_moe_pool *pool, int64_t token);
+
+/* Unpin a token's slots once the work enqueued on `stream` so far has
+ * completed (a CUDA event, polled by later plans). */
+int redlite_moe_pool_release(redlite_moe_pool *pool, int64_t token, void *stream);
+
+/* Slot of a resident expert, or -1; pins of a slot, or -1 for a bad slot. */
+int32_t redlite_moe_pool_slot_of(const redlite_moe_pool *pool, int32_t expert);
+int32_t redlite_moe_pool_pins(const redlite_moe_pool *pool, int32_t slot);
+
+/* The policy step plus the data movement: for every miss the expert's three
+ * matrices are copied host -> device on copy_stream into its slot
+ * (slots_dev + slot * slot_bytes: gate, up at the gate size rounded up to 16
+ * bytes, down after), and table_dev[id] is written; an evicted expert's
+ * entry is cleared first (a stale id then reports BAD_EXPERT).  The work
+ * enqueued next on compute_stream waits for these copies, so a layer call
+ * may follow at once; copies for the next selection overlap the current
+ * layer kernel when copy_stream differs from compute_stream.
+ *   host_experts  host [n_experts]; gate/up/down are HOST pointers to the
+ *                 matrices already in the resident layout
+ *                 (redlite_moe_pack_matrix); pinned host memory makes the
+ *                 copies asynchronous; they must stay valid until the copies
+ *                 complete
+ *   slot_bytes    multiple of 16, >= 2 * round16(gate bytes) + down bytes of
+ *                 every expert acquired (else REDLITE_ENOMEM)
+ * After enqueuing the layer call, pass the token to redlite_moe_pool_release
+ * with compute_stream. */
+int redlite_moe_pool_acquire(redlite_moe_pool *pool, const int32_t *ids, int32_t n,
+                             const redlite_moe_expert *host_experts, int32_t hidden, void *slots_dev,
+                             size_t slot_bytes, redlite_moe_expert *table_dev, void *copy_stream,
+                             void *compute_stream, redlite_moe_pool_counters *counters, int64_t *token);
 
 #ifdef __cplusplus
 }

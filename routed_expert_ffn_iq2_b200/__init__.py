@@ -6,6 +6,7 @@ package is a thin ctypes binding plus a buffer-owning convenience class."""
 from ._native import (  # noqa: F401
     EXPORTS,
     LIB_PATH,
+    REDLITE_EAGAIN,
     REDLITE_EINVAL,
     REDLITE_ENOMEM,
     REDLITE_EUNSUPPORTED,
@@ -16,6 +17,7 @@ from ._native import (  # noqa: F401
     REDLITE_STATUS_BAD_EXPERT,
     REDLITE_STATUS_BAD_ID,
     REDLITE_STATUS_TIMEOUT,
+    SlotPool,
     launches_per_call,
     lib,
     redlite_moe_dequant,
@@ -25,7 +27,11 @@ from ._native import (  # noqa: F401
     redlite_moe_layer,
     redlite_moe_layer_noalloc,
     redlite_moe_matrix_bytes,
+    redlite_moe_block,
+    redlite_moe_block_scratch_bytes,
     redlite_moe_pack_matrix,
+    redlite_moe_pool_counters,
+    redlite_moe_route_topk,
     redlite_moe_table,
     redlite_moe_upload_counters,
     redlite_moe_upload_experts,

@@ -22,6 +22,7 @@ REDLITE_EINVAL = -1
 REDLITE_EUNSUPPORTED = -2
 REDLITE_ENOMEM = -3
 REDLITE_ECUDA = -4
+REDLITE_EAGAIN = -5
 REDLITE_STATUS_BAD_ID = 1
 REDLITE_STATUS_BAD_EXPERT = 2
 REDLITE_STATUS_TIMEOUT = 4
@@ -43,6 +44,11 @@ class redlite_moe_table(ctypes.Structure):
     ]
 
 
+class redlite_moe_pool_counters(ctypes.Structure):
+    _fields_ = [("loads", ctypes.c_int64), ("hits", ctypes.c_int64), ("evictions", ctypes.c_int64),
+                ("copies", ctypes.c_int64), ("bytes", ctypes.c_int64)]
+
+
 class redlite_moe_upload_counters(ctypes.Structure):
     _fields_ = [("loads", ctypes.c_int64), ("copies", ctypes.c_int64), ("bytes", ctypes.c_int64)]
 
@@ -59,6 +65,24 @@ EXPORTS = {
     "redlite_moe_layer_noalloc": (ctypes.c_int, [_c_void_p, ctypes.c_int32, _c_void_p, _c_void_p, ctypes.c_int32,
                                                  ctypes.POINTER(redlite_moe_table),
                                                  ctypes.POINTER(redlite_moe_expert), _c_void_p]),
+    "redlite_moe_route_topk": (ctypes.c_int, [_c_void_p, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, _c_void_p,
+                                              _c_void_p, _c_void_p]),
+    "redlite_moe_block_scratch_bytes": (ctypes.c_size_t, [ctypes.c_int32] * 4),
+    "redlite_moe_block": (ctypes.c_int, [_c_void_p, ctypes.c_int32, _c_void_p, ctypes.c_float, _c_void_p,
+                                         ctypes.c_int32, ctypes.POINTER(redlite_moe_table),
+                                         ctypes.POINTER(redlite_moe_expert), _c_void_p, _c_void_p, ctypes.c_size_t]),
+    "redlite_moe_pool_create": (_c_void_p, [ctypes.c_int32, ctypes.c_int32]),
+    "redlite_moe_pool_destroy": (None, [_c_void_p]),
+    "redlite_moe_pool_plan": (ctypes.c_int, [_c_void_p, _c_void_p, ctypes.c_int32, _c_void_p, _c_void_p, _c_void_p,
+                                             ctypes.POINTER(ctypes.c_int64)]),
+    "redlite_moe_pool_complete": (ctypes.c_int, [_c_void_p, ctypes.c_int64]),
+    "redlite_moe_pool_release": (ctypes.c_int, [_c_void_p, ctypes.c_int64, _c_void_p]),
+    "redlite_moe_pool_slot_of": (ctypes.c_int32, [_c_void_p, ctypes.c_int32]),
+    "redlite_moe_pool_pins": (ctypes.c_int32, [_c_void_p, ctypes.c_int32]),
+    "redlite_moe_pool_acquire": (ctypes.c_int, [_c_void_p, _c_void_p, ctypes.c_int32, _c_void_p, ctypes.c_int32,
+                                                _c_void_p, ctypes.c_size_t, _c_void_p, _c_void_p, _c_void_p,
+                                                ctypes.POINTER(redlite_moe_pool_counters),
+                                                ctypes.POINTER(ctypes.c_int64)]),
     "redlite_moe_pack_matrix": (ctypes.c_int, [ctypes.c_int32, ctypes.c_int64, ctypes.c_int64, _c_void_p,
                                                _c_void_p]),
     "redlite_moe_dequant": (ctypes.c_int, [ctypes.c_int32, _c_void_p, ctypes.c_int64, ctypes.c_int64, _c_void_p,
@@ -167,6 +191,27 @@ def redlite_moe_layer_noalloc(x: torch.Tensor, n_tokens: int, expert_ids: torch.
                                            _ptr(out))
 
 
+def redlite_moe_route_topk(logits: torch.Tensor, n_tokens: int, n_experts: int, top_k: int, expert_ids: torch.Tensor,
+                           router_weights: torch.Tensor, stream=None) -> int:
+    """The router: softmax over the logits, top-k by probability, renormalised weights."""
+    return lib().redlite_moe_route_topk(_ptr(logits), n_tokens, n_experts, top_k, _ptr(expert_ids),
+                                        _ptr(router_weights), _stream_handle(stream))
+
+
+def redlite_moe_block_scratch_bytes(hidden: int, n_experts: int, max_tokens: int, top_k: int) -> int:
+    return int(lib().redlite_moe_block_scratch_bytes(hidden, n_experts, max_tokens, top_k))
+
+
+def redlite_moe_block(h: torch.Tensor, n_tokens: int, norm_weight: torch.Tensor, eps: float, router_w: torch.Tensor,
+                      top_k: int, expert_table: redlite_moe_table, shared_expert: Optional[redlite_moe_expert],
+                      out: torch.Tensor, scratch: torch.Tensor) -> int:
+    """out = h + layer(RMSNorm(h)) with the router's own top-k routing."""
+    return lib().redlite_moe_block(_ptr(h), n_tokens, _ptr(norm_weight), float(eps), _ptr(router_w), top_k,
+                                   ctypes.byref(expert_table),
+                                   ctypes.byref(shared_expert) if shared_expert is not None else None, _ptr(out),
+                                   _ptr(scratch), scratch.numel() * scratch.element_size())
+
+
 def redlite_moe_upload_experts(hidden: int, ids, host_experts, pool: torch.Tensor, pool_offset: int,
                                table_dev: torch.Tensor, n_experts: int, counters=None, stream=None):
     """ids: list of expert ids; host_experts: objects with qtype, ffn and numpy gate/up/down arrays.
@@ -188,6 +233,72 @@ def redlite_moe_upload_experts(hidden: int, ids, host_experts, pool: torch.Tenso
                                           ctypes.byref(ctr), ctypes.byref(end))
     del keep
     return rc, int(end.value)
+
+
+class SlotPool:
+    """The bounded, top-k-aware LRU slot pool (a host object of the library).
+    plan() is the policy step alone (no device work); acquire() also copies
+    the misses' matrices into their device slots and updates the slot table."""
+
+    def __init__(self, n_experts: int, capacity: int):
+        self.n_experts, self.capacity = n_experts, capacity
+        self.handle = lib().redlite_moe_pool_create(n_experts, capacity)
+        if not self.handle:
+            raise RuntimeError("redlite_moe_pool_create failed")
+        self.counters = redlite_moe_pool_counters()
+
+    def close(self):
+        if self.handle:
+            lib().redlite_moe_pool_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+    def plan(self, ids):
+        """(rc, slots, evicted, miss, token) for the selection `ids`."""
+        import numpy as np
+
+        a = np.ascontiguousarray(ids, dtype=np.int32)
+        n = a.size
+        slots = np.zeros(max(n, 1), np.int32)
+        ev = np.zeros(max(n, 1), np.int32)
+        miss = np.zeros(max(n, 1), np.uint8)
+        tok = ctypes.c_int64(0)
+        rc = lib().redlite_moe_pool_plan(self.handle, a.ctypes.data_as(_c_void_p), n, slots.ctypes.data_as(_c_void_p),
+                                         ev.ctypes.data_as(_c_void_p), miss.ctypes.data_as(_c_void_p),
+                                         ctypes.byref(tok))
+        return rc, slots[:n].tolist(), ev[:n].tolist(), miss[:n].astype(bool).tolist(), tok.value
+
+    def complete(self, token: int) -> int:
+        return lib().redlite_moe_pool_complete(self.handle, token)
+
+    def release(self, token: int, stream=None) -> int:
+        return lib().redlite_moe_pool_release(self.handle, token, _stream_handle(stream))
+
+    def slot_of(self, expert: int) -> int:
+        return int(lib().redlite_moe_pool_slot_of(self.handle, expert))
+
+    def pins(self, slot: int) -> int:
+        return int(lib().redlite_moe_pool_pins(self.handle, slot))
+
+    def acquire(self, ids, host_experts, hidden: int, slots: torch.Tensor, slot_bytes: int, table_dev: torch.Tensor,
+                copy_stream, compute_stream):
+        """host_experts: ctypes array [n_experts] of redlite_moe_expert with host pointers (resident layout).
+        Returns (rc, token)."""
+        import numpy as np
+
+        a = np.ascontiguousarray(ids, dtype=np.int32)
+        tok = ctypes.c_int64(0)
+        rc = lib().redlite_moe_pool_acquire(self.handle, a.ctypes.data_as(_c_void_p), a.size,
+                                            ctypes.cast(host_experts, _c_void_p), hidden, _ptr(slots), slot_bytes,
+                                            _ptr(table_dev), _stream_handle(copy_stream),
+                                            _stream_handle(compute_stream), ctypes.byref(self.counters),
+                                            ctypes.byref(tok))
+        return rc, tok.value
 
 
 def launches_per_call(n_tokens: int, top_k: int, has_shared: bool, fast: bool = True) -> int:

@@ -58,8 +58,12 @@ int redlite_moe_workspace_reset(const redlite_moe_table *t) {
              : REDLITE_ECUDA;
 }
 
-int redlite_moe_layer(const float *x, int32_t n_tokens, const int32_t *expert_ids, const float *router_weights,
-                      int32_t top_k, const redlite_moe_table *t, const redlite_moe_expert *shared, float *out) {
+}  // extern "C"
+
+namespace redlite {
+
+int layer_impl(const float *x, int32_t n_tokens, const int32_t *expert_ids, const float *router_weights, int32_t top_k,
+               const redlite_moe_table *t, const redlite_moe_expert *shared, float *out, const float *residual) {
   if (!table_ok(t)) return REDLITE_EINVAL;
   if (n_tokens < 0 || n_tokens > t->max_tokens) return REDLITE_EINVAL;
   if (top_k < 1 || top_k > kMaxTopK) return REDLITE_EINVAL;
@@ -97,9 +101,15 @@ int redlite_moe_layer(const float *x, int32_t n_tokens, const int32_t *expert_id
     fa.ws = ws;
     fa.L = L;
     fa.status = t->status;
+    fa.residual = residual;
     return launch_fused(fa, s) == cudaSuccess ? REDLITE_OK : REDLITE_ECUDA;
   }
-  if (cudaMemsetAsync(out, 0, sizeof(float) * (size_t)n_tokens * t->hidden, s) != cudaSuccess) return REDLITE_ECUDA;
+  const size_t out_bytes = sizeof(float) * (size_t)n_tokens * t->hidden;
+  if (!residual) {
+    if (cudaMemsetAsync(out, 0, out_bytes, s) != cudaSuccess) return REDLITE_ECUDA;
+  } else if (residual != out) {
+    if (cudaMemcpyAsync(out, residual, out_bytes, cudaMemcpyDeviceToDevice, s) != cudaSuccess) return REDLITE_ECUDA;
+  }
   const bool tc = tiled && tc_supported(t->hidden, t->max_ffn);
   RouteArgs ra{expert_ids, router_weights, n_tokens, top_k, t->n_experts, t->hidden, t->max_ffn,
                t->experts, shared != nullptr, shared ? shared->ffn : 0, shared ? shared->qtype : 0, tc, ws, L,
@@ -123,6 +133,15 @@ int redlite_moe_layer(const float *x, int32_t n_tokens, const int32_t *expert_id
   const int max_active = (int)((routed < t->n_experts ? routed : t->n_experts) + (shared ? 1 : 0));
   if (launch_simt_tiles(ta, max_active, s) != cudaSuccess) return REDLITE_ECUDA;
   return REDLITE_OK;
+}
+
+}  // namespace redlite
+
+extern "C" {
+
+int redlite_moe_layer(const float *x, int32_t n_tokens, const int32_t *expert_ids, const float *router_weights,
+                      int32_t top_k, const redlite_moe_table *t, const redlite_moe_expert *shared, float *out) {
+  return layer_impl(x, n_tokens, expert_ids, router_weights, top_k, t, shared, out, nullptr);
 }
 
 int redlite_moe_dequant(int32_t qtype, const void *packed, int64_t rows, int64_t k, const void *grids, float *out_f32,

@@ -862,12 +862,14 @@ __global__ void __launch_bounds__(kCThreads, 1) decode_fused_kernel(FusedArgs a)
       issue(lane);
     }
   } else {
-    // ---- the other warps zero this CTA's slice of out (the down items
-    // add into it after the grid barrier; out does not overlap the inputs)
+    // ---- the other warps zero this CTA's slice of out, or copy the
+    // residual into it (the down items add into it after the grid barrier;
+    // out does not overlap the inputs)
     const unsigned total4 = (unsigned)(T * H / 4);
     const unsigned z0 = cta * total4 / (unsigned)G, z1 = (cta + 1) * total4 / (unsigned)G;
     for (unsigned i = z0 + tid - 32; i < z1; i += kCThreads - 32)
-      reinterpret_cast<float4 *>(a.out)[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+      reinterpret_cast<float4 *>(a.out)[i] =
+          a.residual ? __ldg(reinterpret_cast<const float4 *>(a.residual) + i) : make_float4(0.f, 0.f, 0.f, 0.f);
   }
   uint32_t my_p1;
   uint64_t my_p2;

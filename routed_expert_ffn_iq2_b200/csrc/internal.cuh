@@ -305,6 +305,7 @@ struct FusedArgs {
   const int32_t *ids;
   const float *weights;
   float *out;
+  const float *residual;  // nullptr, or [n_tokens, hidden] added to out (out starts from it)
   int n_tokens, top_k, n_experts, hidden, max_ffn;
   const redlite_moe_expert *experts;
   redlite_moe_expert shared;
@@ -324,5 +325,11 @@ constexpr int kTcTokens = 128;
 bool tc_supported(int hidden, int max_ffn);
 cudaError_t launch_tc(const TileArgs &a, cudaStream_t stream);
 cudaError_t launch_fused(const FusedArgs &a, cudaStream_t stream);
+
+// The layer with an optional residual: out = residual + layer(x) (out =
+// layer(x) when residual is null).  Checks and path choice as
+// redlite_moe_layer.
+int layer_impl(const float *x, int32_t n_tokens, const int32_t *expert_ids, const float *router_weights, int32_t top_k,
+               const redlite_moe_table *t, const redlite_moe_expert *shared, float *out, const float *residual);
 
 }  // namespace redlite

@@ -154,3 +154,25 @@ def test_no_alloc_rejects_on_host(native):
     # widths the fused kernel does not take
     t1 = native.redlite_moe_table(256, 16, 64, 1, 64, 0, 0x1000, 0x2000, 0x3000, 0, 0x4000, None)
     assert L.redlite_moe_layer_noalloc(p, 1, p, p, 4, ctypes.byref(t1), None, p) == native.REDLITE_EUNSUPPORTED
+
+
+def test_router_and_block_reject_on_host(native):
+    L = native.lib()
+    p = ctypes.c_void_p(0x10000)
+    for T, E, k in [(1, 16, 17), (1, 16, 0), (1, 8, 9), (1, 1025, 4), (1, 0, 1), (-1, 16, 4)]:
+        assert L.redlite_moe_route_topk(p, T, E, k, p, p, None) == native.REDLITE_EINVAL, (T, E, k)
+    assert L.redlite_moe_route_topk(p, 0, 512, 10, None, None, None) == native.REDLITE_OK
+    assert L.redlite_moe_route_topk(None, 1, 512, 10, p, p, None) == native.REDLITE_EINVAL
+    t = native.redlite_moe_table(2048, 512, 512, 64, 512, 0, 0x1000, 0x2000, 0x3000, 1 << 30, 0x4000, None)
+    need = native.redlite_moe_block_scratch_bytes(2048, 512, 64, 10)
+    assert need >= 64 * 2048 * 4 + 64 * 512 * 4
+    assert L.redlite_moe_block(p, 4, p, ctypes.c_float(1e-6), p, 10, ctypes.byref(t), None, p, p, need - 1) == \
+        native.REDLITE_ENOMEM
+    assert L.redlite_moe_block(p, 4, p, ctypes.c_float(1e-6), p, 10, ctypes.byref(t), None,
+                               ctypes.c_void_p(0x10004), p, need) == native.REDLITE_EINVAL
+    assert L.redlite_moe_block(p, 65, p, ctypes.c_float(1e-6), p, 10, ctypes.byref(t), None, p, p, need) == \
+        native.REDLITE_EINVAL
+    assert L.redlite_moe_block(p, 4, p, ctypes.c_float(-1.0), p, 10, ctypes.byref(t), None, p, p, need) == \
+        native.REDLITE_EINVAL
+    assert L.redlite_moe_block(None, 0, None, ctypes.c_float(1e-6), None, 10, ctypes.byref(t), None, None, None, 0) == \
+        native.REDLITE_OK
