@@ -353,3 +353,30 @@ def decode_id_sets(seed: int, n_sets: int, k: int, n_experts: int) -> np.ndarray
         used.extend(ids)
         out[s] = ids
     return out
+
+
+# --------------------------------------------------------------------------- projection formats
+
+PROJ_BLOCK = {3: (32, 34), 4: (256, 144)}  # qtype -> (weights, bytes) per block: Q8_0-style, Q4_K-style
+
+
+def make_proj_matrix(seed: int, qtype: int, rows: int, k: int, *tag: int) -> np.ndarray:
+    """Packed bytes of a Q8_0-style (3) or Q4_K-style (4) matrix: uniform random
+    fields, fp16 scales drawn so that |W| stays near 1/sqrt(k) (the scale
+    fields are the only format knowledge here: Q8_0 d at bytes 0-1; Q4_K d and
+    dmin at bytes 0-1 and 2-3)."""
+    bw, bb = PROJ_BLOCK[qtype]
+    nblk = rows * k // bw
+    st = Stream(seed, 9, qtype, rows, k, *tag)
+    raw = st.bytes(nblk * bb).reshape(nblk, bb)
+    bits = st.u64(nblk)
+    mant = (bits & np.uint64(0x3FF)).astype(np.uint16)
+    if qtype == 3:  # d in [2^-13, 2^-12): |w| <= 128 d
+        d = (np.uint16(2) << np.uint16(10)) | mant
+        raw[:, 0], raw[:, 1] = (d & 0xFF).astype(np.uint8), (d >> 8).astype(np.uint8)
+    else:  # d in [2^-12, 2^-11), dmin in [2^-13, 2^-12): |w| <= 63 * 15 d
+        d = (np.uint16(3) << np.uint16(10)) | mant
+        dm = (np.uint16(2) << np.uint16(10)) | ((bits >> np.uint64(10)) & np.uint64(0x3FF)).astype(np.uint16)
+        raw[:, 0], raw[:, 1] = (d & 0xFF).astype(np.uint8), (d >> 8).astype(np.uint8)
+        raw[:, 2], raw[:, 3] = (dm & 0xFF).astype(np.uint8), (dm >> 8).astype(np.uint8)
+    return raw.reshape(-1)

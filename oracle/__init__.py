@@ -20,6 +20,8 @@ _LIB = os.path.join(_HERE, "liboracle.so")
 
 QTYPE_IQ2XS = 1
 QTYPE_IQ1M = 2
+QTYPE_Q8_0 = 3
+QTYPE_Q4_K = 4
 OK = 0
 EINVAL = -1
 SKIPPED_PAIRS = 1
@@ -73,6 +75,10 @@ def lib():
             ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
         ]
         L.oracle_set_threads.argtypes = [ctypes.c_int]
+        L.oracle_dequant_proj.argtypes = [ctypes.c_int, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64,
+                                          ctypes.c_void_p]
+        L.oracle_gemv_proj.argtypes = [ctypes.c_int, ctypes.c_void_p, ctypes.c_int64, ctypes.c_int64, ctypes.c_void_p,
+                                       ctypes.c_int, ctypes.c_void_p]
         L.oracle_route_topk.argtypes = [ctypes.c_void_p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_void_p,
                                         ctypes.c_void_p]
         L.oracle_moe_block.argtypes = [
@@ -221,3 +227,24 @@ def moe_block(h, gamma, eps: float, router_w, top_k: int, experts: Sequence, sha
     if rc < 0:
         raise ValueError(f"oracle_moe_block failed ({rc})")
     return (out, ids, w) if return_routing else out
+
+
+def dequant_proj(qtype: int, packed, rows: int, k: int) -> np.ndarray:
+    """Weights of a Q8_0-style (3) or Q4_K-style (4) matrix as float64 [rows, k]."""
+    p = np.ascontiguousarray(packed, dtype=np.uint8)
+    out = np.zeros(rows * k, dtype=np.float64)
+    rc = lib().oracle_dequant_proj(qtype, _ptr(p), rows, k, _ptr(out))
+    if rc != OK:
+        raise ValueError(f"oracle_dequant_proj failed ({rc})")
+    return out.reshape(rows, k)
+
+
+def gemv_proj(qtype: int, packed, rows: int, k: int, x) -> np.ndarray:
+    """y = W x (float64 [n_tokens, rows]) for a projection-format matrix."""
+    p = np.ascontiguousarray(packed, dtype=np.uint8)
+    xv = np.ascontiguousarray(x, dtype=np.float32).reshape(-1, k)
+    y = np.zeros((xv.shape[0], rows), dtype=np.float64)
+    rc = lib().oracle_gemv_proj(qtype, _ptr(p), rows, k, _ptr(xv), xv.shape[0], _ptr(y))
+    if rc != OK:
+        raise ValueError(f"oracle_gemv_proj failed ({rc})")
+    return y

@@ -158,6 +158,85 @@ int oracle_dequant_matrix(int qtype, const uint8_t *packed, int64_t rows, int64_
   return ORACLE_OK;
 }
 
+/* ------------------------------------------------------------------ projection formats
+ * The dense projections of the model the pages run use other GGUF formats
+ * ("Red Lite dev15 -- DeltaNet projection bring-up", section
+ * "Field-derived recurrent dimensions": ssm_ba Q8_0 (2048,64), ssm_out
+ * Q4_K (4096,2048); "Red Lite dev16", section "Pinned full-attention graph":
+ * attn_k / attn_v Q4_K (2048,512), attn_output Q4_K (4096,2048)).  The
+ * pages print no bit layouts; the readings below are the plainest
+ * packings of the named fields.
+ *
+ * Q8_0-style block, 34 bytes per 32 weights:
+ *   bytes 0-1  d      fp16 block scale
+ *   bytes 2-33 q[32]  signed 8-bit values
+ * weight i = d * q[i].
+ *
+ * Q4_K-style super-block, 144 bytes per 256 weights (eight sub-blocks of 32):
+ *   bytes 0-1   d       fp16 scale of the sub-block scales
+ *   bytes 2-3   dmin    fp16 scale of the sub-block minima
+ *   bytes 4-15  sm[12]  a 96-bit little-endian field: 6-bit scale of
+ *                       sub-block j at bits 6j, 6-bit minimum of sub-block
+ *                       j at bits 48 + 6j
+ *   bytes 16-143 q[128] 4-bit values, weight i in byte i/2 (low nibble for
+ *                       even i)
+ * weight i = d * scale[i/32] * q_i - dmin * min[i/32]. */
+int oracle_proj_block_weights(int qtype) {
+  return qtype == ORACLE_QTYPE_Q8_0 ? 32 : (qtype == ORACLE_QTYPE_Q4_K ? 256 : -1);
+}
+int oracle_proj_block_bytes(int qtype) {
+  return qtype == ORACLE_QTYPE_Q8_0 ? 34 : (qtype == ORACLE_QTYPE_Q4_K ? 144 : -1);
+}
+
+static double q8_0_weight(const uint8_t *blk, int i) {
+  return oracle_fp16_to_double(load_u16(blk)) * (double)(int8_t)blk[2 + i];
+}
+
+static double q4_k_weight(const uint8_t *blk, int i) {
+  const double d = oracle_fp16_to_double(load_u16(blk)), dmin = oracle_fp16_to_double(load_u16(blk + 2));
+  const int j = i / 32;
+  /* bits 6j.. and 48+6j.. of the 96-bit field bytes 4..15 */
+  int sc = 0, mn = 0;
+  for (int b = 0; b < 6; ++b) {
+    const int bs = 6 * j + b, bm = 48 + 6 * j + b;
+    sc |= ((blk[4 + bs / 8] >> (bs % 8)) & 1) << b;
+    mn |= ((blk[4 + bm / 8] >> (bm % 8)) & 1) << b;
+  }
+  const int q = (blk[16 + i / 2] >> (4 * (i % 2))) & 15;
+  return d * sc * q - dmin * mn;
+}
+
+/* Dequantise a rows x k matrix of a projection format (row-major weights
+ * cut into consecutive blocks; k a multiple of the block size). */
+int oracle_dequant_proj(int qtype, const uint8_t *packed, int64_t rows, int64_t k, double *out) {
+  const int bw = oracle_proj_block_weights(qtype), bb = oracle_proj_block_bytes(qtype);
+  if (bw < 0 || !packed || !out || rows <= 0 || k <= 0 || k % bw) return ORACLE_EINVAL;
+  for (int64_t w = 0; w < rows * k; ++w) {
+    const uint8_t *blk = packed + (w / bw) * bb;
+    out[w] = qtype == ORACLE_QTYPE_Q8_0 ? q8_0_weight(blk, (int)(w % bw)) : q4_k_weight(blk, (int)(w % bw));
+  }
+  return ORACLE_OK;
+}
+
+/* y[t][r] = sum_c W[r][c] * x[t][c] for a projection-format matrix, in
+ * double (c ascending).  x: [n_tokens, k] fp32; y: [n_tokens, rows]. */
+int oracle_gemv_proj(int qtype, const uint8_t *packed, int64_t rows, int64_t k, const float *x, int n_tokens,
+                     double *y) {
+  if (n_tokens < 0 || !x || !y) return ORACLE_EINVAL;
+  double *wd = (double *)malloc(sizeof(double) * (size_t)(rows * k));
+  if (!wd) return ORACLE_EINVAL;
+  int rc = oracle_dequant_proj(qtype, packed, rows, k, wd);
+  if (rc == ORACLE_OK)
+    for (int t = 0; t < n_tokens; ++t)
+      for (int64_t r = 0; r < rows; ++r) {
+        double s = 0.0;
+        for (int64_t c = 0; c < k; ++c) s += wd[r * k + c] * (double)x[(int64_t)t * k + c];
+        y[(int64_t)t * rows + r] = s;
+      }
+  free(wd);
+  return rc;
+}
+
 /* ------------------------------------------------------------------ layer */
 
 /* y[r] = sum_c W[r][c] * v[c] for r < rows, c < k, in double, c ascending.

@@ -35,6 +35,8 @@ extern "C" {
 
 #define ORACLE_QTYPE_IQ2XS 1
 #define ORACLE_QTYPE_IQ1M 2
+#define ORACLE_QTYPE_Q8_0 3 /* projection formats (see oracle_dequant_proj) */
+#define ORACLE_QTYPE_Q4_K 4
 
 #define ORACLE_OK 0
 #define ORACLE_EINVAL (-1)
@@ -96,6 +98,16 @@ int oracle_moe_block(const float *h, int n_tokens, int hidden, const float *gamm
                      const float *router_w, int n_experts, int top_k, const oracle_expert *experts,
                      const oracle_expert *shared, const int8_t *grid_iq2, const int8_t *grid_iq1, double *out,
                      int32_t *ids_out, double *weights_out);
+
+/* Projection formats (Q8_0-style: 34 bytes / 32 weights; Q4_K-style: 144
+ * bytes / 256 weights; layouts stated in redlite_oracle.c): weights and
+ * bytes per block (-1 for another qtype), whole-matrix dequantisation and
+ * the fp64 matrix-vector product y = W x for n_tokens vectors. */
+int oracle_proj_block_weights(int qtype);
+int oracle_proj_block_bytes(int qtype);
+int oracle_dequant_proj(int qtype, const uint8_t *packed, int64_t rows, int64_t k, double *out);
+int oracle_gemv_proj(int qtype, const uint8_t *packed, int64_t rows, int64_t k, const float *x, int n_tokens,
+                     double *y);
 
 /* Threads used by oracle_moe_layer (OpenMP build); returns the value in force. */
 int oracle_set_threads(int n);
