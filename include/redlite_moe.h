@@ -63,7 +63,12 @@
 extern "C" {
 #endif
 
-typedef enum { REDLITE_Q_IQ2XS_STYLE = 1, REDLITE_Q_IQ1M_STYLE = 2 } redlite_qtype;
+typedef enum {
+  REDLITE_Q_IQ2XS_STYLE = 1, /* expert formats (the layer) */
+  REDLITE_Q_IQ1M_STYLE = 2,
+  REDLITE_Q_Q8_0_STYLE = 3,  /* projection formats (redlite_proj_gemv) */
+  REDLITE_Q_Q4_K_STYLE = 4
+} redlite_qtype;
 
 enum {
   REDLITE_OK = 0,
@@ -269,6 +274,32 @@ int redlite_moe_upload_experts(int32_t hidden, const int32_t *ids, const redlite
                                void *pool, size_t pool_bytes, size_t pool_offset, redlite_moe_expert *table_dev,
                                int32_t n_experts, void *stream, redlite_moe_upload_counters *counters,
                                size_t *pool_end);
+
+/* ---------------------------------------------------------------- projections
+ * The decode-GEMV for the other weight formats of the model the pages run
+ * ("Red Lite dev15 -- DeltaNet projection bring-up", section "Field-derived
+ * recurrent dimensions": ssm_ba Q8_0, ssm_out Q4_K; "Red Lite dev16",
+ * section "Pinned full-attention graph": attn_k, attn_v, attn_output Q4_K).
+ * The pages print no layouts; the library reads them as:
+ *   Q8_0-style  34 bytes / 32 weights: u16 d (fp16) | int8 q[32];
+ *               w = d * q
+ *   Q4_K-style 144 bytes / 256 weights: u16 d | u16 dmin (fp16) | u8 sm[12]
+ *               (96-bit little-endian field: 6-bit scale of sub-block j =
+ *               weights 32j..32j+31 at bit 6j, 6-bit minimum at bit 48+6j)
+ *               | u8 q[128] (weight i: nibble i & 1 of byte i / 2);
+ *               w = d * scale * q - dmin * minimum
+ * A rows x k matrix is its row-major weights cut into consecutive blocks. */
+
+/* Packed bytes of a rows x k projection matrix (k a multiple of 256), or 0. */
+size_t redlite_proj_matrix_bytes(int32_t qtype, int64_t rows, int64_t k);
+
+/* y[t][r] = sum_c W[r][c] * x[t][c] for t < n_tokens (0..8), fp32.
+ *   W  device, the packed matrix (2-byte aligned for Q8_0-style, 16-byte
+ *      aligned for Q4_K-style); x device [n_tokens, k] fp32, 16-byte aligned;
+ *   y  device [n_tokens, rows] fp32, overwritten.
+ * REDLITE_EUNSUPPORTED if k is not a multiple of 256; enqueued on stream. */
+int redlite_proj_gemv(int32_t qtype, const void *W, int64_t rows, int64_t k, const float *x, int32_t n_tokens,
+                      float *y, void *stream);
 
 /* ---------------------------------------------------------------- slot pool
  * The bounded, top-k-aware LRU pool of expert slots ("Red Metal dev8",

@@ -30,6 +30,8 @@ from ._native import (  # noqa: F401
     redlite_moe_block,
     redlite_moe_block_scratch_bytes,
     redlite_moe_pack_matrix,
+    redlite_proj_gemv,
+    redlite_proj_matrix_bytes,
     redlite_moe_pool_counters,
     redlite_moe_route_topk,
     redlite_moe_table,

@@ -17,6 +17,8 @@ LIB_PATH = os.path.join(_HERE, "libredlite_moe.so")
 
 REDLITE_Q_IQ2XS_STYLE = 1
 REDLITE_Q_IQ1M_STYLE = 2
+REDLITE_Q_Q8_0_STYLE = 3
+REDLITE_Q_Q4_K_STYLE = 4
 REDLITE_OK = 0
 REDLITE_EINVAL = -1
 REDLITE_EUNSUPPORTED = -2
@@ -83,6 +85,9 @@ EXPORTS = {
                                                 _c_void_p, ctypes.c_size_t, _c_void_p, _c_void_p, _c_void_p,
                                                 ctypes.POINTER(redlite_moe_pool_counters),
                                                 ctypes.POINTER(ctypes.c_int64)]),
+    "redlite_proj_matrix_bytes": (ctypes.c_size_t, [ctypes.c_int32, ctypes.c_int64, ctypes.c_int64]),
+    "redlite_proj_gemv": (ctypes.c_int, [ctypes.c_int32, _c_void_p, ctypes.c_int64, ctypes.c_int64, _c_void_p,
+                                         ctypes.c_int32, _c_void_p, _c_void_p]),
     "redlite_moe_pack_matrix": (ctypes.c_int, [ctypes.c_int32, ctypes.c_int64, ctypes.c_int64, _c_void_p,
                                                _c_void_p]),
     "redlite_moe_dequant": (ctypes.c_int, [ctypes.c_int32, _c_void_p, ctypes.c_int64, ctypes.c_int64, _c_void_p,
@@ -233,6 +238,16 @@ def redlite_moe_upload_experts(hidden: int, ids, host_experts, pool: torch.Tenso
                                           ctypes.byref(ctr), ctypes.byref(end))
     del keep
     return rc, int(end.value)
+
+
+def redlite_proj_matrix_bytes(qtype: int, rows: int, k: int) -> int:
+    return int(lib().redlite_proj_matrix_bytes(qtype, rows, k))
+
+
+def redlite_proj_gemv(qtype: int, W: torch.Tensor, rows: int, k: int, x: torch.Tensor, n_tokens: int,
+                      y: torch.Tensor, stream=None) -> int:
+    """y = W x for a Q8_0-style (3) or Q4_K-style (4) projection matrix."""
+    return lib().redlite_proj_gemv(qtype, _ptr(W), rows, k, _ptr(x), n_tokens, _ptr(y), _stream_handle(stream))
 
 
 class SlotPool:

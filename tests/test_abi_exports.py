@@ -176,3 +176,17 @@ def test_router_and_block_reject_on_host(native):
         native.REDLITE_EINVAL
     assert L.redlite_moe_block(None, 0, None, ctypes.c_float(1e-6), None, 10, ctypes.byref(t), None, None, None, 0) == \
         native.REDLITE_OK
+
+
+def test_proj_gemv_rejects_on_host(native):
+    L = native.lib()
+    p = ctypes.c_void_p(0x10000)
+    assert native.redlite_proj_matrix_bytes(3, 64, 2048) == 64 * 64 * 34
+    assert native.redlite_proj_matrix_bytes(4, 2048, 4096) == 2048 * 16 * 144
+    assert native.redlite_proj_matrix_bytes(4, 8, 300) == 0 and native.redlite_proj_matrix_bytes(1, 8, 256) == 0
+    assert L.redlite_proj_gemv(4, p, 8, 300, p, 1, p, None) == native.REDLITE_EUNSUPPORTED
+    assert L.redlite_proj_gemv(4, p, 8, 256, p, 9, p, None) == native.REDLITE_EINVAL
+    assert L.redlite_proj_gemv(5, p, 8, 256, p, 1, p, None) == native.REDLITE_EINVAL
+    assert L.redlite_proj_gemv(4, ctypes.c_void_p(0x10008), 8, 256, p, 1, p, None) == native.REDLITE_EINVAL
+    assert L.redlite_proj_gemv(3, ctypes.c_void_p(0x10001), 8, 256, p, 1, p, None) == native.REDLITE_EINVAL
+    assert L.redlite_proj_gemv(4, p, 8, 256, p, 0, p, None) == native.REDLITE_OK
