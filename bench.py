@@ -116,10 +116,11 @@ class ClockSampler:
         return self.summarise(rows, self.window)
 
 
-# Source files that do not go into a kernel's translation unit: a change there
-# leaves the counters taken for that kernel valid.
-_NOT_IN = {k: ("grouped_tc.cu", "route.cu", "tiles_simt.cu") for k in ("decode", "decode_iq1", "batched")}
-_NOT_IN["prefill"] = ("decode_fused.cu", "noalloc.cu", "tiles_simt.cu")
+# The source files of each measured kernel: counters taken for a kernel stay
+# valid while these files are unchanged.
+_HDRS = ("internal.cuh", "layout.cuh")
+_SRC_OF = {k: ("decode_fused.cu",) + _HDRS for k in ("decode", "decode_iq1", "batched")}
+_SRC_OF["prefill"] = ("grouped_tc.cu", "route.cu", "ptx.cuh") + _HDRS
 
 
 def max_over_ranks(ms, world, device=None):
@@ -157,12 +158,11 @@ def input_views(buf, T, H, k):
             buf[nx + ni:nx + 2 * ni].view(torch.float32).view(T, k))
 
 
-def _source_sha(exclude=()):
+def _source_sha(files):
     h = hashlib.sha256()
     csrc = os.path.join(ROOT, "routed_expert_ffn_iq2_b200", "csrc")
-    for fn in sorted(os.listdir(csrc)):
-        if fn not in exclude:
-            h.update(open(os.path.join(csrc, fn), "rb").read())
+    for fn in sorted(files):
+        h.update(open(os.path.join(csrc, fn), "rb").read())
     return h.hexdigest()[:16]
 
 
@@ -173,7 +173,7 @@ def _traffic(kernel_key: str):
     if not os.path.exists(p):
         return None
     d = json.load(open(p)).get(kernel_key)
-    if not d or d.get("source_sha") != _source_sha(_NOT_IN.get(kernel_key, ())):
+    if not d or d.get("source_sha") != _source_sha(_SRC_OF[kernel_key]):
         return None
     return d.get("dram_bytes_per_launch")
 
@@ -442,6 +442,143 @@ def measure(cfg: int, steps: int, warmup: int, world: int, rank: int, local: int
     }
 
 
+# ------------------------------------------------------------------ the other rows of the path
+
+
+def _graph_time(fn, n_calls, reps, stream):
+    """Device time per call (us) of `fn` captured n_calls times in a CUDA graph."""
+    import torch
+
+    for _ in range(3):
+        fn(0)
+    stream.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(n_calls):
+            fn(i)
+    g.replay()
+    stream.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for _ in range(reps):
+        g.replay()
+    e1.record(stream)
+    e1.synchronize()
+    return e0.elapsed_time(e1) * 1e3 / (reps * n_calls)
+
+
+def measure_components(dev):
+    """Router, block, slot pool and projection GEMVs on their own (one GPU):
+    device time per call and the rate each is bound by."""
+    import ctypes
+
+    import torch
+
+    import routed_expert_ffn_iq2_b200 as R
+
+    peaks = _peaks()
+    stream = torch.cuda.Stream(dev)
+    torch.cuda.set_stream(stream)
+    res = {}
+    # router: 64 tokens x 512 logits -> top-10
+    st = fixtures.Stream(0x5EED0004, 4)
+    lg = torch.from_numpy(st.normal(64 * 512).reshape(64, 512).astype(np.float32)).to(dev)
+    ids = torch.empty((64, 10), dtype=torch.int32, device=dev)
+    wts = torch.empty((64, 10), dtype=torch.float32, device=dev)
+    us = _graph_time(lambda i: R.redlite_moe_route_topk(lg, 64, 512, 10, ids, wts, stream), 100, 20, stream)
+    res["router"] = {"workload": "route-top10-t64-e512", "us_per_call": us, "tokens_per_s": 64 / (us * 1e-6)}
+    # projection GEMVs, one token: the recurrent layer's ssm_ba (Q8_0, 2048 -> 64) and ssm_out (Q4_K,
+    # 4096 -> 2048), the attention layer's attn_k (Q4_K, 2048 -> 512)
+    for name, qt, rows, k in (("ssm_ba-q8_0-2048x64", 3, 64, 2048), ("ssm_out-q4_k-4096x2048", 4, 2048, 4096),
+                              ("attn_k-q4_k-2048x512", 4, 512, 2048)):
+        nmat = max(1, (256 << 20) // R.redlite_proj_matrix_bytes(qt, rows, k))  # cycle > L2 of copies
+        mats = [torch.from_numpy(fixtures.make_proj_matrix(800, qt, rows, k)).to(dev)]
+        big = mats[0].repeat(min(nmat, 64))
+        mb = R.redlite_proj_matrix_bytes(qt, rows, k)
+        nm = big.numel() // mb
+        xv = torch.from_numpy(fixtures.make_x(801, 1, k)).to(dev)
+        yv = torch.empty((1, rows), dtype=torch.float32, device=dev)
+        us = _graph_time(lambda i: R.redlite_proj_gemv(qt, big[(i % nm) * mb:(i % nm + 1) * mb], rows, k, xv, 1, yv,
+                                                        stream), nm, 10, stream)
+        gbs = (mb + 4 * (k + rows)) / (us * 1e-6) / 1e9
+        res["proj_" + name] = {"us_per_call": us, "roofline": {"bound": "hbm", "achieved": gbs,
+                                                               "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                                                               "frac": gbs / peaks["hbm_gbs"]},
+                               "copies_cycled": nm, "l2": "matrix copies cycled" if nm * mb > (126 << 20) else
+                               "matrix copies cycled (inside L2)"}
+    # block and pool: 64 IQ2_XS-style experts of width 512, hidden 2048, top-10, one token per call
+    H, E, F, k = 2048, 64, 512, 10
+    seed = 0x5EED00B0
+    g2, g1 = fixtures.make_grid(seed, 1), fixtures.make_grid(seed, 2)
+    experts = [fixtures.make_expert(seed, 1, H, F, e) for e in range(E)]
+    L = R.MoeLayer(H, E, F, 1, k, g2, g1, pool_bytes=(E + 1) * (fixtures.expert_bytes(1, H, F) + 64), device=str(dev),
+                   stream=stream)
+    for i in range(0, E, 16):
+        R._native._check(L.upload(list(range(i, i + 16)), experts[i:i + 16]), "upload")
+    hs = torch.from_numpy(fixtures.make_x(seed, 48, H)).to(dev)
+    gam = torch.from_numpy((1.0 + 0.1 * fixtures.Stream(seed, 2).normal(H)).astype(np.float32)).to(dev)
+    rw = torch.from_numpy((0.05 * fixtures.Stream(seed, 3).normal(E * H)).reshape(E, H).astype(np.float32)).to(dev)
+    scratch = torch.zeros(R.redlite_moe_block_scratch_bytes(H, E, 1, k), dtype=torch.uint8, device=dev)
+    out = torch.empty((1, H), dtype=torch.float32, device=dev)
+    us = _graph_time(lambda i: R.redlite_moe_block(hs[i % 48:i % 48 + 1], 1, gam, 1e-6, rw, k, L.table, None, out,
+                                                   scratch), 96, 20, stream)
+    if L.read_status() != 0:
+        raise RuntimeError(f"block: device status {L.read_status()}")
+    res["block"] = {"workload": "block-rmsnorm-router-iq2xs-h2048-e64-f512-top10-t1", "us_per_call": us,
+                    "tokens_per_s": 1 / (us * 1e-6)}
+    # slot pool: capacity 24, every call a fresh top-10 (cycling through 6 disjoint sets of the 64
+    # experts), misses filled host -> device on a copy stream while the previous layer call runs
+    pool = R.SlotPool(E, 24)
+    gb = fixtures.matrix_bytes(1, F, H)
+    slot_bytes = 2 * ((gb + 15) // 16 * 16) + fixtures.matrix_bytes(1, H, F)
+    slots = torch.zeros(24 * slot_bytes, dtype=torch.uint8, device=dev)
+    host = (R.redlite_moe_expert * E)()
+    keep = []
+    for e, ex in enumerate(experts):
+        mats = []
+        for m, (r, c) in zip((ex.gate, ex.up, ex.down), ((F, H), (F, H), (H, F))):
+            t = torch.from_numpy(R.redlite_moe_pack_matrix(1, r, c, m)).pin_memory()
+            mats.append(t)
+        keep += mats
+        host[e] = R.redlite_moe_expert(1, F, *[t.data_ptr() for t in mats])
+    PL = R.MoeLayer(H, E, F, 1, k, g2, g1, pool_bytes=16, device=str(dev), stream=stream)
+    PL.table.min_ffn = F
+    sets = [list(range(10 * j, 10 * j + 10)) for j in range(6)]
+    copy_s = torch.cuda.Stream(dev)
+    xin = torch.from_numpy(fixtures.make_x(seed, 1, H)).to(dev)
+    wt = torch.full((1, k), 0.1, dtype=torch.float32, device=dev)
+    idt = [torch.tensor([s], dtype=torch.int32, device=dev) for s in sets]
+    pend = []
+    n_calls = 60
+    for warm in (True, False):
+        stream.synchronize()
+        t0 = time.perf_counter()
+        c0 = (pool.counters.loads, pool.counters.bytes)
+        for i in range(n_calls if not warm else 6):
+            rc, tok = pool.acquire(sets[i % 6], host, H, slots, slot_bytes, PL.table_dev, copy_s, stream)
+            while rc == R.REDLITE_EAGAIN:  # every slot in flight: retire the oldest call
+                torch.cuda.current_stream().synchronize()
+                stream.synchronize()
+                rc, tok = pool.acquire(sets[i % 6], host, H, slots, slot_bytes, PL.table_dev, copy_s, stream)
+            R._native._check(rc, "pool acquire")
+            R._native._check(R.redlite_moe_layer(xin, 1, idt[i % 6], wt, k, PL.table, None, out), "layer")
+            pool.release(tok, stream)
+        stream.synchronize()
+        dt = time.perf_counter() - t0
+    loads = pool.counters.loads - c0[0]
+    nbytes = pool.counters.bytes - c0[1]
+    if PL.read_status() != 0:
+        raise RuntimeError(f"pool: device status {PL.read_status()}")
+    res["pool"] = {"workload": "pool-cap24-e64-iq2xs-top10-t1, a fresh selection per call", "calls": n_calls,
+                   "us_per_call": dt * 1e6 / n_calls, "loads": int(loads), "h2d_gbs": nbytes / dt / 1e9,
+                   "note": "host wall time of acquire + layer per call (fills from pinned host memory on a copy "
+                           "stream)"}
+    pool.close()
+    del keep, L, PL
+    torch.cuda.empty_cache()
+    return res
+
+
 # ------------------------------------------------------------------ main
 
 
@@ -456,6 +593,7 @@ def main():
     ap.add_argument("--cpu-budget", type=float, default=12.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-components", action="store_true", help="skip router/block/pool/projection timings")
     args = ap.parse_args()
     steps = max(1, args.steps)
 
@@ -504,6 +642,7 @@ def main():
                 r.pop("cpu_baseline", None)
                 others[str(c)] = r
 
+    comps = measure_components(dev) if world == 1 and not args.no_components else None
     if rank == 0:
         line = {
             "metric": METRIC, "value": head["value"], "unit": "tokens/s", "n_gpus": world, "steps": steps,
@@ -523,6 +662,8 @@ def main():
         }
         if others:
             line["workloads"] = others
+        if comps:
+            line["components"] = comps
         print(json.dumps(line), flush=True)
     if world > 1:
         import torch.distributed as dist
