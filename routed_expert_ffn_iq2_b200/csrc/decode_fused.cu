@@ -541,6 +541,28 @@ __global__ void __launch_bounds__(kCThreads, 1) decode_fused_kernel(FusedArgs a)
     bulk_g2s(S.sel1, a.grids + kGridQ1Sel, 4096 * 4, &s_lut_bar);
   }
   asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  // Warm L2 with the call's small inputs and the whole slot table while the
+  // previous kernel of the stream finishes: a prefetch reads nothing into
+  // registers, and L2 stays coherent with writes that land after it.  One
+  // 128-byte line per thread of the grid.
+  {
+    const unsigned g = (unsigned)cta * kCThreads + tid;
+    const unsigned l_tab = (unsigned)(E * (int)sizeof(redlite_moe_expert) + 127) / 128u;
+    const unsigned l_ids = (unsigned)(npairs * 4 + 127) / 128u;
+    const unsigned l_x = (unsigned)(T * H * 4 + 127) / 128u;
+    const char *p = nullptr;
+    if (g < l_tab)
+      p = reinterpret_cast<const char *>(a.experts) + 128 * g;
+    else if (g < l_tab + l_ids)
+      p = reinterpret_cast<const char *>(a.ids) + 128 * (g - l_tab);
+    else if (g < l_tab + 2 * l_ids)
+      p = reinterpret_cast<const char *>(a.weights) + 128 * (g - l_tab - l_ids);
+    else if (g < l_tab + 2 * l_ids + l_x)
+      p = reinterpret_cast<const char *>(a.x) + 128 * (g - l_tab - 2 * l_ids);
+    else if (a.residual && g < l_tab + 2 * l_ids + 2 * l_x)
+      p = reinterpret_cast<const char *>(a.residual) + 128 * (g - l_tab - 2 * l_ids - l_x);
+    if (p) asm volatile("prefetch.global.L2 [%0];" ::"l"(p));
+  }
   __syncthreads();  // the mbarriers are initialised before anyone waits on them
   // the call's own inputs may come from the previous kernel
   asm volatile("griddepcontrol.wait;" ::: "memory");
@@ -555,8 +577,6 @@ __global__ void __launch_bounds__(kCThreads, 1) decode_fused_kernel(FusedArgs a)
     my_w[j] = p < npairs ? __ldcg(a.weights + p) : 0.f;
   }
   TR_STAMP(8);
-  if (T <= 4)  // warm L2 for the warps' activation slices
-    for (int i = tid; i < T * H / 32; i += kCThreads) asm volatile("prefetch.global.L2 [%0];" ::"l"(a.x + 32 * i));
 #pragma unroll
   for (int j = 0; j < 2; ++j) {
     const int e = my_ids[j];
@@ -623,6 +643,7 @@ __global__ void __launch_bounds__(kCThreads, 1) decode_fused_kernel(FusedArgs a)
         rank += (kq < key) || (kq == key && q < lane);
         less |= (unsigned)(kq < key) << q;
       }
+      TR_STAMP(17);
       const unsigned same = __match_any_sync(0xffffffffu, key), lt = (1u << lane) - 1u;
       const bool leader = ok && (same & lt) == 0;
       const unsigned leaders = __ballot_sync(0xffffffffu, leader);
@@ -646,6 +667,7 @@ __global__ void __launch_bounds__(kCThreads, 1) decode_fused_kernel(FusedArgs a)
       bad = __reduce_or_sync(0xffffffffu, bad);
       if (lane == 0) s_bad = bad;
       __syncwarp();
+      TR_STAMP(18);
       item_prefix(n_inst);
       TR_STAMP(9);
     } else {
@@ -857,10 +879,12 @@ __global__ void __launch_bounds__(kCThreads, 1) decode_fused_kernel(FusedArgs a)
       S.items[k] = item_word(lo, loc / ng, loc % ng, phase);
     }
     __syncwarp();
+    TR_STAMP(19);
     if (lane < min(kRing, my1 + my2)) {
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");  // the rings were bucketing scratch
       issue(lane);
     }
+    TR_STAMP(20);
   } else {
     // ---- the other warps zero this CTA's slice of out, or copy the
     // residual into it (the down items add into it after the grid barrier;
@@ -921,7 +945,10 @@ __global__ void __launch_bounds__(kCThreads, 1) decode_fused_kernel(FusedArgs a)
   // this warp's activation limbs: the input slice of its current tile-block
   // for the item's token positions (per-slice scales sc0, sc1)
   uint8_t *wl = S.wlimbs + (size_t)warp * kTokChunk * 3 * kWPlane;
-  uint32_t lim_key = 0xFFFFFFFFu;  // (instance, chunk, phase, input block) of the limbs in wl
+  // what the limbs in wl hold: phase 1 (input block, the positions' tokens),
+  // phase 2 (input block, first pair, positions) -- gate/up items of other
+  // experts with the same tokens reuse them
+  uint64_t lim_key = ~0ull;
   float sc0 = 0.f, sc1 = 0.f;
   const uint32_t g2 = smem_u32(S.sel2), g1 = smem_u32(S.sel1);
   const int ncol = lane >> 2, cpos = ncol / 3;  // this lane's B column: limb ncol % 3 of position cpos
@@ -957,7 +984,10 @@ __global__ void __launch_bounds__(kCThreads, 1) decode_fused_kernel(FusedArgs a)
     float acc[4] = {0.f, 0.f, 0.f, 0.f};
     TR(0);
     if (bytes) {
-      const uint32_t key = (w & ~(255u << 19)) | ((uint32_t)kb << 28);
+      const uint64_t key =
+          phase == 1 ? ((uint64_t)kb << 60) | ((uint64_t)(uint32_t)S.pair_tok[pbase] << 30) |
+                           (uint32_t)(ntok > 1 ? S.pair_tok[pbase + 1] + 1 : 0)
+                     : (1ull << 63) | ((uint64_t)kb << 60) | ((uint64_t)(uint32_t)pbase << 30) | (uint32_t)ntok;
       if (key != lim_key) {
         // limbs of the item's token positions, this warp's 256 inputs
         lim_key = key;

@@ -4,11 +4,12 @@
 // "Red Metal dev8 -- resident routed top-k layer", steps 4-6, for a batch of
 // tokens: the (token, slot) pairs are bucketed by expert (route.cu), then
 // every expert's gate/up and down projections run as dense contractions on
-// the 5th-generation tensor cores (tcgen05.mma, bf16 operands in shared
-// memory, fp32 accumulators in tensor memory).  Weights are decoded from the
-// packed tile-blocks into 128-byte-swizzled bf16 tiles (each weight is exact
-// in fp32 and rounded to bf16, nearest even); activations are rounded to bf16
-// the same way.  Accumulation is fp32.
+// the 5th-generation tensor cores (tcgen05.mma, bf16 operands, fp32
+// accumulators in tensor memory).  Weights are decoded from the packed
+// tile-blocks straight into tensor memory (each weight is exact in fp32 and
+// rounded to bf16, nearest even), where the MMA reads its A operand; the
+// activations (B) are rounded to bf16 the same way and staged in shared
+// memory.  Accumulation is fp32.
 //
 // Work unit: (expert, 128 output rows, up to 128 of the expert's tokens).
 //   gate/up  A = the rows of gate and of up, B = the tokens' activations;
@@ -19,14 +20,22 @@
 //   warp 0      one thread bulk-copies the packed tile-blocks of each
 //               256-input column of a unit (8 per matrix) into a 2-deep ring;
 //   warp 1      one thread issues the tcgen05.mma of every 64-input step and
-//               commits them to the step's slot and, per unit, to one of two
-//               accumulator buffers;
-//   warps 2-9   dequant warp w decodes tile-block w (rows 16w..16w+15) of
-//               each matrix into the A tiles of a ring of 64-input steps (3
-//               deep for gate/up, 5 for down) and
-//               fetches rows 16w..16w+15 of B with cp.async, a step ahead;
-//   warps 10-13 the epilogue (TMEM -> registers -> h or out), overlapping
-//               the next unit's contraction.
+//               commits them to the step's slot and, per unit, to an
+//               accumulator buffer (one for gate/up, two for down);
+//   warps 2-9   dequant warps: each decodes one tile-block (16 rows) of each
+//               matrix, in the TMEM lane quarter its warp index may write,
+//               into the A slots of a 4-step ring in tensor memory
+//               (tcgen05.st), and fetches 16 rows of B with cp.async into the
+//               matching shared-memory slot, a step ahead;
+//   warps 10-13 the epilogue (TMEM -> registers -> h or out).
+//
+// Input order inside a 64-input step.  A thread of the 16-lane TMEM store
+// holds four consecutive K positions of its two rows per 16-position chunk,
+// and decodes 8-weight groups t and t + 4 of the step (t = lane % 4).  So
+// TMEM position 32 c + 16 j + 4 t + i holds input 32 c + 8 t + 4 j + i of
+// the step (c, j in {0, 1}, i < 4), and the bf16 copies of x and of h that
+// B is loaded from are stored in that same order (perm64): the contraction
+// over a step is a sum over all 64 inputs either way.
 #include "internal.cuh"
 #include "layout.cuh"
 #include "ptx.cuh"
@@ -38,10 +47,11 @@ constexpr int kDqWarps = 8;
 constexpr int kEpWarps = 4;
 constexpr int kTcWarps = 2 + kDqWarps + kEpWarps;
 constexpr int kTcThreads = 32 * kTcWarps;  // 448
-constexpr int kTile = 128 * 64 * 2;        // 16 KB: 128 rows x 64 bf16
+constexpr int kBTile = 128 * 64 * 2;       // 16 KB: up to 128 token rows x 64 bf16
 constexpr int kPr = 2;                     // packed columns in flight
 constexpr int kMaxUnits = 128;             // unit records per pass
 constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kAccCols = 256;         // accumulators in columns 0..255, A slots above
 
 // Optional per-warp cycle counters (build with -DREDLITE_TC_TRACE): CTA c,
 // warp w adds to 8 words at the end of the workspace layout, slot (c * 32 + w) * 8.
@@ -67,11 +77,43 @@ constexpr uint32_t kTmemCols = 512;
 template <bool DOWN>
 struct Cfg {
   static constexpr int kMats = DOWN ? 1 : 2;
-  static constexpr int kAr = DOWN ? 5 : 3;                  // 64-input steps in flight
-  static constexpr int kStep = (kMats + 1) * kTile;         // A tiles, then the B tile
+  static constexpr int kAr = 4;                             // 64-input steps in flight
+  static constexpr int kStep = kBTile;                      // shared memory per step: the B tile
   static constexpr int kPacked = kMats * 8 * kQ2TileBlock;  // one column, largest format
-  static constexpr uint32_t kBufCols = DOWN ? 128 : 256;    // TMEM columns per accumulator buffer
+  static constexpr uint32_t kSlotCols = kMats * 32;         // TMEM columns of one step's A tiles
+  static_assert(kAccCols + kAr * kSlotCols <= kTmemCols, "TMEM columns");
 };
+
+// Accumulator columns of a unit.  down: buffer b = unit count mod 2, columns
+// 128 b ..  gate/up: two halves, half b = gate columns 64 b .. 64 b + 63 and
+// up columns 128 + 64 b ..; a unit of at most 64 tokens takes the next half
+// in turn, a larger one both (gate 0 .., up 128 ..).  The MMA thread and the
+// epilogue warps replay the same sequence; mask: the halves the unit holds.
+struct AccPlan {
+  uint32_t gate, up;
+  int mask;
+};
+template <bool DOWN>
+__device__ __forceinline__ AccPlan acc_plan(int n_pad, uint32_t ucount, int &next) {
+  AccPlan p;
+  if (DOWN) {
+    const int b = (int)(ucount & 1u);
+    p.gate = 128u * b, p.up = 0u, p.mask = 1 << b;
+  } else if (n_pad <= 64) {
+    p.gate = 64u * next, p.up = 128u + 64u * next, p.mask = 1 << next;
+    next ^= 1;
+  } else {
+    p.gate = 0u, p.up = 128u, p.mask = 3;
+    next = 0;
+  }
+  return p;
+}
+
+// Position of input `in` of a 64-input step in the order the tensor-core
+// kernels contract over (see the header): bit 2 moves to bit 4, bits 3-4 to bits 2-3.
+__host__ __device__ __forceinline__ int perm64(int in) {
+  return (in & ~31) | ((in & 4) << 2) | ((in & 24) >> 1) | (in & 3);
+}
 
 struct Unit {
   const uint8_t *mat0, *mat1;  // gate, up (or down, unused)
@@ -89,12 +131,15 @@ struct Smem {
   Unit *units;
   Bars *bars;
   uint32_t *taddr;
+  float *stage;  // epilogue stages
 };
+
+constexpr int kEpStage = 2 * 16 * 128;  // epilogue: two 16-column x 128-row stages (fp32; bf16 for h)
 
 template <bool DOWN>
 constexpr size_t smem_bytes() {
   return 1024 + (size_t)Cfg<DOWN>::kAr * Cfg<DOWN>::kStep + (size_t)kPr * Cfg<DOWN>::kPacked + 512 * 8 + 2048 * 8 +
-         sizeof(Unit) * kMaxUnits + sizeof(Bars) + 16;
+         sizeof(Unit) * kMaxUnits + sizeof(Bars) + 16 + sizeof(float) * kEpStage;
 }
 
 template <bool DOWN>
@@ -114,6 +159,8 @@ __device__ __forceinline__ Smem carve(uint8_t *smem) {
   S.bars = reinterpret_cast<Bars *>(p);
   p += sizeof(Bars);
   S.taddr = reinterpret_cast<uint32_t *>(p);
+  p += 16;
+  S.stage = reinterpret_cast<float *>(p);
   return S;
 }
 
@@ -161,6 +208,17 @@ __device__ __forceinline__ void cp_async16(void *dst, const void *src) {
 // entries (the scaled grid values of symbols 0, 1, 2) in two registers; the
 // byte-permute selectors of the weights' grid entry then pick a bf16 pair
 // per instruction.  IQ2_XS-style signs are flipped with one XOR per pair.
+// Lane (q, t) decodes rows q and q+8 of its tile-block, groups t and t + 4
+// of each 64-input step, into the sixteen registers of one 16-lane TMEM
+// store: group 4 c + t fills repetitions 2c (weights 0-3) and 2c+1
+// (weights 4-7), row q in registers 0-1 of a repetition, row q+8 in 2-3.
+
+__device__ __forceinline__ void put_group(uint32_t (&r)[16], int c, int h, uint4 v) {
+  r[8 * c + 2 * h] = v.x;
+  r[8 * c + 2 * h + 1] = v.y;
+  r[8 * c + 4 + 2 * h] = v.z;
+  r[8 * c + 4 + 2 * h + 1] = v.w;
+}
 
 // IQ2_XS-style tile-block fields of lane (q, t) (the resident layout's lane
 // order: rows q and q+8, groups 4c + t, field i = 2c + h).
@@ -185,19 +243,13 @@ __device__ __forceinline__ Q2Lane load_q2(uint32_t tb, int lane) {
   return r;
 }
 
-// Step s (inputs 64s..64s+63 of the column) of one IQ2 tile-block into rows
-// row0..row0+15 of the swizzled A tile: fields i = 4s + 2 c2 + h.  `lane` is
-// the layout lane (q, t); the warp runs it on thread q + 8 t, so the eight
-// threads of a quarter-warp store to eight different rows (conflict-free
-// 128-bit stores in the swizzled tile) with a field order fixed at compile time.
-__device__ __forceinline__ void dequant_q2(const Q2Lane &L, int s, uint32_t A, int row0, uint32_t sel2,
-                                           int lane) {
-  const int q = lane >> 2, t = lane & 3;
+// Step s (inputs 64s..64s+63 of the column) of one IQ2 tile-block: fields
+// i = 4s + 2c + h (group 8s + 4c + t of row q+8h).
+__device__ __forceinline__ void dequant_q2(const Q2Lane &L, int s, uint32_t sel2, uint32_t (&r)[16]) {
   const uint32_t qw = s == 0 ? L.qs[0] : s == 1 ? L.qs[1] : s == 2 ? L.qs[2] : L.qs[3];
   const uint32_t sw = s == 0 ? L.sg[0] : s == 1 ? L.sg[1] : s == 2 ? L.sg[2] : L.sg[3];
 #pragma unroll
-  for (int j = 0; j < 2; ++j) {
-    const int c2 = j;
+  for (int c2 = 0; c2 < 2; ++c2) {
     const int c = 2 * s + c2;
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
@@ -217,62 +269,59 @@ __device__ __forceinline__ void dequant_q2(const Q2Lane &L, int s, uint32_t A, i
       v.y = __byte_perm(t0, t1, sel.x >> 16) ^ ((__byte_perm(sgz, 0u, 0x4441u) * 0x08008000u) & 0x80008000u);
       v.z = __byte_perm(t0, t1, sel.y) ^ ((__byte_perm(sgz, 0u, 0x4442u) * 0x08008000u) & 0x80008000u);
       v.w = __byte_perm(t0, t1, sel.y >> 16) ^ ((__byte_perm(sgz, 0u, 0x4443u) * 0x08008000u) & 0x80008000u);
-      ptx::sts128(A + ptx::sw128_offset(row0 + q + 8 * h, 32 * c2 + 8 * t), v);
+      put_group(r, c2, h, v);
     }
   }
 }
 
-// IQ1_M-style tile-block fields of lane (q, t): pair p = t >> 1 (groups
-// 2 sb + p of rows q and q+8, field i = 2 sb + h); half = t & 1 takes
-// sub-blocks 4S + 2 half + {0, 1} of step S.
+// IQ1_M-style tile-block fields of lane (q, t) for groups 8S + 4c + t (c =
+// 0, 1) of every step S, rows q and q+8.  Group g sits in the record of
+// pair p = g & 1 (here t & 1) as entry i = 2 (g >> 1) + h; with u = t >> 1
+// the lane's entries of step S are bytes 2u, 2u+1 of qs words 2S and 2S+1,
+// and its qh nibbles bytes u and 2+u of nibble word S.
 struct Q1Lane {
   uint32_t qs[4], nb[4];
-  uint64_t row0, row1;  // 3-bit sub-block scales of rows q and q+8, from sub-block 2 half
+  uint64_t row0, row1;  // 3-bit sub-block scales of rows q and q+8, from sub-block u
   float d0, d1;
 };
 
 __device__ __forceinline__ Q1Lane load_q1(uint32_t tb, int lane) {
   Q1Lane r;
-  const int q = lane >> 2, p = (lane >> 1) & 1, half = lane & 1;
+  const int q = lane >> 2, p = lane & 1, u = (lane >> 1) & 1;
   const uint32_t pb = tb + 48 * (2 * q + p);
   const uint4 qa = ptx::lds128(pb), qb = ptx::lds128(pb + 16);
   const uint4 nb = ptx::lds128(pb + 32);
-  // qs word 2S + half holds fields 8S + 4 half .. + 3 of step S
-  r.qs[0] = half ? qa.y : qa.x;
-  r.qs[1] = half ? qa.w : qa.z;
-  r.qs[2] = half ? qb.y : qb.x;
-  r.qs[3] = half ? qb.w : qb.z;
-  // nibble word of step S: this lane's half of it
-  r.nb[0] = half ? nb.x >> 16 : nb.x & 0xFFFFu;
-  r.nb[1] = half ? nb.y >> 16 : nb.y & 0xFFFFu;
-  r.nb[2] = half ? nb.z >> 16 : nb.z & 0xFFFFu;
-  r.nb[3] = half ? nb.w >> 16 : nb.w & 0xFFFFu;
+  const uint32_t qsel = u ? 0x7632u : 0x5410u, nsel = u ? 0x4431u : 0x4420u;
+  r.qs[0] = __byte_perm(qa.x, qa.y, qsel);
+  r.qs[1] = __byte_perm(qa.z, qa.w, qsel);
+  r.qs[2] = __byte_perm(qb.x, qb.y, qsel);
+  r.qs[3] = __byte_perm(qb.z, qb.w, qsel);
+  r.nb[0] = __byte_perm(nb.x, 0u, nsel);
+  r.nb[1] = __byte_perm(nb.y, 0u, nsel);
+  r.nb[2] = __byte_perm(nb.z, 0u, nsel);
+  r.nb[3] = __byte_perm(nb.w, 0u, nsel);
   const uint32_t s0 = ptx::lds32(tb + 768 + 12 * q), s1 = ptx::lds32(tb + 772 + 12 * q),
                  s2 = ptx::lds32(tb + 776 + 12 * q);
   r.row0 = (uint64_t)s0 | ((uint64_t)(s1 & 0xFFFFu) << 32);
   r.row1 = (uint64_t)(s1 >> 16) | ((uint64_t)s2 << 16);
-  r.row0 >>= 6 * half;  // this lane's sub-blocks are 4 S + 2 half + {0, 1}
-  r.row1 >>= 6 * half;
+  r.row0 >>= 3 * u;  // sub-block of group 8S + 4c + t is 4S + 2c + u
+  r.row1 >>= 3 * u;
   const uint32_t dw = ptx::lds32(tb + 864 + 4 * q);
   r.d0 = __half2float(__ushort_as_half((unsigned short)(dw & 0xFFFFu)));
   r.d1 = __half2float(__ushort_as_half((unsigned short)(dw >> 16)));
   return r;
 }
 
-__device__ __forceinline__ void dequant_q1(const Q1Lane &L, int S, uint32_t A, int row0, uint32_t sel1,
-                                           int lane) {
-  const int q = lane >> 2, p = (lane >> 1) & 1, half = lane & 1;
+__device__ __forceinline__ void dequant_q1(const Q1Lane &L, int S, uint32_t sel1, uint32_t (&r)[16]) {
   const uint32_t qw = S == 0 ? L.qs[0] : S == 1 ? L.qs[1] : S == 2 ? L.qs[2] : L.qs[3];
   const uint32_t nb16 = S == 0 ? L.nb[0] : S == 1 ? L.nb[1] : S == 2 ? L.nb[2] : L.nb[3];
 #pragma unroll
-  for (int j = 0; j < 2; ++j) {
-    const int s2 = j;
-    const int sb = 4 * S + s2;  // sub-block 4 S + 2 half + s2, counted from the lane's first
+  for (int c2 = 0; c2 < 2; ++c2) {
+    const int sb = 4 * S + 2 * c2;  // sub-block, counted from the lane's first (u)
 #pragma unroll
     for (int h = 0; h < 2; ++h) {
-      const int f = 2 * s2 + h;
-      const uint32_t qsb = (qw >> (8 * f)) & 0xFFu;
-      const uint32_t nib = (nb16 >> (4 * f)) & 15u;
+      const uint32_t qsb = (qw >> (16 * c2 + 8 * h)) & 0xFFu;
+      const uint32_t nib = (nb16 >> (8 * c2 + 4 * h)) & 15u;
       const uint2 sel = ptx::lds64_const(sel1 + 8 * (qsb | ((nib & 7u) << 8)));
       const uint32_t sc3 = (uint32_t)(((h ? L.row1 : L.row0) >> (3 * sb)) & 7u);
       const float sc = (h ? L.d1 : L.d0) * odd_f(sc3);
@@ -283,7 +332,7 @@ __device__ __forceinline__ void dequant_q1(const Q1Lane &L, int S, uint32_t A, i
       v.y = __byte_perm(t0, t1, sel.x >> 16);
       v.z = __byte_perm(t0, t1, sel.y);
       v.w = __byte_perm(t0, t1, sel.y >> 16);
-      ptx::sts128(A + ptx::sw128_offset(row0 + q + 8 * h, 16 * (2 * half + s2) + 8 * p), v);
+      put_group(r, c2, h, v);
     }
   }
 }
@@ -330,6 +379,8 @@ __global__ void __maxnreg__(128) grouped_tc_kernel(TileArgs a) {
   TC_DECL;
   // per-role pipeline positions (they carry over between passes)
   uint32_t col = 0, step = 0, ucount = 0;
+  uint32_t acc_use[2] = {0u, 0u};  // MMA thread / epilogue: uses of each accumulator buffer so far
+  int acc_next = 0;
 
   for (int base = 0; base < my_total; base += kMaxUnits) {
     const int n_this = min(kMaxUnits, my_total - base);
@@ -368,14 +419,19 @@ __global__ void __maxnreg__(128) grouped_tc_kernel(TileArgs a) {
       if (lane == 0) {
         for (int u = 0; u < n_this; ++u, ++ucount) {
           const Unit U = S.units[u];
-          const int buf = ucount & 1;
+          const AccPlan P = acc_plan<DOWN>(U.n_pad, ucount, acc_next);
           {
             TC_T0();
-            if (ucount >= 2 && !ptx::mbar_wait_suspend(&B.accempty[buf], ((ucount >> 1) - 1) & 1u)) bad = true;
+#pragma unroll
+            for (int b = 0; b < 2; ++b)
+              if ((P.mask >> b) & 1) {
+                if (acc_use[b] >= 1 && !ptx::mbar_wait_suspend(&B.accempty[b], (acc_use[b] - 1) & 1u)) bad = true;
+                ++acc_use[b];
+              }
             TC_ADD(0);
           }
           ptx::tc_fence_after();
-          const uint32_t d = tmem + buf * C::kBufCols;
+          const uint32_t d = tmem + P.gate, du = tmem + P.up;
           const uint32_t idesc = ptx::idesc_bf16_f32(128, U.n_pad);
           const int nsteps = U.K / 64;
           for (int k = 0; k < nsteps; ++k, ++step) {
@@ -386,31 +442,31 @@ __global__ void __maxnreg__(128) grouped_tc_kernel(TileArgs a) {
               TC_ADD(1);
             }
             ptx::tc_fence_after();
-            const uint32_t a0 = ptx::smem_u32(S.ring + (size_t)as * C::kStep);
-            // descriptors of the step's tiles; 16 more inputs = 32 bytes = 2 in the start-address field
-            const uint64_t da = ptx::sdesc_k_sw128(a0), du = da + (kTile >> 4),
-                           db = ptx::sdesc_k_sw128(a0 + C::kMats * kTile);
-            if (k == 0) {
-              ptx::umma_bf16(d, da, db, idesc, false);
-              if (!DOWN) ptx::umma_bf16(d + 128, du, db, idesc, false);
-            } else {
-              ptx::umma_bf16_acc(d, da, db, idesc);
-              if (!DOWN) ptx::umma_bf16_acc(d + 128, du, db, idesc);
-            }
+            // A: the step's slot in TMEM (gate, then up 32 columns on); B:
+            // the step's shared-memory tile.  16 more inputs = 8 TMEM columns
+            // = 32 bytes = 2 in the descriptor's start-address field.
+            const uint32_t ag = tmem + kAccCols + (uint32_t)as * C::kSlotCols;
+            const uint64_t db = ptx::sdesc_k_sw128(ptx::smem_u32(S.ring + (size_t)as * C::kStep));
 #pragma unroll
-            for (int ks = 1; ks < 4; ++ks) {
-              ptx::umma_bf16_acc(d, da + 2 * ks, db + 2 * ks, idesc);
-              if (!DOWN) ptx::umma_bf16_acc(d + 128, du + 2 * ks, db + 2 * ks, idesc);
+            for (int ks = 0; ks < 4; ++ks) {
+              const bool acc = k > 0 || ks > 0;
+              ptx::umma_bf16_ts(d, ag + 8 * ks, db + 2 * ks, idesc, acc);
+              if (!DOWN) ptx::umma_bf16_ts(du, ag + 32 + 8 * ks, db + 2 * ks, idesc, acc);
             }
             ptx::umma_commit(&B.aempty[as]);  // the slot is free once these have read it
           }
-          ptx::umma_commit(&B.accfull[buf]);
+#pragma unroll
+          for (int b = 0; b < 2; ++b)
+            if ((P.mask >> b) & 1) ptx::umma_commit(&B.accfull[b]);
         }
       }
     } else if (warp < 2 + kDqWarps) {
-      // ---- dequant warps: A tiles (and this warp's 16 rows of B)
+      // ---- dequant warps: one tile-block of each matrix into TMEM, 16 rows of B
       const int w = warp - 2;
-      const int ll = ((lane & 7) << 2) | (lane >> 3);  // the layout lane this thread decodes
+      // the TMEM lanes this warp may write are 32 (warp % 4) .. + 31: its
+      // tile-block (16 rows of the unit's 128) lies in that quarter
+      const int tbi = 2 * (warp & 3) + (warp >= 6 ? 1 : 0);
+      const uint32_t tlane = tmem + ((uint32_t)(16 * tbi) << 16);
       const uint32_t sel2a = ptx::smem_u32(S.sel2), sel1a = ptx::smem_u32(S.sel1);
       for (int u = 0; u < n_this; ++u) {
         const Unit U = S.units[u];
@@ -427,7 +483,8 @@ __global__ void __maxnreg__(128) grouped_tc_kernel(TileArgs a) {
         }
         const int tbb = tile_block_bytes(U.qtype), nsteps = 4 * nkb;
         // B rows of local step n into ring slot `as`, as one cp.async group;
-        // issued a step ahead so the copies overlap the decode of the step before
+        // issued a step ahead so the copies overlap the decode of the step
+        // before.  Waiting for the slot's release also frees its A slot.
         auto fetch_b = [&](int n, uint32_t gstep) {
           const int as = gstep % C::kAr;
           {
@@ -436,7 +493,7 @@ __global__ void __maxnreg__(128) grouped_tc_kernel(TileArgs a) {
               bad = true;
             TC_ADD(1);
           }
-          uint8_t *bt = S.ring + (size_t)as * C::kStep + C::kMats * kTile;
+          uint8_t *bt = S.ring + (size_t)as * C::kStep;
           const int k0 = 64 * n + 8 * (lane & 7);
 #pragma unroll
           for (int i = 0; i < 4; ++i)
@@ -456,10 +513,10 @@ __global__ void __maxnreg__(128) grouped_tc_kernel(TileArgs a) {
           Q1Lane l1[C::kMats];
           if (U.qtype == kQ2) {
 #pragma unroll
-            for (int m = 0; m < C::kMats; ++m) l2[m] = load_q2(pk + (m * 8 + w) * tbb, ll);
+            for (int m = 0; m < C::kMats; ++m) l2[m] = load_q2(pk + (m * 8 + tbi) * tbb, lane);
           } else {
 #pragma unroll
-            for (int m = 0; m < C::kMats; ++m) l1[m] = load_q1(pk + (m * 8 + w) * tbb, ll);
+            for (int m = 0; m < C::kMats; ++m) l1[m] = load_q1(pk + (m * 8 + tbi) * tbb, lane);
           }
           __syncwarp();
           if (lane == 0) ptx::mbar_arrive(&B.pempty[ps]);
@@ -468,22 +525,28 @@ __global__ void __maxnreg__(128) grouped_tc_kernel(TileArgs a) {
             const int n = 4 * kb + s, as = step % C::kAr;
             const bool more = n + 1 < nsteps;
             if (more) fetch_b(n + 1, step + 1);
-            const uint32_t stg = ptx::smem_u32(S.ring) + as * C::kStep;
+            // the slot's previous MMAs are done (waited for when its B rows were fetched)
+            ptx::tc_fence_after();
+            const uint32_t at = tlane + kAccCols + (uint32_t)as * C::kSlotCols;
             TC_T0();
-            if (U.qtype == kQ2) {
 #pragma unroll
-              for (int m = 0; m < C::kMats; ++m) dequant_q2(l2[m], s, stg + m * kTile, 16 * w, sel2a, ll);
-            } else {
-#pragma unroll
-              for (int m = 0; m < C::kMats; ++m) dequant_q1(l1[m], s, stg + m * kTile, 16 * w, sel1a, ll);
+            for (int m = 0; m < C::kMats; ++m) {
+              uint32_t r[16];
+              if (U.qtype == kQ2)
+                dequant_q2(l2[m], s, sel2a, r);
+              else
+                dequant_q1(l1[m], s, sel1a, r);
+              ptx::tmem_st16x256_x4(at + 32 * m, r);
             }
             TC_ADD(2);
+            ptx::tmem_wait_st();
             // this step's B rows landed (the next step's may still be in flight)
             if (more)
               asm volatile("cp.async.wait_group 1;" ::: "memory");
             else
               asm volatile("cp.async.wait_group 0;" ::: "memory");
             ptx::fence_proxy_async_smem();  // generic-proxy writes -> the tensor cores
+            ptx::tc_fence_before();
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(&B.afull[as]);
           }
@@ -492,22 +555,59 @@ __global__ void __maxnreg__(128) grouped_tc_kernel(TileArgs a) {
     } else {
       // ---- epilogue: warp reads TMEM lanes 32 (warp % 4) .. + 31 (= tile rows)
       const int lq = warp & 3, row = 32 * lq + lane;
+      const bool vec_out = ((uintptr_t)a.out & 15) == 0;  // 4-wide vector adds need 16-byte rows
+      uint32_t ep_stage = 0;
       for (int u = 0; u < n_this; ++u, ++ucount) {
         const Unit U = S.units[u];
-        const int buf = ucount & 1;
+        const AccPlan P = acc_plan<DOWN>(U.n_pad, ucount, acc_next);
         {
           TC_T0();
-          if (!ptx::mbar_wait_suspend(&B.accfull[buf], (ucount >> 1) & 1u)) bad = true;
+#pragma unroll
+          for (int b = 0; b < 2; ++b)
+            if ((P.mask >> b) & 1) {
+              if (!ptx::mbar_wait_suspend(&B.accfull[b], acc_use[b] & 1u)) bad = true;
+              ++acc_use[b];
+            }
           TC_ADD(0);
         }
         ptx::tc_fence_after();
-        const uint32_t d = tmem + buf * C::kBufCols + ((uint32_t)(32 * lq) << 16);
+        const uint32_t lq16 = (uint32_t)(32 * lq) << 16;
+        const uint32_t d = tmem + P.gate + lq16, du = tmem + P.up + lq16;
         const int r = 128 * U.rt + row;
-        Pair pl = {0, 0.f};  // down: pair c0 - (c0 % 32) + lane of the unit, broadcast by shuffles
+        // h is stored in the contraction order of the down kernel's steps
+        const int rp = (r & ~63) | perm64(r & 63);
+        Pair pl = {0, 0.f};  // down, scalar path: pair c0 - (c0 % 32) + lane of the unit, broadcast by shuffles
+        // down, vector path: lane l holds the pair of column lq + 4 l (the
+        // columns this warp adds), read once per unit
+        Pair mine = {0, 0.f};
+        if (DOWN && vec_out && lq + 4 * lane < U.n_real) mine = pairs[U.p0 + lq + 4 * lane];
         for (int c0 = 0; c0 < U.n_pad; c0 += 16) {
           uint32_t d0[16];
           ptx::tmem_ld16(d + (uint32_t)c0, d0);
-          if (DOWN) {
+          if (DOWN && vec_out) {
+            // stage the 16 columns (tokens) x 128 rows, then warp lq adds
+            // columns lq, lq + 4, .. into out, lane j taking rows 4j..4j+3:
+            // one 4-wide vector add per lane, 512 contiguous bytes per column
+            float *T = S.stage + (ep_stage & 1) * 16 * 128;
+            ++ep_stage;
+            ptx::tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 16; ++i) T[i * 128 + row] = __uint_as_float(d0[i]);
+            asm volatile("bar.sync 1, %0;" ::"n"(32 * kEpWarps) : "memory");
+#pragma unroll
+            for (int k = 0; k < 4; ++k) {
+              const int i = lq + 4 * k, col = c0 + i;
+              const int tok = __shfl_sync(0xffffffffu, mine.token, (c0 >> 2) + k);
+              const float wgt = __shfl_sync(0xffffffffu, mine.weight, (c0 >> 2) + k);
+              if (col < U.n_real) {
+                const float4 v = *reinterpret_cast<const float4 *>(T + i * 128 + 4 * lane);
+                float *o = a.out + (size_t)tok * H + 128 * U.rt + 4 * lane;
+                asm volatile("red.global.add.v4.f32 [%0], {%1, %2, %3, %4};" ::"l"(o), "f"(wgt * v.x),
+                             "f"(wgt * v.y), "f"(wgt * v.z), "f"(wgt * v.w)
+                             : "memory");
+              }
+            }
+          } else if (DOWN) {
             if ((c0 & 31) == 0) {
               const int jl = c0 + lane;
               if (jl < U.n_real) pl = pairs[U.p0 + jl];
@@ -521,21 +621,34 @@ __global__ void __maxnreg__(128) grouped_tc_kernel(TileArgs a) {
               if (c0 + i < U.n_real) atomicAdd(a.out + (size_t)tok * H + r, wgt * __uint_as_float(d0[i]));
             }
           } else {
+            // h of 16 pairs x 128 rows staged as bf16 at the rows' permuted
+            // places, then written as 16-byte pieces (pair i, piece g)
             uint32_t d1[16];
-            ptx::tmem_ld16(d + 128 + (uint32_t)c0, d1);
+            ptx::tmem_ld16(du + (uint32_t)c0, d1);
+            __nv_bfloat16 *T = reinterpret_cast<__nv_bfloat16 *>(S.stage) + (ep_stage & 1) * 16 * 128;
+            ++ep_stage;
             ptx::tmem_wait_ld();
+            const int prow = rp - 128 * U.rt;
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              const int jj = c0 + i;
-              if (jj < U.n_real)
-                hbuf[(size_t)(U.p0 + jj) * a.max_ffn + r] =
-                    __float2bfloat16_rn(silu_mul(__uint_as_float(d0[i]), __uint_as_float(d1[i])));
+            for (int i = 0; i < 16; ++i)
+              T[i * 128 + prow] = __float2bfloat16_rn(silu_mul_fast(__uint_as_float(d0[i]), __uint_as_float(d1[i])));
+            asm volatile("bar.sync 1, %0;" ::"n"(32 * kEpWarps) : "memory");
+#pragma unroll
+            for (int k = 0; k < 2; ++k) {
+              const int e = 32 * lq + lane + 128 * k, i = e >> 4, g = e & 15;
+              if (c0 + i < U.n_real)
+                *reinterpret_cast<uint4 *>(hbuf + (size_t)(U.p0 + c0 + i) * a.max_ffn + 128 * U.rt + 8 * g) =
+                    *reinterpret_cast<const uint4 *>(T + i * 128 + 8 * g);
             }
           }
         }
         ptx::tc_fence_before();
         __syncwarp();
-        if (lane == 0) ptx::mbar_arrive(&B.accempty[buf]);
+        if (lane == 0) {
+#pragma unroll
+          for (int b = 0; b < 2; ++b)
+            if ((P.mask >> b) & 1) ptx::mbar_arrive(&B.accempty[b]);
+        }
       }
     }
   }
@@ -547,14 +660,19 @@ __global__ void __maxnreg__(128) grouped_tc_kernel(TileArgs a) {
   if (warp == 0) ptx::tmem_dealloc(tmem, kTmemCols);
 }
 
-// Activations to bf16 (round to nearest even), 8 per thread.
+// Activations to bf16 (round to nearest even), 8 per thread: inputs
+// 8i..8i+7 (group G = i mod 8 of a 64-input step) go to positions perm64,
+// two runs of four.
 __global__ void to_bf16_kernel(const float *__restrict__ x, __nv_bfloat16 *__restrict__ xb, int64_t n8) {
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= n8) return;
   const float4 v0 = __ldg(reinterpret_cast<const float4 *>(x) + 2 * i);
   const float4 v1 = __ldg(reinterpret_cast<const float4 *>(x) + 2 * i + 1);
-  reinterpret_cast<uint4 *>(xb)[i] =
-      make_uint4(bf16x2(v0.x, v0.y), bf16x2(v0.z, v0.w), bf16x2(v1.x, v1.y), bf16x2(v1.z, v1.w));
+  const int64_t base = (i >> 3) << 6;
+  const int g = (int)(i & 7);
+  const int p0 = perm64(8 * g), p1 = perm64(8 * g + 4);
+  *reinterpret_cast<uint2 *>(xb + base + p0) = make_uint2(bf16x2(v0.x, v0.y), bf16x2(v0.z, v0.w));
+  *reinterpret_cast<uint2 *>(xb + base + p1) = make_uint2(bf16x2(v1.x, v1.y), bf16x2(v1.z, v1.w));
 }
 
 }  // namespace
