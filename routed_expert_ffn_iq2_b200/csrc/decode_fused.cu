@@ -23,8 +23,14 @@
 //             load; a warp decodes its tile-block, writes its partial sums
 //             to the item's reduction slot and moves on; the item's reducer
 //             (warp item mod 16) adds the partials once all are in;
-//   barrier   one grid-wide counter between phase 1 and phase 2 (bounded
-//             wait).  Down tiles stream into the rings before it opens.
+//   slices    no grid barrier: the reducer of a gate/up item counts the
+//             16-row tiles of h it wrote per (token chunk, 256-input slice)
+//             with a release add; a warp about to decode a down tile-block
+//             waits (acquire, bounded) until its slice of h is complete and
+//             every CTA has initialised its part of out.  Down tiles stream
+//             into the rings meanwhile.  Two counter sets alternate between
+//             calls: a call zeroes the other set in its prologue, so the
+//             call's end needs no reset pass.
 //
 // Arithmetic: weights are decoded to exact signed int8 values (IQ2: +-8,
 // +-25, +-43; IQ1: 8*(grid + delta) in {+-1, +-7, +-9}) by two byte
@@ -198,14 +204,17 @@ __device__ __forceinline__ void arrive_release(int *counter) {
 }
 
 // Spin until *counter >= target; false (and the TIMEOUT status bit) if that
-// takes longer than kGridWaitNs.  One thread per CTA calls it.
+// takes longer than kGridWaitNs.  One thread per warp calls it; polls are
+// spaced by a short sleep (many warps may wait on a few counters).
 __device__ __noinline__ bool wait_count(const int *counter, int target, int32_t *status) {
+  if (ld_acquire(counter) >= target) return true;
   const uint64_t t_end = global_ns() + kGridWaitNs;
   while (ld_acquire(counter) < target) {
     if (global_ns() > t_end) {
       atomicOr(status, REDLITE_STATUS_TIMEOUT);
       return false;
     }
+    __nanosleep(64);
   }
   return true;  // the acquiring load orders what follows
 }
@@ -512,7 +521,7 @@ __global__ void __launch_bounds__(kCThreads, 1) decode_fused_kernel(FusedArgs a)
   off += sizeof(uint64_t) * kRedSlots;
   S.rfree = reinterpret_cast<uint64_t *>(smem + off);
   off += sizeof(uint64_t) * kRedSlots;
-  __shared__ int s_n_inst, s_n1, s_n2, s_bad, s_scan[33];
+  __shared__ int s_n_inst, s_n1, s_n2, s_bad, s_par, s_scan[33];
   __shared__ uint64_t s_lut_bar;
   TR_STAMP(0);
   // the next layer call may start its own table setup on SMs this grid frees
@@ -567,6 +576,7 @@ __global__ void __launch_bounds__(kCThreads, 1) decode_fused_kernel(FusedArgs a)
   // the call's own inputs may come from the previous kernel
   asm volatile("griddepcontrol.wait;" ::: "memory");
   TR_STAMP(7);
+
   int my_ids[2];
   float my_w[2];
   uint4 my_d[2][2];  // slot-table entry of each of this thread's pairs
@@ -786,17 +796,55 @@ __global__ void __launch_bounds__(kCThreads, 1) decode_fused_kernel(FusedArgs a)
   }
   TR_STAMP(16);
 
-  // ---- the item split: gate/up items evenly over the CTAs, down items in
-  // reverse CTA order (a CTA with one more gate/up item tends to get one
-  // fewer down item).  (The host keeps every CTA's list within kMaxItems;
-  // the clamps only guard the shared-memory list.)
-  auto split = [&](int &b1, int &my1, int &b2, int &my2) {
-    const unsigned uG = (unsigned)G, uN1 = (unsigned)s_n1, uN2 = (unsigned)s_n2;  // products < 2^31
-    b1 = (int)(cta * uN1 / uG);
-    my1 = min(kMaxItems, (int)((cta + 1) * uN1 / uG) - b1);
-    const int rc = G - 1 - cta;
-    b2 = (int)(rc * uN2 / uG);
-    my2 = min(kMaxItems - my1, (int)((rc + 1) * uN2 / uG) - b2);
+  // ---- the item split.  Gate/up items in contiguous ranges of N1 / G, the
+  // first N1 mod G CTAs taking one more (so the h slices that complete last
+  // are those of the first few experts).  Down items in time slots: first one
+  // each for the CTAs without an extra gate/up item, then one per CTA per
+  // round, in reverse item order, so the down items that need the late slices
+  // come last.  (The host keeps every CTA's list within kMaxItems; the clamps
+  // only guard the shared-memory list.)
+  struct Split {
+    int b1, my1, e1, first2, my2, b2;  // b2 >= 0: down items in one contiguous range
+  };
+  auto split = [&]() -> Split {
+    Split p;
+    const int N1 = s_n1, N2 = s_n2;
+    const int r1 = N1 / G;
+    p.e1 = N1 - r1 * G;
+    p.b1 = cta < p.e1 ? (r1 + 1) * cta : (r1 + 1) * p.e1 + r1 * (cta - p.e1);
+    p.my1 = min(r1 + (cta < p.e1), kMaxItems - 1);
+    if (N2 >= 4 * G) {
+      // many down items per CTA: contiguous ranges (consecutive items share
+      // an expert's h slices and weights), in reverse CTA order
+      const unsigned uG = (unsigned)G, uN2 = (unsigned)N2, rc = (unsigned)(G - 1 - cta);
+      p.b2 = (int)(rc * uN2 / uG);
+      p.my2 = (int)((rc + 1) * uN2 / uG) - p.b2;
+      p.first2 = -1;
+    } else {
+      p.b2 = -1;
+      p.first2 = (cta >= p.e1 && cta - p.e1 < N2) ? cta - p.e1 : -1;
+      const int base = G - p.e1 + cta;  // this CTA's first round-robin slot
+      p.my2 = (p.first2 >= 0) + (base < N2 ? (N2 - base + G - 1) / G : 0);
+    }
+    p.my2 = min(p.my2, kMaxItems - p.my1);
+    return p;
+  };
+  // the global index of list entry k (gate/up entries first)
+  auto item_index = [&](const Split &p, int k, int &phase) -> int {
+    if (k < p.my1) {
+      phase = 1;
+      return p.b1 + k;
+    }
+    phase = 2;
+    if (p.b2 >= 0) return p.b2 + (k - p.my1);
+    int k2 = k - p.my1, slot;
+    if (p.first2 >= 0 && k2 == 0) {
+      slot = p.first2;
+    } else {
+      if (p.first2 >= 0) --k2;
+      slot = G - p.e1 + cta + k2 * G;
+    }
+    return s_n2 - 1 - slot;
   };
   // warp wi's place in an item, packed: phase 1 (bits 0-3 tile offset,
   // 4-6 input block, 7 has a tile-block, 8 matrix: gate 0 / up 1); phase 2
@@ -862,12 +910,12 @@ __global__ void __launch_bounds__(kCThreads, 1) decode_fused_kernel(FusedArgs a)
     // every warp (the weights start streaming as soon as the routing is
     // known)
     __syncwarp();
-    int b1, my1, b2, my2;
-    split(b1, my1, b2, my2);
+    const Split sp = split();
+    const int my1 = sp.my1, my2 = sp.my2;
     const int n_inst = s_n_inst;
     for (int k = lane; k < my1 + my2; k += 32) {
-      const int phase = k < my1 ? 1 : 2;
-      const int j = phase == 1 ? b1 + k : b2 + (k - my1);
+      int phase;
+      const int j = item_index(sp, k, phase);
       int lo = 0, hi = n_inst - 1;  // last instance whose base <= j
       while (lo < hi) {
         const int mid = (lo + hi + 1) >> 1;
@@ -886,8 +934,24 @@ __global__ void __launch_bounds__(kCThreads, 1) decode_fused_kernel(FusedArgs a)
     }
     TR_STAMP(20);
   } else {
+    if (warp == 1) {
+      // this call's counter set (by the parity of the call count); the other
+      // one, used by the previous call, is zeroed here, spread over the
+      // grid's warps 1, for the next call
+      const int par = ctrl->epoch & 1;
+      int *other = reinterpret_cast<int *>(a.ws + a.L.slices) + (par ^ 1) * kSliceSetInts;
+      const int n_old = min(ctrl->slice_pairs[par ^ 1], kFusedMaxPairs + 64) * kSlicesPerPair;
+      for (int i = cta * 32 + lane; i < n_old; i += G * 32) other[i * kSliceStride] = 0;
+      if (lane == 0) {
+        s_par = par;
+        if (cta == 0) {
+          ctrl->out_ready[par ^ 1] = 0;
+          ctrl->slice_pairs[par] = npairs + (a.has_shared ? T : 0);
+        }
+      }
+    }
     // ---- the other warps zero this CTA's slice of out, or copy the
-    // residual into it (the down items add into it after the grid barrier;
+    // residual into it (the down items add into it once every CTA has;
     // out does not overlap the inputs)
     const unsigned total4 = (unsigned)(T * H / 4);
     const unsigned z0 = cta * total4 / (unsigned)G, z1 = (cta + 1) * total4 / (unsigned)G;
@@ -899,16 +963,23 @@ __global__ void __launch_bounds__(kCThreads, 1) decode_fused_kernel(FusedArgs a)
   uint64_t my_p2;
   warp_place(warp, my_p1, my_p2);
   __syncthreads();  // the item list and the replicated tables are visible
-  int b1, my1, b2, my2;
-  split(b1, my1, b2, my2);
-  const int my_items = my1 + my2;
+  const int par = s_par;
+  int *slices = reinterpret_cast<int *>(a.ws + a.L.slices) + par * kSliceSetInts;
+  // this CTA's slice of out is initialised
+  if (tid == 0) arrive_release(&ctrl->out_ready[par]);
+  const Split sp = split();
+  const int my1 = sp.my1, my_items = sp.my1 + sp.my2;
+  // slice counters, one per 128-byte line (many warps poll them)
+  auto slice_ctr = [&](int pair, int slice) { return slices + (pair * kSlicesPerPair + slice) * kSliceStride; };
+  bool out_ready = false;  // this warp has seen every CTA's part of out initialised
   TR_STAMP(1);
   TR_DECL;
 
   // The reducer of phase-1 item j (warp j mod 16) adds the item's partials
-  // once all warps have stored them and writes h = SiLU(g) * u for its rows.
-  // Reductions run kRedLag items late, so the reducer rarely waits for a
-  // slower warp; rj is the next item this warp considers.
+  // once all warps have stored them, writes h = SiLU(g) * u for its rows and
+  // counts them for their slice of h.  Reductions run kRedLag items late, so
+  // the reducer rarely waits for a slower warp; rj is the next item this warp
+  // considers.
   int rj = 0;
   auto reduce_until = [&](int upto) {
     for (; rj < upto; ++rj) {
@@ -935,7 +1006,15 @@ __global__ void __launch_bounds__(kCThreads, 1) decode_fused_kernel(FusedArgs a)
           __stcg(hbuf + (size_t)(pbase + pos) * a.max_ffn + tile * 16 + (lane >> 1), silu_mul(g, u));
       }
       __syncwarp();
-      if (lane == 0) mbar_arrive(&S.rfree[r]);
+      if (lane == 0) {
+        mbar_arrive(&S.rfree[r]);
+        // the item's tiles of h are written: count them for their 256-input
+        // slice (it1 divides 16, so they lie in one)
+        const int t0 = grp * it1, nt = min(it1, I.ffn / 16 - t0);
+        if (nt > 0)
+          asm volatile("red.release.gpu.global.add.s32 [%0], %1;" ::"l"(slice_ctr(pbase, t0 >> 4)), "r"(nt)
+                       : "memory");
+      }
       TR(9);
     }
   };
@@ -954,22 +1033,7 @@ __global__ void __launch_bounds__(kCThreads, 1) decode_fused_kernel(FusedArgs a)
   const int ncol = lane >> 2, cpos = ncol / 3;  // this lane's B column: limb ncol % 3 of position cpos
   const uint32_t bp = smem_u32(wl) + (uint32_t)((cpos * 3 + ncol % 3) * kWPlane);
   for (int k = 0; k <= my_items; ++k) {
-    if (k == my1) {
-      // grid barrier: every CTA has written its h rows and zeroed its slice
-      // of out (all of this CTA's phase-1 reductions are done once every
-      // warp has reduced its items below my1 and reached this point)
-      TR(0);
-      TR_STAMP(3);
-      all_sync();
-      TR_STAMP(4);
-      if (tid == 0) {
-        arrive_release(&ctrl->phase1_done);
-        wait_count(&ctrl->phase1_done, G, a.status);
-      }
-      all_sync();
-      TR_STAMP(5);
-      TR(1);
-    }
+    if (k == my1) TR_STAMP(3);
     if (k == my_items) break;
     const int s = k % kRing;
     const uint32_t w = S.items[k];
@@ -989,6 +1053,17 @@ __global__ void __launch_bounds__(kCThreads, 1) decode_fused_kernel(FusedArgs a)
                            (uint32_t)(ntok > 1 ? S.pair_tok[pbase + 1] + 1 : 0)
                      : (1ull << 63) | ((uint64_t)kb << 60) | ((uint64_t)(uint32_t)pbase << 30) | (uint32_t)ntok;
       if (key != lim_key) {
+        if (phase == 2) {
+          // this slice of h is complete (16 tiles), and out is initialised
+          // everywhere before the first down result is added into it
+          if (lane == 0) {
+            wait_count(slice_ctr(pbase, kb), 16, a.status);
+            if (!out_ready) wait_count(&ctrl->out_ready[par], G, a.status);
+          }
+          out_ready = true;
+          __syncwarp();
+          TR(1);
+        }
         // limbs of the item's token positions, this warp's 256 inputs
         lim_key = key;
         for (int j = 0; j < ntok; ++j) {
@@ -1071,18 +1146,13 @@ __global__ void __launch_bounds__(kCThreads, 1) decode_fused_kernel(FusedArgs a)
   TR_STAMP(22);
   TR_FLUSH();
   TR_STAMP(6);
-  // ---- exit: the last CTA resets the counters for the next call
-  __syncthreads();
+  // ---- exit: the last CTA closes the call (the next call starts only once
+  // this grid has completed, so plain stores do)
   TR_STAMP(23);
-  if (tid == 0) {
-    __threadfence();
-    const int prev = atomicAdd(&ctrl->exit_count, 1);
-    if (prev == G - 1) {
-      ctrl->phase1_done = 0;
-      ctrl->phase0_done = 0;
-      __threadfence();
-      ctrl->exit_count = 0;
-    }
+  __syncthreads();
+  if (tid == 0 && atomicAdd(&ctrl->exit_count, 1) == G - 1) {
+    ctrl->exit_count = 0;
+    ctrl->epoch = ctrl->epoch + 1;
   }
 }
 

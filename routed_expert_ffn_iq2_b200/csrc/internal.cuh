@@ -114,26 +114,38 @@ struct Ctrl {
   int n_active;        // entries in the active list (incl. shared)
   int n_pairs;         // pairs in the sorted list
   int ticket;          // next work ticket
-  int exit_count;      // CTAs that finished (the last one resets)
-  int phase1_done;     // CTAs past the gate/up items (fused decode kernel)
-  int phase0_done;     // CTAs past the activation-conversion phase
+  int exit_count;      // fused decode kernel: CTAs that finished (the last one closes the call)
+  int epoch;           // fused decode kernel: calls so far; its parity picks the counter set
+  int out_ready[2];    // per parity: CTAs that initialised their part of out
+  int slice_pairs[2];  // per parity: pairs whose slice counters that call used
   int n_gu_units;      // tensor-core path: gate/up work units
   int n_dn_units;      // tensor-core path: down work units
   int ticket_gu;       // next gate/up unit
   int ticket_dn;       // next down unit
-  int pad[54];
+  int pad[51];
 };
 static_assert(sizeof(Ctrl) == 256, "ctrl block is 256 bytes");
 
 struct WorkspaceLayout {
-  size_t ctrl, active, pairs, counts, hist, h, xb, gu, limbs, exps, total;
+  size_t ctrl, slices, active, pairs, counts, hist, h, xb, gu, total;
   int max_active, max_pairs;
 };
+
+// Fused decode kernel: h slices finished, per (first pair of a token chunk,
+// 256-input slice of the expert width): counts of 16-row tiles written.  Two
+// sets, picked by the parity of the call count: a call uses one and zeroes
+// the part of the other that the previous call used.  They persist between
+// calls, so they sit at a fixed offset, right after the control block,
+// whatever the call's shape.
+constexpr int kSlicesPerPair = 8;  // widths up to 2048
+constexpr int kSliceStride = 32;   // ints between counters: one 128-byte line each
 
 // Largest (token, slot) pair count the fused decode kernel takes.
 constexpr int kRouteBlocks = 32;  // bucketing: blocks that count and place pairs
 constexpr int kFusedMaxPairs = 640;
 constexpr int kFusedMaxInst = kFusedMaxPairs + 2;  // selected experts + the shared expert, rounded up
+constexpr int kSliceSetInts = (kFusedMaxPairs + 64) * kSlicesPerPair * kSliceStride;  // + shared pairs
+constexpr size_t kSliceBytes = sizeof(int) * 2 * (size_t)kSliceSetInts;
 
 inline size_t align256(size_t v) { return (v + 255) & ~size_t(255); }
 
@@ -145,6 +157,8 @@ inline WorkspaceLayout workspace_layout(int hidden, int n_experts, int max_token
   size_t off = 0;
   L.ctrl = off;
   off = align256(off + sizeof(Ctrl));
+  L.slices = off;  // fixed place (see kSliceBytes)
+  off = align256(off + kSliceBytes);
   L.active = off;
   off = align256(off + sizeof(ActiveEntry) * (size_t)L.max_active);
   L.pairs = off;
@@ -157,15 +171,11 @@ inline WorkspaceLayout workspace_layout(int hidden, int n_experts, int max_token
   off = align256(off + sizeof(float) * (size_t)L.max_pairs * (size_t)max_ffn);
   L.xb = off;  // tensor-core path: the call's activations as bf16 [tokens][hidden]
   off = align256(off + 2 * (size_t)max_tokens * (size_t)hidden);
-  // fused decode kernel: gate/up results per pair, activation limbs per token
+  // fused decode kernel: h per pair
   const int64_t ft = std::min<int64_t>(max_tokens, kFusedMaxPairs / (top_k > 0 ? top_k : 1));
   const int64_t fpairs = ft * top_k + ft;
   L.gu = off;
-  off = align256(off + sizeof(float) * (size_t)fpairs * 2 * (size_t)max_ffn);
-  L.limbs = off;
-  off = align256(off + (size_t)ft * 3 * (size_t)(hidden + 32));
-  L.exps = off;
-  off = align256(off + sizeof(int) * (size_t)(ft + 1));
+  off = align256(off + sizeof(float) * (size_t)fpairs * (size_t)max_ffn);
   L.total = off;
   return L;
 }

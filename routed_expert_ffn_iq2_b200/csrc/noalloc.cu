@@ -46,12 +46,10 @@ WorkspaceLayout noalloc_layout(int hidden, int n_tokens, int top_k, int max_ffn)
   size_t off = 0;
   L.ctrl = off;
   off = align256(off + sizeof(Ctrl));
+  L.slices = off;  // fixed place after the control block, as in the workspace layout
+  off = align256(off + kSliceBytes);
   L.gu = off;
-  off = align256(off + sizeof(float) * (size_t)pairs * 2 * (size_t)max_ffn);
-  L.limbs = off;
-  off = align256(off + (size_t)n_tokens * 3 * (size_t)(hidden + 32));
-  L.exps = off;
-  off = align256(off + sizeof(int) * (size_t)(n_tokens + 1));
+  off = align256(off + sizeof(float) * (size_t)pairs * (size_t)max_ffn);
   L.active = L.pairs = L.counts = L.hist = L.h = L.xb = off;
   L.total = off;
   L.max_pairs = (int)pairs;

@@ -147,7 +147,7 @@ def test_no_alloc_rejects_on_host(native):
     for sh, why in _shared_cases(native) + [(native.redlite_moe_expert(1, 128, 0x1000, 0x2000, 0x3000), "not tiled")]:
         rc = L.redlite_moe_layer_noalloc(p, 1, p, p, 10, ctypes.byref(t), ctypes.byref(sh), p)
         assert rc == native.REDLITE_EINVAL, (why, rc)
-    # 64 tokens x top-10 + shared at width 2048: 704 pairs x 2 x 2048 fp32 gate/up values > 4 MiB
+    # 64 tokens x top-10 + shared at width 2048: 704 pairs x 2048 fp32 h values > 4 MiB
     big = native.redlite_moe_table(2048, 512, 2048, 64, 2048, 0, 0x1000, 0x2000, 0x3000, 0, 0x4000, None)
     sh = native.redlite_moe_expert(1, 2048, 0x1000, 0x2000, 0x3000)
     assert L.redlite_moe_layer_noalloc(p, 64, p, p, 10, ctypes.byref(big), ctypes.byref(sh), p) == native.REDLITE_ENOMEM

@@ -377,7 +377,8 @@ def test_tensor_core_path_matches_bf16_operand_reference(P, oracle_lib):
 
 
 def test_grid_wait_gives_up_and_reports(P):
-    """A grid-wide wait that can never be met (the gate/up barrier counter is
+    """A grid-wide wait that can never be met (the count of CTAs that have
+    initialised their part of out, which every down warp waits for, is
     corrupted from the host) gives up after its time limit, sets
     REDLITE_STATUS_TIMEOUT, and leaves the context and the workspace usable:
     the next call returns the right result with a clean status."""
@@ -386,7 +387,7 @@ def test_grid_wait_gives_up_and_reports(P):
     ref = _run(L, w.x, w.ids, w.weights)
     assert L.read_status() == 0
     ctrl = L.workspace.view(torch.int32)
-    ctrl[4] = -(1 << 30)  # control word 4: CTAs past their gate/up items
+    ctrl[5] = ctrl[6] = -(1 << 30)  # control words 5, 6: CTAs that initialised their part of out (per call parity)
     torch.cuda.synchronize()
     _run(L, w.x, w.ids, w.weights)
     assert L.read_status() & P.REDLITE_STATUS_TIMEOUT

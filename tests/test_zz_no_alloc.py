@@ -69,7 +69,7 @@ def test_no_alloc_refusals_leave_out_untouched(P):
     ids = torch.from_numpy(w.ids).cuda()
     wt = torch.from_numpy(w.weights).cuda()
     out = torch.full_like(x, 3.5)
-    # declared max_ffn 2048: 704 pairs x 2 x 2048 fp32 gate/up values do not fit 4 MiB
+    # declared max_ffn 2048: 704 pairs x 2048 fp32 h values do not fit 4 MiB
     big = P.redlite_moe_table.from_buffer_copy(bytes(L.table))
     big.max_ffn = 2048
     rc = P.redlite_moe_layer_noalloc(x, x.shape[0], ids, wt, w.top_k, big, L.shared, out)
