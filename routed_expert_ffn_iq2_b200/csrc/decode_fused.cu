@@ -644,31 +644,44 @@ __global__ void __launch_bounds__(kCThreads, 1) decode_fused_kernel(FusedArgs a)
       const int e = inrange ? my_ids[0] : -1;
       const bool ok = e >= 0 && e < E;
       int bad = (inrange && !ok) ? REDLITE_STATUS_BAD_ID : 0;
-      const int key = ok ? e : 0x7fffffff;
-      int rank = 0;        // position of this pair in (expert, pair index) order
-      unsigned less = 0u;  // lanes whose expert id is smaller
+      const unsigned lt = (1u << lane) - 1u;
+      int n_inst, n_routed_pairs;
+      redlite_moe_expert d;
+      memcpy(reinterpret_cast<uint8_t *>(&d), &my_d[0][0], 16);
+      memcpy(reinterpret_cast<uint8_t *>(&d) + 16, &my_d[0][1], 16);
+      if (T == 1) {
+        // one token: every valid pair is its own instance, in pair order (a
+        // repeated id runs twice, each time with its own weight)
+        const unsigned okm = __ballot_sync(0xffffffffu, ok);
+        const int rank = __popc(okm & lt);
+        if (ok) {
+          S.pair_tok[rank] = 0;
+          S.pair_w[rank] = my_w[0];
+          set_inst(S.inst[rank], d, 1, rank, bad);
+        }
+        n_inst = n_routed_pairs = __popc(okm);
+      } else {
+        const int key = ok ? e : 0x7fffffff;
+        int rank = 0;        // position of this pair in (expert, pair index) order
+        unsigned less = 0u;  // lanes whose expert id is smaller
 #pragma unroll 4
-      for (int q = 0; q < 32; ++q) {
-        const int kq = __shfl_sync(0xffffffffu, key, q);
-        rank += (kq < key) || (kq == key && q < lane);
-        less |= (unsigned)(kq < key) << q;
+        for (int q = 0; q < 32; ++q) {
+          const int kq = __shfl_sync(0xffffffffu, key, q);
+          rank += (kq < key) || (kq == key && q < lane);
+          less |= (unsigned)(kq < key) << q;
+        }
+        const unsigned same = __match_any_sync(0xffffffffu, key);
+        const bool leader = ok && (same & lt) == 0;
+        const unsigned leaders = __ballot_sync(0xffffffffu, leader);
+        if (ok) {
+          S.pair_tok[rank] = lane / K;
+          S.pair_w[rank] = my_w[0];
+        }
+        if (leader) set_inst(S.inst[__popc(leaders & less)], d, __popc(same), rank, bad);
+        n_inst = __popc(leaders);
+        n_routed_pairs = __popc(__ballot_sync(0xffffffffu, ok));
       }
       TR_STAMP(17);
-      const unsigned same = __match_any_sync(0xffffffffu, key), lt = (1u << lane) - 1u;
-      const bool leader = ok && (same & lt) == 0;
-      const unsigned leaders = __ballot_sync(0xffffffffu, leader);
-      if (ok) {
-        S.pair_tok[rank] = lane / K;
-        S.pair_w[rank] = my_w[0];
-      }
-      if (leader) {
-        redlite_moe_expert d;
-        memcpy(reinterpret_cast<uint8_t *>(&d), &my_d[0][0], 16);
-        memcpy(reinterpret_cast<uint8_t *>(&d) + 16, &my_d[0][1], 16);
-        set_inst(S.inst[__popc(leaders & less)], d, __popc(same), rank, bad);
-      }
-      int n_inst = __popc(leaders);
-      const int n_routed_pairs = __popc(__ballot_sync(0xffffffffu, ok));
       if (a.has_shared) {
         if (lane == 0) set_inst(S.inst[n_inst], a.shared, T, n_routed_pairs, bad);
         if (lane < T) S.pair_tok[n_routed_pairs + lane] = lane, S.pair_w[n_routed_pairs + lane] = 1.f;
@@ -963,12 +976,12 @@ __global__ void __launch_bounds__(kCThreads, 1) decode_fused_kernel(FusedArgs a)
   uint64_t my_p2;
   warp_place(warp, my_p1, my_p2);
   __syncthreads();  // the item list and the replicated tables are visible
+  const Split sp = split();
+  const int my1 = sp.my1, my_items = sp.my1 + sp.my2;
   const int par = s_par;
   int *slices = reinterpret_cast<int *>(a.ws + a.L.slices) + par * kSliceSetInts;
   // this CTA's slice of out is initialised
   if (tid == 0) arrive_release(&ctrl->out_ready[par]);
-  const Split sp = split();
-  const int my1 = sp.my1, my_items = sp.my1 + sp.my2;
   // slice counters, one per 128-byte line (many warps poll them)
   auto slice_ctr = [&](int pair, int slice) { return slices + (pair * kSlicesPerPair + slice) * kSliceStride; };
   bool out_ready = false;  // this warp has seen every CTA's part of out initialised
