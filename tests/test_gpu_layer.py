@@ -418,3 +418,35 @@ def test_overstated_min_ffn_is_reported_not_read(P, T):
     got = _run(L, x, ids, wt)
     assert L.read_status() & P.REDLITE_STATUS_BAD_EXPERT
     assert np.all(got == 0.0)
+
+
+def test_alternating_call_shapes_share_one_workspace(P, oracle_lib):
+    """The fused kernel keeps completion counters in the workspace between
+    calls (at a fixed place, two sets alternating by call parity).  One
+    workspace serves a sequence of calls that change the token count, the
+    top-k, the shared expert and the path (fused decode for up to 640 pairs,
+    the tensor-core path above); every call matches the fp64 oracle."""
+    H, E, F, kmax, Tmax = 512, 32, 256, 6, 160
+    seed = 6060
+    g2, g1 = fixtures.make_grid(seed, 1), fixtures.make_grid(seed, 2)
+    G2, G1 = oracle_lib.expand_grid(1, g2), oracle_lib.expand_grid(2, g1)
+    experts = [fixtures.make_expert(seed, 1 + (e % 2), H, F, e) for e in range(E)]
+    shared = fixtures.make_expert(seed, 1, H, F, 999)
+    L = P.MoeLayer(H, E, F, Tmax, kmax, g2, g1, pool_bytes=(E + 2) * fixtures.expert_bytes(1, H, F) + 4096)
+    assert L.upload(list(range(E)), experts) == 0
+    assert L.set_shared(shared) == 0
+    shared_desc = L.shared
+    st = fixtures.Stream(seed, 7)
+    # (tokens, top-k, with shared expert): the fused path up to 640 pairs
+    # (kmax * Tmax = 960 > 640: the last shapes take the tensor-core path)
+    for T, k, sh in [(1, 6, False), (1, 5, False), (3, 6, True), (1, 6, True), (48, 6, False),
+                     (1, 2, False), (150, 6, True), (2, 6, False), (160, 6, False), (1, 6, False)]:
+        ids = st.randint(T * k, E).astype(np.int32).reshape(T, k)
+        wt = (0.1 + st.uniform(T * k)).astype(np.float32).reshape(T, k)
+        x = fixtures.make_x(seed + T + 10 * k, T, H)
+        L.shared = shared_desc if sh else None
+        got = _run(L, x, ids, wt)
+        ref = oracle_lib.moe_layer(x, ids, wt, experts, shared if sh else None, G2, G1)
+        assert L.read_status() == 0, (T, k, sh)
+        tol = TOL_BF16 if T * k > 640 else TOL_FP32
+        assert _rel_err(got, ref) <= tol, (T, k, sh, _rel_err(got, ref))
