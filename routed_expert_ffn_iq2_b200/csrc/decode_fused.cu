@@ -114,6 +114,36 @@ struct Smem {
   uint64_t *rfree;   // [kRedSlots]: the reducer is done with the slot
 };
 
+// Byte offsets of the shared-memory regions, each rounded up to 16 bytes
+// (bulk-copy destinations need 16, mbarriers 8).
+struct SmemPlan {
+  size_t sel2, sel1, ring, red, wlimbs, inst, items, pair_tok, pair_w, full, left, rfull, rfree, total;
+};
+__host__ __device__ constexpr size_t r16(size_t v) { return (v + 15) & ~(size_t)15; }
+__host__ __device__ constexpr SmemPlan smem_plan() {
+  SmemPlan p{};
+  size_t off = 0;
+  p.sel2 = off, off = r16(off + 512 * kRep2 * 4);
+  p.sel1 = off, off = r16(off + 4096 * kRep1 * 4);
+  p.ring = off, off = r16(off + (size_t)kCWarps * kRing * kStageBytes);
+  p.red = off, off = r16(off + sizeof(float) * kRedSlots * kCWarps * kRedFloats);
+  p.wlimbs = off, off = r16(off + (size_t)kCWarps * kTokChunk * 3 * kWPlane);
+  p.inst = off, off = r16(off + sizeof(Inst) * kFusedMaxInst);
+  p.items = off, off = r16(off + sizeof(uint32_t) * kMaxItems);
+  p.pair_tok = off, off = r16(off + sizeof(int) * (kFusedMaxPairs + 64));
+  p.pair_w = off, off = r16(off + sizeof(float) * (kFusedMaxPairs + 64));
+  p.full = off, off = r16(off + sizeof(uint64_t) * kRing);
+  p.left = off, off = r16(off + sizeof(int) * kRing);
+  p.rfull = off, off = r16(off + sizeof(uint64_t) * kRedSlots);
+  p.rfree = off, off = r16(off + sizeof(uint64_t) * kRedSlots);
+  p.total = off;
+  return p;
+}
+static_assert(smem_plan().total + 64 <= 227 * 1024, "shared memory of the fused kernel");
+static_assert(smem_plan().ring % 16 == 0 && smem_plan().full % 8 == 0 && smem_plan().rfull % 8 == 0 &&
+                  smem_plan().rfree % 8 == 0 && (kStageBytes % 16) == 0 && (kQ1TileBlock % 16) == 0,
+              "alignment of bulk-copy destinations and mbarriers");
+
 // ------------------------------------------------------------------ PTX wrappers
 
 __device__ __forceinline__ uint32_t smem_u32(const void *p) { return (uint32_t)__cvta_generic_to_shared(p); }
@@ -493,34 +523,21 @@ __global__ void __launch_bounds__(kCThreads, 1) decode_fused_kernel(FusedArgs a)
   float *hbuf = reinterpret_cast<float *>(a.ws + a.L.gu);  // h per pair: [pairs][max_ffn]
 
   // ---- shared memory carve
+  constexpr SmemPlan P = smem_plan();
   Smem S;
-  size_t off = 0;
-  S.sel2 = reinterpret_cast<uint32_t *>(smem + off);
-  off += 512 * kRep2 * 4;
-  S.sel1 = reinterpret_cast<uint32_t *>(smem + off);
-  off += 4096 * kRep1 * 4;
-  S.ring = smem + off;
-  off += (size_t)kCWarps * kRing * kStageBytes;
-  S.red = reinterpret_cast<float *>(smem + off);
-  off += sizeof(float) * kRedSlots * kCWarps * kRedFloats;
-  S.wlimbs = smem + off;
-  off += (size_t)kCWarps * kTokChunk * 3 * kWPlane;
-  S.inst = reinterpret_cast<Inst *>(smem + off);
-  off += sizeof(Inst) * kFusedMaxInst;
-  S.items = reinterpret_cast<uint32_t *>(smem + off);
-  off += sizeof(uint32_t) * kMaxItems;
-  S.pair_tok = reinterpret_cast<int *>(smem + off);
-  off += sizeof(int) * (kFusedMaxPairs + 64);
-  S.pair_w = reinterpret_cast<float *>(smem + off);
-  off += sizeof(float) * (kFusedMaxPairs + 64);
-  S.full = reinterpret_cast<uint64_t *>(smem + off);
-  off += sizeof(uint64_t) * kRing;
-  S.left = reinterpret_cast<int *>(smem + off);
-  off += sizeof(int) * kRing;
-  S.rfull = reinterpret_cast<uint64_t *>(smem + off);
-  off += sizeof(uint64_t) * kRedSlots;
-  S.rfree = reinterpret_cast<uint64_t *>(smem + off);
-  off += sizeof(uint64_t) * kRedSlots;
+  S.sel2 = reinterpret_cast<uint32_t *>(smem + P.sel2);
+  S.sel1 = reinterpret_cast<uint32_t *>(smem + P.sel1);
+  S.ring = smem + P.ring;
+  S.red = reinterpret_cast<float *>(smem + P.red);
+  S.wlimbs = smem + P.wlimbs;
+  S.inst = reinterpret_cast<Inst *>(smem + P.inst);
+  S.items = reinterpret_cast<uint32_t *>(smem + P.items);
+  S.pair_tok = reinterpret_cast<int *>(smem + P.pair_tok);
+  S.pair_w = reinterpret_cast<float *>(smem + P.pair_w);
+  S.full = reinterpret_cast<uint64_t *>(smem + P.full);
+  S.left = reinterpret_cast<int *>(smem + P.left);
+  S.rfull = reinterpret_cast<uint64_t *>(smem + P.rfull);
+  S.rfree = reinterpret_cast<uint64_t *>(smem + P.rfree);
   __shared__ int s_n_inst, s_n1, s_n2, s_bad, s_par, s_scan[33];
   __shared__ uint64_t s_lut_bar;
   TR_STAMP(0);
@@ -1169,17 +1186,7 @@ __global__ void __launch_bounds__(kCThreads, 1) decode_fused_kernel(FusedArgs a)
   }
 }
 
-size_t fused_smem_bytes(int hidden, int max_ffn) {
-  size_t off = 512 * kRep2 * 4 + 4096 * kRep1 * 4;
-  off += (size_t)kCWarps * kRing * kStageBytes;
-  off += sizeof(float) * kRedSlots * kCWarps * kRedFloats;
-  off += (size_t)kCWarps * kTokChunk * 3 * kWPlane;
-  off += sizeof(Inst) * kFusedMaxInst;
-  off += sizeof(uint32_t) * kMaxItems;
-  off += 2 * sizeof(int) * (kFusedMaxPairs + 64);
-  off += sizeof(uint64_t) * (kRing + 2 * kRedSlots) + sizeof(int) * kRing;
-  return off + 64;
-}
+size_t fused_smem_bytes(int hidden, int max_ffn) { return smem_plan().total + 64; }
 
 bool fused_supported(int hidden, int max_ffn, int n_tokens, int top_k, int n_experts, bool has_shared, int sms) {
   if (hidden % 256 || hidden > 2048 || max_ffn % 256 || max_ffn > 2048) return false;
