@@ -14,6 +14,7 @@
 // reads the row's bytes for those 256 inputs with coalesced loads; x is
 // read through L1 (every row reads the same x).
 #include "internal.cuh"
+#include "ptx.cuh"
 
 namespace redlite {
 
@@ -43,25 +44,47 @@ __device__ __forceinline__ void step_load(const uint8_t *row, int64_t s, int lan
   }
 }
 
-// The lane's 8 weights from the words of step_load.
+// Exact small integers as floats without a conversion instruction: byte i
+// of v, placed in the low mantissa byte of 2^23, minus 2^23 + bias (the
+// result is an exact integer in fp32).
+__device__ __forceinline__ float byte_f(uint32_t v, int i, float bias = 0.f) {
+  return __uint_as_float(__byte_perm(v, 0x4B000000u, 0x7650u | (uint32_t)i)) - (8388608.f + bias);
+}
+
+// This lane's partial dot product of one row over one 256-input step, with
+// the lane's 8 inputs xa, xb and their sum xs (the same for every row).
+// Q8_0-style: d * sum(q x); Q4_K-style: d sc sum(q x) - dmin m sum(x),
+// both per sub-block (the lane's 8 weights share one).  sh: the bit offset
+// of the lane's 6-bit scale in the 96-bit scale field (6 j, j = lane / 4).
 template <int QT>
-__device__ __forceinline__ void step_weights(const uint32_t wd[5], int lane, float w[8]) {
+__device__ __forceinline__ float step_dot(const uint32_t wd[5], int sh, float4 xa, float4 xb, float xs) {
   if constexpr (QT == 3) {
+    // signed int8 q as unsigned q + 128 (xor 0x80 per byte); byte_f removes
+    // the 128 again, so every q is exact before it multiplies x
+    const uint32_t u01 = __byte_perm(__byte_perm(wd[1], wd[2], 0x0040u), __byte_perm(wd[3], wd[4], 0x0040u), 0x5410u) ^
+                         0x80808080u;
+    const uint32_t u23 = __byte_perm(__byte_perm(wd[1], wd[2], 0x0051u), __byte_perm(wd[3], wd[4], 0x0051u), 0x5410u) ^
+                         0x80808080u;
+    // weights 2i (u01 byte i) and 2i+1 (u23 byte i)
+    float dot = byte_f(u01, 0, 128.f) * xa.x + byte_f(u23, 0, 128.f) * xa.y;
+    dot += byte_f(u01, 1, 128.f) * xa.z + byte_f(u23, 1, 128.f) * xa.w;
+    dot += byte_f(u01, 2, 128.f) * xb.x + byte_f(u23, 2, 128.f) * xb.y;
+    dot += byte_f(u01, 3, 128.f) * xb.z + byte_f(u23, 3, 128.f) * xb.w;
+    (void)xs;
     const float d = __half2float(__ushort_as_half((unsigned short)wd[0]));
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      w[2 * i] = d * (float)(int8_t)(wd[1 + i] & 0xFF);
-      w[2 * i + 1] = d * (float)(int8_t)((wd[1 + i] >> 8) & 0xFF);
-    }
+    return d * dot;
   } else {
-    const int j = lane >> 2;  // sub-block of inputs 8l..8l+7
-    const uint64_t lo = (uint64_t)wd[1] | ((uint64_t)wd[2] << 32), hi = (uint64_t)wd[2] | ((uint64_t)wd[3] << 32);
-    const int sc = (int)((lo >> (6 * j)) & 63u), mn = (int)((hi >> (16 + 6 * j)) & 63u);
+    const uint32_t lo = wd[4] & 0x0F0F0F0Fu, hi = (wd[4] >> 4) & 0x0F0F0F0Fu;  // weights 2i, 2i+1
+    float dot = byte_f(lo, 0) * xa.x + byte_f(hi, 0) * xa.y;
+    dot += byte_f(lo, 1) * xa.z + byte_f(hi, 1) * xa.w;
+    dot += byte_f(lo, 2) * xb.x + byte_f(hi, 2) * xb.y;
+    dot += byte_f(lo, 3) * xb.z + byte_f(hi, 3) * xb.w;
+    const uint64_t f = (uint64_t)wd[1] | ((uint64_t)wd[2] << 32);
+    const uint64_t g = (uint64_t)wd[2] | ((uint64_t)wd[3] << 32);
+    const int sc = (int)((f >> sh) & 63u), mn = (int)((g >> (16 + sh)) & 63u);
     const float d = __half2float(__ushort_as_half((unsigned short)(wd[0] & 0xFFFFu)));
     const float dmin = __half2float(__ushort_as_half((unsigned short)(wd[0] >> 16)));
-    const float av = d * (float)sc, bv = dmin * (float)mn;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) w[i] = av * (float)((wd[4] >> (4 * i)) & 15u) - bv;
+    return d * (float)sc * dot - dmin * (float)mn * xs;
   }
 }
 
@@ -78,6 +101,7 @@ __global__ void __launch_bounds__(32 * kGemvWarps) gemv_proj_kernel(const uint8_
   const int64_t r0 = (int64_t)blockIdx.x * kGemvRows;
   const int64_t steps = k / 256;
   const size_t row_bytes = QT == 3 ? (size_t)(k / 32) * 34 : (size_t)steps * 144;
+  const int sh = 6 * (lane >> 2);  // this lane's sub-block (Q4_K-style scale field offset)
   float acc[kGemvRows][NT];
 #pragma unroll
   for (int h = 0; h < kGemvRows; ++h)
@@ -102,22 +126,21 @@ __global__ void __launch_bounds__(32 * kGemvWarps) gemv_proj_kernel(const uint8_
       const int64_t s = s0 + (int64_t)u * kGemvWarps;
       if (s >= steps) break;
       float4 xa[NT], xb[NT];
+      float xs[NT];
 #pragma unroll
-      for (int t = 0; t < NT; ++t)
+      for (int t = 0; t < NT; ++t) {
+        xa[t] = xb[t] = make_float4(0.f, 0.f, 0.f, 0.f);
         if (t < ntok) {
           const float4 *xp = reinterpret_cast<const float4 *>(x + t * k + 256 * s + 8 * lane);
           xa[t] = __ldg(xp), xb[t] = __ldg(xp + 1);
         }
+        xs[t] = (xa[t].x + xa[t].y) + (xa[t].z + xa[t].w) + (xb[t].x + xb[t].y) + (xb[t].z + xb[t].w);
+      }
 #pragma unroll
-      for (int h = 0; h < kGemvRows; ++h) {
-        float w[8];
-        step_weights<QT>(wd[u][h], lane, w);
+      for (int h = 0; h < kGemvRows; ++h)
 #pragma unroll
         for (int t = 0; t < NT; ++t)
-          if (t < ntok)
-            acc[h][t] += w[0] * xa[t].x + w[1] * xa[t].y + w[2] * xa[t].z + w[3] * xa[t].w + w[4] * xb[t].x +
-                         w[5] * xb[t].y + w[6] * xb[t].z + w[7] * xb[t].w;
-      }
+          if (t < ntok) acc[h][t] += step_dot<QT>(wd[u][h], sh, xa[t], xb[t], xs[t]);
     }
   }
 #pragma unroll
@@ -140,9 +163,142 @@ __global__ void __launch_bounds__(32 * kGemvWarps) gemv_proj_kernel(const uint8_
   }
 }
 
+// The words of step_load for a row held in shared memory.
+template <int QT>
+__device__ __forceinline__ void step_load_smem(const uint8_t *row, int64_t s, int lane, uint32_t wd[5]) {
+  if constexpr (QT == 3) {
+    const uint8_t *blk = row + (8 * s + lane / 4) * 34;
+    const unsigned short *qv = reinterpret_cast<const unsigned short *>(blk + 2 + 8 * (lane & 3));
+    wd[0] = *reinterpret_cast<const unsigned short *>(blk);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) wd[1 + i] = qv[i];
+  } else {
+    const uint8_t *blk = row + s * 144;
+    const uint4 hd = *reinterpret_cast<const uint4 *>(blk);
+    wd[0] = hd.x, wd[1] = hd.y, wd[2] = hd.z, wd[3] = hd.w;
+    wd[4] = reinterpret_cast<const uint32_t *>(blk + 16)[lane];
+  }
+}
+
+constexpr int kGsStages = 4;                 // row groups in flight per CTA
+constexpr int kGsMaxStage = 24 * 1024;       // bytes of one row group (kGemvRows rows)
+
+// Streaming form for matrices whose rows are 16-byte aligned: a persistent
+// grid, each CTA walking row groups g = blockIdx.x, + gridDim.x, ...; a group
+// (kGemvRows consecutive rows, contiguous in memory) arrives in a 4-stage
+// shared-memory ring by one bulk copy, so every CTA keeps four groups of
+// HBM reads in flight.  The 8 warps split each group's 256-input steps as in
+// gemv_proj_kernel; one CTA barrier per group closes the reduction and frees
+// the stage.  A bulk copy that does not land within the wait bound leaves NaN
+// in that group's outputs.
+template <int QT, int NT>
+__global__ void __launch_bounds__(32 * kGemvWarps) gemv_stream_kernel(const uint8_t *__restrict__ W, int64_t rows,
+                                                                     int64_t k, const float *__restrict__ x,
+                                                                     int ntok, float *__restrict__ y,
+                                                                     int64_t row_bytes, int n_groups) {
+  extern __shared__ __align__(128) uint8_t ring[];
+  __shared__ uint64_t full[kGsStages];
+  __shared__ float red[2][kGemvWarps][kGemvRows][NT];
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int G = gridDim.x, c = blockIdx.x;
+  const int my_n = n_groups > c ? (n_groups - c + G - 1) / G : 0;
+  const int64_t steps = k / 256;
+  const size_t stage_bytes = (size_t)kGemvRows * row_bytes;
+  if (tid == 0) {
+    for (int i = 0; i < kGsStages; ++i) ptx::mbar_init(&full[i], 1);
+    ptx::mbar_fence_init();
+  }
+  __syncthreads();
+  auto issue = [&](int i) {
+    const int st = i % kGsStages;
+    const int64_t r0 = (int64_t)(c + (int64_t)i * G) * kGemvRows;
+    const uint32_t bytes = (uint32_t)(min((int64_t)kGemvRows, rows - r0) * row_bytes);
+    ptx::mbar_expect_tx(&full[st], bytes);
+    ptx::bulk_g2s(ring + st * stage_bytes, W + r0 * row_bytes, bytes, &full[st]);
+  };
+  if (tid == 0)
+    for (int i = 0; i < min(kGsStages, my_n); ++i) issue(i);
+  const int sh = 6 * (lane >> 2);  // this lane's sub-block (Q4_K-style scale field offset)
+  for (int i = 0; i < my_n; ++i) {
+    const int st = i % kGsStages;
+    const int64_t r0 = (int64_t)(c + (int64_t)i * G) * kGemvRows;
+    const bool landed = ptx::mbar_wait(&full[st], (uint32_t)((i / kGsStages) & 1));
+    const uint8_t *stage = ring + st * stage_bytes;
+    float acc[kGemvRows][NT];
+#pragma unroll
+    for (int h = 0; h < kGemvRows; ++h)
+#pragma unroll
+      for (int t = 0; t < NT; ++t) acc[h][t] = 0.f;
+    for (int64_t s = warp; s < steps; s += kGemvWarps) {
+      float4 xa[NT], xb[NT];
+      float xs[NT];
+#pragma unroll
+      for (int t = 0; t < NT; ++t) {
+        xa[t] = xb[t] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (t < ntok) {
+          const float4 *xp = reinterpret_cast<const float4 *>(x + t * k + 256 * s + 8 * lane);
+          xa[t] = __ldg(xp), xb[t] = __ldg(xp + 1);
+        }
+        xs[t] = (xa[t].x + xa[t].y) + (xa[t].z + xa[t].w) + (xb[t].x + xb[t].y) + (xb[t].z + xb[t].w);
+      }
+#pragma unroll
+      for (int h = 0; h < kGemvRows; ++h) {
+        if (r0 + h >= rows) break;
+        uint32_t wd[5];
+        step_load_smem<QT>(stage + h * row_bytes, s, lane, wd);
+#pragma unroll
+        for (int t = 0; t < NT; ++t)
+          if (t < ntok) acc[h][t] += step_dot<QT>(wd, sh, xa[t], xb[t], xs[t]);
+      }
+    }
+#pragma unroll
+    for (int h = 0; h < kGemvRows; ++h)
+#pragma unroll
+      for (int t = 0; t < NT; ++t) {
+        float v = acc[h][t];
+#pragma unroll
+        for (int o = 16; o; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+        if (lane == 0) red[i & 1][warp][h][t] = v;
+      }
+    __syncthreads();  // every warp is done with the stage and has stored its sums
+    if (tid == 0 && i + kGsStages < my_n) {
+      asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+      issue(i + kGsStages);
+    }
+    const int tr = tid / NT, tt = tid % NT;
+    if (tr < kGemvRows && tt < ntok && r0 + tr < rows) {
+      float v = 0.f;
+#pragma unroll
+      for (int w = 0; w < kGemvWarps; ++w) v += red[i & 1][w][tr][tt];
+      y[tt * rows + r0 + tr] = landed ? v : __int_as_float(0x7fc00000);
+    }
+  }
+}
+
+template <int QT, int NT>
+cudaError_t launch_stream(const uint8_t *W, int64_t rows, int64_t k, const float *x, int ntok, float *y,
+                          int64_t row_bytes, cudaStream_t s) {
+  const int n_groups = (int)((rows + kGemvRows - 1) / kGemvRows);
+  const size_t smem = (size_t)kGsStages * kGemvRows * row_bytes;
+  cudaError_t e = cudaFuncSetAttribute(gemv_stream_kernel<QT, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       (int)smem);
+  if (e != cudaSuccess) return e;
+  const int sms = device_sms();
+  const int grid = min(n_groups, 2 * (sms > 0 ? sms : 148));
+  gemv_stream_kernel<QT, NT><<<grid, 32 * kGemvWarps, smem, s>>>(W, rows, k, x, ntok, y, row_bytes, n_groups);
+  return cudaGetLastError();
+}
+
 template <int QT>
 cudaError_t launch_gemv(const uint8_t *W, int64_t rows, int64_t k, const float *x, int ntok, float *y,
                         cudaStream_t s) {
+  const int64_t row_bytes = QT == 3 ? (k / 32) * 34 : (k / 256) * 144;
+  if ((((uintptr_t)W) & 15) == 0 && row_bytes % 16 == 0 && kGemvRows * row_bytes <= kGsMaxStage) {
+    if (ntok <= 1) return launch_stream<QT, 1>(W, rows, k, x, ntok, y, row_bytes, s);
+    if (ntok <= 2) return launch_stream<QT, 2>(W, rows, k, x, ntok, y, row_bytes, s);
+    if (ntok <= 4) return launch_stream<QT, 4>(W, rows, k, x, ntok, y, row_bytes, s);
+    return launch_stream<QT, 8>(W, rows, k, x, ntok, y, row_bytes, s);
+  }
   const unsigned blocks = (unsigned)((rows + kGemvRows - 1) / kGemvRows);
   if (ntok <= 1)
     gemv_proj_kernel<QT, 1><<<blocks, 32 * kGemvWarps, 0, s>>>(W, rows, k, x, ntok, y);

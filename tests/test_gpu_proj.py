@@ -40,3 +40,23 @@ def test_proj_gemv_matches_oracle(P, oracle_lib, qtype, rows, k, T):
     got = y.cpu().numpy().astype(np.float64)
     ref = oracle_lib.gemv_proj(qtype, m, rows, k, x)
     assert np.abs(got - ref).max() <= 1e-5 * np.abs(ref).max()
+
+
+@pytest.mark.parametrize("qtype,rows,k,T,offset", [(3, 96, 2048, 2, 2), (3, 33, 512, 1, 6), (4, 40, 11008, 1, 0),
+                                                   (4, 9, 11008, 3, 0)])
+def test_proj_gemv_fallback_layouts(P, oracle_lib, qtype, rows, k, T, offset):
+    """Matrices the streaming kernel does not take: Q8_0-style at a 2-byte
+    (not 16-byte) aligned address, and Q4_K-style rows of more than 6 KB (a
+    4-row group above the 24 KB stage).  The per-CTA kernel serves them."""
+    m = fixtures.make_proj_matrix(900 + rows, qtype, rows, k)
+    buf = torch.zeros(m.size + 64, dtype=torch.uint8, device="cuda")
+    buf[offset:offset + m.size] = torch.from_numpy(m).cuda()
+    W = buf[offset:offset + m.size]
+    x = fixtures.make_x(901, T, k)
+    xd = torch.from_numpy(x).cuda()
+    y = torch.full((T, rows), float("nan"), dtype=torch.float32, device="cuda")
+    assert P.redlite_proj_gemv(qtype, W, rows, k, xd, T, y) == P.REDLITE_OK
+    torch.cuda.synchronize()
+    got = y.cpu().numpy().astype(np.float64)
+    ref = oracle_lib.gemv_proj(qtype, m, rows, k, x)
+    assert np.abs(got - ref).max() <= 1e-5 * np.abs(ref).max()
