@@ -569,10 +569,27 @@ def measure_components(dev):
     nbytes = pool.counters.bytes - c0[1]
     if PL.read_status() != 0:
         raise RuntimeError(f"pool: device status {PL.read_status()}")
+    # the link's own rate for reference: one 64 MB copy from pinned host memory, device-timed
+    hbig = torch.empty(64 << 20, dtype=torch.uint8).pin_memory()
+    dbig = torch.empty(64 << 20, dtype=torch.uint8, device=dev)
+    for _ in range(2):
+        dbig.copy_(hbig, non_blocking=True)
+    torch.cuda.synchronize()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record()
+    for _ in range(4):
+        dbig.copy_(hbig, non_blocking=True)
+    e1.record()
+    e1.synchronize()
+    peak = 4 * (64 << 20) / (e0.elapsed_time(e1) * 1e-3) / 1e9
+    del hbig, dbig
     res["pool"] = {"workload": "pool-cap24-e64-iq2xs-top10-t1, a fresh selection per call", "calls": n_calls,
                    "us_per_call": dt * 1e6 / n_calls, "loads": int(loads), "h2d_gbs": nbytes / dt / 1e9,
-                   "note": "host wall time of acquire + layer per call (fills from pinned host memory on a copy "
-                           "stream)"}
+                   "roofline": {"bound": "h2d", "achieved": nbytes / dt / 1e9, "peak": peak, "unit": "GB/s",
+                                "frac": nbytes / dt / 1e9 / peak,
+                                "peak_kind": "measured: one 64 MB pinned host-to-device copy"},
+                   "note": "host wall time of acquire + layer per call (fills from pinned host memory on the "
+                           "pool's copy streams)"}
     pool.close()
     del keep, L, PL
     torch.cuda.empty_cache()

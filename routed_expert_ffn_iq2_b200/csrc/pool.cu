@@ -10,10 +10,13 @@
 //
 // The policy is host code with no device dependence (redlite_moe_pool_plan,
 // testable without a GPU); redlite_moe_pool_acquire adds the data movement:
-// the misses' three matrices are copied host -> device on a copy stream into
-// their slots, the slot table is updated (an evicted expert's entry is
-// cleared first, so a stale id reports BAD_EXPERT instead of reading a
-// reused slot), and the compute stream waits for those copies.  Pinned
+// the misses' three matrices are copied host -> device into their slots, the
+// slot table is updated (an evicted expert's entry is cleared first, so a
+// stale id reports BAD_EXPERT instead of reading a reused slot), and the
+// compute stream waits for those copies.  The copies are spread over the
+// pool's own copy streams, forked from the caller's copy stream and joined
+// back into it, so several are in flight at once (a fill of one expert is
+// three transfers of ~0.3 MB, where per-copy overhead is a large share).  Pinned
 // slots are released when the caller says the work using them is done
 // (redlite_moe_pool_complete) or when a CUDA event recorded after that work
 // completes (redlite_moe_pool_release).
@@ -35,6 +38,12 @@ struct redlite_moe_pool {
     cudaEvent_t event;  // nullptr until released with an event
   };
   std::vector<Pending> pending;
+  // copy streams of this pool (created on the first fill) with the events
+  // that fork them from, and join them back into, the caller's copy stream
+  static constexpr int kStreams = 8;
+  cudaStream_t streams[kStreams] = {};
+  cudaEvent_t fork = nullptr, join[kStreams] = {};
+  bool streams_ok = false;
 };
 
 namespace {
@@ -60,6 +69,22 @@ void poll_events(redlite_moe_pool *p) {
   }
 }
 
+// Slot-table updates of one acquire, passed by value: entry id[i] of the
+// table becomes d[i] (an empty entry for an eviction).  One launch replaces
+// a small pageable host -> device copy per entry.
+constexpr int kMaxUpdates = 64;
+struct TableUpdates {
+  int32_t n;
+  int32_t id[kMaxUpdates];
+  redlite_moe_expert d[kMaxUpdates];
+};
+static_assert(sizeof(TableUpdates) <= 4096, "kernel parameters");
+
+__global__ void table_update_kernel(const TableUpdates u, redlite_moe_expert *table) {
+  const int i = threadIdx.x;
+  if (i < u.n) table[u.id[i]] = u.d[i];
+}
+
 }  // namespace
 
 extern "C" {
@@ -81,6 +106,11 @@ void redlite_moe_pool_destroy(redlite_moe_pool *p) {
   if (!p) return;
   for (auto &q : p->pending)
     if (q.event) cudaEventDestroy(q.event);
+  for (int i = 0; i < redlite_moe_pool::kStreams; ++i) {
+    if (p->streams[i]) cudaStreamDestroy(p->streams[i]);
+    if (p->join[i]) cudaEventDestroy(p->join[i]);
+  }
+  if (p->fork) cudaEventDestroy(p->fork);
   delete p;
 }
 
@@ -226,11 +256,40 @@ int redlite_moe_pool_acquire(redlite_moe_pool *p, const int32_t *ids, int32_t n,
   cudaStream_t cs = (cudaStream_t)copy_stream;
   int64_t loads = 0, hits = 0, evictions = 0, bytes = 0;
   static const redlite_moe_expert kEmpty = {0, 0, nullptr, nullptr, nullptr};
+  TableUpdates upd;
+  upd.n = 0;
+  // table entries are written after every fill has landed: evicted entries
+  // cleared, loaded entries set (flushed early if the batch is full)
+  auto flush = [&]() -> bool {
+    if (!upd.n) return true;
+    table_update_kernel<<<1, kMaxUpdates, 0, cs>>>(upd, table_dev);
+    upd.n = 0;
+    return cudaGetLastError() == cudaSuccess;
+  };
+  int n_miss = 0;
+  for (int i = 0; i < n; ++i) n_miss += miss[i] != 0;
+  constexpr int S = redlite_moe_pool::kStreams;
+  if (n_miss > 1 && !p->streams_ok) {
+    bool ok = cudaEventCreateWithFlags(&p->fork, cudaEventDisableTiming) == cudaSuccess;
+    for (int j = 0; ok && j < S; ++j)
+      ok = cudaStreamCreateWithFlags(&p->streams[j], cudaStreamNonBlocking) == cudaSuccess &&
+           cudaEventCreateWithFlags(&p->join[j], cudaEventDisableTiming) == cudaSuccess;
+    if (!ok) return REDLITE_ECUDA;
+    p->streams_ok = true;
+  }
+  // with several fills: fork the pool's streams from the caller's copy stream
+  const int n_used = n_miss > 1 ? (n_miss < S ? n_miss : S) : 0;
+  if (n_used) {
+    if (cudaEventRecord(p->fork, cs) != cudaSuccess) return REDLITE_ECUDA;
+    for (int j = 0; j < n_used; ++j)
+      if (cudaStreamWaitEvent(p->streams[j], p->fork, 0) != cudaSuccess) return REDLITE_ECUDA;
+  }
   for (int i = 0; i < n; ++i) {
     if (!miss[i]) {
       ++hits;
       continue;
     }
+    const cudaStream_t fs = n_used ? p->streams[loads % n_used] : cs;
     const redlite_moe_expert &h = host_experts[ids[i]];
     const size_t gb = matrix_bytes(h.qtype, h.ffn, hidden), db = matrix_bytes(h.qtype, hidden, h.ffn);
     const size_t ga = (gb + 15) & ~size_t(15);
@@ -238,17 +297,30 @@ int redlite_moe_pool_acquire(redlite_moe_pool *p, const int32_t *ids, int32_t n,
     redlite_moe_expert d{h.qtype, h.ffn, base, base + ga, base + 2 * ga};
     if (ev[i] >= 0) {
       ++evictions;
-      if (cudaMemcpyAsync(table_dev + ev[i], &kEmpty, sizeof kEmpty, cudaMemcpyHostToDevice, cs) != cudaSuccess)
-        return REDLITE_ECUDA;
+      upd.id[upd.n] = ev[i], upd.d[upd.n] = kEmpty, ++upd.n;
     }
-    if (cudaMemcpyAsync(base, h.gate, gb, cudaMemcpyHostToDevice, cs) != cudaSuccess ||
-        cudaMemcpyAsync(base + ga, h.up, gb, cudaMemcpyHostToDevice, cs) != cudaSuccess ||
-        cudaMemcpyAsync(base + 2 * ga, h.down, db, cudaMemcpyHostToDevice, cs) != cudaSuccess ||
-        cudaMemcpyAsync(table_dev + ids[i], &d, sizeof d, cudaMemcpyHostToDevice, cs) != cudaSuccess)
+    if (cudaMemcpyAsync(base, h.gate, gb, cudaMemcpyHostToDevice, fs) != cudaSuccess ||
+        cudaMemcpyAsync(base + ga, h.up, gb, cudaMemcpyHostToDevice, fs) != cudaSuccess ||
+        cudaMemcpyAsync(base + 2 * ga, h.down, db, cudaMemcpyHostToDevice, fs) != cudaSuccess)
       return REDLITE_ECUDA;
+    upd.id[upd.n] = ids[i], upd.d[upd.n] = d, ++upd.n;
     ++loads;
     bytes += (int64_t)(2 * gb + db);
+    if (upd.n > kMaxUpdates - 2) {
+      // a full batch: its entries' fills must land first
+      for (int j = 0; j < n_used; ++j)
+        if (cudaEventRecord(p->join[j], p->streams[j]) != cudaSuccess ||
+            cudaStreamWaitEvent(cs, p->join[j], 0) != cudaSuccess)
+          return REDLITE_ECUDA;
+      if (!flush()) return REDLITE_ECUDA;
+    }
   }
+  // join the pool's streams back into the caller's copy stream, then write
+  // the table entries
+  for (int j = 0; j < n_used; ++j)
+    if (cudaEventRecord(p->join[j], p->streams[j]) != cudaSuccess || cudaStreamWaitEvent(cs, p->join[j], 0) != cudaSuccess)
+      return REDLITE_ECUDA;
+  if (!flush()) return REDLITE_ECUDA;
   if (loads && copy_stream != compute_stream) {
     // the work enqueued next on the compute stream waits for the fills
     cudaEvent_t e;
