@@ -354,11 +354,14 @@ int32_t redlite_moe_pool_slot_of(const redlite_moe_pool *pool, int32_t expert);
 int32_t redlite_moe_pool_pins(const redlite_moe_pool *pool, int32_t slot);
 
 /* The policy step plus the data movement: for every miss the expert's three
- * matrices are copied host -> device on copy_stream into its slot
- * (slots_dev + slot * slot_bytes: gate, up at the gate size rounded up to 16
- * bytes, down after), and table_dev[id] is written; an evicted expert's
- * entry is cleared first (a stale id then reports BAD_EXPERT).  The work
- * enqueued next on compute_stream waits for these copies, so a layer call
+ * matrices are copied host -> device into its slot (slots_dev + slot *
+ * slot_bytes: gate, up at the gate size rounded up to 16 bytes, down after),
+ * then table_dev[id] is written and an evicted expert's entry cleared (a
+ * stale id then reports BAD_EXPERT).  The copies run on the pool's own copy
+ * streams (created on the current device at the first acquire with several
+ * misses), forked from copy_stream and joined back into it, so they are
+ * ordered after earlier work on copy_stream and before later work on it.
+ * The work enqueued next on compute_stream waits for them, so a layer call
  * may follow at once; copies for the next selection overlap the current
  * layer kernel when copy_stream differs from compute_stream.
  *   host_experts  host [n_experts]; gate/up/down are HOST pointers to the
