@@ -115,7 +115,8 @@ typedef struct {
   void *stream;                      /* cudaStream_t */
 } redlite_moe_table;
 
-/* Bytes of the expanded-grid buffer expand_grids writes. */
+/* Bytes of the expanded-grid buffer expand_grids writes.  (Library
+ * convenience: no counterpart on the pages.) */
 size_t redlite_moe_grids_bytes(void);
 
 /* Grid expansion ("Red Lite dev10", section "Quant grids"; done once before
@@ -128,14 +129,17 @@ size_t redlite_moe_grids_bytes(void);
 int redlite_moe_expand_grids(const uint16_t *iq2_compact, const uint16_t *iq1_compact, void *grids_dev,
                              void *stream);
 
-/* Packed bytes of a rows x k matrix, or 0 if the shape is not supported. */
+/* Packed bytes of a rows x k matrix, or 0 if the shape is not supported.
+ * (Library convenience: no counterpart on the pages.) */
 size_t redlite_moe_matrix_bytes(int32_t qtype, int64_t rows, int64_t k);
 
-/* Device scratch a layer call needs for these limits. */
+/* Device scratch a layer call needs for these limits.  (Library
+ * convenience: no counterpart on the pages.) */
 size_t redlite_moe_workspace_bytes(int32_t hidden, int32_t n_experts, int32_t max_tokens, int32_t top_k,
                                    int32_t max_ffn);
 
-/* Zero the workspace (table->workspace_bytes): its control words and
+/* (Library convenience: no counterpart on the pages.)
+ * Zero the workspace (table->workspace_bytes): its control words and
  * completion counters.  Call once after allocating it; layer calls leave it
  * ready for the next call, a call that reported REDLITE_STATUS_TIMEOUT
  * included.  Enqueued on table->stream. */
@@ -234,13 +238,14 @@ int redlite_moe_layer_noalloc(const float *x, int32_t n_tokens, const int32_t *e
                               const redlite_moe_expert *shared_expert, float *out);
 
 /* Host-side conversion of one matrix from the interchange layout to the
- * resident layout.  src, dst: host buffers of redlite_moe_matrix_bytes()
+ * resident layout (library convenience: the resident layout is this
+ * library's own; the pages keep the file's byte order).  src, dst: host buffers of redlite_moe_matrix_bytes()
  * bytes, not overlapping.  REDLITE_EUNSUPPORTED for shapes the kernels do
  * not take.  Pure host code: no device work. */
 int redlite_moe_pack_matrix(int32_t qtype, int64_t rows, int64_t k, const void *src, void *dst);
 
 /* Dequantise one matrix held in the resident layout (the bit-exactness
- * check of the decoders).  packed: device; out_f32: device [rows*k] fp32 or
+ * check of the decoders; library convenience, no counterpart on the pages).  packed: device; out_f32: device [rows*k] fp32 or
  * NULL; out_bf16: device [rows*k] bf16 bits (round to nearest even) or
  * NULL; outputs 16-byte aligned.  grids: expanded.  Enqueued on stream. */
 int redlite_moe_dequant(int32_t qtype, const void *packed, int64_t rows, int64_t k, const void *grids, float *out_f32,
