@@ -450,3 +450,28 @@ def test_alternating_call_shapes_share_one_workspace(P, oracle_lib):
         assert L.read_status() == 0, (T, k, sh)
         tol = TOL_BF16 if T * k > 640 else TOL_FP32
         assert _rel_err(got, ref) <= tol, (T, k, sh, _rel_err(got, ref))
+
+
+def test_tensor_core_path_odd_widths(P, oracle_lib):
+    """The tcgen05 path on hidden 768 (three 256-input columns per row tile)
+    with experts of widths 256, 512 and 768 in one call (down contractions of
+    4, 8 and 12 steps of 64 inputs; 2 to 6 row tiles of 128) and a shared
+    expert of width 512: 300 tokens x top-4 = 1200 pairs."""
+    H, E, k, T = 768, 12, 4, 300
+    seed = 7070
+    widths = [256, 512, 768]
+    g2, g1 = fixtures.make_grid(seed, 1), fixtures.make_grid(seed, 2)
+    experts = [fixtures.make_expert(seed, 1 + (e % 2), H, widths[e % 3], e) for e in range(E)]
+    shared = fixtures.make_expert(seed, 2, H, 512, 999)
+    L = P.MoeLayer(H, E, 768, T, k, g2, g1, pool_bytes=(E + 2) * fixtures.expert_bytes(1, H, 768) + 4096)
+    assert L.upload(list(range(E)), experts) == 0
+    assert L.set_shared(shared) == 0
+    st = fixtures.Stream(seed, 9)
+    ids = np.stack([st.randint(k, E) for _ in range(T)]).astype(np.int32)
+    wt = (0.1 + st.uniform(T * k)).astype(np.float32).reshape(T, k)
+    x = fixtures.make_x(seed, T, H)
+    got = _run(L, x, ids, wt)
+    ref = oracle_lib.moe_layer(x, ids, wt, experts, shared, oracle_lib.expand_grid(1, g2),
+                               oracle_lib.expand_grid(2, g1))
+    assert L.read_status() == 0
+    assert _rel_err(got, ref) <= TOL_BF16
