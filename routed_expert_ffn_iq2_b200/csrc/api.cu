@@ -102,6 +102,8 @@ int layer_impl(const float *x, int32_t n_tokens, const int32_t *expert_ids, cons
     fa.L = L;
     fa.status = t->status;
     fa.residual = residual;
+    fa.wide = fused_wide_items(t->hidden, n_tokens * top_k, t->min_ffn, t->max_ffn, shared != nullptr,
+                               shared ? shared->ffn : 0);
     return launch_fused(fa, s) == cudaSuccess ? REDLITE_OK : REDLITE_ECUDA;
   }
   const size_t out_bytes = sizeof(float) * (size_t)n_tokens * t->hidden;

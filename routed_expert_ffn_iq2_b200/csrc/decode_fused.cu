@@ -11,18 +11,20 @@
 //             memory, buckets the (token, slot) pairs by expert (stable,
 //             identical in every CTA), reads the selected slots'
 //             descriptors and converts the activations to fixed-point limbs;
-//   items     the work is a list of items of up to 16 tile-blocks (16 rows
-//             x 256 inputs of a packed matrix) for a chunk of <= 2 tokens:
+//   items     the work is a list of items of up to 16 warp units (a unit is
+//             one tile-block, 16 rows x 256 inputs of a packed matrix, or
+//             for large calls two adjacent ones) for a chunk of <= 2 tokens:
 //             phase 1 items are gate and up tiles of the same rows (their
 //             reduction yields h = SiLU(g) * u for those rows), phase 2
 //             items are groups of down tiles (their reduction is added to
 //             out with the router weight).  Items are split evenly over the
-//             CTAs; warp w of a CTA handles tile-block w of each item;
-//   streams   each warp streams its own tile-blocks by bulk copy into a
-//             private 4-stage ring, so warps do not wait for each other to
-//             load; a warp decodes its tile-block, writes its partial sums
-//             to the item's reduction slot and moves on; the item's reducer
-//             (warp item mod 16) adds the partials once all are in;
+//             CTAs; warp w of a CTA handles unit w of each item;
+//   streams   each warp streams its own units by bulk copy into a private
+//             ring (4 stages, 2 for two-block units), so warps do not wait
+//             for each other to load; a warp decodes its unit, writes its
+//             partial sums to the item's reduction slot and moves on; the
+//             item's reducer (warp item mod 16) adds the partials once all
+//             are in;
 //   slices    no grid barrier: the reducer of a gate/up item counts the
 //             16-row tiles of h it wrote per (token chunk, 256-input slice)
 //             with a release add; a warp about to decode a down tile-block
@@ -48,17 +50,27 @@ namespace redlite {
 
 constexpr int kCWarps = 16;                // warps per CTA (all consume)
 constexpr int kCThreads = 32 * kCWarps;    // 512
-constexpr int kRing = 4;                   // item stages in flight
-constexpr int kStageBytes = kQ2TileBlock;  // per warp and stage: 1184 >= kQ1TileBlock
+constexpr int kStageBytes = kQ2TileBlock;  // per tile-block slot of a stage: 1184 >= kQ1TileBlock
 constexpr int kLimbPadW = 32;              // padding per limb plane (spreads shared-memory banks)
 constexpr int kRedSlots = 6;               // reduction slots (items in flight)
 constexpr int kRedLag = 2;                 // an item is reduced this many items after its own
 constexpr int kMaxItems = 1536;            // items of one CTA (the host checks the bound)
 constexpr int kRedFloats = 32;             // per warp and item: 16 rows x 2 token positions
 constexpr int kTokChunk = 2;               // token positions per item
-constexpr int kWPlane = 256 + kLimbPadW;    // bytes per limb plane of a warp's input slice
-constexpr int kRep2 = 16;                  // replicas of the IQ2 selector table (bank spread)
-constexpr int kRep1 = 2;                   // replicas of the IQ1 selector table
+
+// Item shape.  W = 1: a warp decodes one tile-block per item (16 per item);
+// W = 2 (calls with many items): two consecutive tile-blocks of the same 16
+// rows (input blocks kb, kb + 1), accumulated together, so items, partial
+// sums and reductions per tile-block halve.  W = 2 makes its room in shared
+// memory with fewer selector-table replicas.
+template <int W>
+struct Shape {
+  static constexpr int kRing = W == 1 ? 4 : 2;          // item stages in flight
+  static constexpr int kStageTB = 16 * W;               // tile-block slots per stage
+  static constexpr int kWPlane = 256 * W + kLimbPadW;  // bytes per limb plane of a warp's inputs
+  static constexpr int kRep2 = W == 1 ? 16 : 8;         // replicas of the IQ2 selector table (bank spread)
+  static constexpr int kRep1 = W == 1 ? 2 : 1;          // replicas of the IQ1 selector table
+};
 constexpr uint32_t kSpinLimit = 1u << 24;
 
 // 8-byte tables the selector nibbles index: IQ2 +8,+25,+43,0,-8,-25,-43,0;
@@ -88,24 +100,13 @@ __device__ __forceinline__ int item_phase(uint32_t w) { return 1 + (int)(w >> 27
 constexpr uint64_t kIt2Tab = 0x0202020304050810ull;
 __device__ __forceinline__ int it2_of(int nkb) { return (int)((kIt2Tab >> (8 * (nkb - 1))) & 0xFFu); }
 
-// Tiles per item (phase 1: gate and up tiles of nkb = hidden / 256
-// tile-blocks each, 8 tile-blocks per matrix; phase 2: down tiles of nkb =
-// ffn / 256 tile-blocks, 16 per item) and item groups per token chunk.
-__device__ __forceinline__ int tiles_per_item(int nkb, int phase) {
-  return phase == 1 ? max(1, 8 / nkb) : max(1, 16 / nkb);
-}
-__device__ __forceinline__ int groups_of(int rows, int nkb, int phase) {
-  const int it = tiles_per_item(nkb, phase);
-  return (rows / 16 + it - 1) / it;
-}
-
 struct Smem {
   uint32_t *sel2, *sel1;
   uint32_t *items;  // [kMaxItems] this CTA's item list
-  uint8_t *ring;   // [kRing][kCWarps][kStageBytes]: stage s holds item k = s mod kRing
+  uint8_t *ring;   // [kRing][kStageTB][kStageBytes]: stage s holds item k = s mod kRing
   int *left;       // [kRing]: warps not yet done with the stage's item
   float *red;      // [kRedSlots][kCWarps][kRedFloats]
-  uint8_t *wlimbs;  // [kCWarps][2 positions][3 limbs][kWPlane]: each warp's input slice
+  uint8_t *wlimbs;  // [kCWarps][2 positions][3 limbs][kWPlane]: each warp's inputs
   Inst *inst;
   int *pair_tok;
   float *pair_w;
@@ -120,29 +121,36 @@ struct SmemPlan {
   size_t sel2, sel1, ring, red, wlimbs, inst, items, pair_tok, pair_w, full, left, rfull, rfree, total;
 };
 __host__ __device__ constexpr size_t r16(size_t v) { return (v + 15) & ~(size_t)15; }
+template <int W>
 __host__ __device__ constexpr SmemPlan smem_plan() {
+  using Sh = Shape<W>;
   SmemPlan p{};
   size_t off = 0;
-  p.sel2 = off, off = r16(off + 512 * kRep2 * 4);
-  p.sel1 = off, off = r16(off + 4096 * kRep1 * 4);
-  p.ring = off, off = r16(off + (size_t)kCWarps * kRing * kStageBytes);
+  p.sel2 = off, off = r16(off + 512 * Sh::kRep2 * 4);
+  p.sel1 = off, off = r16(off + 4096 * Sh::kRep1 * 4);
+  p.ring = off, off = r16(off + (size_t)Sh::kStageTB * Sh::kRing * kStageBytes);
   p.red = off, off = r16(off + sizeof(float) * kRedSlots * kCWarps * kRedFloats);
-  p.wlimbs = off, off = r16(off + (size_t)kCWarps * kTokChunk * 3 * kWPlane);
+  p.wlimbs = off, off = r16(off + (size_t)kCWarps * kTokChunk * 3 * Sh::kWPlane);
   p.inst = off, off = r16(off + sizeof(Inst) * kFusedMaxInst);
   p.items = off, off = r16(off + sizeof(uint32_t) * kMaxItems);
   p.pair_tok = off, off = r16(off + sizeof(int) * (kFusedMaxPairs + 64));
   p.pair_w = off, off = r16(off + sizeof(float) * (kFusedMaxPairs + 64));
-  p.full = off, off = r16(off + sizeof(uint64_t) * kRing);
-  p.left = off, off = r16(off + sizeof(int) * kRing);
+  p.full = off, off = r16(off + sizeof(uint64_t) * Sh::kRing);
+  p.left = off, off = r16(off + sizeof(int) * Sh::kRing);
   p.rfull = off, off = r16(off + sizeof(uint64_t) * kRedSlots);
   p.rfree = off, off = r16(off + sizeof(uint64_t) * kRedSlots);
   p.total = off;
   return p;
 }
-static_assert(smem_plan().total + 64 <= 227 * 1024, "shared memory of the fused kernel");
-static_assert(smem_plan().ring % 16 == 0 && smem_plan().full % 8 == 0 && smem_plan().rfull % 8 == 0 &&
-                  smem_plan().rfree % 8 == 0 && (kStageBytes % 16) == 0 && (kQ1TileBlock % 16) == 0,
-              "alignment of bulk-copy destinations and mbarriers");
+template <int W>
+constexpr bool plan_ok() {
+  constexpr SmemPlan p = smem_plan<W>();
+  return p.total + 64 <= 227 * 1024 && p.ring % 16 == 0 && p.full % 8 == 0 && p.rfull % 8 == 0 &&
+         p.rfree % 8 == 0 && p.wlimbs % 16 == 0 && (kStageBytes % 16) == 0 && (kQ1TileBlock % 16) == 0;
+}
+static_assert(plan_ok<1>() && plan_ok<2>(), "shared memory size and alignment of the fused kernel");
+// both shapes hold the same ring bytes (the bucketing scratch of large calls lives there)
+static_assert(Shape<1>::kRing * Shape<1>::kStageTB == Shape<2>::kRing * Shape<2>::kStageTB, "ring bytes");
 
 // ------------------------------------------------------------------ PTX wrappers
 
@@ -315,12 +323,15 @@ __device__ __forceinline__ void to_limbs(float v, float scale, int &l0, int &l1,
 // group: the 9-bit index (one byte extract, one bit), one table load for
 // the symbols' selector, the signs moved into bit 2 of each selector nibble
 // by one shift and one mask of the group's sign word, two byte permutes.
+template <int R2>
 __device__ __forceinline__ void tb_q2(uint32_t tb, uint32_t g2, uint32_t bp, bool bv, float acc[4]) {
+  static_assert(R2 == 16 || R2 == 8, "IQ2 table replicas");
+  constexpr int kSh = R2 == 16 ? 14 : 13;  // byte offset of index bit 8: 256 entries x 4 R2 bytes
   const int lane = threadIdx.x & 31, q = lane >> 2, t = lane & 3;
-  const uint32_t r4 = (uint32_t)(lane & 15) << 2;
+  const uint32_t r4 = (uint32_t)(lane & (R2 - 1)) << 2;
   const uint4 qs = lds_v4(tb + 32 * lane);
   const uint4 sg = lds_v4(tb + 32 * lane + 16);
-  const uint32_t qh14 = lds_b16(tb + 1024 + 2 * lane) << 14;
+  const uint32_t qhs = lds_b16(tb + 1024 + 2 * lane) << kSh;
   const uint2 scw = lds_v2(tb + 1088 + 8 * q);
   const uint32_t dw = lds_b32(tb + 1152 + 4 * q);
   uint2 b[8];
@@ -332,7 +343,7 @@ __device__ __forceinline__ void tb_q2(uint32_t tb, uint32_t g2, uint32_t bp, boo
 #pragma unroll
   for (int i = 0; i < 16; ++i) {
     const uint32_t qsb = __byte_perm(qsw[i >> 2], 0u, 0x4440u | (uint32_t)(i & 3));
-    const uint32_t go = qsb * 64u + (((qh14 >> i) & 0x4000u) | r4);  // index bit 8; 16 replicas
+    const uint32_t go = qsb * (4u * R2) + (((qhs >> i) & (1u << kSh)) | r4);  // index bit 8; R2 replicas
     const int m = i & 3;  // sign word i >> 2 holds this field's sign bit j at bit 4j + m
     const uint32_t sgn = (m <= 2 ? (sgw[i >> 2] << (2 - m)) : (sgw[i >> 2] >> 1)) & 0x44444444u;
     sel[i] = lds_table(g2 + go) | sgn;
@@ -367,8 +378,9 @@ __device__ __forceinline__ void tb_q2(uint32_t tb, uint32_t g2, uint32_t bp, boo
 
 // IQ1_M-style tile-block: one k16 mma per 16-weight sub-block; lane t holds
 // weights 4t..4t+3 of the sub-block (half of group 2s + (t >> 1)).
+template <int R1>
 __device__ __forceinline__ void tb_q1(uint32_t tb, uint32_t sel1, uint32_t bp, bool bv, float acc[4]) {
-  const int lane = threadIdx.x & 31, q = lane >> 2, t = lane & 3, r = lane & (kRep1 - 1);
+  const int lane = threadIdx.x & 31, q = lane >> 2, t = lane & 3, r = lane & (R1 - 1);
   const uint32_t pb = tb + 48 * (2 * q + (t >> 1));
   const uint4 qa = lds_v4(pb);
   const uint4 qb = lds_v4(pb + 16);
@@ -392,7 +404,7 @@ __device__ __forceinline__ void tb_q1(uint32_t tb, uint32_t sel1, uint32_t bp, b
       const int i = 2 * s + h;  // entry i = 2s + h
       const uint32_t qsb = (qsw[i >> 2] >> (8 * (i & 3))) & 0xFFu;
       const uint32_t nib = (nbw[i >> 3] >> (4 * (i & 7))) & 0xFu;
-      sel[h] = lds_table(sel1 + 4 * ((qsb | (nib << 8)) * kRep1 + r)) >> hshift;
+      sel[h] = lds_table(sel1 + 4 * ((qsb | (nib << 8)) * R1 + r)) >> hshift;
     }
     const uint32_t a0 = __byte_perm(kQ1Pos, kQ1Neg, sel[0]);
     const uint32_t a1 = __byte_perm(kQ1Pos, kQ1Neg, sel[1]);
@@ -444,27 +456,38 @@ __device__ __forceinline__ void store_partials(const float acc[4], float sc0, fl
   }
 }
 
-// Limbs of the 256 consecutive floats src[0..255] (the input slice of one
-// token position that a warp's tile-blocks read): three planes of 256
-// signed 7-bit limbs at dst, dst + kWPlane, dst + 2 kWPlane.  Returns the
-// slice's scale 2^(e - 20), 2^e > max |src[i]|.  Lane l converts inputs
-// 8l..8l+7.  coherent: read through L2 only (data other CTAs wrote during
-// this kernel).  Out of line: it runs once per token chunk.
+// Limbs of the 256 W consecutive floats src[0 .. 256 W - 1] (the inputs of
+// one token position that a warp's tile-blocks read): three planes of
+// 256 W signed 7-bit limbs at dst, dst + kWPlane, dst + 2 kWPlane, with one
+// scale for all of them.  Returns the scale 2^(e - 20), 2^e > max |src[i]|.
+// Lane l converts inputs 8 W l .. 8 W l + 8 W - 1.  coherent: read through
+// L2 only (data other CTAs wrote during this kernel).  Out of line: it runs
+// once per token chunk.
+template <int W>
 __device__ __noinline__ float warp_slice_limbs(const float *src, bool coherent, uint8_t *dst) {
+  constexpr int NV = 8 * W, kWPlane = Shape<W>::kWPlane;
   const int lane = threadIdx.x & 31;
-  const float4 *s4 = reinterpret_cast<const float4 *>(src) + 2 * lane;
-  const float4 v0 = coherent ? __ldcg(s4) : __ldg(s4), v1 = coherent ? __ldcg(s4 + 1) : __ldg(s4 + 1);
-  const float f[8] = {v0.x, v0.y, v0.z, v0.w, v1.x, v1.y, v1.z, v1.w};
+  const float4 *s4 = reinterpret_cast<const float4 *>(src) + (NV / 4) * lane;
+  float f[NV];
+#pragma unroll
+  for (int j = 0; j < NV / 4; ++j) {
+    const float4 v = coherent ? __ldcg(s4 + j) : __ldg(s4 + j);
+    f[4 * j] = v.x, f[4 * j + 1] = v.y, f[4 * j + 2] = v.z, f[4 * j + 3] = v.w;
+  }
   float m = 0.f;
 #pragma unroll
-  for (int i = 0; i < 8; ++i) m = fmaxf(m, fabsf(f[i]));
+  for (int i = 0; i < NV; ++i) m = fmaxf(m, fabsf(f[i]));
 #pragma unroll
   for (int o = 16; o; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
   const int e = pow2_above(m);
   const float sc = pow2f(20 - e);
-  uint32_t p[3][2] = {{0u, 0u}, {0u, 0u}, {0u, 0u}};
+  uint32_t p[3][NV / 4];
 #pragma unroll
-  for (int i = 0; i < 8; ++i) {
+  for (int l = 0; l < 3; ++l)
+#pragma unroll
+    for (int j = 0; j < NV / 4; ++j) p[l][j] = 0u;
+#pragma unroll
+  for (int i = 0; i < NV; ++i) {
     int l0, l1, l2;
     to_limbs(f[i], sc, l0, l1, l2);
     p[0][i >> 2] |= (uint32_t)(l0 & 0xFF) << (8 * (i & 3));
@@ -472,7 +495,12 @@ __device__ __noinline__ float warp_slice_limbs(const float *src, bool coherent, 
     p[2][i >> 2] |= (uint32_t)(l2 & 0xFF) << (8 * (i & 3));
   }
 #pragma unroll
-  for (int l = 0; l < 3; ++l) *reinterpret_cast<uint2 *>(dst + l * kWPlane + 8 * lane) = make_uint2(p[l][0], p[l][1]);
+  for (int l = 0; l < 3; ++l) {
+    if constexpr (W == 1)
+      *reinterpret_cast<uint2 *>(dst + l * kWPlane + 8 * lane) = make_uint2(p[l][0], p[l][1]);
+    else
+      *reinterpret_cast<uint4 *>(dst + l * kWPlane + 16 * lane) = make_uint4(p[l][0], p[l][1], p[l][2], p[l][3]);
+  }
   __syncwarp();
   return pow2f(e - 20);
 }
@@ -481,49 +509,55 @@ __device__ __noinline__ float warp_slice_limbs(const float *src, bool coherent, 
 // holds source word w / r; replicas spread lanes over banks): warps 1..15
 // (t = 0..479), named barrier 2.  Every source word is read before any is
 // overwritten.  Out of line: it runs once per call.
+template <int R2, int R1>
 __device__ __noinline__ void replicate_tables(uint32_t *sel2, uint32_t *sel1, int t) {
   constexpr int NT = 480, BAR = 2;
-  struct {
-    uint32_t *sel2, *sel1;
-  } S{sel2, sel1};
-  static_assert(kRep2 == 16 && kRep1 == 2, "replication below assumes 16 / 2 replicas");
-  constexpr int N2 = (512 + NT - 1) / NT, N1 = (4096 + NT - 1) / NT;
-  uint32_t v2[N2], v1[N1];
+  static_assert((R2 == 16 || R2 == 8) && (R1 == 2 || R1 == 1), "replication below assumes 16 or 8 / 2 or 1 replicas");
+  constexpr int N2 = (512 + NT - 1) / NT, N1 = R1 == 2 ? (4096 + NT - 1) / NT : 0;
+  uint32_t v2[N2], v1[N1 > 0 ? N1 : 1];
 #pragma unroll
-  for (int i = 0; i < N2; ++i) v2[i] = t + NT * i < 512 ? S.sel2[t + NT * i] : 0u;
+  for (int i = 0; i < N2; ++i) v2[i] = t + NT * i < 512 ? sel2[t + NT * i] : 0u;
 #pragma unroll
-  for (int i = 0; i < N1; ++i) v1[i] = t + NT * i < 4096 ? S.sel1[t + NT * i] : 0u;
+  for (int i = 0; i < N1; ++i) v1[i] = t + NT * i < 4096 ? sel1[t + NT * i] : 0u;
   asm volatile("bar.sync %0, %1;" ::"n"(BAR), "n"(NT) : "memory");
-  const int rot = (t & 31) >> 1;  // lanes of one store wavefront cover distinct banks
+  constexpr int Q = R2 / 4;  // 16-byte stores per entry
+  const int rot = (t & 31) / (8 / Q > 0 ? 8 / Q : 1);  // lanes of one store wavefront cover distinct banks
 #pragma unroll
-  for (int r = 0; r < 4; ++r) {
-    const int q = (r + rot) & 3;
+  for (int r = 0; r < Q; ++r) {
+    const int q = (r + rot) % Q;
 #pragma unroll
     for (int i = 0; i < N2; ++i)
       if (t + NT * i < 512)
-        reinterpret_cast<uint4 *>(S.sel2)[(t + NT * i) * 4 + q] = make_uint4(v2[i], v2[i], v2[i], v2[i]);
+        reinterpret_cast<uint4 *>(sel2)[(t + NT * i) * Q + q] = make_uint4(v2[i], v2[i], v2[i], v2[i]);
   }
+  if constexpr (R1 == 2) {
 #pragma unroll
-  for (int i = 0; i < N1; ++i)
-    if (t + NT * i < 4096) reinterpret_cast<uint2 *>(S.sel1)[t + NT * i] = make_uint2(v1[i], v1[i]);
+    for (int i = 0; i < N1; ++i)
+      if (t + NT * i < 4096) reinterpret_cast<uint2 *>(sel1)[t + NT * i] = make_uint2(v1[i], v1[i]);
+  }
   asm volatile("bar.sync %0, %1;" ::"n"(BAR), "n"(NT) : "memory");
 }
 
 // ------------------------------------------------------------------ the kernel
 
+template <int W>
 __global__ void __launch_bounds__(kCThreads, 1) decode_fused_kernel(FusedArgs a) {
+  using Sh = Shape<W>;
+  constexpr int kRing = Sh::kRing, kWPlane = Sh::kWPlane;
   extern __shared__ __align__(128) uint8_t smem[];
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = gridDim.x, cta = blockIdx.x;
   const int H = a.hidden, T = a.n_tokens, K = a.top_k, E = a.n_experts;
   const int nkbH = H >> 8;
-  const int it1 = max(1, 8 / nkbH);  // gate (and up) tiles per phase-1 item
+  // gate (and up) tiles per phase-1 item (W = 2 needs hidden 2048: two tiles
+  // of 8 input blocks, each warp two blocks of one tile)
+  const int it1 = W * max(1, 8 / nkbH);
   const int npairs = T * K;
   Ctrl *ctrl = reinterpret_cast<Ctrl *>(a.ws + a.L.ctrl);
   float *hbuf = reinterpret_cast<float *>(a.ws + a.L.gu);  // h per pair: [pairs][max_ffn]
 
   // ---- shared memory carve
-  constexpr SmemPlan P = smem_plan();
+  constexpr SmemPlan P = smem_plan<W>();
   Smem S;
   S.sel2 = reinterpret_cast<uint32_t *>(smem + P.sel2);
   S.sel1 = reinterpret_cast<uint32_t *>(smem + P.sel1);
@@ -623,7 +657,8 @@ __global__ void __launch_bounds__(kCThreads, 1) decode_fused_kernel(FusedArgs a)
       if (u < n_inst) {
         Inst &I = S.inst[u];
         const int nch = (I.count + kTokChunk - 1) / kTokChunk;
-        const int ng1 = (I.ffn / 16 + it1 - 1) / it1, it2 = it2_of(I.ffn >> 8), ng2 = (H / 16 + it2 - 1) / it2;
+        const int it2 = W == 1 ? it2_of(I.ffn >> 8) : 32 / (I.ffn >> 8);  // down tiles per item
+        const int ng1 = (I.ffn / 16 + it1 - 1) / it1, ng2 = (H / 16 + it2 - 1) / it2;
         I.ng1 = (int16_t)ng1, I.ng2 = (int16_t)ng2;
         c1 = nch * ng1;
         c2 = nch * ng2;
@@ -644,7 +679,8 @@ __global__ void __launch_bounds__(kCThreads, 1) decode_fused_kernel(FusedArgs a)
     }
   };
   auto set_inst = [&](Inst &I, const redlite_moe_expert &d, int count, int pair_start, int &bad) {
-    if (expert_ok(d, H, a.max_ffn, true)) {
+    // (the W = 2 item shape pairs down input blocks: widths a multiple of 512)
+    if (expert_ok(d, H, a.max_ffn, true) && (W == 1 || d.ffn % 512 == 0)) {
       I.gate = (const uint8_t *)d.gate, I.up = (const uint8_t *)d.up, I.down = (const uint8_t *)d.down;
       I.qtype = (int16_t)d.qtype, I.ffn = (int16_t)d.ffn, I.count = count;
     } else {
@@ -714,7 +750,7 @@ __global__ void __launch_bounds__(kCThreads, 1) decode_fused_kernel(FusedArgs a)
       // meanwhile the other warps replicate the selector tables
       mbar_wait(&s_lut_bar, 0, a.status);
       if (warp == 1) TR_STAMP(10);
-      replicate_tables(S.sel2, S.sel1, tid - 32);
+      replicate_tables<Sh::kRep2, Sh::kRep1>(S.sel2, S.sel1, tid - 32);
       if (warp == 1) TR_STAMP(11);
     }
   } else {
@@ -821,7 +857,7 @@ __global__ void __launch_bounds__(kCThreads, 1) decode_fused_kernel(FusedArgs a)
     // not touched)
     if (warp > 0) {
       mbar_wait(&s_lut_bar, 0, a.status);
-      replicate_tables(S.sel2, S.sel1, tid - 32);
+      replicate_tables<Sh::kRep2, Sh::kRep1>(S.sel2, S.sel1, tid - 32);
     }
   }
   TR_STAMP(16);
@@ -895,6 +931,24 @@ __global__ void __launch_bounds__(kCThreads, 1) decode_fused_kernel(FusedArgs a)
   auto tile_of = [&](uint32_t p1, uint64_t p2, uint32_t w, const uint8_t *&src, int &kb, int &tile) -> uint32_t {
     const Inst &I = S.inst[item_inst(w)];
     const int tbb = tile_block_bytes(I.qtype);
+    if constexpr (W == 2) {
+      // phase 1: warp = matrix (bit 3), tile of the item (bit 2), input
+      // blocks 2 (warp & 3) and + 1; phase 2: nkb / 2 warps per down tile,
+      // each two consecutive input blocks
+      if (item_phase(w) == 1) {
+        tile = item_grp(w) * 2 + ((warp >> 2) & 1);
+        kb = 2 * (warp & 3);
+        if (tile >= I.ffn / 16) return 0;
+        src = ((warp >> 3) ? I.up : I.gate) + (size_t)(tile * nkbH + kb) * tbb;
+      } else {
+        const int nkb = I.ffn >> 8, half = nkb >> 1;
+        tile = item_grp(w) * (32 / nkb) + warp / half;
+        kb = 2 * (warp % half);
+        if (tile >= H / 16) return 0;
+        src = I.down + (size_t)(tile * nkb + kb) * tbb;
+      }
+      return (uint32_t)tbb;
+    }
     if (item_phase(w) == 1) {
       tile = item_grp(w) * it1 + (int)(p1 & 15u);
       kb = (int)((p1 >> 4) & 7u);
@@ -918,16 +972,16 @@ __global__ void __launch_bounds__(kCThreads, 1) decode_fused_kernel(FusedArgs a)
     const uint32_t w = S.items[k];
     const Inst &I = S.inst[item_inst(w)];
     const int tbb = tile_block_bytes(I.qtype);
-    uint8_t *dst = S.ring + (size_t)s * kCWarps * kStageBytes;
+    uint8_t *dst = S.ring + (size_t)s * Sh::kStageTB * kStageBytes;
     if (item_phase(w) == 1) {
       const int t0 = item_grp(w) * it1, nt = min(it1, I.ffn / 16 - t0);
       const uint32_t bytes = (uint32_t)(nt * nkbH * tbb);
       const size_t off0 = (size_t)t0 * nkbH * tbb;
       mbar_expect_tx(&S.full[s], 2 * bytes);
       bulk_g2s(dst, I.gate + off0, bytes, &S.full[s]);
-      bulk_g2s(dst + 8 * kStageBytes, I.up + off0, bytes, &S.full[s]);
+      bulk_g2s(dst + 8 * W * kStageBytes, I.up + off0, bytes, &S.full[s]);
     } else {
-      const int nkb = I.ffn >> 8, it = it2_of(nkb);
+      const int nkb = I.ffn >> 8, it = W == 1 ? it2_of(nkb) : 32 / nkb;
       const int t0 = item_grp(w) * it, nt = min(it, H / 16 - t0);
       const uint32_t bytes = (uint32_t)(nt * nkb * tbb);
       mbar_expect_tx(&S.full[s], bytes);
@@ -1028,9 +1082,10 @@ __global__ void __launch_bounds__(kCThreads, 1) decode_fused_kernel(FusedArgs a)
         const int tile = grp * it1 + ti;
         if (tile >= I.ffn / 16) break;
         float g = 0.f, u = 0.f;
-        for (int kb = 0; kb < nkbH; ++kb) {
-          g += red[(ti * nkbH + kb) * kRedFloats + lane];
-          u += red[(8 + ti * nkbH + kb) * kRedFloats + lane];
+        // the warps of tile ti: ti * (nkbH / W) + j (gate), 8 + that (up)
+        for (int j = 0; j < nkbH / W; ++j) {
+          g += red[(ti * (nkbH / W) + j) * kRedFloats + lane];
+          u += red[(8 + ti * (nkbH / W) + j) * kRedFloats + lane];
         }
         if (pos < ntok)
           __stcg(hbuf + (size_t)(pbase + pos) * a.max_ffn + tile * 16 + (lane >> 1), silu_mul(g, u));
@@ -1088,6 +1143,7 @@ __global__ void __launch_bounds__(kCThreads, 1) decode_fused_kernel(FusedArgs a)
           // everywhere before the first down result is added into it
           if (lane == 0) {
             wait_count(slice_ctr(pbase, kb), 16, a.status);
+            if (W == 2) wait_count(slice_ctr(pbase, kb + 1), 16, a.status);
             if (!out_ready) wait_count(&ctrl->out_ready[par], G, a.status);
           }
           out_ready = true;
@@ -1099,7 +1155,7 @@ __global__ void __launch_bounds__(kCThreads, 1) decode_fused_kernel(FusedArgs a)
         for (int j = 0; j < ntok; ++j) {
           const float *x = phase == 1 ? a.x + (size_t)S.pair_tok[pbase + j] * H + 256 * kb
                                       : hbuf + (size_t)(pbase + j) * a.max_ffn + 256 * kb;
-          const float scj = warp_slice_limbs(x, phase == 2, wl + j * 3 * kWPlane);
+          const float scj = warp_slice_limbs<W>(x, phase == 2, wl + j * 3 * kWPlane);
           if (j == 0) sc0 = scj; else sc1 = scj;
         }
         TR(2);
@@ -1117,12 +1173,23 @@ __global__ void __launch_bounds__(kCThreads, 1) decode_fused_kernel(FusedArgs a)
       // part from slot 8; phase 2: down tiles from slot 0), tile-blocks at
       // their own size
       const int tbb = tile_block_bytes(I.qtype);
-      const uint32_t tb = smem_u32(S.ring + (size_t)s * kCWarps * kStageBytes) +
-                          (uint32_t)(phase == 1 ? (warp >> 3) * 8 * kStageBytes + (warp & 7) * tbb : warp * tbb);
-      if (I.qtype == kQ2)
-        tb_q2(tb, g2, bp, bv, acc);
-      else
-        tb_q1(tb, g1, bp, bv, acc);
+      uint32_t slot;  // this warp's first tile-block in the stage, in tile-blocks
+      if constexpr (W == 1) {
+        slot = phase == 1 ? (uint32_t)(warp & 7) : (uint32_t)warp;
+      } else {
+        const int nkb = I.ffn >> 8;
+        slot = phase == 1 ? (uint32_t)(((warp >> 2) & 1) * 8 + 2 * (warp & 3))
+                          : (uint32_t)((warp / (nkb >> 1)) * nkb + 2 * (warp % (nkb >> 1)));
+      }
+      const uint32_t tb = smem_u32(S.ring + (size_t)s * Sh::kStageTB * kStageBytes) +
+                          (uint32_t)(phase == 1 ? (warp >> 3) * 8 * W * kStageBytes : 0) + slot * (uint32_t)tbb;
+#pragma unroll
+      for (int b = 0; b < W; ++b) {  // (W = 2: input blocks kb and kb + 1, limbs 256 bytes on)
+        if (I.qtype == kQ2)
+          tb_q2<Sh::kRep2>(tb + b * tbb, g2, bp + 256 * b, bv, acc);
+        else
+          tb_q1<Sh::kRep1>(tb + b * tbb, g1, bp + 256 * b, bv, acc);
+      }
       if (warp == 0 && k == 0) TR_STAMP(13);
       if (warp == 0 && k == my1) TR_STAMP(15);
       TR(4);
@@ -1186,7 +1253,7 @@ __global__ void __launch_bounds__(kCThreads, 1) decode_fused_kernel(FusedArgs a)
   }
 }
 
-size_t fused_smem_bytes(int hidden, int max_ffn) { return smem_plan().total + 64; }
+size_t fused_smem_bytes(int w) { return (w == 2 ? smem_plan<2>().total : smem_plan<1>().total) + 64; }
 
 bool fused_supported(int hidden, int max_ffn, int n_tokens, int top_k, int n_experts, bool has_shared, int sms) {
   if (hidden % 256 || hidden > 2048 || max_ffn % 256 || max_ffn > 2048) return false;
@@ -1206,8 +1273,10 @@ bool fused_supported(int hidden, int max_ffn, int n_tokens, int top_k, int n_exp
     if ((n1 + g - 1) / g + (n2 + g - 1) / g > kMaxItems) return false;
   }
   // bucketing scratch (slot-table entries, counts, first pairs, ids, weights) lives in the rings
-  if ((size_t)n_experts * 8 + 40 * (size_t)kFusedMaxPairs > (size_t)kCWarps * kRing * kStageBytes) return false;
-  return fused_smem_bytes(hidden, max_ffn) <= 227 * 1024;
+  if ((size_t)n_experts * 8 + 40 * (size_t)kFusedMaxPairs >
+      (size_t)Shape<1>::kStageTB * Shape<1>::kRing * kStageBytes)
+    return false;
+  return true;  // both item shapes fit shared memory (checked at compile time)
 }
 
 int device_sms() {
@@ -1217,12 +1286,15 @@ int device_sms() {
   return sms;
 }
 
-cudaError_t launch_fused(const FusedArgs &a, cudaStream_t stream) {
-  const int sms = device_sms();
-  if (sms <= 0) return cudaErrorNoDevice;
-  cudaError_t e;
-  const size_t smem = fused_smem_bytes(a.hidden, a.max_ffn);
-  e = cudaFuncSetAttribute(decode_fused_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+bool fused_wide_items(int hidden, int n_pairs, int min_ffn, int max_ffn, bool has_shared, int shared_ffn) {
+  return hidden == 2048 && n_pairs > 32 && min_ffn == max_ffn && max_ffn % 512 == 0 &&
+         (!has_shared || shared_ffn % 512 == 0);
+}
+
+template <int W>
+static cudaError_t launch_shape(const FusedArgs &a, cudaStream_t stream, int sms) {
+  const size_t smem = fused_smem_bytes(W);
+  cudaError_t e = cudaFuncSetAttribute(decode_fused_kernel<W>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
   if (e != cudaSuccess) return e;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(sms);
@@ -1237,17 +1309,23 @@ cudaError_t launch_fused(const FusedArgs &a, cudaStream_t stream) {
   cfg.attrs = attr;
   static bool pdl_ok = true;  // dependent launch lets a call's table setup overlap the previous call
   cfg.numAttrs = pdl_ok ? 2 : 1;
-  e = cudaLaunchKernelEx(&cfg, decode_fused_kernel, a);
+  e = cudaLaunchKernelEx(&cfg, decode_fused_kernel<W>, a);
   if (e != cudaSuccess && pdl_ok) {
     (void)cudaGetLastError();
     pdl_ok = false;
     cfg.numAttrs = 1;
-    e = cudaLaunchKernelEx(&cfg, decode_fused_kernel, a);
+    e = cudaLaunchKernelEx(&cfg, decode_fused_kernel<W>, a);
   }
 #ifdef REDLITE_DEBUG_LAUNCH
   if (e != cudaSuccess) fprintf(stderr, "decode_fused_kernel launch: %s\n", cudaGetErrorString(e));
 #endif
   return e;
+}
+
+cudaError_t launch_fused(const FusedArgs &a, cudaStream_t stream) {
+  const int sms = device_sms();
+  if (sms <= 0) return cudaErrorNoDevice;
+  return a.wide ? launch_shape<2>(a, stream, sms) : launch_shape<1>(a, stream, sms);
 }
 
 }  // namespace redlite

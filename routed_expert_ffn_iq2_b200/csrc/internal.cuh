@@ -324,7 +324,12 @@ struct FusedArgs {
   uint8_t *ws;
   WorkspaceLayout L;
   int32_t *status;
+  int wide;  // item shape: 0 one tile-block per warp and item, 1 two (fused_wide_items)
 };
+// Whether a fused call uses items of two tile-blocks per warp: hidden 2048,
+// more than 32 (token, slot) pairs, one expert width, a multiple of 512
+// (the kernel reports an expert of another width as BAD_EXPERT).
+bool fused_wide_items(int hidden, int n_pairs, int min_ffn, int max_ffn, bool has_shared, int shared_ffn);
 // Whether the fused decode kernel takes a call; sms: the device's SM count
 // (0 if unknown: a B200's 148 is assumed).
 bool fused_supported(int hidden, int max_ffn, int n_tokens, int top_k, int n_experts, bool has_shared, int sms);

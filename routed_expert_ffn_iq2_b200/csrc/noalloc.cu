@@ -100,5 +100,7 @@ extern "C" int redlite_moe_layer_noalloc(const float *x, int32_t n_tokens, const
   fa.ws = scratch;
   fa.L = L;
   fa.status = t->status;
+  fa.wide = fused_wide_items(t->hidden, n_tokens * top_k, t->min_ffn, t->max_ffn, shared != nullptr,
+                             shared ? shared->ffn : 0);
   return launch_fused(fa, s) == cudaSuccess ? REDLITE_OK : REDLITE_ECUDA;
 }

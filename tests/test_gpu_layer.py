@@ -239,6 +239,24 @@ def test_batched_token_counts(P, oracle_lib, T):
     assert _rel_err(got, ref) <= TOL_FP32
 
 
+@pytest.mark.parametrize("T,k", [(8, 4), (11, 3)])
+def test_batched_item_shape_boundary(P, oracle_lib, T, k):
+    """32 (token, slot) pairs run items of one tile-block per warp, 33 pairs
+    items of two; both against the oracle on the mixed-format workload with
+    the shared expert (the first k slots of each token's routing)."""
+    w = fixtures.workload(4, n_tokens=T)
+    L = layer_for_workload(w)
+    ids, wt = np.ascontiguousarray(w.ids[:, :k]), np.ascontiguousarray(w.weights[:, :k])
+    got = _run(L, w.x, ids, wt)
+    experts = [None] * w.n_experts
+    for e in w.selected():
+        experts[e] = w.expert(e)
+    ref = oracle_lib.moe_layer(w.x, ids, wt, experts, w.shared(), oracle_lib.expand_grid(1, w.grid_iq2),
+                               oracle_lib.expand_grid(2, w.grid_iq1))
+    assert L.read_status() == 0
+    assert _rel_err(got, ref) <= TOL_FP32
+
+
 def test_general_path_agrees_with_fast_path(P):
     w = fixtures.workload(4, n_tokens=9)
     L = layer_for_workload(w)
