@@ -22,20 +22,21 @@
 //   warp 1      one thread issues the tcgen05.mma of every 64-input step and
 //               commits them to the step's slot and, per unit, to an
 //               accumulator buffer (one for gate/up, two for down);
-//   warps 2-9   dequant warps: each decodes one tile-block (16 rows) of each
-//               matrix, in the TMEM lane quarter its warp index may write,
-//               into the A slots of a 4-step ring in tensor memory
-//               (tcgen05.st), and fetches 16 rows of B with cp.async into the
-//               matching shared-memory slot, a step ahead;
+//   warps 2-9   dequant warps, two per TMEM lane quarter: thread i of a warp
+//               whose lane quarter is qd owns row 32 qd + i of the unit's 128
+//               rows (TMEM lane 32 qd + i) and writes, per step and matrix,
+//               its 64 consecutive weights into 32 consecutive columns of the
+//               step's A slot (tcgen05.st 32x32b).  Half kh of the quarter's
+//               two warps takes steps 2 kh and 2 kh + 1 of every 256-input
+//               column; the four warps of a half also fetch the 128 B rows of
+//               their steps with cp.async into the step's shared-memory slot;
 //   warps 10-13 the epilogue (TMEM -> registers -> h or out).
 //
-// Input order inside a 64-input step.  A thread of the 16-lane TMEM store
-// holds four consecutive K positions of its two rows per 16-position chunk,
-// and decodes 8-weight groups t and t + 4 of the step (t = lane % 4).  So
-// TMEM position 32 c + 16 j + 4 t + i holds input 32 c + 8 t + 4 j + i of
-// the step (c, j in {0, 1}, i < 4), and the bf16 copies of x and of h that
-// B is loaded from are stored in that same order (perm64): the contraction
-// over a step is a sum over all 64 inputs either way.
+// A and B hold every step's 64 inputs in input order: TMEM column c of an A
+// slot holds inputs 2c and 2c + 1 of its row, and a B row is the 64 inputs
+// of the step as 128 contiguous bytes (before the hardware swizzle).
+#include <type_traits>
+
 #include "internal.cuh"
 #include "layout.cuh"
 #include "ptx.cuh"
@@ -109,12 +110,6 @@ __device__ __forceinline__ AccPlan acc_plan(int n_pad, uint32_t ucount, int &nex
   return p;
 }
 
-// Position of input `in` of a 64-input step in the order the tensor-core
-// kernels contract over (see the header): bit 2 moves to bit 4, bits 3-4 to bits 2-3.
-__host__ __device__ __forceinline__ int perm64(int in) {
-  return (in & ~31) | ((in & 4) << 2) | ((in & 24) >> 1) | (in & 3);
-}
-
 struct Unit {
   const uint8_t *mat0, *mat1;  // gate, up (or down, unused)
   int qtype, K, rt, p0, n_real, n_pad, pad0, pad1;
@@ -138,7 +133,7 @@ constexpr int kEpStage = 2 * 16 * 128;  // epilogue: two 16-column x 128-row sta
 
 template <bool DOWN>
 constexpr size_t smem_bytes() {
-  return 1024 + (size_t)Cfg<DOWN>::kAr * Cfg<DOWN>::kStep + (size_t)kPr * Cfg<DOWN>::kPacked + 512 * 8 + 2048 * 8 +
+  return 1024 + (size_t)Cfg<DOWN>::kAr * Cfg<DOWN>::kStep + (size_t)kPr * Cfg<DOWN>::kPacked + 512 * 8 + 4096 * 8 +
          sizeof(Unit) * kMaxUnits + sizeof(Bars) + 16 + sizeof(float) * kEpStage;
 }
 
@@ -153,7 +148,7 @@ __device__ __forceinline__ Smem carve(uint8_t *smem) {
   S.sel2 = reinterpret_cast<const uint2 *>(p);
   p += 512 * 8;
   S.sel1 = reinterpret_cast<const uint2 *>(p);
-  p += 2048 * 8;
+  p += 4096 * 8;
   S.units = reinterpret_cast<Unit *>(p);
   p += sizeof(Unit) * kMaxUnits;
   S.bars = reinterpret_cast<Bars *>(p);
@@ -189,9 +184,6 @@ __device__ Unit make_unit(const TileArgs &a, const ActiveEntry *act, int n_activ
   return u;
 }
 
-// (float)(2 n + 1) for 0 <= n < 2^22, exactly, without a conversion instruction.
-__device__ __forceinline__ float odd_f(uint32_t n) { return __uint_as_float(0x4B000001u + 2 * n) - 8388608.f; }
-
 __device__ __forceinline__ uint32_t bf16x2(float lo, float hi) {
   uint32_t r;
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
@@ -204,135 +196,136 @@ __device__ __forceinline__ void cp_async16(void *dst, const void *src) {
 
 // --------------------------------------------------------------- dequant
 //
-// A lane builds the bf16 values of one (row, sub-block) as a table of three
-// entries (the scaled grid values of symbols 0, 1, 2) in two registers; the
-// byte-permute selectors of the weights' grid entry then pick a bf16 pair
-// per instruction.  IQ2_XS-style signs are flipped with one XOR per pair.
-// Lane (q, t) decodes rows q and q+8 of its tile-block, groups t and t + 4
-// of each 64-input step, into the sixteen registers of one 16-lane TMEM
-// store: group 4 c + t fills repetitions 2c (weights 0-3) and 2c+1
-// (weights 4-7), row q in registers 0-1 of a repetition, row q+8 in 2-3.
+// A thread decodes the weights of one row: per 16-weight (IQ1_M-style) or
+// 32-weight (IQ2_XS-style) sub-block it builds the bf16 values the row's
+// grid symbols can take, scaled by d and the sub-scale, in two registers;
+// the byte-permute selectors of a grid entry then pick one bf16 pair per
+// instruction.  Every value is exact in fp32 before its one rounding to bf16
+// (nearest even), so it equals redlite_moe_dequant's bf16 output.
+//
+// Row 32 qd + i of a unit lies in tile-block 2 qd + (i >> 4) of each column,
+// at row rr = i & 15 of it (q = rr & 7, hh = rr >> 3 in the tiled layout).
+// Half kh of a lane quarter reads the fields of its two steps (inputs 128 kh
+// .. 128 kh + 127 of the column) once per column.
 
-__device__ __forceinline__ void put_group(uint32_t (&r)[16], int c, int h, uint4 v) {
-  r[8 * c + 2 * h] = v.x;
-  r[8 * c + 2 * h + 1] = v.y;
-  r[8 * c + 4 + 2 * h] = v.z;
-  r[8 * c + 4 + 2 * h + 1] = v.w;
-}
-
-// IQ2_XS-style tile-block fields of lane (q, t) (the resident layout's lane
-// order: rows q and q+8, groups 4c + t, field i = 2c + h).
-struct Q2Lane {
-  uint32_t qs[4], sg[4], qh, sc0, sc1;
-  float d0, d1;  // d / 8 of rows q and q+8
+// IQ1_M-style fields of one row for half kh of a column.  Records p = 0, 1 of
+// the tile-block (groups 2 s + p, s = 0..15) give, for the half's local
+// sub-blocks s' = 0..7 (s = 8 kh + s'): qs word s' >> 1 (byte 2 (s' & 1) +
+// hh), and nibble word s' >> 2 (byte s' & 3, shifted so the row's nibble is
+// the byte's low nibble).
+struct Q1Row {
+  uint32_t qa[2][4], nb[2][2];
+  uint32_t sc;  // 3-bit sub-scales of the local sub-blocks, s' at bit 3 s'
+  float d8;     // d / 8
 };
 
-__device__ __forceinline__ Q2Lane load_q2(uint32_t tb, int lane) {
-  Q2Lane r;
-  const uint4 qs = ptx::lds128(tb + 32 * lane);
-  const uint4 sg = ptx::lds128(tb + 32 * lane + 16);
-  r.qs[0] = qs.x, r.qs[1] = qs.y, r.qs[2] = qs.z, r.qs[3] = qs.w;
-  r.sg[0] = sg.x, r.sg[1] = sg.y, r.sg[2] = sg.z, r.sg[3] = sg.w;
-  r.qh = ptx::lds16(tb + 1024 + 2 * lane);
-  const int q = lane >> 2;
-  const uint2 sc = ptx::lds64(tb + 1088 + 8 * q);
-  r.sc0 = sc.x, r.sc1 = sc.y;
-  const uint32_t dw = ptx::lds32(tb + 1152 + 4 * q);
-  r.d0 = __half2float(__ushort_as_half((unsigned short)(dw & 0xFFFFu))) * 0.125f;
-  r.d1 = __half2float(__ushort_as_half((unsigned short)(dw >> 16))) * 0.125f;
+__device__ __forceinline__ Q1Row load_q1_row(uint32_t tb, int q, int hh, int kh) {
+  Q1Row r;
+#pragma unroll
+  for (int p = 0; p < 2; ++p) {
+    const uint32_t rec = tb + 48 * (2 * q + p);
+    const uint4 a = ptx::lds128(rec + 16 * kh);
+    const uint2 b = ptx::lds64(rec + 32 + 8 * kh);
+    r.qa[p][0] = a.x, r.qa[p][1] = a.y, r.qa[p][2] = a.z, r.qa[p][3] = a.w;
+    r.nb[p][0] = b.x >> (4 * hh), r.nb[p][1] = b.y >> (4 * hh);
+  }
+  // the 48-bit sub-scale fields of rows q and q + 8 are bytes 0-5 and 6-11
+  const uint32_t s0 = ptx::lds32(tb + 768 + 12 * q), s1 = ptx::lds32(tb + 772 + 12 * q),
+                 s2 = ptx::lds32(tb + 776 + 12 * q);
+  const uint32_t lo = hh ? (s1 >> 16) | (s2 << 16) : s0, hi = hh ? s2 >> 16 : s1 & 0xFFFFu;
+  r.sc = kh ? (lo >> 24) | (hi << 8) : lo & 0xFFFFFFu;
+  const uint32_t dw = ptx::lds32(tb + 864 + 4 * q);
+  r.d8 = __half2float(__ushort_as_half((unsigned short)(hh ? dw >> 16 : dw & 0xFFFFu))) * 0.125f;
   return r;
 }
 
-// Step s (inputs 64s..64s+63 of the column) of one IQ2 tile-block: fields
-// i = 4s + 2c + h (group 8s + 4c + t of row q+8h).
-__device__ __forceinline__ void dequant_q2(const Q2Lane &L, int s, uint32_t sel2, uint32_t (&r)[16]) {
-  const uint32_t qw = s == 0 ? L.qs[0] : s == 1 ? L.qs[1] : s == 2 ? L.qs[2] : L.qs[3];
-  const uint32_t sw = s == 0 ? L.sg[0] : s == 1 ? L.sg[1] : s == 2 ? L.sg[2] : L.sg[3];
+// Local step j (0, 1) of one IQ1 row into r[32]: group 2m + p of the step
+// (sub-block s' = 4 j + m) fills registers 4 (2m + p) .. + 3.  The table
+// sel1 has 4096 entries indexed by qs | nibble << 8 (the delta bit is index
+// bit 11); its selectors pick from (X, Q) with X = P for delta +1/8 and
+// X = R for delta -1/8, where P = (-7, 1), R = (-9, -1), Q = (9, 7) times
+// d (2 sc + 1) / 8 -- the values 8 (grid + delta) of symbols 0, 1, 2 are
+// slots 0, 1, 2 for +1/8 and 0, 1, 3 for -1/8.  selc[n]: the byte-permute
+// that moves qs byte 2 (n & 1) + hh and nibble byte n into bytes 0 and 1.
+__device__ __forceinline__ void dequant_q1_row(const Q1Row &R, int j, uint32_t sel1, const uint32_t (&selc)[4],
+                                               uint32_t (&r)[32]) {
 #pragma unroll
-  for (int c2 = 0; c2 < 2; ++c2) {
-    const int c = 2 * s + c2;
+  for (int m = 0; m < 4; ++m) {
+    const int s = 4 * j + m;
+    const uint32_t n2 = (s == 0 ? R.sc << 1 : R.sc >> (3 * s - 1)) & 14u;  // 2 * sub-scale
+    const float sc8 = R.d8 * (__uint_as_float(0x4B000001u | n2) - 8388608.f);
+    const uint32_t P = bf16x2(-7.f * sc8, sc8), Rv = bf16x2(-9.f * sc8, -sc8), Q = bf16x2(9.f * sc8, 7.f * sc8);
+    const uint32_t RmP = Rv - P;
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int f = 2 * c2 + h;
-      // sign word s holds bit j of field 4s + f at bit 4j + f
-      const uint32_t qsb = (qw >> (8 * f)) & 0xFFu, sgz = (sw >> f) & 0x11111111u;
-      const uint32_t idx = qsb | (((L.qh >> (4 * s + f)) & 1u) << 8);
-      const uint2 sel = ptx::lds64_const(sel2 + 8 * idx);
-      const uint32_t nib = ((h ? L.sc1 : L.sc0) >> (4 * c)) & 15u;
-      const float sc = (h ? L.d1 : L.d0) * odd_f(nib);
-      const uint32_t t0 = bf16x2(sc * 8.f, sc * 25.f), t1 = bf16x2(sc * 43.f, 0.f);
-      // sign bits 2w, 2w+1 sit at bits 0 and 4 of byte w of sgz: that byte
-      // times 2^15 + 2^27 puts them at bits 15 and 31 of pair w (masked; the
-      // two shifted copies never overlap, so no carries)
-      uint4 v;
-      v.x = __byte_perm(t0, t1, sel.x) ^ ((__byte_perm(sgz, 0u, 0x4440u) * 0x08008000u) & 0x80008000u);
-      v.y = __byte_perm(t0, t1, sel.x >> 16) ^ ((__byte_perm(sgz, 0u, 0x4441u) * 0x08008000u) & 0x80008000u);
-      v.z = __byte_perm(t0, t1, sel.y) ^ ((__byte_perm(sgz, 0u, 0x4442u) * 0x08008000u) & 0x80008000u);
-      v.w = __byte_perm(t0, t1, sel.y >> 16) ^ ((__byte_perm(sgz, 0u, 0x4443u) * 0x08008000u) & 0x80008000u);
-      put_group(r, c2, h, v);
+    for (int p = 0; p < 2; ++p) {
+      const uint32_t idx = __byte_perm(R.qa[p][s >> 1], R.nb[p][s >> 2], selc[s & 3]) & 0xFFFu;
+      const uint2 sel = ptx::lds64_const(sel1 + 8 * idx);
+      const uint32_t X = (idx >> 11) * RmP + P;
+      const int g = 2 * m + p;
+      r[4 * g + 0] = __byte_perm(X, Q, sel.x);
+      r[4 * g + 1] = __byte_perm(X, Q, sel.x >> 16);
+      r[4 * g + 2] = __byte_perm(X, Q, sel.y);
+      r[4 * g + 3] = __byte_perm(X, Q, sel.y >> 16);
     }
   }
 }
 
-// IQ1_M-style tile-block fields of lane (q, t) for groups 8S + 4c + t (c =
-// 0, 1) of every step S, rows q and q+8.  Group g sits in the record of
-// pair p = g & 1 (here t & 1) as entry i = 2 (g >> 1) + h; with u = t >> 1
-// the lane's entries of step S are bytes 2u, 2u+1 of qs words 2S and 2S+1,
-// and its qh nibbles bytes u and 2+u of nibble word S.
-struct Q1Lane {
-  uint32_t qs[4], nb[4];
-  uint64_t row0, row1;  // 3-bit sub-block scales of rows q and q+8, from sub-block u
-  float d0, d1;
+// IQ2_XS-style fields of one row for half kh of a column.  Records t = 0..3
+// of the tile-block (lanes 4q + t: groups 4c + t) give, for the local
+// sub-blocks c' = c - 4 kh = 0..3: qs word c' >> 1 (byte 2 (c' & 1) after a
+// shift by 8 hh), sign word c' >> 1 (bit 4 j' + 2 (c' & 1) = sign of weight
+// j' after a shift by hh), and index bit 8 at bit 0 of byte t of vq[c'].
+struct Q2Row {
+  uint32_t qs[4][2], sg[4][2], vq[4];
+  uint32_t sc;  // 4-bit sub-scales of the local sub-blocks, c' at bit 4 c'
+  float d8;
 };
 
-__device__ __forceinline__ Q1Lane load_q1(uint32_t tb, int lane) {
-  Q1Lane r;
-  const int q = lane >> 2, p = lane & 1, u = (lane >> 1) & 1;
-  const uint32_t pb = tb + 48 * (2 * q + p);
-  const uint4 qa = ptx::lds128(pb), qb = ptx::lds128(pb + 16);
-  const uint4 nb = ptx::lds128(pb + 32);
-  const uint32_t qsel = u ? 0x7632u : 0x5410u, nsel = u ? 0x4431u : 0x4420u;
-  r.qs[0] = __byte_perm(qa.x, qa.y, qsel);
-  r.qs[1] = __byte_perm(qa.z, qa.w, qsel);
-  r.qs[2] = __byte_perm(qb.x, qb.y, qsel);
-  r.qs[3] = __byte_perm(qb.z, qb.w, qsel);
-  r.nb[0] = __byte_perm(nb.x, 0u, nsel);
-  r.nb[1] = __byte_perm(nb.y, 0u, nsel);
-  r.nb[2] = __byte_perm(nb.z, 0u, nsel);
-  r.nb[3] = __byte_perm(nb.w, 0u, nsel);
-  const uint32_t s0 = ptx::lds32(tb + 768 + 12 * q), s1 = ptx::lds32(tb + 772 + 12 * q),
-                 s2 = ptx::lds32(tb + 776 + 12 * q);
-  r.row0 = (uint64_t)s0 | ((uint64_t)(s1 & 0xFFFFu) << 32);
-  r.row1 = (uint64_t)(s1 >> 16) | ((uint64_t)s2 << 16);
-  r.row0 >>= 3 * u;  // sub-block of group 8S + 4c + t is 4S + 2c + u
-  r.row1 >>= 3 * u;
-  const uint32_t dw = ptx::lds32(tb + 864 + 4 * q);
-  r.d0 = __half2float(__ushort_as_half((unsigned short)(dw & 0xFFFFu)));
-  r.d1 = __half2float(__ushort_as_half((unsigned short)(dw >> 16)));
+__device__ __forceinline__ Q2Row load_q2_row(uint32_t tb, int q, int hh, int kh) {
+  Q2Row r;
+#pragma unroll
+  for (int t = 0; t < 4; ++t) {
+    const uint32_t rec = tb + 32 * (4 * q + t);
+    const uint2 a = ptx::lds64(rec + 8 * kh), b = ptx::lds64(rec + 16 + 8 * kh);
+    r.qs[t][0] = a.x >> (8 * hh), r.qs[t][1] = a.y >> (8 * hh);
+    r.sg[t][0] = b.x >> hh, r.sg[t][1] = b.y >> hh;
+  }
+  // index bit 8 of field i = 2c + hh is bit i of record t's u16
+  const uint2 qh = ptx::lds64(tb + 1024 + 8 * q);
+  const int sh = 8 * kh + hh;
+  const uint32_t v = __byte_perm(__byte_perm(qh.x >> sh, qh.x >> (16 + sh), 0x0040u),
+                                 __byte_perm(qh.y >> sh, qh.y >> (16 + sh), 0x0040u), 0x5410u);
+#pragma unroll
+  for (int c = 0; c < 4; ++c) r.vq[c] = v >> (2 * c);
+  r.sc = ptx::lds32(tb + 1088 + 8 * q + 4 * hh) >> (16 * kh);
+  const uint32_t dw = ptx::lds32(tb + 1152 + 4 * q);
+  r.d8 = __half2float(__ushort_as_half((unsigned short)(hh ? dw >> 16 : dw & 0xFFFFu))) * 0.125f;
   return r;
 }
 
-__device__ __forceinline__ void dequant_q1(const Q1Lane &L, int S, uint32_t sel1, uint32_t (&r)[16]) {
-  const uint32_t qw = S == 0 ? L.qs[0] : S == 1 ? L.qs[1] : S == 2 ? L.qs[2] : L.qs[3];
-  const uint32_t nb16 = S == 0 ? L.nb[0] : S == 1 ? L.nb[1] : S == 2 ? L.nb[2] : L.nb[3];
+// Local step j (0, 1) of one IQ2 row into r[32]: group 4 cc + t of the step
+// (local sub-block c' = 2 j + cc) fills registers 4 (4 cc + t) .. + 3.  The
+// value table is (8, 25 | 43, 0) times d (2 sc + 1) / 8; each pair's two
+// sign bits become bits 15 and 31 of an XOR mask.
+__device__ __forceinline__ void dequant_q2_row(const Q2Row &R, int j, uint32_t sel2, uint32_t (&r)[32]) {
 #pragma unroll
-  for (int c2 = 0; c2 < 2; ++c2) {
-    const int sb = 4 * S + 2 * c2;  // sub-block, counted from the lane's first (u)
+  for (int cc = 0; cc < 2; ++cc) {
+    const int c = 2 * j + cc;
+    const uint32_t n2 = (c == 0 ? R.sc << 1 : R.sc >> (4 * c - 1)) & 30u;  // 2 * sub-scale
+    const float sc8 = R.d8 * (__uint_as_float(0x4B000001u | n2) - 8388608.f);
+    const uint32_t t0 = bf16x2(sc8 * 8.f, sc8 * 25.f), t1 = bf16x2(sc8 * 43.f, 0.f);
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const uint32_t qsb = (qw >> (16 * c2 + 8 * h)) & 0xFFu;
-      const uint32_t nib = (nb16 >> (8 * c2 + 4 * h)) & 15u;
-      const uint2 sel = ptx::lds64_const(sel1 + 8 * (qsb | ((nib & 7u) << 8)));
-      const uint32_t sc3 = (uint32_t)(((h ? L.row1 : L.row0) >> (3 * sb)) & 7u);
-      const float sc = (h ? L.d1 : L.d0) * odd_f(sc3);
-      const float dl = (nib & 8u) ? -0.125f : 0.125f;
-      const uint32_t t0 = bf16x2(sc * (dl - 1.f), sc * dl), t1 = bf16x2(sc * (dl + 1.f), 0.f);
-      uint4 v;
-      v.x = __byte_perm(t0, t1, sel.x);
-      v.y = __byte_perm(t0, t1, sel.x >> 16);
-      v.z = __byte_perm(t0, t1, sel.y);
-      v.w = __byte_perm(t0, t1, sel.y >> 16);
-      put_group(r, c2, h, v);
+    for (int t = 0; t < 4; ++t) {
+      const uint32_t idx = __byte_perm(R.qs[t][j], R.vq[c], (uint32_t)(2 * cc) | ((4u + t) << 4)) & 0x1FFu;
+      const uint2 sel = ptx::lds64_const(sel2 + 8 * idx);
+      const uint32_t sgz = (R.sg[t][j] >> (2 * cc)) & 0x11111111u;
+      const int g = 4 * cc + t;
+#pragma unroll
+      for (int w = 0; w < 4; ++w) {
+        const uint32_t sw = w & 1 ? (w & 2 ? sel.y : sel.x) >> 16 : (w & 2 ? sel.y : sel.x);
+        const uint32_t m = __byte_perm(sgz, 0u, 0x4440u + w) * 0x08008000u;
+        r[4 * g + w] = __byte_perm(t0, t1, sw) ^ (m & 0x80008000u);
+      }
     }
   }
 }
@@ -355,12 +348,23 @@ __global__ void __maxnreg__(128) grouped_tc_kernel(TileArgs a) {
   Bars &B = *S.bars;
 
   // selector tables, barriers, TMEM
-  for (int i = tid; i < (512 + 2048) * 8 / 16; i += kTcThreads)
-    reinterpret_cast<uint4 *>(const_cast<uint2 *>(S.sel2))[i] =
-        __ldg(reinterpret_cast<const uint4 *>(a.grids + kGridQ2Bsel) + i);
+  // (the IQ1 table gets a second half for delta -1/8: slot 2 -> 3, i.e.
+  // selector nibbles 4, 5 -> 6, 7)
+  {
+    const uint4 *g = reinterpret_cast<const uint4 *>(a.grids + kGridQ2Bsel);
+    uint4 *t2 = reinterpret_cast<uint4 *>(const_cast<uint2 *>(S.sel2));
+    uint4 *t1 = reinterpret_cast<uint4 *>(const_cast<uint2 *>(S.sel1));
+    for (int i = tid; i < 512 * 8 / 16; i += kTcThreads) t2[i] = __ldg(g + i);
+    for (int i = tid; i < 2048 * 8 / 16; i += kTcThreads) {
+      const uint4 v = __ldg(g + 512 * 8 / 16 + i);
+      t1[i] = v;
+      t1[i + 2048 * 8 / 16] = make_uint4(v.x + ((v.x & 0x44444444u) >> 1), v.y + ((v.y & 0x44444444u) >> 1),
+                                         v.z + ((v.z & 0x44444444u) >> 1), v.w + ((v.w & 0x44444444u) >> 1));
+    }
+  }
   if (tid == 0) {
     for (int i = 0; i < kPr; ++i) ptx::mbar_init(&B.pfull[i], 1), ptx::mbar_init(&B.pempty[i], kDqWarps);
-    for (int i = 0; i < C::kAr; ++i) ptx::mbar_init(&B.afull[i], kDqWarps), ptx::mbar_init(&B.aempty[i], 1);
+    for (int i = 0; i < C::kAr; ++i) ptx::mbar_init(&B.afull[i], kDqWarps / 2), ptx::mbar_init(&B.aempty[i], 1);
     for (int i = 0; i < 2; ++i) ptx::mbar_init(&B.accfull[i], 1), ptx::mbar_init(&B.accempty[i], kEpWarps);
     ptx::mbar_fence_init();
   }
@@ -461,30 +465,30 @@ __global__ void __maxnreg__(128) grouped_tc_kernel(TileArgs a) {
         }
       }
     } else if (warp < 2 + kDqWarps) {
-      // ---- dequant warps: one tile-block of each matrix into TMEM, 16 rows of B
-      const int w = warp - 2;
-      // the TMEM lanes this warp may write are 32 (warp % 4) .. + 31: its
-      // tile-block (16 rows of the unit's 128) lies in that quarter
-      const int tbi = 2 * (warp & 3) + (warp >= 6 ? 1 : 0);
-      const uint32_t tlane = tmem + ((uint32_t)(16 * tbi) << 16);
+      // ---- dequant warps: rows 32 qd .. 32 qd + 31 of every matrix, steps
+      // 2 kh and 2 kh + 1 of every column, and the B rows of those steps
+      const int qd = warp & 3, kh = warp >= 6 ? 1 : 0;
+      const int tbi = 2 * qd + (lane >> 4), rr = lane & 15, q = rr & 7, hh = rr >> 3;
+      const uint32_t tlane = tmem + ((uint32_t)(32 * qd) << 16);
       const uint32_t sel2a = ptx::smem_u32(S.sel2), sel1a = ptx::smem_u32(S.sel1);
+      uint32_t selc[4];
+#pragma unroll
+      for (int n = 0; n < 4; ++n) selc[n] = (uint32_t)(2 * (n & 1) + hh) | ((4u + n) << 4);
       for (int u = 0; u < n_this; ++u) {
         const Unit U = S.units[u];
         const int nkb = U.K / 256;
-        // B rows 16w + (lane >> 3) + 4i, 16-byte chunk lane & 7 of each step
-        const __nv_bfloat16 *brow[4];
-        int nb = 0;
+        // B rows 32 qd + (lane >> 3) + 4 i (i < 8), 16-byte chunk lane & 7:
+        // the row of x (the pair's token) or of h (the pair) they copy
+        int brow[8], nb = 0;
 #pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const int j = 16 * w + (lane >> 3) + 4 * i;
-          const int jj = min(j, U.n_real - 1);  // pad rows read a real row; their results are dropped
-          if (j < U.n_pad) nb = i + 1;
-          brow[i] = DOWN ? hbuf + (size_t)(U.p0 + jj) * a.max_ffn : xb + (size_t)pairs[U.p0 + jj].token * H;
+        for (int i = 0; i < 8; ++i) {
+          const int jr = 32 * qd + (lane >> 3) + 4 * i;
+          const int jj = min(jr, U.n_real - 1);  // pad rows read a real row; their results are dropped
+          if (jr < U.n_pad) nb = i + 1;
+          brow[i] = DOWN ? U.p0 + jj : pairs[U.p0 + jj].token;
         }
-        const int tbb = tile_block_bytes(U.qtype), nsteps = 4 * nkb;
-        // B rows of local step n into ring slot `as`, as one cp.async group;
-        // issued a step ahead so the copies overlap the decode of the step
-        // before.  Waiting for the slot's release also frees its A slot.
+        // B rows of local step n into ring slot gstep % kAr, as one cp.async
+        // group; waiting for the slot's release also frees its A slot
         auto fetch_b = [&](int n, uint32_t gstep) {
           const int as = gstep % C::kAr;
           {
@@ -496,12 +500,17 @@ __global__ void __maxnreg__(128) grouped_tc_kernel(TileArgs a) {
           uint8_t *bt = S.ring + (size_t)as * C::kStep;
           const int k0 = 64 * n + 8 * (lane & 7);
 #pragma unroll
-          for (int i = 0; i < 4; ++i)
-            if (i < nb) cp_async16(bt + ptx::sw128_offset(16 * w + (lane >> 3) + 4 * i, 8 * (lane & 7)), brow[i] + k0);
+          for (int i = 0; i < 8; ++i)
+            if (i < nb) {
+              const __nv_bfloat16 *src = DOWN ? hbuf + (size_t)brow[i] * a.max_ffn : xb + (size_t)brow[i] * H;
+              cp_async16(bt + ptx::sw128_offset(32 * qd + (lane >> 3) + 4 * i, 8 * (lane & 7)), src + k0);
+            }
           asm volatile("cp.async.commit_group;" ::: "memory");
         };
-        fetch_b(0, step);
         for (int kb = 0; kb < nkb; ++kb, ++col) {
+          const uint32_t g0 = step + 4 * kb + 2 * kh;  // this half's first step of the column
+          fetch_b(4 * kb + 2 * kh, g0);
+          fetch_b(4 * kb + 2 * kh + 1, g0 + 1);
           const int ps = col % kPr;
           {
             TC_T0();
@@ -509,48 +518,56 @@ __global__ void __maxnreg__(128) grouped_tc_kernel(TileArgs a) {
             TC_ADD(0);
           }
           const uint32_t pk = ptx::smem_u32(S.packed) + ps * C::kPacked;
-          Q2Lane l2[C::kMats];
-          Q1Lane l1[C::kMats];
-          if (U.qtype == kQ2) {
-#pragma unroll
-            for (int m = 0; m < C::kMats; ++m) l2[m] = load_q2(pk + (m * 8 + tbi) * tbb, lane);
-          } else {
-#pragma unroll
-            for (int m = 0; m < C::kMats; ++m) l1[m] = load_q1(pk + (m * 8 + tbi) * tbb, lane);
-          }
-          __syncwarp();
-          if (lane == 0) ptx::mbar_arrive(&B.pempty[ps]);
-#pragma unroll
-          for (int s = 0; s < 4; ++s, ++step) {
-            const int n = 4 * kb + s, as = step % C::kAr;
-            const bool more = n + 1 < nsteps;
-            if (more) fetch_b(n + 1, step + 1);
-            // the slot's previous MMAs are done (waited for when its B rows were fetched)
-            ptx::tc_fence_after();
-            const uint32_t at = tlane + kAccCols + (uint32_t)as * C::kSlotCols;
-            TC_T0();
+          // the column's fields of every matrix, then its two steps; one
+          // instance per format so only one format's fields are live
+          auto column = [&](auto fmt) {
+            constexpr bool kIsQ2 = decltype(fmt)::value == kQ2;
+            using Row = typename std::conditional<kIsQ2, Q2Row, Q1Row>::type;
+            Row rows[C::kMats];
 #pragma unroll
             for (int m = 0; m < C::kMats; ++m) {
-              uint32_t r[16];
-              if (U.qtype == kQ2)
-                dequant_q2(l2[m], s, sel2a, r);
+              if constexpr (kIsQ2)
+                rows[m] = load_q2_row(pk + (m * 8 + tbi) * kQ2TileBlock, q, hh, kh);
               else
-                dequant_q1(l1[m], s, sel1a, r);
-              ptx::tmem_st16x256_x4(at + 32 * m, r);
+                rows[m] = load_q1_row(pk + (m * 8 + tbi) * kQ1TileBlock, q, hh, kh);
             }
-            TC_ADD(2);
-            ptx::tmem_wait_st();
-            // this step's B rows landed (the next step's may still be in flight)
-            if (more)
-              asm volatile("cp.async.wait_group 1;" ::: "memory");
-            else
-              asm volatile("cp.async.wait_group 0;" ::: "memory");
-            ptx::fence_proxy_async_smem();  // generic-proxy writes -> the tensor cores
-            ptx::tc_fence_before();
             __syncwarp();
-            if (lane == 0) ptx::mbar_arrive(&B.afull[as]);
-          }
+            if (lane == 0) ptx::mbar_arrive(&B.pempty[ps]);
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+              const int as = (int)((g0 + j) % C::kAr);
+              // the slot's previous MMAs are done (waited for when its B rows were fetched)
+              ptx::tc_fence_after();
+              const uint32_t at = tlane + kAccCols + (uint32_t)as * C::kSlotCols;
+              TC_T0();
+#pragma unroll
+              for (int m = 0; m < C::kMats; ++m) {
+                uint32_t r[32];
+                if constexpr (kIsQ2)
+                  dequant_q2_row(rows[m], j, sel2a, r);
+                else
+                  dequant_q1_row(rows[m], j, sel1a, selc, r);
+                ptx::tmem_st32x32b_x32(at + 32 * m, r);
+              }
+              TC_ADD(2);
+              ptx::tmem_wait_st();
+              // this step's B rows landed (the next step's may still be in flight)
+              if (j == 0)
+                asm volatile("cp.async.wait_group 1;" ::: "memory");
+              else
+                asm volatile("cp.async.wait_group 0;" ::: "memory");
+              ptx::fence_proxy_async_smem();  // generic-proxy writes -> the tensor cores
+              ptx::tc_fence_before();
+              __syncwarp();
+              if (lane == 0) ptx::mbar_arrive(&B.afull[as]);
+            }
+          };
+          if (U.qtype == kQ2)
+            column(std::integral_constant<int, kQ2>());
+          else
+            column(std::integral_constant<int, kQ1>());
         }
+        step += 4 * nkb;
       }
     } else {
       // ---- epilogue: warp reads TMEM lanes 32 (warp % 4) .. + 31 (= tile rows)
@@ -574,8 +591,6 @@ __global__ void __maxnreg__(128) grouped_tc_kernel(TileArgs a) {
         const uint32_t lq16 = (uint32_t)(32 * lq) << 16;
         const uint32_t d = tmem + P.gate + lq16, du = tmem + P.up + lq16;
         const int r = 128 * U.rt + row;
-        // h is stored in the contraction order of the down kernel's steps
-        const int rp = (r & ~63) | perm64(r & 63);
         Pair pl = {0, 0.f};  // down, scalar path: pair c0 - (c0 % 32) + lane of the unit, broadcast by shuffles
         // down, vector path: lane l holds the pair of column lq + 4 l (the
         // columns this warp adds), read once per unit
@@ -628,10 +643,9 @@ __global__ void __maxnreg__(128) grouped_tc_kernel(TileArgs a) {
             __nv_bfloat16 *T = reinterpret_cast<__nv_bfloat16 *>(S.stage) + (ep_stage & 1) * 16 * 128;
             ++ep_stage;
             ptx::tmem_wait_ld();
-            const int prow = rp - 128 * U.rt;
 #pragma unroll
             for (int i = 0; i < 16; ++i)
-              T[i * 128 + prow] = __float2bfloat16_rn(silu_mul_fast(__uint_as_float(d0[i]), __uint_as_float(d1[i])));
+              T[i * 128 + row] = __float2bfloat16_rn(silu_mul_fast(__uint_as_float(d0[i]), __uint_as_float(d1[i])));
             asm volatile("bar.sync 1, %0;" ::"n"(32 * kEpWarps) : "memory");
 #pragma unroll
             for (int k = 0; k < 2; ++k) {
@@ -660,19 +674,14 @@ __global__ void __maxnreg__(128) grouped_tc_kernel(TileArgs a) {
   if (warp == 0) ptx::tmem_dealloc(tmem, kTmemCols);
 }
 
-// Activations to bf16 (round to nearest even), 8 per thread: inputs
-// 8i..8i+7 (group G = i mod 8 of a 64-input step) go to positions perm64,
-// two runs of four.
+// Activations to bf16 (round to nearest even), 8 per thread.
 __global__ void to_bf16_kernel(const float *__restrict__ x, __nv_bfloat16 *__restrict__ xb, int64_t n8) {
   const int64_t i = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
   if (i >= n8) return;
   const float4 v0 = __ldg(reinterpret_cast<const float4 *>(x) + 2 * i);
   const float4 v1 = __ldg(reinterpret_cast<const float4 *>(x) + 2 * i + 1);
-  const int64_t base = (i >> 3) << 6;
-  const int g = (int)(i & 7);
-  const int p0 = perm64(8 * g), p1 = perm64(8 * g + 4);
-  *reinterpret_cast<uint2 *>(xb + base + p0) = make_uint2(bf16x2(v0.x, v0.y), bf16x2(v0.z, v0.w));
-  *reinterpret_cast<uint2 *>(xb + base + p1) = make_uint2(bf16x2(v1.x, v1.y), bf16x2(v1.z, v1.w));
+  reinterpret_cast<uint4 *>(xb)[i] =
+      make_uint4(bf16x2(v0.x, v0.y), bf16x2(v0.z, v0.w), bf16x2(v1.x, v1.y), bf16x2(v1.z, v1.w));
 }
 
 }  // namespace
