@@ -497,6 +497,9 @@ __global__ void __maxnreg__(128) grouped_tc_kernel(TileArgs a) {
               bad = true;
             TC_ADD(1);
           }
+          // the tensor cores read the slot's previous rows through the async
+          // proxy; order those reads before these generic-proxy writes
+          ptx::fence_proxy_async_smem();
           uint8_t *bt = S.ring + (size_t)as * C::kStep;
           const int k0 = 64 * n + 8 * (lane & 7);
 #pragma unroll
@@ -509,8 +512,6 @@ __global__ void __maxnreg__(128) grouped_tc_kernel(TileArgs a) {
         };
         for (int kb = 0; kb < nkb; ++kb, ++col) {
           const uint32_t g0 = step + 4 * kb + 2 * kh;  // this half's first step of the column
-          fetch_b(4 * kb + 2 * kh, g0);
-          fetch_b(4 * kb + 2 * kh + 1, g0 + 1);
           const int ps = col % kPr;
           {
             TC_T0();
@@ -531,8 +532,16 @@ __global__ void __maxnreg__(128) grouped_tc_kernel(TileArgs a) {
               else
                 rows[m] = load_q1_row(pk + (m * 8 + tbi) * kQ1TileBlock, q, hh, kh);
             }
+            // the fields were read through the generic proxy and the slot's
+            // next bytes arrive through the async proxy (bulk copy): order
+            // the reads before the release that lets the producer refill it
+            ptx::fence_proxy_async_smem();
             __syncwarp();
             if (lane == 0) ptx::mbar_arrive(&B.pempty[ps]);
+            // the B rows of the two steps (after the fence, which would
+            // otherwise wait for these copies too)
+            fetch_b(4 * kb + 2 * kh, g0);
+            fetch_b(4 * kb + 2 * kh + 1, g0 + 1);
 #pragma unroll
             for (int j = 0; j < 2; ++j) {
               const int as = (int)((g0 + j) % C::kAr);
