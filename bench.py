@@ -383,8 +383,9 @@ def measure(cfg: int, steps: int, warmup: int, world: int, rank: int, local: int
     launches_per_call = R.launches_per_call(dx[0].shape[0], w.top_k, sh is not None)
     del graph
 
-    # end-to-end through the public call with host buffers (pinned), per call:
-    # H2D of the call's x, ids and weights (one packed transfer); the layer; D2H of out.
+    # end-to-end through the public call with host buffers (pinned), per call
+    # (redlite_moe_layer_host): H2D of the call's x, ids and weights (one
+    # packed transfer); the layer; D2H of out.
     e2e = None
     if e2e_on:
         hbuf = [torch.from_numpy(pk).pin_memory() for pk in packed]
@@ -392,10 +393,11 @@ def measure(cfg: int, steps: int, warmup: int, world: int, rank: int, local: int
         e_calls = min(steps * cps, 2400 if nsets > 1 else steps * cps)
 
         def e2e_call(i):
+            # one public call: the packed inputs host -> device, the layer, out device -> host
             j = i % nsets
-            dbuf[j].copy_(hbuf[j], non_blocking=True)
-            call(j)
-            ho[j].copy_(do[j], non_blocking=True)
+            rc = R.redlite_moe_layer_host(hbuf[j], dbuf[j], dx[j].shape[0], w.top_k, L.table, L.shared, do[j], ho[j])
+            if rc != 0:
+                raise RuntimeError(f"redlite_moe_layer_host rc={rc}")
 
         for i in range(3):
             e2e_call(i)

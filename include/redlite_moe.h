@@ -164,6 +164,35 @@ int redlite_moe_layer(const float *x, int32_t n_tokens, const int32_t *expert_id
                       int32_t top_k, const redlite_moe_table *expert_table, const redlite_moe_expert *shared_expert,
                       float *out);
 
+/* The layer for inputs and output held in host memory (a library
+ * convenience with no page counterpart; the arithmetic is
+ * redlite_moe_layer's).  On expert_table->stream it copies the call's
+ * packed inputs host -> device in one transfer, runs the layer on the
+ * device copy and copies out back to the host:
+ *   inputs_host  host buffer (page-locked for an asynchronous copy) of
+ *                redlite_moe_host_input_bytes(hidden, n_tokens, top_k)
+ *                bytes: x [n_tokens, hidden] fp32, then expert_ids
+ *                [n_tokens, top_k] int32, then router_weights [n_tokens,
+ *                top_k] fp32, contiguous
+ *   inputs_dev   device buffer of the same size, 16-byte aligned: the
+ *                staging copy the kernels read (caller-owned)
+ *   out_dev      device [n_tokens, hidden] fp32, 16-byte aligned, written
+ *   out_host     host [n_tokens, hidden] fp32 (page-locked for an
+ *                asynchronous copy), written
+ * n_tokens, top_k, expert_table and shared_expert as for redlite_moe_layer.
+ * Asynchronous: the host buffers must stay valid, inputs_host unchanged and
+ * out_host unread, until the stream has passed the call.  Errors: the
+ * checks of redlite_moe_layer plus null or misaligned buffers, found on the
+ * host before anything is enqueued; REDLITE_ECUDA if a copy or a launch
+ * cannot be enqueued.  n_tokens = 0 returns REDLITE_OK and enqueues nothing. */
+int redlite_moe_layer_host(const void *inputs_host, void *inputs_dev, int32_t n_tokens, int32_t top_k,
+                           const redlite_moe_table *expert_table, const redlite_moe_expert *shared_expert,
+                           float *out_dev, float *out_host);
+
+/* Bytes of the packed host input buffer of redlite_moe_layer_host: 4
+ * (hidden + 2 top_k) n_tokens; 0 for a negative or zero size. */
+size_t redlite_moe_host_input_bytes(int32_t hidden, int32_t n_tokens, int32_t top_k);
+
 /* The router that feeds the layer ("Red Metal dev8", section "Field
  * validation": router-network integration is the milestone after the
  * routed layer; "Red Lite dev10", section "What dev10 does not yet claim":

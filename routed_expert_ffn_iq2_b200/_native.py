@@ -67,6 +67,10 @@ EXPORTS = {
     "redlite_moe_layer_noalloc": (ctypes.c_int, [_c_void_p, ctypes.c_int32, _c_void_p, _c_void_p, ctypes.c_int32,
                                                  ctypes.POINTER(redlite_moe_table),
                                                  ctypes.POINTER(redlite_moe_expert), _c_void_p]),
+    "redlite_moe_layer_host": (ctypes.c_int, [_c_void_p, _c_void_p, ctypes.c_int32, ctypes.c_int32,
+                                              ctypes.POINTER(redlite_moe_table), ctypes.POINTER(redlite_moe_expert),
+                                              _c_void_p, _c_void_p]),
+    "redlite_moe_host_input_bytes": (ctypes.c_size_t, [ctypes.c_int32, ctypes.c_int32, ctypes.c_int32]),
     "redlite_moe_route_topk": (ctypes.c_int, [_c_void_p, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32, _c_void_p,
                                               _c_void_p, _c_void_p]),
     "redlite_moe_block_scratch_bytes": (ctypes.c_size_t, [ctypes.c_int32] * 4),
@@ -194,6 +198,21 @@ def redlite_moe_layer_noalloc(x: torch.Tensor, n_tokens: int, expert_ids: torch.
                                            ctypes.byref(expert_table),
                                            ctypes.byref(shared_expert) if shared_expert is not None else None,
                                            _ptr(out))
+
+
+def redlite_moe_layer_host(inputs_host: torch.Tensor, inputs_dev: torch.Tensor, n_tokens: int, top_k: int,
+                           expert_table: redlite_moe_table, shared_expert: Optional[redlite_moe_expert],
+                           out_dev: torch.Tensor, out_host: torch.Tensor) -> int:
+    """The layer on inputs and output in host memory: one packed host -> device
+    copy (x, ids, weights), the layer, the device -> host copy of out."""
+    return lib().redlite_moe_layer_host(_ptr(inputs_host), _ptr(inputs_dev), n_tokens, top_k,
+                                        ctypes.byref(expert_table),
+                                        ctypes.byref(shared_expert) if shared_expert is not None else None,
+                                        _ptr(out_dev), _ptr(out_host))
+
+
+def redlite_moe_host_input_bytes(hidden: int, n_tokens: int, top_k: int) -> int:
+    return int(lib().redlite_moe_host_input_bytes(hidden, n_tokens, top_k))
 
 
 def redlite_moe_route_topk(logits: torch.Tensor, n_tokens: int, n_experts: int, top_k: int, expert_ids: torch.Tensor,

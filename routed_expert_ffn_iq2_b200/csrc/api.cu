@@ -62,24 +62,33 @@ int redlite_moe_workspace_reset(const redlite_moe_table *t) {
 
 namespace redlite {
 
-int layer_impl(const float *x, int32_t n_tokens, const int32_t *expert_ids, const float *router_weights, int32_t top_k,
-               const redlite_moe_table *t, const redlite_moe_expert *shared, float *out, const float *residual) {
+// The checks of a layer call that do not involve its data pointers:
+// REDLITE_OK, or the error code the call returns before enqueuing anything.
+static int layer_call_ok(int32_t n_tokens, int32_t top_k, const redlite_moe_table *t, const redlite_moe_expert *shared) {
   if (!table_ok(t)) return REDLITE_EINVAL;
   if (n_tokens < 0 || n_tokens > t->max_tokens) return REDLITE_EINVAL;
   if (top_k < 1 || top_k > kMaxTopK) return REDLITE_EINVAL;
-  if (n_tokens == 0) return REDLITE_OK;
-  if (!x || !expert_ids || !router_weights || !out) return REDLITE_EINVAL;
-  if (!aligned16(x) || !aligned16(out)) return REDLITE_EINVAL;
+  if (n_tokens == 0) return REDLITE_OK;  // the call enqueues nothing
   // min_ffn >= 256 declares every slot tiled: the fast kernels then run, and
   // the shared expert must be one they can read (selected slots are checked
   // on the device and reported in the status word)
+  if (shared && !shared_ok(*shared, t, t->min_ffn >= 256)) return REDLITE_EINVAL;
+  // the largest top_k this workspace can hold for the table's token limit
+  if (workspace_layout(t->hidden, t->n_experts, t->max_tokens, top_k, t->max_ffn).total > t->workspace_bytes)
+    return REDLITE_ENOMEM;
+  return REDLITE_OK;
+}
+
+int layer_impl(const float *x, int32_t n_tokens, const int32_t *expert_ids, const float *router_weights, int32_t top_k,
+               const redlite_moe_table *t, const redlite_moe_expert *shared, float *out, const float *residual) {
+  const int ok = layer_call_ok(n_tokens, top_k, t, shared);
+  if (ok != REDLITE_OK) return ok;
+  if (n_tokens == 0) return REDLITE_OK;
+  if (!x || !expert_ids || !router_weights || !out) return REDLITE_EINVAL;
+  if (!aligned16(x) || !aligned16(out)) return REDLITE_EINVAL;
   const bool tiled = t->min_ffn >= 256;
-  if (shared && !shared_ok(*shared, t, tiled)) return REDLITE_EINVAL;
-  // the largest top_k this workspace can hold for n_tokens
-  WorkspaceLayout L = workspace_layout(t->hidden, t->n_experts, n_tokens, top_k, t->max_ffn);
-  WorkspaceLayout Lmax = workspace_layout(t->hidden, t->n_experts, t->max_tokens, top_k, t->max_ffn);
-  if (Lmax.total > t->workspace_bytes) return REDLITE_ENOMEM;
-  L = Lmax;  // region offsets are fixed by the table limits
+  // region offsets are fixed by the table limits
+  const WorkspaceLayout L = workspace_layout(t->hidden, t->n_experts, t->max_tokens, top_k, t->max_ffn);
   cudaStream_t s = (cudaStream_t)t->stream;
   uint8_t *ws = (uint8_t *)t->workspace;
 
@@ -214,6 +223,36 @@ int redlite_moe_upload_experts(int32_t hidden, const int32_t *ids, const redlite
   }
   if (pool_end) *pool_end = off;
   return REDLITE_OK;
+}
+
+}  // extern "C"
+
+extern "C" {
+
+size_t redlite_moe_host_input_bytes(int32_t hidden, int32_t n_tokens, int32_t top_k) {
+  if (hidden <= 0 || n_tokens <= 0 || top_k <= 0) return 0;
+  return sizeof(float) * ((size_t)hidden + 2 * (size_t)top_k) * (size_t)n_tokens;
+}
+
+int redlite_moe_layer_host(const void *inputs_host, void *inputs_dev, int32_t n_tokens, int32_t top_k,
+                           const redlite_moe_table *t, const redlite_moe_expert *shared, float *out_dev,
+                           float *out_host) {
+  const int ok = layer_call_ok(n_tokens, top_k, t, shared);
+  if (ok != REDLITE_OK) return ok;
+  if (n_tokens == 0) return REDLITE_OK;
+  if (!inputs_host || !inputs_dev || !out_dev || !out_host) return REDLITE_EINVAL;
+  if (!aligned16(inputs_dev) || !aligned16(out_dev)) return REDLITE_EINVAL;
+  cudaStream_t s = (cudaStream_t)t->stream;
+  const size_t nx = sizeof(float) * (size_t)n_tokens * (size_t)t->hidden;
+  const size_t nk = sizeof(float) * (size_t)n_tokens * (size_t)top_k;
+  if (cudaMemcpyAsync(inputs_dev, inputs_host, nx + 2 * nk, cudaMemcpyHostToDevice, s) != cudaSuccess)
+    return REDLITE_ECUDA;
+  const uint8_t *in = (const uint8_t *)inputs_dev;
+  const int rc = layer_impl((const float *)in, n_tokens, (const int32_t *)(in + nx), (const float *)(in + nx + nk),
+                            top_k, t, shared, out_dev, nullptr);
+  if (rc != REDLITE_OK) return rc;
+  return cudaMemcpyAsync(out_host, out_dev, nx, cudaMemcpyDeviceToHost, s) == cudaSuccess ? REDLITE_OK
+                                                                                          : REDLITE_ECUDA;
 }
 
 }  // extern "C"

@@ -1282,7 +1282,10 @@ bool fused_supported(int hidden, int max_ffn, int n_tokens, int top_k, int n_exp
 int device_sms() {
   int dev = 0, sms = 0;
   if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  static int cached[64] = {};  // per device; a repeated store writes the same value
+  if (dev >= 0 && dev < 64 && cached[dev] > 0) return cached[dev];
   if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  if (dev >= 0 && dev < 64) cached[dev] = sms;
   return sms;
 }
 
@@ -1294,8 +1297,16 @@ bool fused_wide_items(int hidden, int n_pairs, int min_ffn, int max_ffn, bool ha
 template <int W>
 static cudaError_t launch_shape(const FusedArgs &a, cudaStream_t stream, int sms) {
   const size_t smem = fused_smem_bytes(W);
-  cudaError_t e = cudaFuncSetAttribute(decode_fused_kernel<W>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+  // the shared-memory limit is a per-device attribute of the kernel: set once per device
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
+  static bool smem_set[64] = {};
+  if (dev < 0 || dev >= 64 || !smem_set[dev]) {
+    e = cudaFuncSetAttribute(decode_fused_kernel<W>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    if (dev >= 0 && dev < 64) smem_set[dev] = true;
+  }
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(sms);
   cfg.blockDim = dim3(kCThreads);

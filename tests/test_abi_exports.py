@@ -156,6 +156,34 @@ def test_no_alloc_rejects_on_host(native):
     assert L.redlite_moe_layer_noalloc(p, 1, p, p, 4, ctypes.byref(t1), None, p) == native.REDLITE_EUNSUPPORTED
 
 
+def test_host_buffer_layer_rejects_on_host(native):
+    """The host-buffer entry point refuses null or misaligned buffers, a bad
+    shared expert and an undersized workspace before it enqueues anything
+    (without a GPU any copy or launch would return ECUDA instead), and a
+    zero-token call is a no-op."""
+    L = native.lib()
+    h = ctypes.c_void_p(0x20000)
+    d = ctypes.c_void_p(0x10000)
+    t = native.redlite_moe_table(2048, 512, 512, 64, 512, 0, 0x1000, 0x2000, 0x3000, 1 << 30, 0x4000, None)
+    T = ctypes.byref(t)
+    assert L.redlite_moe_layer_host(h, d, 0, 10, T, None, d, h) == native.REDLITE_OK
+    assert L.redlite_moe_layer_host(None, d, 1, 10, T, None, d, h) == native.REDLITE_EINVAL
+    assert L.redlite_moe_layer_host(h, None, 1, 10, T, None, d, h) == native.REDLITE_EINVAL
+    assert L.redlite_moe_layer_host(h, d, 1, 10, T, None, None, h) == native.REDLITE_EINVAL
+    assert L.redlite_moe_layer_host(h, d, 1, 10, T, None, d, None) == native.REDLITE_EINVAL
+    assert L.redlite_moe_layer_host(h, ctypes.c_void_p(0x10008), 1, 10, T, None, d, h) == native.REDLITE_EINVAL
+    assert L.redlite_moe_layer_host(h, d, 1, 10, T, None, ctypes.c_void_p(0x10004), h) == native.REDLITE_EINVAL
+    assert L.redlite_moe_layer_host(h, d, 65, 10, T, None, d, h) == native.REDLITE_EINVAL  # > max_tokens
+    assert L.redlite_moe_layer_host(h, d, 1, 17, T, None, d, h) == native.REDLITE_EINVAL  # top_k
+    for sh, why in _shared_cases(native):
+        assert L.redlite_moe_layer_host(h, d, 1, 10, T, ctypes.byref(sh), d, h) == native.REDLITE_EINVAL, why
+    small = native.redlite_moe_table(2048, 512, 512, 64, 512, 0, 0x1000, 0x2000, 0x3000, 4096, 0x4000, None)
+    assert L.redlite_moe_layer_host(h, d, 1, 10, ctypes.byref(small), None, d, h) == native.REDLITE_ENOMEM
+    # the packed input buffer: x, then ids, then weights
+    assert L.redlite_moe_host_input_bytes(2048, 64, 10) == 4 * (2048 + 20) * 64
+    assert L.redlite_moe_host_input_bytes(2048, 0, 10) == 0
+
+
 def test_router_and_block_reject_on_host(native):
     L = native.lib()
     p = ctypes.c_void_p(0x10000)

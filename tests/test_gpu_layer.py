@@ -495,3 +495,34 @@ def test_tensor_core_path_odd_widths(P, oracle_lib):
                                oracle_lib.expand_grid(2, g1))
     assert L.read_status() == 0
     assert _rel_err(got, ref) <= TOL_BF16
+
+
+@pytest.mark.parametrize("cfg,T", [(2, None), (4, 9), (5, 200)])
+def test_host_buffer_entry_point_matches_device_call(P, oracle_lib, cfg, T):
+    """redlite_moe_layer_host (packed host inputs -> device, the layer, out ->
+    host, on the table's stream) gives redlite_moe_layer's results, twice in a
+    row, on the fused decode path (1 and 9 tokens) and on the tensor-core path
+    (200 tokens); the first call also matches the fp64 oracle."""
+    from bench import pack_inputs
+
+    w = fixtures.workload(cfg, n_tokens=T) if T else fixtures.workload(cfg)
+    L = layer_for_workload(w)
+    n, H, k = w.x.shape[0], w.hidden, w.top_k
+    ref = _run(L, w.x, w.ids, w.weights)
+    hin = torch.from_numpy(pack_inputs(w.x, w.ids, w.weights)).pin_memory()
+    assert hin.numel() == P.redlite_moe_host_input_bytes(H, n, k)
+    din = torch.empty(hin.numel(), dtype=torch.uint8, device="cuda")
+    dout = torch.empty((n, H), dtype=torch.float32, device="cuda")
+    hout = torch.empty((n, H), dtype=torch.float32).pin_memory()
+    tol = 1e-4 if cfg != 5 else 2e-2
+    for i in range(2):
+        hout.fill_(float("nan"))
+        rc = P.redlite_moe_layer_host(hin, din, n, k, L.table, L.shared, dout, hout)
+        assert rc == P.REDLITE_OK
+        L.stream.synchronize()
+        got = hout.numpy().astype(np.float64)
+        assert np.isfinite(got).all()
+        assert np.abs(got - ref).max() <= 1e-5 * np.abs(ref).max()  # up to the order of fp32 atomic adds
+        if i == 0:
+            assert _rel_err(got, oracle_lib.workload_layer(w)) <= tol
+    assert L.read_status() == 0
