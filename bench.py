@@ -385,35 +385,54 @@ def measure(cfg: int, steps: int, warmup: int, world: int, rank: int, local: int
 
     # end-to-end through the public call with host buffers (pinned), per call
     # (redlite_moe_layer_host): H2D of the call's x, ids and weights (one
-    # packed transfer); the layer; D2H of out.
+    # packed transfer); the layer; D2H of out.  Two pipelines -- each its own
+    # stream, workspace and staging buffers over the same resident experts --
+    # take the calls in turn, so one call's transfers run on the copy engines
+    # while the other's kernels compute.
     e2e = None
     if e2e_on:
-        hbuf = [torch.from_numpy(pk).pin_memory() for pk in packed]
-        ho = [torch.empty((s[0].shape[0], w.hidden), dtype=torch.float32).pin_memory() for s in P.sets]
+        streams = [stream, torch.cuda.Stream(dev)]
+        tables = [L.table, R._native.redlite_moe_table.from_buffer_copy(bytes(L.table))]
+        ws2 = torch.zeros(L.workspace.numel(), dtype=torch.uint8, device=dev)
+        tables[1].workspace = ws2.data_ptr()
+        tables[1].stream = streams[1].cuda_stream
+        R._native._check(R._native.redlite_moe_workspace_reset(tables[1]), "redlite_moe_workspace_reset")
+        hbuf = [[torch.from_numpy(pk).pin_memory() for pk in packed] for _ in range(2)]
+        ho = [[torch.empty((s[0].shape[0], w.hidden), dtype=torch.float32).pin_memory() for s in P.sets]
+              for _ in range(2)]
+        db2 = [dbuf, [torch.empty_like(b) for b in dbuf]]
+        do2 = [do, [torch.empty_like(o) for o in do]]
         e_calls = min(steps * cps, 2400 if nsets > 1 else steps * cps)
+        e_calls += e_calls & 1  # whole pairs of calls
 
         def e2e_call(i):
-            # one public call: the packed inputs host -> device, the layer, out device -> host
-            j = i % nsets
-            rc = R.redlite_moe_layer_host(hbuf[j], dbuf[j], dx[j].shape[0], w.top_k, L.table, L.shared, do[j], ho[j])
+            p, j = i & 1, (i >> 1) % nsets
+            rc = R.redlite_moe_layer_host(hbuf[p][j], db2[p][j], dx[j].shape[0], w.top_k, tables[p], L.shared,
+                                          do2[p][j], ho[p][j])
             if rc != 0:
                 raise RuntimeError(f"redlite_moe_layer_host rc={rc}")
 
-        for i in range(3):
+        for i in range(4):
             e2e_call(i)
-        stream.synchronize()
+        torch.cuda.synchronize()
         barrier()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
+        start_ev, done_ev = torch.cuda.Event(), torch.cuda.Event()
+        e0.record(streams[0])
+        start_ev.record(streams[0])
+        streams[1].wait_event(start_ev)
         for i in range(e_calls):
             e2e_call(i)
-        e1.record(stream)
+        done_ev.record(streams[1])
+        streams[0].wait_event(done_ev)
+        e1.record(streams[0])
         e1.synchronize()
         barrier()
         ems = max_over_ranks(e0.elapsed_time(e1), world, dev)
         e2e = {"value": job_rate(world, e_calls, P.tokens_per_call, ems), "unit": "tokens/s",
-               "h2d_bytes_per_step": int(hbuf[0].nbytes) * cps, "d2h_bytes_per_step": int(ho[0].nbytes) * cps,
-               "calls": e_calls}
+               "h2d_bytes_per_step": int(hbuf[0][0].nbytes) * cps, "d2h_bytes_per_step": int(ho[0][0].nbytes) * cps,
+               "calls": e_calls, "pipelines": 2}
+        del ws2, db2, do2
 
     status = L.read_status()
     if status != 0:

@@ -526,3 +526,40 @@ def test_host_buffer_entry_point_matches_device_call(P, oracle_lib, cfg, T):
         if i == 0:
             assert _rel_err(got, oracle_lib.workload_layer(w)) <= tol
     assert L.read_status() == 0
+
+
+@pytest.mark.parametrize("cfg,T", [(2, None), (5, 200)])
+def test_two_workspaces_on_two_streams(P, cfg, T):
+    """Two tables over the same resident experts, each with its own workspace
+    and stream, take calls in turn (host-buffer entry point) and overlap on
+    the device: every call gives the single-stream result, on the fused
+    decode path and on the tensor-core path."""
+    from bench import pack_inputs
+
+    w = fixtures.workload(cfg, n_tokens=T) if T else fixtures.workload(cfg)
+    L = layer_for_workload(w)
+    n, H, k = w.x.shape[0], w.hidden, w.top_k
+    ref = _run(L, w.x, w.ids, w.weights)
+    streams = [L.stream, torch.cuda.Stream()]
+    t2 = P.redlite_moe_table.from_buffer_copy(bytes(L.table))
+    ws2 = torch.zeros(L.workspace.numel(), dtype=torch.uint8, device="cuda")
+    t2.workspace, t2.stream = ws2.data_ptr(), streams[1].cuda_stream
+    assert P.redlite_moe_workspace_reset(t2) == P.REDLITE_OK
+    tables = [L.table, t2]
+    packed = pack_inputs(w.x, w.ids, w.weights)
+    hin = [torch.from_numpy(packed).pin_memory() for _ in range(2)]
+    din = [torch.empty(hin[0].numel(), dtype=torch.uint8, device="cuda") for _ in range(2)]
+    dout = [torch.empty((n, H), dtype=torch.float32, device="cuda") for _ in range(2)]
+    hout = [[torch.full((n, H), float("nan")).pin_memory() for _ in range(2)] for _ in range(4)]
+    torch.cuda.synchronize()
+    for i in range(8):
+        p = i & 1
+        rc = P.redlite_moe_layer_host(hin[p], din[p], n, k, tables[p], L.shared, dout[p], hout[i >> 1][p])
+        assert rc == P.REDLITE_OK
+    torch.cuda.synchronize()
+    for row in hout:
+        for h in row:
+            got = h.numpy().astype(np.float64)
+            assert np.isfinite(got).all()
+            assert np.abs(got - ref).max() <= 1e-5 * np.abs(ref).max()
+    assert L.read_status() == 0
