@@ -645,8 +645,8 @@ __global__ void __maxnreg__(128) grouped_tc_kernel(TileArgs a) {
               if (c0 + i < U.n_real) atomicAdd(a.out + (size_t)tok * H + r, wgt * __uint_as_float(d0[i]));
             }
           } else {
-            // h of 16 pairs x 128 rows staged as bf16 at the rows' permuted
-            // places, then written as 16-byte pieces (pair i, piece g)
+            // h of 16 pairs x 128 rows staged as bf16 in row order, then
+            // written as 16-byte pieces (pair i, piece g)
             uint32_t d1[16];
             ptx::tmem_ld16(du + (uint32_t)c0, d1);
             __nv_bfloat16 *T = reinterpret_cast<__nv_bfloat16 *>(S.stage) + (ep_stage & 1) * 16 * 128;
