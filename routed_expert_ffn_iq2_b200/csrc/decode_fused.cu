@@ -1302,7 +1302,8 @@ static cudaError_t launch_shape(const FusedArgs &a, cudaStream_t stream, int sms
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
   static bool smem_set[64] = {};
-  if (dev < 0 || dev >= 64 || !smem_set[dev]) {
+  const bool cached = dev >= 0 && dev < 64 && smem_set[dev];
+  if (!cached) {
     e = cudaFuncSetAttribute(decode_fused_kernel<W>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return e;
     if (dev >= 0 && dev < 64) smem_set[dev] = true;
@@ -1321,6 +1322,13 @@ static cudaError_t launch_shape(const FusedArgs &a, cudaStream_t stream, int sms
   static bool pdl_ok = true;  // dependent launch lets a call's table setup overlap the previous call
   cfg.numAttrs = pdl_ok ? 2 : 1;
   e = cudaLaunchKernelEx(&cfg, decode_fused_kernel<W>, a);
+  if (e != cudaSuccess && cached) {
+    // the device's context may have been reset since the attribute was set
+    (void)cudaGetLastError();
+    e = cudaFuncSetAttribute(decode_fused_kernel<W>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return e;
+    e = cudaLaunchKernelEx(&cfg, decode_fused_kernel<W>, a);
+  }
   if (e != cudaSuccess && pdl_ok) {
     (void)cudaGetLastError();
     pdl_ok = false;
