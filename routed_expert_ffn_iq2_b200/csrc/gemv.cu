@@ -180,7 +180,8 @@ __device__ __forceinline__ void step_load_smem(const uint8_t *row, int64_t s, in
   }
 }
 
-constexpr int kGsStages = 4;                 // row groups in flight per CTA
+constexpr int kGsStages = 4;                 // row groups in flight per CTA, at most
+constexpr int kGsPre = 2;                    // steps per warp whose inputs are held in registers
 constexpr int kGsMaxStage = 24 * 1024;       // bytes of one row group (kGemvRows rows)
 
 // Streaming form for matrices whose rows are 16-byte aligned: a persistent
@@ -195,7 +196,7 @@ template <int QT, int NT>
 __global__ void __launch_bounds__(32 * kGemvWarps) gemv_stream_kernel(const uint8_t *__restrict__ W, int64_t rows,
                                                                      int64_t k, const float *__restrict__ x,
                                                                      int ntok, float *__restrict__ y,
-                                                                     int64_t row_bytes, int n_groups) {
+                                                                     int64_t row_bytes, int n_groups, int nst) {
   extern __shared__ __align__(128) uint8_t ring[];
   __shared__ uint64_t full[kGsStages];
   __shared__ float red[2][kGemvWarps][kGemvRows][NT];
@@ -205,42 +206,55 @@ __global__ void __launch_bounds__(32 * kGemvWarps) gemv_stream_kernel(const uint
   const int64_t steps = k / 256;
   const size_t stage_bytes = (size_t)kGemvRows * row_bytes;
   if (tid == 0) {
-    for (int i = 0; i < kGsStages; ++i) ptx::mbar_init(&full[i], 1);
+    for (int i = 0; i < nst; ++i) ptx::mbar_init(&full[i], 1);
     ptx::mbar_fence_init();
   }
   __syncthreads();
   auto issue = [&](int i) {
-    const int st = i % kGsStages;
+    const int st = i % nst;
     const int64_t r0 = (int64_t)(c + (int64_t)i * G) * kGemvRows;
     const uint32_t bytes = (uint32_t)(min((int64_t)kGemvRows, rows - r0) * row_bytes);
     ptx::mbar_expect_tx(&full[st], bytes);
     ptx::bulk_g2s(ring + st * stage_bytes, W + r0 * row_bytes, bytes, &full[st]);
   };
   if (tid == 0)
-    for (int i = 0; i < min(kGsStages, my_n); ++i) issue(i);
+    for (int i = 0; i < min(nst, my_n); ++i) issue(i);
   const int sh = 6 * (lane >> 2);  // this lane's sub-block (Q4_K-style scale field offset)
+  // this lane's 8 inputs of a step (and their sum) for every token
+  auto load_x = [&](int64_t s, float4 (&xa)[NT], float4 (&xb)[NT], float (&xs)[NT]) {
+#pragma unroll
+    for (int t = 0; t < NT; ++t) {
+      xa[t] = xb[t] = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (t < ntok) {
+        const float4 *xp = reinterpret_cast<const float4 *>(x + t * k + 256 * s + 8 * lane);
+        xa[t] = __ldg(xp), xb[t] = __ldg(xp + 1);
+      }
+      xs[t] = (xa[t].x + xa[t].y) + (xa[t].z + xa[t].w) + (xb[t].x + xb[t].y) + (xb[t].z + xb[t].w);
+    }
+  };
+  // a warp's steps are the same for every row group: for one or two tokens
+  // and at most kGsPre steps per warp their inputs are loaded once, while
+  // the first group's weights are still in flight
+  constexpr int kPre = NT <= 2 ? kGsPre : 1;
+  const bool pre = NT <= 2 && steps <= (int64_t)kGemvWarps * kPre;
+  float4 pxa[kPre][NT], pxb[kPre][NT];
+  float pxs[kPre][NT];
+  if (pre) {
+#pragma unroll
+    for (int j = 0; j < kPre; ++j)
+      if (warp + kGemvWarps * j < steps) load_x(warp + kGemvWarps * j, pxa[j], pxb[j], pxs[j]);
+  }
   for (int i = 0; i < my_n; ++i) {
-    const int st = i % kGsStages;
+    const int st = i % nst;
     const int64_t r0 = (int64_t)(c + (int64_t)i * G) * kGemvRows;
-    const bool landed = ptx::mbar_wait(&full[st], (uint32_t)((i / kGsStages) & 1));
+    const bool landed = ptx::mbar_wait(&full[st], (uint32_t)((i / nst) & 1));
     const uint8_t *stage = ring + st * stage_bytes;
     float acc[kGemvRows][NT];
 #pragma unroll
     for (int h = 0; h < kGemvRows; ++h)
 #pragma unroll
       for (int t = 0; t < NT; ++t) acc[h][t] = 0.f;
-    for (int64_t s = warp; s < steps; s += kGemvWarps) {
-      float4 xa[NT], xb[NT];
-      float xs[NT];
-#pragma unroll
-      for (int t = 0; t < NT; ++t) {
-        xa[t] = xb[t] = make_float4(0.f, 0.f, 0.f, 0.f);
-        if (t < ntok) {
-          const float4 *xp = reinterpret_cast<const float4 *>(x + t * k + 256 * s + 8 * lane);
-          xa[t] = __ldg(xp), xb[t] = __ldg(xp + 1);
-        }
-        xs[t] = (xa[t].x + xa[t].y) + (xa[t].z + xa[t].w) + (xb[t].x + xb[t].y) + (xb[t].z + xb[t].w);
-      }
+    auto step_rows = [&](int64_t s, const float4 (&xa)[NT], const float4 (&xb)[NT], const float (&xs)[NT]) {
 #pragma unroll
       for (int h = 0; h < kGemvRows; ++h) {
         if (r0 + h >= rows) break;
@@ -249,6 +263,18 @@ __global__ void __launch_bounds__(32 * kGemvWarps) gemv_stream_kernel(const uint
 #pragma unroll
         for (int t = 0; t < NT; ++t)
           if (t < ntok) acc[h][t] += step_dot<QT>(wd, sh, xa[t], xb[t], xs[t]);
+      }
+    };
+    if (pre) {
+#pragma unroll
+      for (int j = 0; j < kPre; ++j)
+        if (warp + kGemvWarps * j < steps) step_rows(warp + kGemvWarps * j, pxa[j], pxb[j], pxs[j]);
+    } else {
+      for (int64_t s = warp; s < steps; s += kGemvWarps) {
+        float4 xa[NT], xb[NT];
+        float xs[NT];
+        load_x(s, xa, xb, xs);
+        step_rows(s, xa, xb, xs);
       }
     }
 #pragma unroll
@@ -261,9 +287,9 @@ __global__ void __launch_bounds__(32 * kGemvWarps) gemv_stream_kernel(const uint
         if (lane == 0) red[i & 1][warp][h][t] = v;
       }
     __syncthreads();  // every warp is done with the stage and has stored its sums
-    if (tid == 0 && i + kGsStages < my_n) {
+    if (tid == 0 && i + nst < my_n) {
       asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-      issue(i + kGsStages);
+      issue(i + nst);
     }
     const int tr = tid / NT, tt = tid % NT;
     if (tr < kGemvRows && tt < ntok && r0 + tr < rows) {
@@ -279,13 +305,17 @@ template <int QT, int NT>
 cudaError_t launch_stream(const uint8_t *W, int64_t rows, int64_t k, const float *x, int ntok, float *y,
                           int64_t row_bytes, cudaStream_t s) {
   const int n_groups = (int)((rows + kGemvRows - 1) / kGemvRows);
-  const size_t smem = (size_t)kGsStages * kGemvRows * row_bytes;
+  // one row group per CTA up to eight CTAs per SM (every group's copy is in
+  // flight from the start and no CTA works through two); beyond that a
+  // persistent grid with a ring of up to kGsStages groups per CTA
+  const int sms = device_sms();
+  const int grid = min(n_groups, 8 * (sms > 0 ? sms : 148));
+  const int nst = min(kGsStages, (n_groups + grid - 1) / grid);
+  const size_t smem = (size_t)nst * kGemvRows * row_bytes;
   cudaError_t e = cudaFuncSetAttribute(gemv_stream_kernel<QT, NT>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                        (int)smem);
   if (e != cudaSuccess) return e;
-  const int sms = device_sms();
-  const int grid = min(n_groups, 2 * (sms > 0 ? sms : 148));
-  gemv_stream_kernel<QT, NT><<<grid, 32 * kGemvWarps, smem, s>>>(W, rows, k, x, ntok, y, row_bytes, n_groups);
+  gemv_stream_kernel<QT, NT><<<grid, 32 * kGemvWarps, smem, s>>>(W, rows, k, x, ntok, y, row_bytes, n_groups, nst);
   return cudaGetLastError();
 }
 
