@@ -178,6 +178,12 @@ def _traffic(kernel_key: str):
     return d.get("dram_bytes_per_launch")
 
 
+# end-to-end leg: pipelines (stream, workspace, staging buffers) that take the
+# calls in turn; three keep the copy engines and the SMs busy for the
+# prefill call (copy in, layer and copy out of ~0.6 + 0.8 + 0.6 ms)
+E2E_PIPES = 3
+
+
 def layer_for_workload(w, experts=None, max_tokens=None, extra_pool: int = 0, device: str = "cuda"):
     """A MoeLayer holding the experts of a fixtures.Workload (by default the
     selected ones) and its shared expert, uploaded through the C ABI."""
@@ -385,54 +391,62 @@ def measure(cfg: int, steps: int, warmup: int, world: int, rank: int, local: int
 
     # end-to-end through the public call with host buffers (pinned), per call
     # (redlite_moe_layer_host): H2D of the call's x, ids and weights (one
-    # packed transfer); the layer; D2H of out.  Two pipelines -- each its own
-    # stream, workspace and staging buffers over the same resident experts --
-    # take the calls in turn, so one call's transfers run on the copy engines
-    # while the other's kernels compute.
+    # packed transfer); the layer; D2H of out.  E2E_PIPES pipelines -- each
+    # its own stream, workspace and staging buffers over the same resident
+    # experts -- take the calls in turn, so calls' transfers run on the copy
+    # engines while other calls' kernels compute (a pipeline's own copy in,
+    # layer and copy out stay in order on its stream).
     e2e = None
     if e2e_on:
-        streams = [stream, torch.cuda.Stream(dev)]
-        tables = [L.table, R._native.redlite_moe_table.from_buffer_copy(bytes(L.table))]
-        ws2 = torch.zeros(L.workspace.numel(), dtype=torch.uint8, device=dev)
-        tables[1].workspace = ws2.data_ptr()
-        tables[1].stream = streams[1].cuda_stream
-        R._native._check(R._native.redlite_moe_workspace_reset(tables[1]), "redlite_moe_workspace_reset")
-        hbuf = [[torch.from_numpy(pk).pin_memory() for pk in packed] for _ in range(2)]
+        NP = E2E_PIPES
+        streams = [stream] + [torch.cuda.Stream(dev) for _ in range(NP - 1)]
+        tables, extra_ws = [L.table], []
+        for p in range(1, NP):
+            t = R._native.redlite_moe_table.from_buffer_copy(bytes(L.table))
+            ws = torch.zeros(L.workspace.numel(), dtype=torch.uint8, device=dev)
+            t.workspace, t.stream = ws.data_ptr(), streams[p].cuda_stream
+            R._native._check(R._native.redlite_moe_workspace_reset(t), "redlite_moe_workspace_reset")
+            tables.append(t)
+            extra_ws.append(ws)
+        hbuf = [[torch.from_numpy(pk).pin_memory() for pk in packed] for _ in range(NP)]
         ho = [[torch.empty((s[0].shape[0], w.hidden), dtype=torch.float32).pin_memory() for s in P.sets]
-              for _ in range(2)]
-        db2 = [dbuf, [torch.empty_like(b) for b in dbuf]]
-        do2 = [do, [torch.empty_like(o) for o in do]]
+              for _ in range(NP)]
+        db2 = [dbuf] + [[torch.empty_like(b) for b in dbuf] for _ in range(NP - 1)]
+        do2 = [do] + [[torch.empty_like(o) for o in do] for _ in range(NP - 1)]
         e_calls = min(steps * cps, 2400 if nsets > 1 else steps * cps)
-        e_calls += e_calls & 1  # whole pairs of calls
+        e_calls = max(NP, e_calls - e_calls % NP)  # whole rounds of the pipelines
 
         def e2e_call(i):
-            p, j = i & 1, (i >> 1) % nsets
+            p, j = i % NP, (i // NP) % nsets
             rc = R.redlite_moe_layer_host(hbuf[p][j], db2[p][j], dx[j].shape[0], w.top_k, tables[p], L.shared,
                                           do2[p][j], ho[p][j])
             if rc != 0:
                 raise RuntimeError(f"redlite_moe_layer_host rc={rc}")
 
-        for i in range(4):
+        for i in range(2 * NP):
             e2e_call(i)
         torch.cuda.synchronize()
         barrier()
         e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        start_ev, done_ev = torch.cuda.Event(), torch.cuda.Event()
+        start_ev = torch.cuda.Event()
         e0.record(streams[0])
         start_ev.record(streams[0])
-        streams[1].wait_event(start_ev)
+        for st in streams[1:]:
+            st.wait_event(start_ev)
         for i in range(e_calls):
             e2e_call(i)
-        done_ev.record(streams[1])
-        streams[0].wait_event(done_ev)
+        for st in streams[1:]:
+            ev = torch.cuda.Event()
+            ev.record(st)
+            streams[0].wait_event(ev)
         e1.record(streams[0])
         e1.synchronize()
         barrier()
         ems = max_over_ranks(e0.elapsed_time(e1), world, dev)
         e2e = {"value": job_rate(world, e_calls, P.tokens_per_call, ems), "unit": "tokens/s",
                "h2d_bytes_per_step": int(hbuf[0][0].nbytes) * cps, "d2h_bytes_per_step": int(ho[0][0].nbytes) * cps,
-               "calls": e_calls, "pipelines": 2}
-        del ws2, db2, do2
+               "calls": e_calls, "pipelines": NP}
+        del extra_ws, db2, do2
 
     status = L.read_status()
     if status != 0:

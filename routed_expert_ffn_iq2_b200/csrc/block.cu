@@ -27,6 +27,9 @@ __global__ void __launch_bounds__(256) norm_router_kernel(const float *__restric
                                                           const float *__restrict__ router_w, int n_experts,
                                                           float *__restrict__ xn, float *__restrict__ logits) {
   extern __shared__ float4 sx[];  // [kNrTok][hidden / 4]
+  // the router kernel that follows may launch now; it waits for this grid
+  // before it reads the logits
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int t0 = blockIdx.y * kNrTok, nt = min(kNrTok, n_tokens - t0);
   const int h4 = hidden / 4;

@@ -28,6 +28,11 @@ template <int PER>
 __global__ void __launch_bounds__(32 * kRouterWarps) route_topk_kernel(const float *__restrict__ logits, int n_tokens,
                                                                     int n_experts, int top_k, int32_t *__restrict__ ids,
                                                                     float *__restrict__ weights) {
+  // launched as a programmatic dependent of the kernel that writes the
+  // logits: wait for it, then let the layer kernel that follows start its
+  // own prologue (it waits for this grid before it reads ids and weights)
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
   const int lane = threadIdx.x & 31;
   const int t = blockIdx.x * kRouterWarps + (threadIdx.x >> 5);
   if (t >= n_tokens) return;
@@ -78,12 +83,28 @@ __global__ void __launch_bounds__(32 * kRouterWarps) route_topk_kernel(const flo
 cudaError_t launch_route_topk(const float *logits, int n_tokens, int n_experts, int top_k, int32_t *ids,
                               float *weights, cudaStream_t stream) {
   const unsigned blocks = (unsigned)((n_tokens + kRouterWarps - 1) / kRouterWarps);
-  if (n_experts <= 32 * 16)
-    route_topk_kernel<16><<<blocks, 32 * kRouterWarps, 0, stream>>>(logits, n_tokens, n_experts, top_k, ids, weights);
-  else
-    route_topk_kernel<kRouterPerLane>
-        <<<blocks, 32 * kRouterWarps, 0, stream>>>(logits, n_tokens, n_experts, top_k, ids, weights);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(blocks);
+  cfg.blockDim = dim3(32 * kRouterWarps);
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  auto launch = [&](cudaLaunchConfig_t &c) {
+    return n_experts <= 32 * 16
+               ? cudaLaunchKernelEx(&c, route_topk_kernel<16>, logits, n_tokens, n_experts, top_k, ids, weights)
+               : cudaLaunchKernelEx(&c, route_topk_kernel<kRouterPerLane>, logits, n_tokens, n_experts, top_k, ids,
+                                    weights);
+  };
+  cudaError_t e = launch(cfg);
+  if (e != cudaSuccess) {  // without the dependent-launch attribute
+    (void)cudaGetLastError();
+    cfg.numAttrs = 0;
+    e = launch(cfg);
+  }
+  return e;
 }
 
 }  // namespace redlite
