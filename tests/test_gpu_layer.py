@@ -583,3 +583,31 @@ def test_fused_decode_is_repeatable(P, cfg):
     scale = np.abs(ref).max()
     for o in outs[1:]:
         assert np.abs(o.cpu().numpy().astype(np.float64) - ref).max() <= 1e-5 * scale
+
+
+@pytest.mark.parametrize("H,F,T,k,with_shared", [(768, 512, 1, 6, False), (768, 256, 5, 4, True),
+                                                 (1280, 512, 1, 8, True), (1280, 256, 3, 6, False)])
+def test_fused_decode_odd_block_counts(P, oracle_lib, H, F, T, k, with_shared):
+    """The fused decode kernel on hidden sizes whose 256-input block count is
+    not a power of two (768: 3 blocks, items of two row tiles with some warps
+    idle; 1280: 5 blocks, items of one tile), tiled widths 256 and 512, one
+    and several tokens, with and without a shared expert, against the fp64
+    oracle."""
+    E, seed = 16, 8080 + H + F + T
+    g2, g1 = fixtures.make_grid(seed, 1), fixtures.make_grid(seed, 2)
+    experts = [fixtures.make_expert(seed, 1 + (e % 2), H, F, e) for e in range(E)]
+    shared = fixtures.make_expert(seed, 2, H, F, 999) if with_shared else None
+    L = P.MoeLayer(H, E, F, T, k, g2, g1, pool_bytes=(E + 2) * fixtures.expert_bytes(1, H, F) + 4096)
+    assert L.upload(list(range(E)), experts) == 0
+    if with_shared:
+        assert L.set_shared(shared) == 0
+    assert L.table.min_ffn >= 256  # the tiled fast path
+    st = fixtures.Stream(seed, 3)
+    ids = np.stack([np.argsort(st.uniform(E))[:k] for _ in range(T)]).astype(np.int32)
+    wt = (0.1 + st.uniform(T * k)).astype(np.float32).reshape(T, k)
+    x = fixtures.make_x(seed, T, H)
+    got = _run(L, x, ids, wt)
+    ref = oracle_lib.moe_layer(x, ids, wt, experts, shared, oracle_lib.expand_grid(1, g2),
+                               oracle_lib.expand_grid(2, g1))
+    assert L.read_status() == 0
+    assert _rel_err(got, ref) <= TOL_FP32
