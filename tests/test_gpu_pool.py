@@ -109,3 +109,60 @@ def test_pool_feeds_the_layer(P, oracle_lib):
     assert np.abs(got - ref(A)).max() <= TOL * np.abs(ref(A)).max()
     pool.close()
     del keep
+
+
+def test_pool_pipelined_calls_with_evictions(P, oracle_lib):
+    """Sixteen top-10 calls over 40 experts through a 24-slot pool, enqueued
+    back to back: each call's slots are released by an event recorded after
+    it, with no host synchronisation in between except when the pool reports
+    every candidate slot in flight (EAGAIN).  A fill for a later selection
+    must never land in a slot that an earlier, still running call reads, so
+    every call's output matches the fp64 oracle at the end."""
+    w = fixtures.workload(2)
+    H, E, F, k = w.hidden, w.n_experts, w.ffn, w.top_k
+    st = fixtures.Stream(fixtures.SEED_BASE + 2, 77)
+    sels = [[12 * u + 3 for u in fixtures.draw_distinct_nonadjacent(st, k, 40)] for _ in range(16)]
+    cap = 24
+    L = P.MoeLayer(H, E, F, 1, k, w.grid_iq2, w.grid_iq1, pool_bytes=16)
+    L.table.min_ffn = F
+    gb = fixtures.matrix_bytes(1, F, H)
+    slot_bytes = 2 * ((gb + 15) // 16 * 16) + fixtures.matrix_bytes(1, H, F)
+    slots = torch.zeros(cap * slot_bytes, dtype=torch.uint8, device="cuda")
+    host = (P.redlite_moe_expert * E)()
+    keep = []
+    for e in sorted(set(sum(sels, []))):
+        ex = w.expert(e)
+        mats = [np.ascontiguousarray(P.redlite_moe_pack_matrix(1, r, c, m))
+                for m, (r, c) in zip((ex.gate, ex.up, ex.down), ((F, H), (F, H), (H, F)))]
+        keep += mats
+        host[e] = P.redlite_moe_expert(1, F, *[m.ctypes.data for m in mats])
+    pool = P.SlotPool(E, cap)
+    copy_s, comp_s = torch.cuda.Stream(), torch.cuda.current_stream()
+    x = torch.from_numpy(w.x).cuda()
+    wt = torch.from_numpy(w.weights).cuda()
+    outs, waits = [], 0
+    for sel in sels:
+        ids = torch.tensor([sel], dtype=torch.int32, device="cuda")
+        while True:
+            rc, tok = pool.acquire(sel, host, H, slots, slot_bytes, L.table_dev, copy_s, comp_s)
+            if rc == P.REDLITE_OK:
+                break
+            assert rc == P.REDLITE_EAGAIN
+            waits += 1
+            assert waits < 64
+            comp_s.synchronize()  # the calls in flight end; their events complete
+        outs.append(L(x, ids, wt))
+        assert pool.release(tok, comp_s) == 0
+    torch.cuda.synchronize()
+    assert L.read_status() == 0
+    assert pool.counters.evictions > 0 and pool.counters.hits > 0
+    g2 = oracle_lib.expand_grid(1, w.grid_iq2)
+    for sel, o in zip(sels, outs):
+        experts = [None] * E
+        for e in sel:
+            experts[e] = w.expert(e)
+        ref = oracle_lib.moe_layer(w.x, np.array([sel], np.int32), w.weights, experts, None, g2, None)
+        got = o.cpu().numpy().astype(np.float64)
+        assert np.abs(got - ref).max() <= TOL * np.abs(ref).max()
+    pool.close()
+    del keep
