@@ -864,11 +864,13 @@ __global__ void __launch_bounds__(kCThreads, 1) decode_fused_kernel(FusedArgs a)
 
   // ---- the item split.  Gate/up items in contiguous ranges of N1 / G, the
   // first N1 mod G CTAs taking one more (so the h slices that complete last
-  // are those of the first few experts).  Down items in time slots: first one
-  // each for the CTAs without an extra gate/up item, then one per CTA per
-  // round, in reverse item order, so the down items that need the late slices
-  // come last.  (The host keeps every CTA's list within kMaxItems; the clamps
-  // only guard the shared-memory list.)
+  // are those of the first few experts).  Down items: many per CTA in
+  // contiguous ranges; few (at most two per CTA without an extra gate/up
+  // item) in ranges of one or two on those CTAs only; otherwise in time
+  // slots: first one each for the CTAs without an extra gate/up item, then
+  // one per CTA per round, in reverse item order, so the down items that need
+  // the late slices come last.  (The host keeps every CTA's list within
+  // kMaxItems; the clamps only guard the shared-memory list.)
   struct Split {
     int b1, my1, e1, first2, my2, b2;  // b2 >= 0: down items in one contiguous range
   };
@@ -885,6 +887,16 @@ __global__ void __launch_bounds__(kCThreads, 1) decode_fused_kernel(FusedArgs a)
       const unsigned uG = (unsigned)G, uN2 = (unsigned)N2, rc = (unsigned)(G - 1 - cta);
       p.b2 = (int)(rc * uN2 / uG);
       p.my2 = (int)((rc + 1) * uN2 / uG) - p.b2;
+      p.first2 = -1;
+    } else if (N2 <= 2 * (G - p.e1)) {
+      // few down items: only the CTAs without an extra gate/up item take
+      // them, in contiguous ranges of one or two (two consecutive items of an
+      // expert share its h slices and the warps' limbs), the single ones
+      // first: the lowest items, whose h comes from the extra gate/up items
+      // and so completes last, go to CTAs that have one down item
+      const int nA = G - p.e1, q = N2 / nA, n_lo = nA - (N2 - q * nA), ia = cta - p.e1;
+      p.b2 = ia < 0 ? 0 : ia < n_lo ? ia * q : n_lo * q + (ia - n_lo) * (q + 1);
+      p.my2 = ia < 0 ? 0 : q + (ia >= n_lo);
       p.first2 = -1;
     } else {
       p.b2 = -1;
