@@ -8,23 +8,30 @@
 // Structure (one CTA of 16 warps per SM, cooperative launch so all CTAs are
 // resident):
 //   prologue  every CTA copies the byte-permute selector tables into shared
-//             memory, buckets the (token, slot) pairs by expert (stable,
-//             identical in every CTA), reads the selected slots'
-//             descriptors and converts the activations to fixed-point limbs;
+//             memory and replicates them, buckets the (token, slot) pairs by
+//             expert (identical in every CTA; one warp for calls of at most
+//             32 pairs), reads the selected slots' descriptors, builds its
+//             own item list and starts the first copies;
 //   items     the work is a list of items of up to 16 warp units (a unit is
 //             one tile-block, 16 rows x 256 inputs of a packed matrix, or
 //             for large calls two adjacent ones) for a chunk of <= 2 tokens:
 //             phase 1 items are gate and up tiles of the same rows (their
 //             reduction yields h = SiLU(g) * u for those rows), phase 2
 //             items are groups of down tiles (their reduction is added to
-//             out with the router weight).  Items are split evenly over the
-//             CTAs; warp w of a CTA handles unit w of each item;
-//   streams   each warp streams its own units by bulk copy into a private
-//             ring (4 stages, 2 for two-block units), so warps do not wait
-//             for each other to load; a warp decodes its unit, writes its
+//             out with the router weight).  Gate/up items go to the CTAs in
+//             contiguous ranges; down items in contiguous ranges, or, when
+//             there are few, one or two consecutive ones to each CTA without
+//             an extra gate/up item, or in time slots (see the item split);
+//             warp w of a CTA handles unit w of each item;
+//   streams   stage-major rings: a stage holds one item's units, filled by
+//             one or two bulk copies (an item's tile-blocks are contiguous
+//             in the resident layout); 4 stages, 2 for two-block units; the
+//             last warp done with a stage refills it with the item a ring
+//             ahead.  A warp converts its inputs to limbs when the item's
+//             tokens or input block change, decodes its unit, writes its
 //             partial sums to the item's reduction slot and moves on; the
-//             item's reducer (warp item mod 16) adds the partials once all
-//             are in;
+//             item's reducer (warp item mod 16) adds the partials a few
+//             items later;
 //   slices    no grid barrier: the reducer of a gate/up item counts the
 //             16-row tiles of h it wrote per (token chunk, 256-input slice)
 //             with a release add; a warp about to decode a down tile-block
