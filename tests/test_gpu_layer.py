@@ -586,13 +586,17 @@ def test_fused_decode_is_repeatable(P, cfg):
 
 
 @pytest.mark.parametrize("H,F,T,k,with_shared", [(768, 512, 1, 6, False), (768, 256, 5, 4, True),
-                                                 (1280, 512, 1, 8, True), (1280, 256, 3, 6, False)])
+                                                 (1280, 512, 1, 8, True), (1280, 256, 3, 6, False),
+                                                 (1280, 256, 1, 8, False), (1792, 1280, 1, 3, False)])
 def test_fused_decode_odd_block_counts(P, oracle_lib, H, F, T, k, with_shared):
     """The fused decode kernel on hidden sizes whose 256-input block count is
     not a power of two (768: 3 blocks, items of two row tiles with some warps
-    idle; 1280: 5 blocks, items of one tile), tiled widths 256 and 512, one
-    and several tokens, with and without a shared expert, against the fp64
-    oracle."""
+    idle; 1280: 5 blocks, items of one tile; 1792: 7), tiled widths 256 to
+    1280, one and several tokens, with and without a shared expert, against
+    the fp64 oracle.  On 148 SMs the last two sit on either side of the
+    split's few-down-items rule: 128 gate/up and 40 down items (exactly two
+    down items for each of the 20 CTAs without an extra gate/up item), and
+    240 and 114 (two more than such CTAs can take in pairs: time slots)."""
     E, seed = 16, 8080 + H + F + T
     g2, g1 = fixtures.make_grid(seed, 1), fixtures.make_grid(seed, 2)
     experts = [fixtures.make_expert(seed, 1 + (e % 2), H, F, e) for e in range(E)]
